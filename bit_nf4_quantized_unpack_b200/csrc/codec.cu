@@ -1,0 +1,238 @@
+// codec.cu -- NF4 quantization with double-quantized constants, and the standalone
+// double dequantization (page "QLoRA", itwiki.kr, sections "4비트 NormalFloat(NF4)" and
+// "이중 양자화"). All three kernels are HBM-bound streaming passes.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "nf4_device.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kQuantThreads = 256;
+constexpr int kMaxQuantCtas = 148 * 8;
+
+// NF4 code of x in [-1, 1]: the number of thresholds <= x, by a 4-level bisection in
+// registers (thresholds are kernel parameters).
+__device__ __forceinline__ uint32_t nf4_code(float x, const Nf4Thresholds& th) {
+  uint32_t c = (x >= th.t[7]) ? 8u : 0u;
+  const float t1 = c ? th.t[11] : th.t[3];
+  c += (x >= t1) ? 4u : 0u;
+  const float t2 = (c & 8u) ? ((c & 4u) ? th.t[13] : th.t[9]) : ((c & 4u) ? th.t[5] : th.t[1]);
+  c += (x >= t2) ? 2u : 0u;
+  const float a0 = (c & 4u) ? th.t[4] : th.t[0];
+  const float a1 = (c & 4u) ? th.t[6] : th.t[2];
+  const float b0 = (c & 4u) ? th.t[12] : th.t[8];
+  const float b1 = (c & 4u) ? th.t[14] : th.t[10];
+  const float lo = (c & 2u) ? a1 : a0;
+  const float hi = (c & 2u) ? b1 : b0;
+  const float t3 = (c & 8u) ? hi : lo;
+  c += (x >= t3) ? 1u : 0u;
+  return c;
+}
+
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const uint16_t* p, float (&v)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Level 1: one 64-block per group of 8 lanes (8 elements per lane). Writes the packed
+// codes, the fp32 absmax of each block, and one fp64 partial sum of absmax per CTA.
+template <typename T>
+__global__ void __launch_bounds__(kQuantThreads)
+    k_quantize_blocks(const T* __restrict__ W, int64_t nblocks, const Nf4Thresholds th,
+                      uint8_t* __restrict__ codes, float* __restrict__ absmax,
+                      double* __restrict__ partial) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 7;
+  const unsigned gmask = 0xFFu << (lane & 24);
+  const int64_t per_cta = kQuantThreads / 8;
+  double acc = 0.0;
+  for (int64_t b = blockIdx.x * per_cta + threadIdx.x / 8; b < nblocks;
+       b += static_cast<int64_t>(gridDim.x) * per_cta) {
+    float v[8];
+    load8(W + b * 64 + sub * 8, v);
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+    m = fmaxf(m, __shfl_xor_sync(gmask, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(gmask, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(gmask, m, 4));
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float x = (m > 0.f) ? __fdiv_rn(v[i], m) : 0.f;
+      packed |= nf4_code(x, th) << (4 * i);
+    }
+    reinterpret_cast<uint32_t*>(codes + b * 32)[sub] = packed;
+    if (sub == 0) {
+      absmax[b] = m;
+      acc += static_cast<double>(m);
+    }
+  }
+  __shared__ double red[kQuantThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if (lane == 0) red[threadIdx.x / 32] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < kQuantThreads / 32; ++i) s += red[i];
+    partial[blockIdx.x] = s;
+  }
+}
+
+// Level 2a: the one mean of all block constants (fp64 sum, one rounding to fp32).
+__global__ void __launch_bounds__(1024)
+    k_constants_mean(const double* __restrict__ partial, int nparts, int64_t nblocks,
+                     float* __restrict__ mean) {
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) acc += partial[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < static_cast<int>(blockDim.x / 32); ++i) s += red[i];
+    mean[0] = __double2float_rn(s / static_cast<double>(nblocks));
+  }
+}
+
+// Index of entry i of T8 (ascending) -> its E4M3 bit pattern.
+__device__ __forceinline__ uint32_t t8_index_to_code(int i) {
+  return (i < 126) ? (0xFEu - static_cast<uint32_t>(i)) : (i == 126 ? 0u : static_cast<uint32_t>(i - 126));
+}
+
+// Level 2b: one warp per 256-block of constants, 8 constants per lane.
+__global__ void __launch_bounds__(256)
+    k_double_quantize(const float* __restrict__ absmax, int64_t nblocks,
+                      const float* __restrict__ mean_p, const T8Thresholds th,
+                      uint8_t* __restrict__ c2, float* __restrict__ c1) {
+  __shared__ float sth[kT8Size - 1];
+  for (int i = threadIdx.x; i < kT8Size - 1; i += blockDim.x) sth[i] = th.t[i];
+  __syncthreads();
+  const float mean = *mean_p;
+  const int lane = threadIdx.x & 31;
+  const int64_t ndq = (nblocks + 255) / 256;
+  for (int64_t b = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; b < ndq;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x / 32) {
+    const int64_t j0 = b * 256 + lane * 8;
+    float cc[8];
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      cc[i] = (j0 + i < nblocks) ? __fsub_rn(absmax[j0 + i], mean) : 0.f;
+      m = fmaxf(m, fabsf(cc[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float y = (m > 0.f) ? __fdiv_rn(cc[i], m) : 0.f;
+      int pos = 0;  // number of thresholds <= y
+#pragma unroll
+      for (int step = 128; step >= 1; step >>= 1)
+        if (pos + step <= kT8Size - 1 && sth[pos + step - 1] <= y) pos += step;
+      out[i / 4] |= t8_index_to_code(pos) << (8 * (i % 4));
+    }
+    if (j0 + 8 <= nblocks) {
+      reinterpret_cast<uint2*>(c2 + j0)[0] = make_uint2(out[0], out[1]);
+    } else {
+      for (int i = 0; i < 8 && j0 + i < nblocks; ++i)
+        c2[j0 + i] = static_cast<uint8_t>(out[i / 4] >> (8 * (i % 4)));
+    }
+    if (lane == 0) c1[b] = m;
+  }
+}
+
+// Standalone double dequantization: one thread per 8 codes (one 32-bit word).
+__global__ void __launch_bounds__(256)
+    k_dequant(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ c2,
+              const float* __restrict__ c1, const float* __restrict__ mean_p, int64_t nwords,
+              uint4* __restrict__ out) {
+  __shared__ float lut[16];
+  if (threadIdx.x < 16) lut[threadIdx.x] = nf4_level(threadIdx.x);
+  __syncthreads();
+  const float mean = *mean_p;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = i >> 3;  // 64-block of this word
+    const float s = block_scale(c2[j], c1[j >> 8], mean);
+    const uint32_t w = __ldg(codes + i);
+    uint32_t o[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float a = __fmul_rn(lut[(w >> (8 * p)) & 15u], s);
+      const float b = __fmul_rn(lut[(w >> (8 * p + 4)) & 15u], s);
+      o[p] = pack_bf16x2_rn(a, b);
+    }
+    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+int quant_ctas(int64_t nblocks) {
+  const int64_t want = (nblocks + kQuantThreads / 8 - 1) / (kQuantThreads / 8);
+  const int cap = num_sms() * 8 < kMaxQuantCtas ? num_sms() * 8 : kMaxQuantCtas;
+  return static_cast<int>(want < cap ? (want < 1 ? 1 : want) : cap);
+}
+
+}  // namespace
+
+size_t quantize_workspace_bytes(int64_t n, int64_t k) {
+  const int64_t nblocks = n * k / 64;
+  return align_up(static_cast<size_t>(nblocks) * 4, 256) + kMaxQuantCtas * sizeof(double);
+}
+
+cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, uint8_t* codes,
+                            uint8_t* c2, float* c1, float* mean, void* ws, cudaStream_t st) {
+  const int64_t nblocks = n * k / 64;
+  float* absmax = static_cast<float*>(ws);
+  double* partial = reinterpret_cast<double*>(static_cast<char*>(ws) +
+                                              align_up(static_cast<size_t>(nblocks) * 4, 256));
+  const int ctas = quant_ctas(nblocks);
+  if (w_bf16)
+    k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
+        static_cast<const uint16_t*>(W), nblocks, nf4_thresholds(), codes, absmax, partial);
+  else
+    k_quantize_blocks<float><<<ctas, kQuantThreads, 0, st>>>(
+        static_cast<const float*>(W), nblocks, nf4_thresholds(), codes, absmax, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_constants_mean<<<1, 1024, 0, st>>>(partial, ctas, nblocks, mean);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t ndq = (nblocks + 255) / 256;
+  int64_t g = (ndq + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (g > cap) g = cap;
+  k_double_quantize<<<static_cast<int>(g), 256, 0, st>>>(absmax, nblocks, mean, t8_thresholds(),
+                                                         c2, c1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t st) {
+  const int64_t nwords = w.n_out * w.k_in / 8;
+  int64_t g = (nwords + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+  if (g > cap) g = cap;
+  k_dequant<<<static_cast<int>(g), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(w.codes),
+                                                 w.c2, w.c1, w.mean, nwords,
+                                                 reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

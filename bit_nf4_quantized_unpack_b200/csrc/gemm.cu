@@ -1,0 +1,752 @@
+// gemm.cu -- the QLoRA linear layer on the 5th-generation tensor cores (tcgen05, TMEM
+// accumulators, TMA-fed shared memory) for M > 16 tokens.
+//
+// Forward (page "QLoRA", itwiki.kr, section "계산 방식"; alpha/r from page
+// "quantization", minnong511 blog):  Y = X W_hat^T + scale (X A) B
+// Backward (same sections): G = dY B^T, dX = dY W_hat + scale G A^T,
+//                           dA = scale X^T G, dB = scale T^T dY.
+//
+// Kernels
+//  k_fused_nf4_gemm<kForward>: D[n, m] = sum_k W_hat[n, k] X[m, k] + sum_j B[j, n] Ts[m, j]
+//      W_hat is never written to memory: packed codes arrive by TMA, eight dequant
+//      warps expand them (double dequantization, bit-exact bf16) straight into the
+//      128B-swizzled shared-memory operand layout, and one thread issues
+//      tcgen05.mma into a 128 x 256 fp32 TMEM accumulator. The LoRA product is one
+//      more pipeline step on the same accumulator with operands Ts = bf16(scale T)
+//      and B (r padded to a multiple of 16 with zeros by TMA).
+//  k_fused_nf4_gemm<kDgrad>: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[k, j] Gs[m, j]
+//      the same pipeline with W_hat dequantized into the MN-major operand layout
+//      (contraction over the output features n).
+//  k_lora_gemm: the rank-r products T = X A, G = dY B^T (split over the contraction)
+//      and dA, dB (contraction over tokens; G and T enter as bf16 hi + lo pairs so
+//      that the gradients keep fp32-level accuracy).
+// Small elementwise kernels finalize the split partial sums.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "internal.h"
+#include "nf4_device.cuh"
+
+namespace qlora {
+namespace {
+
+// ================================================================== fused NF4 GEMM
+enum class Mode { kForward, kDgrad };
+
+constexpr int kFusedThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 dequant + epilogue
+constexpr int kStages = 4;
+constexpr int kTileRows = 128;  // D rows on the weight side (n forward, k dgrad) = TMEM lanes
+constexpr int kTileCols = 256;  // D columns on the token side (m) = TMEM columns
+constexpr int kBK = 64;         // contraction per pipeline step
+constexpr uint32_t kActBytes = kTileCols * kBK * 2;   // 32 KB
+constexpr uint32_t kWBytes = kTileRows * kBK * 2;     // 16 KB
+constexpr uint32_t kCodeBytes = kTileRows * kBK / 2;  // 4 KB
+constexpr uint32_t kFusedSmem = kStages * (kActBytes + kWBytes + kCodeBytes) + 1024 + 256;
+
+struct FusedArgs {
+  const uint8_t* c2;
+  const float* c1;
+  const float* mean;
+  int64_t N, K, M;    // W is N x K, M tokens
+  int ext_mmas;       // 16-wide MMAs of the LoRA step (0: no LoRA step)
+  uint16_t* out;      // [M, out_ld] bf16
+  int64_t out_ld;     // N (forward) or K (dgrad)
+  int64_t out_rows;   // valid D rows: N (forward) or K (dgrad)
+  int* err;
+};
+
+__device__ __forceinline__ void record_error(int* err, volatile int* abort, int code) {
+  atomicCAS(err, 0, code);
+  *abort = 1;
+}
+
+// Wait bounded by time only (used while draining after an abort).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
+}
+
+template <Mode MODE>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    k_fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_codes,
+                     const __grid_constant__ CUtensorMap tm_act,
+                     const __grid_constant__ CUtensorMap tm_ext_w,
+                     const __grid_constant__ CUtensorMap tm_ext_act, const FusedArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* act_s = smem;                           // [kStages][kActBytes]  token-side operand
+  uint8_t* w_s = act_s + kStages * kActBytes;      // [kStages][kWBytes]    weight-side operand
+  uint8_t* code_s = w_s + kStages * kWBytes;       // [kStages][kCodeBytes] packed codes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(code_s + kStages * kCodeBytes);
+  uint64_t* full = bars;                 // TMA data of the stage landed
+  uint64_t* deq = bars + kStages;        // dequantized weight tile of the stage written
+  uint64_t* empty = bars + 2 * kStages;  // MMAs reading the stage completed
+  uint64_t* acc_full = bars + 3 * kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileRows;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kTileCols;
+  const int64_t contraction = (MODE == Mode::kForward) ? args.K : args.N;
+  const int ksteps = static_cast<int>((contraction + kBK - 1) / kBK);
+  const int total = ksteps + (args.ext_mmas > 0 ? 1 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&deq[s], 4);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_act);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTileCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int step = 0; step < total; ++step) {
+        const int s = step % kStages;
+        const uint32_t use = step / kStages;
+        if (step >= kStages && !mbar_wait(&empty[s], (use - 1) & 1u, abort_flag)) {
+          record_error(args.err, abort_flag, kErrTimeoutProducer);
+          break;
+        }
+        if (step < ksteps) {
+          mbar_arrive_expect_tx(&full[s], kActBytes + kCodeBytes);
+          if (MODE == Mode::kForward)
+            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &full[s], step * (kBK / 2),
+                        static_cast<int>(row0));
+          else
+            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &full[s],
+                        static_cast<int>(row0 / 2), step * kBK);
+          tma_load_2d(act_s + s * kActBytes, &tm_act, &full[s], step * kBK,
+                      static_cast<int>(m0));
+        } else {
+          mbar_arrive_expect_tx(&full[s], kWBytes + kActBytes);
+          if (MODE == Mode::kForward) {
+            // B [r, N] as an MN-major operand: two 64-wide chunks of n, rows j >= r are 0
+            tma_load_2d(w_s + s * kWBytes, &tm_ext_w, &full[s], static_cast<int>(row0), 0);
+            tma_load_2d(w_s + s * kWBytes + 8192, &tm_ext_w, &full[s],
+                        static_cast<int>(row0) + 64, 0);
+          } else {
+            // A [K, r] as a K-major operand (columns j >= r are 0)
+            tma_load_2d(w_s + s * kWBytes, &tm_ext_w, &full[s], 0, static_cast<int>(row0));
+          }
+          tma_load_2d(act_s + s * kActBytes, &tm_ext_act, &full[s], 0, static_cast<int>(m0));
+        }
+        ++issued;
+      }
+      if (*abort_flag) {  // let copies already in flight land before the CTA exits
+        for (int step = std::max(0, issued - kStages); step < issued; ++step)
+          mbar_wait_drain(&full[step % kStages], (step / kStages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_main =
+          idesc_bf16_f32(kTileRows, kTileCols, MODE == Mode::kDgrad, false);
+      constexpr uint32_t idesc_ext =
+          idesc_bf16_f32(kTileRows, kTileCols, MODE == Mode::kForward, false);
+      bool ok = true;
+      for (int step = 0; step < total && ok; ++step) {
+        const int s = step % kStages;
+        const uint32_t par = (step / kStages) & 1u;
+        if (!mbar_wait(&full[s], par, abort_flag) ||
+            (step < ksteps && !mbar_wait(&deq[s], par, abort_flag))) {
+          record_error(args.err, abort_flag, kErrTimeoutMma);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(w_s + s * kWBytes);
+        const uint32_t b0 = smem_u32(act_s + s * kActBytes);
+        if (step < ksteps) {
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = (MODE == Mode::kForward)
+                                    ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
+                                    : smem_desc_sw128(a0 + kk * 4096, 1024, 2048);
+            const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16(tmem_d, ad, bd, idesc_main, (step | kk) != 0);
+          }
+        } else {
+          for (int kk = 0; kk < args.ext_mmas; ++kk) {
+            const uint64_t ad = (MODE == Mode::kForward)
+                                    ? smem_desc_sw128(a0 + kk * 2048, 8192, 1024)
+                                    : smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16(tmem_d, ad, bd, idesc_ext, 1u);
+          }
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_full);
+      if (!ok) mbar_wait_drain(acc_full, 0);  // MMAs in flight finish before TMEM is freed
+    }
+  } else {
+    // ------------------------------------------------------------ dequant warps
+    const int dw = warp - 2;
+    const int wg = dw >> 2;                  // warpgroup: even / odd pipeline steps
+    const int local = (dw & 3) * 32 + lane;  // 0..127
+    const float mean = *args.mean;
+    const int64_t bpr = args.K / 64;  // 64-blocks per weight row
+    for (int step = wg; step < ksteps; step += 2) {
+      const int s = step % kStages;
+      const uint32_t par = (step / kStages) & 1u;
+      int64_t n, kb;
+      if (MODE == Mode::kForward) {
+        n = row0 + local;
+        kb = step;
+      } else {
+        n = static_cast<int64_t>(step) * kBK + (local >> 1);
+        kb = row0 / 64 + (local & 1);
+      }
+      float sc = 0.f;  // rows / blocks outside W dequantize to zeros
+      if (n < args.N && kb < bpr) {
+        const int64_t j = n * bpr + kb;
+        sc = block_scale(__ldg(args.c2 + j), __ldg(args.c1 + (j >> 8)), mean);
+      }
+      if (!mbar_wait(&full[s], par, abort_flag)) {
+        record_error(args.err, abort_flag, kErrTimeoutDequant);
+        break;
+      }
+      const uint8_t* src = (MODE == Mode::kForward)
+                               ? code_s + s * kCodeBytes + local * 32
+                               : code_s + s * kCodeBytes + (local >> 1) * 64 + (local & 1) * 32;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(src);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(src + 16);
+      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      Nf4Lut lut;
+      build_lut(sc, lut);
+      uint8_t* dst = w_s + s * kWBytes;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t o[4];
+        lut_decode8(words[ch], lut, o);
+        uint32_t off;
+        if (MODE == Mode::kForward) {
+          off = sw128_kmajor_offset(local, ch);
+        } else {
+          const uint32_t nr = local >> 1;  // K-row (contraction) index inside the tile
+          off = (nr >> 3) * 2048u + (local & 1) * 1024u + (nr & 7u) * 128u +
+                ((ch ^ (nr & 7u)) << 4);
+        }
+        *reinterpret_cast<uint4*>(dst + off) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&deq[s]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (mbar_wait(acc_full, 0, abort_flag) && !*abort_flag) {
+      tc_fence_after();
+      const int quarter = warp & 3;  // TMEM lanes this warp may read
+      const int64_t orow = row0 + quarter * 32 + lane;
+      const int colbase = wg * (kTileCols / 2);
+#pragma unroll 1
+      for (int c = 0; c < kTileCols / 2 / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(quarter * 32) << 16) + colbase + c * 32,
+                           v);
+        tmem_ld_wait();
+        if (orow < args.out_rows) {
+          const int64_t mb = m0 + colbase + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (mb + i < args.M)
+              args.out[(mb + i) * args.out_ld + orow] = bf16_bits_rn(__uint_as_float(v[i]));
+        }
+      }
+    } else if (!*abort_flag) {
+      record_error(args.err, abort_flag, kErrTimeoutEpilogue);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, kTileCols);
+  }
+}
+
+// ================================================================== LoRA GEMMs
+constexpr int kLoraThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kLoraStages = 6;
+constexpr uint32_t kLoraABytes = 128 * kBK * 2;  // 16 KB
+constexpr uint32_t kLoraBMax = 128 * kBK * 2;    // 16 KB (NC = 128)
+constexpr uint32_t kLoraSmem = kLoraStages * (kLoraABytes + kLoraBMax) + 1024 + 256;
+
+struct LoraArgs {
+  int64_t rows;      // D rows (128-row tiles)
+  int steps_total;   // 64-wide contraction steps
+  int steps_per;     // steps per split
+  float* partial;    // [splits][rows_pad][NC] fp32
+  int64_t rows_pad;
+  int* err;
+};
+
+// D[128-row tile, NC] = sum over this CTA's contraction range of A^T B (both bf16,
+// K-major or MN-major 128B-swizzled tiles loaded by TMA).
+template <bool A_MN, bool B_MN, int NC>
+__global__ void __launch_bounds__(kLoraThreads, 1)
+    k_lora_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                const LoraArgs args) {
+  constexpr uint32_t kB = NC * kBK * 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* a_s = smem;
+  uint8_t* b_s = a_s + kLoraStages * kLoraABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_s + kLoraStages * kB);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kLoraStages;
+  uint64_t* acc_full = bars + 2 * kLoraStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kLoraStages + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const int s_begin = blockIdx.y * args.steps_per;
+  const int s_end = std::min(args.steps_total, s_begin + args.steps_per);
+  const int nsteps = std::max(0, s_end - s_begin);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kLoraStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, NC);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % kLoraStages;
+        const uint32_t use = i / kLoraStages;
+        if (i >= kLoraStages && !mbar_wait(&empty[s], (use - 1) & 1u, abort_flag)) {
+          record_error(args.err, abort_flag, kErrTimeoutProducer);
+          break;
+        }
+        const int kc = (s_begin + i) * kBK;  // contraction coordinate
+        mbar_arrive_expect_tx(&full[s], kLoraABytes + kB);
+        if (A_MN) {
+          tma_load_2d(a_s + s * kLoraABytes, &tm_a, &full[s], static_cast<int>(row0), kc);
+          tma_load_2d(a_s + s * kLoraABytes + 8192, &tm_a, &full[s], static_cast<int>(row0) + 64,
+                      kc);
+        } else {
+          tma_load_2d(a_s + s * kLoraABytes, &tm_a, &full[s], kc, static_cast<int>(row0));
+        }
+        if (B_MN) {
+#pragma unroll
+          for (int c = 0; c < NC / 64; ++c)
+            tma_load_2d(b_s + s * kB + c * 8192, &tm_b, &full[s], c * 64, kc);
+        } else {
+          tma_load_2d(b_s + s * kB, &tm_b, &full[s], kc, 0);
+        }
+        ++issued;
+      }
+      if (*abort_flag)
+        for (int i = std::max(0, issued - kLoraStages); i < issued; ++i)
+          mbar_wait_drain(&full[i % kLoraStages], (i / kLoraStages) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, NC, A_MN, B_MN);
+      bool ok = true;
+      for (int i = 0; i < nsteps; ++i) {
+        const int s = i % kLoraStages;
+        if (!mbar_wait(&full[s], (i / kLoraStages) & 1u, abort_flag)) {
+          record_error(args.err, abort_flag, kErrTimeoutMma);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(a_s + s * kLoraABytes);
+        const uint32_t b0 = smem_u32(b_s + s * kB);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = A_MN ? smem_desc_sw128(a0 + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(a0 + kk * 32, 16, 1024);
+          const uint64_t bd = B_MN ? smem_desc_sw128(b0 + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(b0 + kk * 32, 16, 1024);
+          umma_bf16(tmem_d, ad, bd, idesc, (i | kk) != 0);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_full);
+      if (!ok) mbar_wait_drain(acc_full, 0);
+    }
+  } else {
+    const bool have = nsteps > 0;
+    if (!have || (mbar_wait(acc_full, 0, abort_flag) && !*abort_flag)) {
+      tc_fence_after();
+      const int quarter = warp & 3;
+      const int64_t row = row0 + quarter * 32 + lane;
+      float* dst = args.partial + (static_cast<int64_t>(blockIdx.y) * args.rows_pad + row) * NC;
+#pragma unroll 1
+      for (int c = 0; c < NC / 32; ++c) {
+        uint32_t v[32];
+        if (have) {
+          tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(quarter * 32) << 16) + c * 32, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<uint4*>(dst + c * 32 + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    } else if (!*abort_flag) {
+      record_error(args.err, abort_flag, kErrTimeoutEpilogue);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, NC);
+  }
+}
+
+// ================================================================== finalize kernels
+// T (or G) = sum of split partials [S][rows_pad][64]. Writes, where asked:
+//   plain fp32 [M, r], scaled bf16 [M, 64] (K-extension operand), hi/lo bf16 [M, 128].
+__global__ void k_finalize_rank(const float* __restrict__ part, int splits, int64_t rows_pad,
+                                int64_t M, int r, float scale, float* __restrict__ plain,
+                                uint16_t* __restrict__ scaled, uint16_t* __restrict__ hilo) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= M * 64) return;
+  const int64_t m = i >> 6;
+  const int j = static_cast<int>(i & 63);
+  float v = 0.f;
+  for (int s = 0; s < splits; ++s) v += part[(s * rows_pad + m) * 64 + j];
+  if (j >= r) v = 0.f;
+  if (plain && j < r) plain[m * r + j] = v;
+  if (scaled) scaled[m * 64 + j] = bf16_bits_rn(v * scale);
+  if (hilo) {
+    const uint16_t hi = bf16_bits_rn(v);
+    const float hv = __uint_as_float(static_cast<uint32_t>(hi) << 16);
+    hilo[m * 128 + j] = hi;
+    hilo[m * 128 + 64 + j] = bf16_bits_rn(v - hv);
+  }
+}
+
+// hi/lo bf16 pair [M, 128] from a saved fp32 T [M, r].
+__global__ void k_hilo_from_plain(const float* __restrict__ t, int64_t M, int r,
+                                  uint16_t* __restrict__ hilo) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= M * 64) return;
+  const int64_t m = i >> 6;
+  const int j = static_cast<int>(i & 63);
+  const float v = (j < r) ? t[m * r + j] : 0.f;
+  const uint16_t hi = bf16_bits_rn(v);
+  hilo[m * 128 + j] = hi;
+  hilo[m * 128 + 64 + j] = bf16_bits_rn(v - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+}
+
+// grad[row, j] (or its transpose) = scale * sum_s (P[s][row][j] + P[s][row][64 + j]).
+__global__ void k_finalize_grad(const float* __restrict__ part, int splits, int64_t rows_pad,
+                                int64_t rows, int r, float scale, bool transpose,
+                                float* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * r) return;
+  int64_t row;
+  int j;
+  if (transpose) {  // out [r, rows]: consecutive threads walk rows (coalesced store)
+    j = static_cast<int>(i / rows);
+    row = i % rows;
+  } else {          // out [rows, r]
+    row = i / r;
+    j = static_cast<int>(i % r);
+  }
+  float v = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float* p = part + (s * rows_pad + row) * 128;
+    v += p[j] + p[64 + j];
+  }
+  out[transpose ? (static_cast<int64_t>(j) * rows + row) : (row * r + j)] = scale * v;
+}
+
+// ================================================================== host side
+constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+constexpr CUtensorMapSwizzle kSW128 = CU_TENSOR_MAP_SWIZZLE_128B;
+
+struct SplitPlan {
+  int splits, steps_per, steps_total;
+  int64_t tiles, rows_pad;
+};
+
+SplitPlan plan_split(int64_t rows, int64_t contraction) {
+  SplitPlan p;
+  p.tiles = (rows + 127) / 128;
+  p.rows_pad = p.tiles * 128;
+  p.steps_total = static_cast<int>((contraction + kBK - 1) / kBK);
+  const int64_t target = 2LL * num_sms();
+  int64_t want = (target + p.tiles - 1) / p.tiles;
+  want = std::max<int64_t>(1, std::min<int64_t>(want, (p.steps_total + 1) / 2));
+  p.steps_per = static_cast<int>((p.steps_total + want - 1) / want);
+  p.splits = (p.steps_total + p.steps_per - 1) / p.steps_per;
+  return p;
+}
+
+// Largest partial buffer (floats) the plans of one call may need.
+size_t partial_floats(int64_t rows, int64_t contraction, int nc) {
+  const SplitPlan p = plan_split(rows, contraction);
+  return static_cast<size_t>(p.splits) * p.rows_pad * nc;
+}
+
+template <bool A_MN, bool B_MN, int NC>
+cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
+                          int64_t contraction, float* partial, cudaStream_t st, int* splits_out) {
+  const SplitPlan p = plan_split(rows, contraction);
+  LoraArgs a;
+  a.rows = rows;
+  a.steps_total = p.steps_total;
+  a.steps_per = p.steps_per;
+  a.partial = partial;
+  a.rows_pad = p.rows_pad;
+  a.err = device_error_word();
+  auto kern = k_lora_gemm<A_MN, B_MN, NC>;
+  const uint32_t smem = kLoraStages * (kLoraABytes + NC * kBK * 2) + 1024 + 256;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(static_cast<unsigned>(p.tiles), static_cast<unsigned>(p.splits)), kLoraThreads, smem,
+         st>>>(ta, tb, a);
+  *splits_out = p.splits;
+  return cudaGetLastError();
+}
+
+template <Mode MODE>
+cudaError_t run_fused(const CUtensorMap& tc, const CUtensorMap& ta, const CUtensorMap& tw,
+                      const CUtensorMap& tx, const FusedArgs& args, cudaStream_t st) {
+  auto kern = k_fused_nf4_gemm<MODE>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = (MODE == Mode::kForward) ? args.N : args.K;
+  dim3 grid(static_cast<unsigned>((rows + kTileRows - 1) / kTileRows),
+            static_cast<unsigned>((args.M + kTileCols - 1) / kTileCols));
+  cudaEvent_t before, after;
+  profile_events(&before, &after);
+  if (before) {
+    e = cudaEventRecord(before, st);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<grid, kFusedThreads, kFusedSmem, st>>>(tc, ta, tw, tx, args);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && after) e = cudaEventRecord(after, st);
+  return e;
+}
+
+inline unsigned blocks_for(int64_t n, int t) { return static_cast<unsigned>((n + t - 1) / t); }
+
+// Workspace carving: a bump allocator over the caller's buffer.
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    off = align_up(off, 256);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+size_t fwd_layout(const LinearShape& s, void* ws, float** part, uint16_t** ts) {
+  Carve c(ws);
+  *part = c.take<float>(partial_floats(s.M, s.K, 64));
+  *ts = c.take<uint16_t>(static_cast<size_t>(s.M) * 64);
+  return c.off + 256;
+}
+
+size_t bwd_layout(const LinearShape& s, void* ws, float** part, uint16_t** gs, uint16_t** ghl,
+                  uint16_t** thl, float** t) {
+  Carve c(ws);
+  size_t pf = partial_floats(s.M, s.N, 64);                    // G = dY B^T
+  pf = std::max(pf, partial_floats(s.M, s.K, 64));             // T = X A (recompute)
+  pf = std::max(pf, partial_floats(s.K, s.M, 128));            // dA
+  pf = std::max(pf, partial_floats(s.N, s.M, 128));            // dB
+  *part = c.take<float>(pf);
+  *gs = c.take<uint16_t>(static_cast<size_t>(s.M) * 64);
+  *ghl = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
+  *thl = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
+  *t = c.take<float>(static_cast<size_t>(s.M) * s.r);
+  return c.off + 256;
+}
+
+#define QL_TRY(expr)                                  \
+  do {                                                \
+    cudaError_t _e = (expr);                          \
+    if (_e != cudaSuccess) return cuda_status(_e);    \
+  } while (0)
+#define QL_MAP(...)                                                    \
+  do {                                                                 \
+    if (!make_tmap_2d(__VA_ARGS__)) return QLORA_ERR_CUDA;             \
+  } while (0)
+
+// T = X A (fp32, split partials) then T_save / bf16(scale T).
+qlora_status lora_down_T(const uint16_t* X, const uint16_t* A, const LinearShape& s, float* part,
+                         float* t_plain, uint16_t* t_scaled, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 128, kSW128);   // X K-major
+  QL_MAP(&tb, kBF16, A, s.r, s.K, s.r * 2, 64, 64, kSW128);    // A as MN-major (j inner)
+  int splits = 0;
+  QL_TRY((run_lora_gemm<false, true, 64>(ta, tb, s.M, s.K, part, st, &splits)));
+  const int64_t rows_pad = plan_split(s.M, s.K).rows_pad;
+  k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(part, splits, rows_pad, s.M, s.r,
+                                                              s.scale, t_plain, t_scaled, nullptr);
+  QL_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+}  // namespace
+
+size_t gemm_fwd_workspace(const LinearShape& s) {
+  float* p;
+  uint16_t* t;
+  return fwd_layout(s, nullptr, &p, &t);
+}
+
+size_t gemm_bwd_workspace(const LinearShape& s) {
+  float *p, *t;
+  uint16_t *g, *gh, *th;
+  return bwd_layout(s, nullptr, &p, &g, &gh, &th, &t);
+}
+
+qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
+                          const uint16_t* B, const LinearShape& s, uint16_t* Y, float* T_save,
+                          void* ws, cudaStream_t st) {
+  float* part;
+  uint16_t* ts;
+  fwd_layout(s, ws, &part, &ts);
+  qlora_status q = lora_down_T(X, A, s, part, T_save, ts, st);
+  if (q != QLORA_OK) return q;
+
+  CUtensorMap tc, ta, tw, tx;
+  QL_MAP(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, s.K / 2, s.N, s.K / 2, 32, 128,
+         CU_TENSOR_MAP_SWIZZLE_NONE);
+  QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 256, kSW128);
+  QL_MAP(&tw, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);   // B [r, N], MN-major chunks
+  QL_MAP(&tx, kBF16, ts, 64, s.M, 128, 64, 256, kSW128);      // bf16(scale T) [M, 64]
+  FusedArgs a;
+  a.c2 = w.c2;
+  a.c1 = w.c1;
+  a.mean = w.mean;
+  a.N = s.N;
+  a.K = s.K;
+  a.M = s.M;
+  a.ext_mmas = (s.r + 15) / 16;
+  a.out = Y;
+  a.out_ld = s.N;
+  a.out_rows = s.N;
+  a.err = device_error_word();
+  QL_TRY(run_fused<Mode::kForward>(tc, ta, tw, tx, a, st));
+  return QLORA_OK;
+}
+
+qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T_saved,
+                           const qlora_nf4_weight& w, const uint16_t* A, const uint16_t* B,
+                           const LinearShape& s, uint16_t* dX, float* dA, float* dB, void* ws,
+                           cudaStream_t st) {
+  float *part, *tbuf;
+  uint16_t *gs, *ghl, *thl;
+  bwd_layout(s, ws, &part, &gs, &ghl, &thl, &tbuf);
+  int splits = 0;
+
+  // G = dY B^T -> bf16(scale G) for the dX extension, bf16 hi/lo for dA.
+  {
+    CUtensorMap ta, tb;
+    QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 128, kSW128);  // dY K-major (over n)
+    QL_MAP(&tb, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);    // B [r, N] K-major
+    QL_TRY((run_lora_gemm<false, false, 64>(ta, tb, s.M, s.N, part, st, &splits)));
+    k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
+        part, splits, plan_split(s.M, s.N).rows_pad, s.M, s.r, s.scale, nullptr, gs, ghl);
+    QL_TRY(cudaGetLastError());
+  }
+  // T (saved, or recomputed) -> bf16 hi/lo for dB.
+  const float* t = T_saved;
+  if (!t) {
+    qlora_status q = lora_down_T(X, A, s, part, tbuf, nullptr, st);
+    if (q != QLORA_OK) return q;
+    t = tbuf;
+  }
+  k_hilo_from_plain<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(t, s.M, s.r, thl);
+  QL_TRY(cudaGetLastError());
+
+  // dX = dY W_hat + scale G A^T
+  if (dX) {
+    CUtensorMap tc, ta, tw, tx;
+    QL_MAP(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, s.K / 2, s.N, s.K / 2, 64, 64,
+           CU_TENSOR_MAP_SWIZZLE_NONE);
+    QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 256, kSW128);
+    QL_MAP(&tw, kBF16, A, s.r, s.K, s.r * 2, 64, 128, kSW128);   // A [K, r] K-major
+    QL_MAP(&tx, kBF16, gs, 64, s.M, 128, 64, 256, kSW128);       // bf16(scale G) [M, 64]
+    FusedArgs a;
+    a.c2 = w.c2;
+    a.c1 = w.c1;
+    a.mean = w.mean;
+    a.N = s.N;
+    a.K = s.K;
+    a.M = s.M;
+    a.ext_mmas = (s.r + 15) / 16;
+    a.out = dX;
+    a.out_ld = s.K;
+    a.out_rows = s.K;
+    a.err = device_error_word();
+    QL_TRY(run_fused<Mode::kDgrad>(tc, ta, tw, tx, a, st));
+  }
+  // dA = scale X^T G  (rows k, contraction over tokens)
+  {
+    CUtensorMap ta, tb;
+    QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 64, kSW128);    // X as MN-major (k inner)
+    QL_MAP(&tb, kBF16, ghl, 128, s.M, 256, 64, 64, kSW128);      // G hi/lo MN-major
+    QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits)));
+    k_finalize_grad<<<blocks_for(s.K * s.r, 256), 256, 0, st>>>(
+        part, splits, plan_split(s.K, s.M).rows_pad, s.K, s.r, s.scale, false, dA);
+    QL_TRY(cudaGetLastError());
+  }
+  // dB = scale T^T dY  (rows n, contraction over tokens), stored [r, N]
+  {
+    CUtensorMap ta, tb;
+    QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);   // dY as MN-major (n inner)
+    QL_MAP(&tb, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);      // T hi/lo MN-major
+    QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.N, s.M, part, st, &splits)));
+    k_finalize_grad<<<blocks_for(s.N * s.r, 256), 256, 0, st>>>(
+        part, splits, plan_split(s.N, s.M).rows_pad, s.N, s.r, s.scale, true, dB);
+    QL_TRY(cudaGetLastError());
+  }
+  return QLORA_OK;
+}
+
+}  // namespace qlora

@@ -1,0 +1,64 @@
+// internal.h -- declarations shared by the library's translation units (not installed).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/qlora.h"
+
+namespace qlora {
+
+// ---- code tables (tables.cpp) ---------------------------------------------------
+// NF4 levels as fp32 bit patterns, ascending; index 7 is the exact zero.
+extern const uint32_t kNf4Bits[16];
+constexpr int kT8Size = 253;  // distinct finite E4M3 values
+struct Nf4Thresholds { float t[15]; };
+struct T8Thresholds { float t[kT8Size - 1]; };
+const Nf4Thresholds& nf4_thresholds();
+const T8Thresholds& t8_thresholds();
+const float* t8_values();        // [253] ascending
+const uint8_t* t8_codes();       // [253] E4M3 bit pattern of each entry
+
+// ---- host helpers (api.cu) -------------------------------------------------------
+void set_last_error(const char* msg);
+qlora_status cuda_status(cudaError_t e);          // records the message, maps the code
+int num_sms();                                     // of the current device
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                  uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                  uint32_t box_outer, CUtensorMapSwizzle swizzle);
+int* device_error_word();                          // per-device error flag of the kernels
+// CUDA events (or NULL) this thread asked to have recorded around each launch of the
+// fused NF4 GEMM kernel (qlora_profile_events).
+void profile_events(cudaEvent_t* before, cudaEvent_t* after);
+
+// ---- launchers (codec.cu) -------------------------------------------------------
+size_t quantize_workspace_bytes(int64_t n, int64_t k);
+cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, uint8_t* codes,
+                            uint8_t* c2, float* c1, float* mean, void* ws, cudaStream_t st);
+cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t st);
+
+// ---- launchers (gemm.cu) --------------------------------------------------------
+struct LinearShape { int64_t M, N, K; int r; float scale; };
+size_t gemm_fwd_workspace(const LinearShape& s);
+size_t gemm_bwd_workspace(const LinearShape& s);
+qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
+                          const uint16_t* B, const LinearShape& s, uint16_t* Y, float* T_save,
+                          void* ws, cudaStream_t st);
+qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T_saved,
+                           const qlora_nf4_weight& w, const uint16_t* A, const uint16_t* B,
+                           const LinearShape& s, uint16_t* dX, float* dA, float* dB, void* ws,
+                           cudaStream_t st);
+
+// ---- launchers (decode.cu) ------------------------------------------------------
+constexpr int64_t kDecodeMaxM = 16;
+size_t decode_workspace(const LinearShape& s);
+qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
+                            const uint16_t* B, const LinearShape& s, uint16_t* Y,
+                            float* T_save, void* ws, cudaStream_t st);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace qlora

@@ -1,0 +1,82 @@
+// nf4_device.cuh -- device-side pieces of the double dequantization shared by the
+// standalone dequant, the fused GEMM and the decode kernels:
+//   s_j   = fl32(fl32(T8[c2_j] * c1[j / 256]) + mean)     (T8[e] = fl32(e4m3(e) / 448))
+//   W_hat = bf16_rn(fl32(NF4[code] * s_j))
+// (page "QLoRA", itwiki.kr: sections "4비트 NormalFloat(NF4)" and "이중 양자화", and
+// doubleDequant in section "계산 방식").
+#pragma once
+
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace qlora {
+
+// NF4 level i as an fp32 constant (bit patterns of the table, ascending).
+__device__ __forceinline__ float nf4_level(int i) {
+  constexpr uint32_t bits[16] = {0xbf800000u, 0xbf3239b3u, 0xbf066b30u, 0xbeca32a0u,
+                                 0xbe91a24cu, 0xbe3d353fu, 0xbdba786bu, 0x00000000u,
+                                 0x3da2fb03u, 0x3e24cae1u, 0x3e7c04dcu, 0x3ead0338u,
+                                 0x3ee1a4b7u, 0x3f1007aau, 0x3f3913b1u, 0x3f800000u};
+  return __uint_as_float(bits[i]);
+}
+
+// Value of an OCP FP8 E4M3 bit pattern (exact in fp32).
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  const float v = (e == 0u) ? static_cast<float>(m) * 0.001953125f  // m * 2^-9
+                            : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  return (b & 0x80u) ? -v : v;
+}
+
+// Reconstructed absmax of one 64-block from its double-quantized constants.
+__device__ __forceinline__ float block_scale(uint32_t c2, float c1, float mean) {
+  const float t8 = __fdiv_rn(e4m3_value(c2), 448.0f);
+  return __fadd_rn(__fmul_rn(t8, c1), mean);
+}
+
+// 16-entry bf16 table {bf16(NF4[i] * s)} split into byte planes for prmt lookups:
+// lo[q] holds the low bytes of entries 4q..4q+3, hi[q] their high bytes.
+struct Nf4Lut {
+  uint32_t lo[4];
+  uint32_t hi[4];
+};
+
+__device__ __forceinline__ void build_lut(float s, Nf4Lut& t) {
+  uint32_t p[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    p[i] = pack_bf16x2_rn(__fmul_rn(nf4_level(2 * i), s), __fmul_rn(nf4_level(2 * i + 1), s));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = prmt(p[2 * q], p[2 * q + 1], 0x6420u);
+    t.hi[q] = prmt(p[2 * q], p[2 * q + 1], 0x7531u);
+  }
+}
+
+// Eight 4-bit codes (nibble i of w = code of element i) -> four bf16x2 registers
+// o[i] = (element 2i in the low half, element 2i+1 in the high half).
+// Bits 0-2 of a code index a byte inside an 8-byte prmt window; bit 3 picks the
+// window (entries 0-7 or 8-15) through a byte mask.
+__device__ __forceinline__ void lut_decode8(uint32_t w, const Nf4Lut& t, uint32_t (&o)[4]) {
+  const uint32_t sel = w & 0x77777777u;
+  const uint32_t msel = ((w >> 3) & 0x11111111u) * 9u;  // nibble 9 -> 0xFF byte, 0 -> 0x00
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t s4 = h ? (sel >> 16) : sel;
+    const uint32_t m4 = h ? (msel >> 16) : msel;
+    const uint32_t mask = prmt(0x00008000u, 0u, m4);
+    const uint32_t lo = (prmt(t.lo[0], t.lo[1], s4) & ~mask) | (prmt(t.lo[2], t.lo[3], s4) & mask);
+    const uint32_t hi = (prmt(t.hi[0], t.hi[1], s4) & ~mask) | (prmt(t.hi[2], t.hi[3], s4) & mask);
+    o[2 * h] = prmt(lo, hi, 0x5140u);
+    o[2 * h + 1] = prmt(lo, hi, 0x7362u);
+  }
+}
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(x));
+  return static_cast<uint16_t>(d & 0xFFFFu);
+}
+
+}  // namespace qlora

@@ -1,0 +1,236 @@
+"""Python binding of the C ABI in ``include/qlora.h`` (``lib/libqlora.so``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. PyTorch supplies device memory and the current stream. There is no
+fallback: if the library is missing or the device is not sm_100, calls raise.
+
+Names follow the C entry points:
+    qlora_quantize_nf4_dq(W)                          -> NF4Weight
+    qlora_dequant(w)                                  -> W_hat bf16 [N, K]
+    qlora_linear_fwd(X, w, A, B, scale)               -> (Y, T)
+    qlora_linear_bwd(dY, X, T, w, A, B, scale)        -> (dX, dA, dB)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libqlora.so")
+
+STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGN",
+          4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_CUDA", 6: "QLORA_ERR_DEVICE",
+          7: "QLORA_ERR_TIMEOUT"}
+F32, BF16 = 0, 1
+
+
+class QLoraError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}" + (f" ({detail})" if detail else ""))
+
+
+class CNF4Weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p),
+                ("mean", ctypes.c_void_p), ("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64)]
+
+
+_lib = None
+_vp, _i64, _i32, _sz, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+
+_SIGNATURES = {
+    "qlora_status_str": (ctypes.c_char_p, [_i32]),
+    "qlora_last_error": (ctypes.c_char_p, []),
+    "qlora_version": (_i32, []),
+    "qlora_device_error": (_i32, [_i32]),
+    "qlora_profile_events": (None, [_vp, _vp]),
+    "qlora_nf4_table": (None, [_vp]),
+    "qlora_nf4_thresholds": (None, [_vp]),
+    "qlora_fp8_thresholds": (None, [_vp, _vp, _vp]),
+    "qlora_quantize_workspace_size": (_sz, [_i64, _i64]),
+    "qlora_quantize_nf4_dq": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_dequant": (_i32, [CNF4Weight, _vp, _vp]),
+    "qlora_linear_fwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
+    "qlora_linear_fwd": (_i32, [_vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
+    "qlora_linear_bwd": (_i32, [_vp, _vp, _vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp,
+                                _vp, _vp, _sz, _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m bit_nf4_quantized_unpack_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise QLoraError(status, where, lib().qlora_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _as_bits(t: torch.Tensor) -> torch.Tensor:
+    """bf16 tensors travel as their uint16 bit patterns."""
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"expected bfloat16, got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return t
+
+
+@dataclass
+class NF4Weight:
+    """A quantized weight [n_out, k_in] in the library's storage format (device)."""
+    codes: torch.Tensor   # uint8 [N*K/2]
+    c2: torch.Tensor      # uint8 [N*K/64]  E4M3 bit patterns
+    c1: torch.Tensor      # float32 [ceil(N*K/16384)]
+    mean: torch.Tensor    # float32 [1]
+    n_out: int
+    k_in: int
+
+    def c_struct(self) -> CNF4Weight:
+        return CNF4Weight(self.codes.data_ptr(), self.c2.data_ptr(), self.c1.data_ptr(),
+                          self.mean.data_ptr(), self.n_out, self.k_in)
+
+    @staticmethod
+    def empty(n_out: int, k_in: int, device="cuda") -> "NF4Weight":
+        nb = n_out * k_in // 64
+        return NF4Weight(torch.empty(n_out * k_in // 2, dtype=torch.uint8, device=device),
+                         torch.empty(nb, dtype=torch.uint8, device=device),
+                         torch.empty((nb + 255) // 256, dtype=torch.float32, device=device),
+                         torch.empty(1, dtype=torch.float32, device=device), n_out, k_in)
+
+
+# ------------------------------------------------------------------ host-only tables
+
+def nf4_table() -> torch.Tensor:
+    out = (ctypes.c_float * 16)()
+    lib().qlora_nf4_table(ctypes.cast(out, ctypes.c_void_p))
+    return torch.tensor(list(out), dtype=torch.float32)
+
+
+def nf4_thresholds() -> torch.Tensor:
+    out = (ctypes.c_float * 15)()
+    lib().qlora_nf4_thresholds(ctypes.cast(out, ctypes.c_void_p))
+    return torch.tensor(list(out), dtype=torch.float32)
+
+
+def fp8_thresholds():
+    th, vals, codes = (ctypes.c_float * 252)(), (ctypes.c_float * 253)(), (ctypes.c_uint8 * 253)()
+    lib().qlora_fp8_thresholds(ctypes.cast(th, ctypes.c_void_p), ctypes.cast(vals, ctypes.c_void_p),
+                               ctypes.cast(codes, ctypes.c_void_p))
+    return (torch.tensor(list(th), dtype=torch.float32), torch.tensor(list(vals), dtype=torch.float32),
+            torch.tensor(list(codes), dtype=torch.uint8))
+
+
+# ------------------------------------------------------------------ entry points
+
+def qlora_quantize_workspace_size(n_out: int, k_in: int) -> int:
+    return int(lib().qlora_quantize_workspace_size(n_out, k_in))
+
+
+def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Weight | None = None,
+                          workspace: torch.Tensor | None = None) -> NF4Weight:
+    """NF4 + double quantization of W [N, K] (fp32 or bf16, CUDA, contiguous)."""
+    if W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D CUDA tensor")
+    dtype = {torch.float32: F32, torch.bfloat16: BF16}.get(W.dtype)
+    if dtype is None:
+        raise TypeError(f"unsupported weight dtype {W.dtype}")
+    n, k = W.shape
+    q = out if out is not None else NF4Weight.empty(n, k, W.device)
+    need = qlora_quantize_workspace_size(n, k)
+    ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8,
+                                                             device=W.device)
+    _check(lib().qlora_quantize_nf4_dq(_ptr(W), dtype, n, k, _ptr(q.codes), _ptr(q.c2), _ptr(q.c1),
+                                       _ptr(q.mean), _ptr(ws), ws.numel(), _stream()),
+           "qlora_quantize_nf4_dq")
+    return q
+
+
+def qlora_dequant(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """doubleDequant of the stored weight to bf16 [N, K]."""
+    y = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16,
+                                                device=w.codes.device)
+    _check(lib().qlora_dequant(w.c_struct(), _ptr(_as_bits(y)), _stream()), "qlora_dequant")
+    return y
+
+
+def qlora_linear_fwd_workspace_size(M: int, n_out: int, k_in: int, r: int) -> int:
+    return int(lib().qlora_linear_fwd_workspace_size(M, n_out, k_in, r))
+
+
+def qlora_linear_bwd_workspace_size(M: int, n_out: int, k_in: int, r: int) -> int:
+    return int(lib().qlora_linear_bwd_workspace_size(M, n_out, k_in, r))
+
+
+def qlora_linear_fwd(X: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor, scale: float,
+                     save_T: bool = True, Y: torch.Tensor | None = None,
+                     T: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """Y = bf16(X W_hat^T + scale (X A) B). Returns (Y, T) with T = X A (fp32) or None."""
+    M, K = X.shape
+    r = A.shape[1]
+    dev = X.device
+    Y = Y if Y is not None else torch.empty(M, w.n_out, dtype=torch.bfloat16, device=dev)
+    if save_T and T is None:
+        T = torch.empty(M, r, dtype=torch.float32, device=dev)
+    need = qlora_linear_fwd_workspace_size(M, w.n_out, w.k_in, r)
+    ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().qlora_linear_fwd(_ptr(_as_bits(X)), M, w.c_struct(), _ptr(_as_bits(A)),
+                                  _ptr(_as_bits(B)), r, float(scale), _ptr(_as_bits(Y)),
+                                  _ptr(T if save_T else None), _ptr(ws), ws.numel(), _stream()),
+           "qlora_linear_fwd")
+    return Y, (T if save_T else None)
+
+
+def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, w: NF4Weight,
+                     A: torch.Tensor, B: torch.Tensor, scale: float, need_dX: bool = True,
+                     dX: torch.Tensor | None = None, dA: torch.Tensor | None = None,
+                     dB: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """Gradients (dX bf16 or None, dA fp32 [K, r], dB fp32 [r, N]); W is frozen."""
+    M = X.shape[0]
+    r = A.shape[1]
+    dev = X.device
+    if need_dX and dX is None:
+        dX = torch.empty(M, w.k_in, dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty(w.k_in, r, dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty(r, w.n_out, dtype=torch.float32, device=dev)
+    need = qlora_linear_bwd_workspace_size(M, w.n_out, w.k_in, r)
+    ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().qlora_linear_bwd(_ptr(_as_bits(dY)), _ptr(_as_bits(X)), _ptr(T), M, w.c_struct(),
+                                  _ptr(_as_bits(A)), _ptr(_as_bits(B)), r, float(scale),
+                                  _ptr(_as_bits(dX) if need_dX else None), _ptr(dA), _ptr(dB),
+                                  _ptr(ws), ws.numel(), _stream()),
+           "qlora_linear_bwd")
+    return (dX if need_dX else None), dA, dB
+
+
+def qlora_profile_events(before=None, after=None):
+    """Record torch.cuda.Event pair (or None) around each fused-GEMM launch of this thread."""
+    lib().qlora_profile_events(ctypes.c_void_p(before.cuda_event) if before is not None else None,
+                               ctypes.c_void_p(after.cuda_event) if after is not None else None)
+
+
+def qlora_device_error(clear: bool = True) -> int:
+    """Status of the device error word (QLORA_ERR_TIMEOUT after a timed-out wait)."""
+    return int(lib().qlora_device_error(1 if clear else 0))

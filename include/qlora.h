@@ -1,0 +1,206 @@
+/*
+ * qlora.h -- C ABI of a B200 (sm_100a) library for the QLoRA linear layer.
+ *
+ * The layer (page "QLoRA", itwiki.kr, section "계산 방식" / computation, and page
+ * "quantization", minnong511 blog, section "QLoRA에서 학습은 어떻게 되는 걸까?"):
+ *
+ *     Y = X * doubleDequant(c1, c2, W_NF4)^T + (alpha / r) * (X * A) * B
+ *
+ * with W stored as 4-bit NormalFloat codes in blocks of 64 weights (itwiki "QLoRA",
+ * section "4비트 NormalFloat(NF4)"), the per-block absmax constants double-quantized
+ * to FP8 E4M3 codes c2 in blocks of 256 after subtracting one mean per tensor, with
+ * one fp32 constant c1 per 256-block (itwiki "QLoRA", section "이중 양자화").
+ * The backward produces dX through the frozen quantized W and the LoRA gradients
+ * dA and dB only (itwiki "QLoRA", computation section; minnong511 "quantization",
+ * section on why a 4-bit base model can be trained).
+ *
+ * Conventions shared by every entry point:
+ *  - Matrices are row-major. W is N x K (out x in) with K % 64 == 0. X is M x K,
+ *    Y is M x N, A is K x r, B is r x N.
+ *  - bf16 data is passed as uint16_t bit patterns.
+ *  - Every pointer argument named "device" is CUDA device memory owned by the
+ *    caller; the library never allocates, frees or keeps device memory. Scratch
+ *    space comes from the caller through (workspace, workspace_bytes); the
+ *    matching *_workspace_size query says how much.
+ *  - Device pointers must be 16-byte aligned (QLORA_ERR_ALIGN otherwise).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *    and runs asynchronously. Argument errors are detected on the host before
+ *    anything is launched; then nothing is enqueued and an error code is
+ *    returned. QLORA_ERR_CUDA reports a failed launch; qlora_last_error() gives
+ *    the CUDA message. Device-side faults surface at the caller's next
+ *    synchronisation, as with any CUDA call.
+ *  - All entry points are thread-safe; calls on different streams may overlap,
+ *    provided their outputs and workspaces do not alias.
+ *
+ * Storage of a quantized weight W [N, K] (all device memory):
+ *    codes : uint8 [N*K/2]   byte b = code(2b) | code(2b+1) << 4 (row-major order)
+ *    c2    : uint8 [N*K/64]  E4M3 bit pattern of each block constant after
+ *                            mean subtraction and 256-block scaling
+ *    c1    : float [ceil(N*K/16384)] absmax of each 256-block of centred constants
+ *    mean  : float [1]       mean of all N*K/64 block absmax values
+ * Double dequantization of block j (flat index, 64 weights each):
+ *    s_j = fl32(fl32(T8[c2_j] * c1[j/256]) + mean),  T8[e] = fl32(e4m3(e) / 448)
+ *    W_hat = bf16_rn(fl32(NF4[code] * s_j))
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1, /* null pointer, unknown dtype, r or scale out of range */
+  QLORA_ERR_SHAPE = 2,       /* unsupported sizes (K % 64 != 0, negative sizes, ...) */
+  QLORA_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+  QLORA_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than the size query */
+  QLORA_ERR_CUDA = 5,        /* a CUDA call failed; see qlora_last_error() */
+  QLORA_ERR_DEVICE = 6,      /* current device is not sm_100 (B200 class) */
+  QLORA_ERR_TIMEOUT = 7      /* a kernel's bounded wait ran out (qlora_device_error) */
+} qlora_status;
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/* A quantized weight as produced by qlora_quantize_nf4_dq (device pointers). */
+typedef struct {
+  const uint8_t *codes;
+  const uint8_t *c2;
+  const float *c1;
+  const float *mean;
+  int64_t n_out; /* N: rows (output features) */
+  int64_t k_in;  /* K: columns (input features), K % 64 == 0 */
+} qlora_nf4_weight;
+
+/* Human-readable name of a status code (static storage). */
+const char *qlora_status_str(qlora_status status);
+
+/* Message of the last CUDA error seen by this thread inside the library, or "". */
+const char *qlora_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int qlora_version(void);
+
+/*
+ * qlora_device_error: synchronous check of the current device's error word. Every
+ * wait inside the kernels is bounded (2 s); a wait that runs out records a code
+ * there and the kernel drains its copies, frees its tensor memory and exits
+ * without writing its outputs. Returns QLORA_ERR_TIMEOUT when a code is set (and
+ * clears it when `clear` != 0), QLORA_OK otherwise. Blocks until the device copy of
+ * the word is read (a synchronous cudaMemcpy on the legacy stream).
+ */
+qlora_status qlora_device_error(int clear);
+
+/*
+ * qlora_profile_events: measurement aid. For the calling thread, record the CUDA
+ * events `before` and `after` (cudaEvent_t, or NULL to stop) on the launch stream
+ * immediately before and after each launch of the fused NF4 tensor-core GEMM
+ * (forward or dX), so that cudaEventElapsedTime gives that kernel's own duration.
+ * The events are owned by the caller; each later launch re-records them.
+ */
+void qlora_profile_events(void *before, void *after);
+
+/*
+ * qlora_nf4_table: writes the 16 NF4 levels (fp32, ascending, NF4[7] == 0) that the
+ * kernels use, to host memory `out16`. Host-only, needs no GPU.
+ * Definition: itwiki "QLoRA", section "4비트 NormalFloat(NF4)": N(0,1) quantiles at
+ * evenly spaced probabilities from 0.9677083 down to 1/2, 8 positive and 7
+ * negative plus an exact zero, normalised by the largest magnitude.
+ */
+void qlora_nf4_table(float *out16);
+
+/*
+ * qlora_nf4_thresholds: writes the 15 decision thresholds of the NF4 code search to
+ * host memory `out15`: code(x) = number of i with x >= out15[i], for every fp32 x in
+ * [-1, 1]. They reproduce argmin_i fl32(|x - NF4[i]|) with ties to the lower index
+ * exactly. Host-only.
+ */
+void qlora_nf4_thresholds(float *out15);
+
+/*
+ * qlora_fp8_thresholds: the same for the 253-entry double-quantization table T8
+ * (distinct finite E4M3 values / 448, ascending): 252 thresholds to host memory
+ * `out252`; also writes T8 itself to `t8_out253` and the E4M3 bit pattern of each
+ * entry to `codes_out253` when those are not NULL. Host-only.
+ */
+void qlora_fp8_thresholds(float *out252, float *t8_out253, uint8_t *codes_out253);
+
+/* Device bytes of workspace qlora_quantize_nf4_dq needs for an N x K weight. */
+size_t qlora_quantize_workspace_size(int64_t n_out, int64_t k_in);
+
+/*
+ * qlora_quantize_nf4_dq: quantize W [n_out, k_in] (device, fp32 or bf16 per
+ * `w_dtype`) to NF4 with double-quantized constants.
+ * Steps (itwiki "QLoRA", NF4 and double-quantization sections):
+ *   1. per 64-block absmax a_j = max |w|; x = fl32(w / a_j) (x = 0 when a_j = 0);
+ *      code = nearest NF4 level (ties to the lower index); two codes per byte.
+ *   2. mean = fl32(sum_j a_j / (N*K/64)) summed in fp64.
+ *   3. per 256-block of centred constants cc_j = fl32(a_j - mean):
+ *      c1 = max |cc|; y = fl32(cc_j / c1) (0 when c1 = 0); c2_j = E4M3 bit pattern
+ *      of the nearest T8 entry (ties to the lower index).
+ * Outputs (device): codes [N*K/2], c2 [N*K/64], c1 [ceil(N*K/16384)], mean [1].
+ * Workspace: at least qlora_quantize_workspace_size(n_out, k_in) bytes (device).
+ * Errors: QLORA_ERR_SHAPE unless n_out >= 1, k_in >= 64 and k_in % 64 == 0;
+ *         QLORA_ERR_INVALID_ARG for a NULL pointer or unknown dtype.
+ * Inputs must be finite.
+ */
+qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, int64_t n_out,
+                                   int64_t k_in, uint8_t *codes, uint8_t *c2, float *c1,
+                                   float *mean, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+/*
+ * qlora_dequant: W_out [n_out, k_in] bf16 (device) = doubleDequant(c1, c2, W_NF4)
+ * (itwiki "QLoRA", computation section; formula in the storage notes above).
+ * Bit-exact with the definition. No workspace.
+ */
+qlora_status qlora_dequant(qlora_nf4_weight w, uint16_t *W_out, void *stream);
+
+/* Device bytes of workspace qlora_linear_fwd needs (0 < r <= 64, r % 8 == 0). */
+size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
+
+/*
+ * qlora_linear_fwd: Y [M, N] bf16 = bf16(X W_hat^T + scale (X A) B), fp32 accumulation.
+ * (itwiki "QLoRA", computation section, with the alpha/r scale of minnong511
+ * "quantization": scale = alpha / r.)
+ *   X      [M, K] bf16 device        A [K, r] bf16 device     B [r, N] bf16 device
+ *   Y      [M, N] bf16 device (written)
+ *   T_save [M, r] fp32 device or NULL: when given, receives T = X A (unscaled) for
+ *          the backward.
+ * M >= 0 (M == 0 enqueues nothing and X, Y may be NULL); r in {8, 16, ..., 64}. M <= 16 runs the decode
+ * (GEMV) kernels, larger M the fused tensor-core GEMM; both dequantize W in
+ * registers without writing it to memory.
+ */
+qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, qlora_nf4_weight w,
+                              const uint16_t *A, const uint16_t *B, int r, float scale,
+                              uint16_t *Y, float *T_save, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/* Device bytes of workspace qlora_linear_bwd needs. */
+size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
+
+/*
+ * qlora_linear_bwd: gradients of qlora_linear_fwd for the upstream gradient dY.
+ *   G  = dY B^T                         [M, r]
+ *   dX = bf16(dY W_hat + scale G A^T)   [M, K] bf16 device, or NULL to skip
+ *   dA = scale X^T G                    [K, r] fp32 device (overwritten)
+ *   dB = scale T^T dY                   [r, N] fp32 device (overwritten)
+ * T_saved [M, r] fp32 device is T = X A from the forward, or NULL to recompute it.
+ * The quantized W is frozen: no gradient for it (itwiki "QLoRA", computation
+ * section; minnong511 "quantization": W is not updated, A and B get gradients).
+ * M == 0 writes zeros to dA and dB (dY, X, dX may be NULL).
+ */
+qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float *T_saved,
+                              int64_t M, qlora_nf4_weight w, const uint16_t *A,
+                              const uint16_t *B, int r, float scale, uint16_t *dX,
+                              float *dA, float *dB, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

@@ -1,0 +1,161 @@
+"""Host-side checks of the C-ABI library: it loads, exports every declared entry point,
+carries the same code tables as the oracle, derives exact nearest-entry thresholds,
+and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_nf4_quantized_unpack_b200 import build, qlora
+from oracle import nf4_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return qlora.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "qlora.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_nf4_table_matches_oracle_bits(L):
+    got = qlora.nf4_table().numpy()
+    assert np.array_equal(got.view(np.uint32), O.nf4_levels().view(np.uint32))
+
+
+def _next_up(x, n=1):
+    return np.nextafter(x, np.float32(np.inf), dtype=np.float32) if n == 1 else None
+
+
+def _ulp_window(center, half):
+    """All fp32 values within `half` ulps of center (ordered-bit walk)."""
+    c = np.float32(center)
+    out = [c]
+    lo, hi = c, c
+    for _ in range(half):
+        lo = np.nextafter(lo, np.float32(-np.inf))
+        hi = np.nextafter(hi, np.float32(np.inf))
+        out += [lo, hi]
+    return np.array(out, np.float32)
+
+
+def _count_leq(th, x):
+    return np.searchsorted(th, x, side="right")
+
+
+def test_nf4_thresholds_reproduce_argmin(L):
+    th = qlora.nf4_thresholds().numpy()
+    table = O.nf4_levels()
+    assert np.all(np.diff(th) > 0)
+    xs = [np.random.default_rng(0).uniform(-1, 1, 1 << 18).astype(np.float32), table,
+          np.array([-1.0, 1.0, 0.0, -0.0], np.float32)]
+    for t in th:
+        xs.append(_ulp_window(t, 2048))
+        mid = np.float32((np.float64(t)))
+        xs.append(_ulp_window(mid, 16))
+    # every midpoint of neighbouring levels, rounded both ways
+    mids = (table[:-1].astype(np.float64) + table[1:]) / 2
+    for m in mids:
+        xs.append(_ulp_window(np.float32(m), 64))
+    x = np.concatenate(xs)
+    x = x[(x >= -1) & (x <= 1)]
+    assert np.array_equal(O.nearest_code(x, table), _count_leq(th, x))
+
+
+def test_fp8_table_and_thresholds_match_oracle(L):
+    th, vals, codes = (t.numpy() for t in qlora.fp8_thresholds())
+    ovals, ocodes = O.fp8_table()
+    assert np.array_equal(vals.view(np.uint32), ovals.view(np.uint32))
+    assert np.array_equal(codes, ocodes)
+    assert th.size == 252 and np.all(np.diff(th) > 0)
+    xs = [np.random.default_rng(1).uniform(-1, 1, 1 << 16).astype(np.float32), ovals]
+    for t in th:
+        xs.append(_ulp_window(t, 24))
+    x = np.concatenate(xs)
+    x = x[(x >= -1) & (x <= 1)]
+    assert np.array_equal(O.nearest_code(x, ovals), _count_leq(th, x))
+
+
+def test_status_strings(L):
+    for code, name in qlora.STATUS.items():
+        assert L.qlora_status_str(code).decode() == name
+    assert L.qlora_version() >= 100
+
+
+# ----------------------------------------------------------------- argument errors
+# Fake, never dereferenced device addresses: every case below is rejected on the
+# host before any CUDA call.
+P = 1 << 20          # 16-byte aligned fake pointer
+Q = (1 << 20) + 8    # misaligned fake pointer
+
+
+def W(codes=P, c2=P, c1=P, mean=P, n=512, k=1024):
+    return qlora.CNF4Weight(codes, c2, c1, mean, n, k)
+
+
+def test_quantize_rejects_bad_arguments(L):
+    f = L.qlora_quantize_nf4_dq
+    ws = L.qlora_quantize_workspace_size(512, 1024)
+    assert ws > 0 and L.qlora_quantize_workspace_size(512, 1000) == 0
+    ok = [P, 0, 512, 1024, P, P, P, P, P, ws, None]
+    def call(**kw):
+        a = list(ok)
+        idx = {"W": 0, "dtype": 1, "n": 2, "k": 3, "codes": 4, "ws": 8, "wsb": 9}
+        for k_, v in kw.items():
+            a[idx[k_]] = v
+        return f(*a)
+    assert call(W=None) == 1
+    assert call(dtype=7) == 1
+    assert call(k=1000) == 2
+    assert call(k=0) == 2
+    assert call(n=0) == 2
+    assert call(codes=Q) == 3
+    assert call(ws=None) == 4
+    assert call(wsb=ws - 1) == 4
+
+
+def test_linear_rejects_bad_arguments(L):
+    fwd = L.qlora_linear_fwd
+    need = L.qlora_linear_fwd_workspace_size(64, 512, 1024, 8)
+    assert need > 0
+    base = dict(X=P, M=64, w=W(), A=P, B=P, r=8, scale=2.0, Y=P, T=None, ws=P, wsb=need)
+    def call(**kw):
+        a = dict(base, **kw)
+        return fwd(a["X"], a["M"], a["w"], a["A"], a["B"], a["r"], a["scale"], a["Y"], a["T"],
+                   a["ws"], a["wsb"], None)
+    assert call(X=None) == 1
+    assert call(r=0) == 1 and call(r=12) == 1 and call(r=72) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(w=W(k=1000)) == 2
+    assert call(w=W(n=500)) == 2
+    assert call(M=-1) == 2
+    assert call(w=W(codes=None)) == 1
+    assert call(w=W(c2=Q)) == 3
+    assert call(Y=Q) == 3
+    assert call(ws=None) == 4
+    assert call(wsb=need - 1) == 4
+    assert call(M=0) == 0          # empty input: nothing to do, nothing launched
+    bwd = L.qlora_linear_bwd
+    bneed = L.qlora_linear_bwd_workspace_size(64, 512, 1024, 8)
+    assert bneed > 0
+    assert bwd(None, P, None, 64, W(), P, P, 8, 2.0, P, P, P, P, bneed, None) == 1
+    assert bwd(P, P, None, 64, W(), P, P, 8, 2.0, P, None, P, P, bneed, None) == 1
+    assert bwd(P, P, None, 64, W(), P, P, 8, 2.0, P, P, P, P, bneed - 1, None) == 4
+    assert bwd(P, P, Q, 64, W(), P, P, 8, 2.0, P, P, P, P, bneed, None) == 3
+    assert L.qlora_dequant(W(k=100), P, None) == 2
+    assert L.qlora_dequant(W(), None, None) == 1

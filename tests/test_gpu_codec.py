@@ -1,0 +1,134 @@
+"""GPU parity of the codec (quantize, double quantization, dequant) against the oracle.
+Codes, c2, c1, mean and the dequantized bf16 weights must be bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_unpack_b200 import inputs, qlora
+from oracle import nf4_oracle as O
+from tests.gpu_util import host, need_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def quantize_on_gpu(W, bf16):
+    t = torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
+    if bf16:
+        t = t.to(torch.bfloat16)
+    q = qlora.qlora_quantize_nf4_dq(t)
+    torch.cuda.synchronize()
+    return q
+
+
+def compare_full(W, bf16):
+    q = quantize_on_gpu(W, bf16)
+    ref = O.quantize_nf4_dq(W)
+    assert np.array_equal(q.codes.cpu().numpy(), ref["codes"])
+    assert np.array_equal(q.c2.cpu().numpy(), ref["c2"])
+    assert np.array_equal(q.c1.cpu().numpy().view(np.uint32), ref["c1"].view(np.uint32))
+    assert q.mean.cpu().numpy().view(np.uint32)[0] == np.float32(ref["mean"]).view(np.uint32)
+    wd = qlora.qlora_dequant(q)
+    torch.cuda.synchronize()
+    got = wd.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, O.bf16_bits(O.double_dequant(ref)))
+    return q, ref
+
+
+def test_pr1_weight_bit_exact():
+    case = inputs.pr1()
+    compare_full(case["W"], bf16=False)
+
+
+@pytest.mark.parametrize("shape", [(5, 192), (1, 64), (3, 4096), (64, 11008), (300, 704)])
+def test_ragged_and_small_shapes(shape):
+    rng = np.random.default_rng(sum(shape))
+    W = inputs.to_bf16_values(rng.normal(0, 0.02, shape).astype(np.float32))
+    compare_full(W, bf16=True)
+
+
+def test_edge_values():
+    rng = np.random.default_rng(21)
+    W = rng.normal(0, 0.02, (40, 640)).astype(np.float32)
+    W[0] = 0.0                                 # all-zero rows / blocks
+    W[1, :64] = 0.0
+    W[2, 5] = 7.5                              # isolated outliers of both signs
+    W[3, 70] = -9.0
+    W[4] = 1e-30                               # tiny magnitudes
+    W[5, :64] = -0.5                           # constant blocks
+    W[6, 64:128] = np.float32(2.0 ** -20) * np.arange(64)
+    compare_full(W, bf16=False)
+
+
+def test_codes_at_every_threshold_window():
+    """Blocks whose absmax is exactly 1 carry x = w unchanged, so weights taken from
+    windows around every NF4 decision threshold probe the code search directly."""
+    th = qlora.nf4_thresholds().numpy()
+    probes = []
+    for t in th:
+        x = np.float32(t)
+        lo = hi = x
+        probes.append(x)
+        for _ in range(300):
+            lo = np.nextafter(lo, np.float32(-2))
+            hi = np.nextafter(hi, np.float32(2))
+            probes += [lo, hi]
+    probes = np.array(probes, np.float32)
+    probes = np.concatenate([probes, O.nf4_levels(), np.array([0.0, -0.0], np.float32)])
+    per = 63
+    nblk = -(-probes.size // per)
+    probes = np.concatenate([probes, np.zeros(nblk * per - probes.size, np.float32)])
+    W = np.concatenate([np.ones((nblk, 1), np.float32), probes.reshape(nblk, per)], axis=1)
+    W = W.reshape(-1, 640)[: (nblk * 64) // 640]
+    q = quantize_on_gpu(W, bf16=False)
+    codes, _ = O.quantize_blocks(W, O.nf4_levels())
+    assert np.array_equal(q.codes.cpu().numpy(), O.pack_nibbles(codes))
+
+
+@pytest.mark.parametrize("n,k", [(4096, 4096), (4096, 11008), (11008, 4096)])
+def test_llama7b_shapes_with_outliers(n, k):
+    """Full-size codec case: all constants compared, codes and dequantized weights on
+    sampled rows (the oracle quantizes rows independently once the mean is known)."""
+    rng = np.random.default_rng(1)
+    W = inputs.weight(rng, n, k, bf16=True, outlier_frac=1e-3)
+    q = quantize_on_gpu(W, bf16=True)
+    absmax = np.max(np.abs(W.reshape(-1, 64)), axis=1)   # block absmax (exact in fp32)
+    c2, c1, mean = O.double_quantize(absmax)
+    assert q.mean.cpu().numpy()[0] == mean
+    assert np.array_equal(q.c1.cpu().numpy().view(np.uint32), c1.view(np.uint32))
+    assert np.array_equal(q.c2.cpu().numpy(), c2)
+    rows = np.unique(np.concatenate([[0, n - 1], rng.choice(n, 256, replace=False)]))
+    codes, _ = O.quantize_blocks(W[rows], O.nf4_levels())
+    got = q.codes.cpu().numpy().reshape(n, k // 2)[rows]
+    assert np.array_equal(got.ravel(), O.pack_nibbles(codes))
+    ref = {"codes": q.codes.cpu().numpy(), "c2": c2, "c1": c1, "mean": mean, "shape": (n, k)}
+    wd = qlora.qlora_dequant(q)
+    torch.cuda.synchronize()
+    got_w = wd.view(torch.int16).cpu().numpy().view(np.uint16)[rows]
+    assert np.array_equal(got_w, O.bf16_bits(O.double_dequant_rows(ref, rows)))
+    # round-trip error stays at the NF4 level
+    mae = np.mean(np.abs(host(wd)[rows] - W[rows]))
+    assert mae < 2.5e-3
+
+
+def test_dequant_of_handmade_constants():
+    """Dequantize constants that no quantizer would produce (negative and subnormal
+    scales, every E4M3 code) and compare with the definition."""
+    n, k = 16, 1024
+    nb = n * k // 64
+    rng = np.random.default_rng(4)
+    codes = rng.integers(0, 256, n * k // 2).astype(np.uint8)
+    c2 = np.array([b for b in range(256) if b not in (0x7F, 0xFF)] * 2, np.uint8)[:nb]
+    c1 = np.array([0.37, -0.0, 1e-38, 3.0], np.float32)[: -(-nb // 256)]
+    mean = np.float32(-0.01)
+    ref = {"codes": codes, "c2": c2, "c1": c1, "mean": mean, "shape": (n, k)}
+    q = qlora.NF4Weight(torch.from_numpy(codes).cuda(), torch.from_numpy(c2).cuda(),
+                        torch.from_numpy(c1).cuda(), torch.tensor([mean]).cuda(), n, k)
+    wd = qlora.qlora_dequant(q)
+    torch.cuda.synchronize()
+    got = wd.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, O.bf16_bits(O.double_dequant(ref)))
