@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA linear layer on B200.
+
+Headline: forward + dX + dA/dB TFLOP/s of a 7B-shaped decoder layer training step
+(q,k,v,o 4096x4096; gate/up 4096->11008; down 11008->4096; NF4 with double
+quantization, LoRA r=64 alpha=16 on each; M=4096 tokens per GPU). Also reported:
+the M=1 decode weight-read bandwidth on 4096x11008 and 8192x28672 NF4 weights.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one rank per GPU: data-parallel replicas, each with its
+own 4096 tokens, and one NCCL all-reduce of the LoRA gradients per step (weak
+scaling). Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s (M=4096); M=1 decode weight GB/s vs HBM peak"
+WORKLOAD = ("7B-shaped decoder layer training step: q,k,v,o 4096x4096, gate/up 4096->11008, "
+            "down 11008->4096, NF4 + double-quantized constants, LoRA r=64 alpha=16 on each; "
+            "M=4096 tokens per GPU (4x1024); forward + dX + dA/dB through all 7 linears")
+M_TOKENS, RANK_R, ALPHA = 4096, 64, 16.0
+INPUT_OF = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out",
+            "gate": "mlp_in", "up": "mlp_in", "down": "mlp_act"}
+KERNELS_PER_LINEAR_STEP = 3 + 8   # forward 3 launches, backward 8 launches
+
+
+def layer_flops(linears, M, r):
+    """Algorithmic FLOPs of forward + dX + dA/dB: 4MNK + 6Mr(K+N) per linear."""
+    return sum(4 * M * n * k + 6 * M * r * (k + n) for _, n, k in linears)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) leg
+def oracle_sample(min_seconds=8.0):
+    """Time the CPU oracle on a bounded sample of the workload: the q linear
+    (4096x4096) of the layer at 512 tokens, r=64: double dequantization of the stored
+    weight, forward, dX and dA/dB in fp64. Returns (TFLOP/s, seconds, description)."""
+    from bit_nf4_quantized_unpack_b200 import inputs
+    from oracle import nf4_oracle as O
+    case = inputs.linear_case(3, 512, 4096, 4096, RANK_R, ALPHA)
+    q = O.quantize_nf4_dq(case["W"])
+    flops, secs, reps = 0.0, 0.0, 0
+    while secs < min_seconds or reps == 0:
+        t0 = time.perf_counter()
+        What = O.double_dequant(q)
+        Y, T = O.linear_forward(case["X"], What, case["A"], case["B"], case["scale"])
+        O.linear_backward(case["dY"], case["X"], What, case["A"], case["B"], case["scale"], T=T)
+        secs += time.perf_counter() - t0
+        flops += layer_flops([("q", 4096, 4096)], 512, RANK_R)
+        reps += 1
+    desc = (f"oracle (NumPy fp64) on the q linear 4096x4096, 512 tokens, r=64: double dequant + "
+            f"forward + dX + dA/dB, {reps} repetition(s)")
+    return flops / secs / 1e12, secs, desc
+
+
+def host_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        blas = 1
+    return max(1, min(len(os.sched_getaffinity(0)), blas))
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(min_seconds=0.0)
+    per_step = []
+    for _ in range(args.steps):
+        v, secs, desc = oracle_sample(min_seconds=0.0)
+        per_step.append((v, secs))
+    value = sum(v for v, _ in per_step) / len(per_step)
+    ms = 1000.0 * sum(s for _, s in per_step) / len(per_step)
+    cores = host_cores()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU leg
+def build_layer(device, seed):
+    from bit_nf4_quantized_unpack_b200 import inputs, qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    M, r = M_TOKENS, RANK_R
+    layer = []
+    for name, n, k in inputs.LLAMA7B_LINEARS:
+        W = (torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16)
+        q = qlora.qlora_quantize_nf4_dq(W)
+        del W
+        A = (torch.randn(k, r, generator=g, device=device) * 0.02).to(torch.bfloat16)
+        B = (torch.randn(r, n, generator=g, device=device) * 0.02).to(torch.bfloat16)
+        layer.append(dict(name=name, n=n, k=k, q=q, A=A, B=B))
+    xs = {}
+    for lin in layer:
+        key = INPUT_OF[lin["name"]]
+        if key not in xs:
+            xs[key] = torch.randn(M, lin["k"], generator=g, device=device).to(torch.bfloat16)
+    grad_numel = sum(lin["k"] * r + r * lin["n"] for lin in layer)
+    grads = torch.empty(grad_numel, dtype=torch.float32, device=device)
+    off = 0
+    ws_f = max(qlora.qlora_linear_fwd_workspace_size(M, l["n"], l["k"], r) for l in layer)
+    ws_b = max(qlora.qlora_linear_bwd_workspace_size(M, l["n"], l["k"], r) for l in layer)
+    for lin in layer:
+        lin["dY"] = torch.randn(M, lin["n"], generator=g, device=device).to(torch.bfloat16)
+        lin["Y"] = torch.empty(M, lin["n"], dtype=torch.bfloat16, device=device)
+        lin["T"] = torch.empty(M, r, dtype=torch.float32, device=device)
+        lin["dX"] = torch.empty(M, lin["k"], dtype=torch.bfloat16, device=device)
+        lin["dA"] = grads[off:off + lin["k"] * r].view(lin["k"], r)
+        off += lin["k"] * r
+        lin["dB"] = grads[off:off + r * lin["n"]].view(r, lin["n"])
+        off += r * lin["n"]
+    return dict(layer=layer, xs=xs, grads=grads,
+                ws_f=torch.empty(ws_f, dtype=torch.uint8, device=device),
+                ws_b=torch.empty(ws_b, dtype=torch.uint8, device=device))
+
+
+def event_pair():
+    """Two timing events whose CUDA handles exist (torch creates them on first record)."""
+    pair = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    for e in pair:
+        e.record()
+    return pair
+
+
+def layer_step(L, scale, world, events=None, pool=None):
+    from bit_nf4_quantized_unpack_b200 import qlora
+    xs = L["xs"]
+    for lin in L["layer"]:
+        if events is not None:
+            events.append((*pool.pop(), "fwd", lin))
+            qlora.qlora_profile_events(events[-1][0], events[-1][1])
+        qlora.qlora_linear_fwd(xs[INPUT_OF[lin["name"]]], lin["q"], lin["A"], lin["B"], scale,
+                               Y=lin["Y"], T=lin["T"], workspace=L["ws_f"])
+    for lin in reversed(L["layer"]):
+        if events is not None:
+            events.append((*pool.pop(), "dgrad", lin))
+            qlora.qlora_profile_events(events[-1][0], events[-1][1])
+        qlora.qlora_linear_bwd(lin["dY"], xs[INPUT_OF[lin["name"]]], lin["T"], lin["q"], lin["A"],
+                               lin["B"], scale, dX=lin["dX"], dA=lin["dA"], dB=lin["dB"],
+                               workspace=L["ws_b"])
+    if events is not None:
+        qlora.qlora_profile_events(None, None)
+    if world > 1:
+        torch.distributed.all_reduce(L["grads"])   # data-parallel LoRA gradient exchange
+
+
+def time_steps(fn, steps, world):
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        fn()
+    stop.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(stop) / steps
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def decode_bandwidth(device, M=1, iters=40):
+    """Weight-read bandwidth of the M-token forward, CUDA-graph timed, cycling through
+    enough copies of the weight that no call finds it in L2."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    out = {}
+    r, alpha = 16, 32.0
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    g = torch.Generator(device=device)
+    g.manual_seed(2)
+    for (n, k) in ((4096, 11008), (8192, 28672)):
+        W = (torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16)
+        q0 = qlora.qlora_quantize_nf4_dq(W)
+        del W
+        wbytes = q0.codes.numel() + q0.c2.numel() + q0.c1.numel() * 4 + 4
+        copies = max(2, int(np.ceil(4 * l2 / wbytes)))
+        qs = [q0] + [qlora.NF4Weight(q0.codes.clone(), q0.c2.clone(), q0.c1.clone(), q0.mean.clone(),
+                                     n, k) for _ in range(copies - 1)]
+        A = (torch.randn(k, r, generator=g, device=device) * 0.02).to(torch.bfloat16)
+        B = (torch.randn(r, n, generator=g, device=device) * 0.02).to(torch.bfloat16)
+        X = torch.randn(M, k, generator=g, device=device).to(torch.bfloat16)
+        Y = torch.empty(M, n, dtype=torch.bfloat16, device=device)
+        ws = torch.empty(qlora.qlora_linear_fwd_workspace_size(M, n, k, r), dtype=torch.uint8,
+                         device=device)
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for i in range(3):
+                qlora.qlora_linear_fwd(X, qs[i % copies], A, B, alpha / r, save_T=False, Y=Y, workspace=ws)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=s):
+                for i in range(iters):
+                    qlora.qlora_linear_fwd(X, qs[i % copies], A, B, alpha / r, save_T=False, Y=Y,
+                                           workspace=ws)
+            graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            e0.record(s)
+            for _ in range(reps):
+                graph.replay()
+            e1.record(s)
+            torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / (reps * iters)
+        algo = 0.515869140625 * n * k + (k + n) * r * 2 + M * k * 2 + M * n * 2
+        out[f"{n}x{k}"] = {"M": M, "us_per_call": us, "algorithmic_bytes": int(algo),
+                           "GBps": algo / us / 1e3, "weight_copies": copies}
+        del graph, qs, q0
+        torch.cuda.empty_cache()
+    return out
+
+
+def e2e_steps(L, scale, world, steps):
+    """The same step through the public API with host-resident inputs: every step copies
+    the activations and upstream gradients from pinned host memory and reads the LoRA
+    gradients back."""
+    host_x = {k: v.cpu().pin_memory() for k, v in L["xs"].items()}
+    host_dy = [lin["dY"].cpu().pin_memory() for lin in L["layer"]]
+    host_grads = torch.empty(L["grads"].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_x.values()) + \
+        sum(t.numel() * t.element_size() for t in host_dy)
+    d2h = host_grads.numel() * 4
+
+    def step():
+        for k, v in host_x.items():
+            L["xs"][k].copy_(v, non_blocking=True)
+        for lin, h in zip(L["layer"], host_dy):
+            lin["dY"].copy_(h, non_blocking=True)
+        layer_step(L, scale, world)
+        host_grads.copy_(L["grads"], non_blocking=True)
+
+    step()
+    ms = time_steps(step, steps, world)
+    return ms, h2d, d2h
+
+
+def profile_linear(device, scale, warmup, steps):
+    """One linear (gate, 11008 x 4096) forward + backward at M=4096, for ncu captures."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(5)
+    n, k, M, r = 11008, 4096, M_TOKENS, RANK_R
+    W = (torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    q = qlora.qlora_quantize_nf4_dq(W)
+    del W
+    A = (torch.randn(k, r, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    B = (torch.randn(r, n, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    X = torch.randn(M, k, generator=g, device=device).to(torch.bfloat16)
+    dY = torch.randn(M, n, generator=g, device=device).to(torch.bfloat16)
+    for _ in range(warmup + steps):
+        _, T = qlora.qlora_linear_fwd(X, q, A, B, scale)
+        qlora.qlora_linear_bwd(dY, X, T, q, A, B, scale)
+    torch.cuda.synchronize()
+    if qlora.qlora_device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-linear", action="store_true",
+                    help="only run forward + backward of the gate linear (11008x4096, M=4096) "
+                         "--steps times: a small, self-contained case for profiler captures")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    from bit_nf4_quantized_unpack_b200 import build, inputs, qlora
+    build.build()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    scale = ALPHA / RANK_R
+    if args.profile_linear:
+        profile_linear(device, scale, args.warmup, args.steps)
+        return
+    L = build_layer(device, seed=3 + 1000 * rank)
+    flops = layer_flops(inputs.LLAMA7B_LINEARS, M_TOKENS, RANK_R)
+    step = lambda: layer_step(L, scale, world)  # noqa: E731
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if qlora.qlora_device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_steps(step, args.steps, world)
+    clk = clocks.stop()
+    value = world * flops / (ms / 1e3) / 1e12
+    print(f"[bench] layer step {ms:.3f} ms -> {value:.1f} TFLOP/s per {world} GPU(s)",
+          file=sys.stderr, flush=True)
+
+    # dominant kernel: the fused NF4 GEMM, timed per launch with events on its stream
+    events = []
+    pool = [event_pair() for _ in range(2 * len(L["layer"]) * args.steps)]
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        layer_step(L, scale, world, events=events, pool=pool)
+    torch.cuda.synchronize()
+    fused_ms = sum(b.elapsed_time(a) for b, a, _, _ in events)
+    fused_flops = 0
+    for _, _, kind, lin in events:
+        other = lin["n"] if kind == "fwd" else lin["k"]
+        fused_flops += 2 * M_TOKENS * lin["n"] * lin["k"] + 2 * M_TOKENS * RANK_R * other
+    peaks, peaks_src = load_peaks()
+    achieved = fused_flops / (fused_ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    roofline = {"bound": "tensor", "kernel": "k_fused_nf4_gemm (forward + dX)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peaks_src} bf16_tflops_sustained",
+                "fused_share_of_step": fused_ms / args.steps / ms, "traffic": None}
+
+    e2e_ms, h2d, d2h = e2e_steps(L, scale, world, max(2, args.steps // 2))
+    e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    decode = None
+    if not args.no_decode and rank == 0:
+        del L
+        torch.cuda.empty_cache()
+        decode = decode_bandwidth(device)
+        hbm = float(peaks["hbm_gbs"])
+        for v in decode.values():
+            v["frac_of_hbm"] = v["GBps"] / hbm
+        decode["hbm_peak_GBps"] = hbm
+        decode["hbm_peak_source"] = f"{peaks_src} hbm_gbs"
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, secs, desc = oracle_sample()
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+               "sample": desc, "seconds": secs}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": WORKLOAD, "tokens_per_gpu": M_TOKENS,
+                           "global_tokens": M_TOKENS * world, "lora_rank": RANK_R,
+                           "lora_alpha": ALPHA, "parallelism": f"dp{world}",
+                           "flops_per_step_per_gpu": flops,
+                           "l2": "inputs larger than L2 (weights + activations ~1.3 GB per step)"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": KERNELS_PER_LINEAR_STEP * len(inputs.LLAMA7B_LINEARS) * args.steps,
+                "clocks": clk, "decode": decode}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

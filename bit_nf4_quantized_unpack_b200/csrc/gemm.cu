@@ -11,9 +11,10 @@
 //      W_hat is never written to memory: packed codes arrive by TMA, eight dequant
 //      warps expand them (double dequantization, bit-exact bf16) straight into the
 //      128B-swizzled shared-memory operand layout, and one thread issues
-//      tcgen05.mma into a 128 x 256 fp32 TMEM accumulator. The LoRA product is one
-//      more pipeline step on the same accumulator with operands Ts = bf16(scale T)
-//      and B (r padded to a multiple of 16 with zeros by TMA).
+//      tcgen05.mma into a 128 x 256 fp32 TMEM accumulator. The LoRA product is two
+//      more pipeline steps on the same accumulator with operands B (r padded to a
+//      multiple of 16 with zeros by TMA) and Ts = scale T split into a bf16 hi part
+//      and a bf16 lo part (scale T - hi), which keeps it at fp32-level accuracy.
 //  k_fused_nf4_gemm<kDgrad>: D[k, m] = sum_n W_hat[n, k] dY[m, n] + sum_j A[k, j] Gs[m, j]
 //      the same pipeline with W_hat dequantized into the MN-major operand layout
 //      (contraction over the output features n).
@@ -93,7 +94,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kTileCols;
   const int64_t contraction = (MODE == Mode::kForward) ? args.K : args.N;
   const int ksteps = static_cast<int>((contraction + kBK - 1) / kBK);
-  const int total = ksteps + (args.ext_mmas > 0 ? 1 : 0);
+  // the LoRA product enters as two steps: bf16 hi part, then bf16 lo part of scale*T
+  const int total = ksteps + (args.ext_mmas > 0 ? 2 : 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -148,7 +150,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             // A [K, r] as a K-major operand (columns j >= r are 0)
             tma_load_2d(w_s + s * kWBytes, &tm_ext_w, &full[s], 0, static_cast<int>(row0));
           }
-          tma_load_2d(act_s + s * kActBytes, &tm_ext_act, &full[s], 0, static_cast<int>(m0));
+          tma_load_2d(act_s + s * kActBytes, &tm_ext_act, &full[s], (step - ksteps) * 64,
+                      static_cast<int>(m0));
         }
         ++issued;
       }
@@ -439,7 +442,8 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
 
 // ================================================================== finalize kernels
 // T (or G) = sum of split partials [S][rows_pad][64]. Writes, where asked:
-//   plain fp32 [M, r], scaled bf16 [M, 64] (K-extension operand), hi/lo bf16 [M, 128].
+//   plain fp32 [M, r]; bf16 hi/lo of scale * v [M, 128] (the K-extension operand);
+//   bf16 hi/lo of v [M, 128] (operand of the LoRA gradients).
 __global__ void k_finalize_rank(const float* __restrict__ part, int splits, int64_t rows_pad,
                                 int64_t M, int r, float scale, float* __restrict__ plain,
                                 uint16_t* __restrict__ scaled, uint16_t* __restrict__ hilo) {
@@ -451,7 +455,12 @@ __global__ void k_finalize_rank(const float* __restrict__ part, int splits, int6
   for (int s = 0; s < splits; ++s) v += part[(s * rows_pad + m) * 64 + j];
   if (j >= r) v = 0.f;
   if (plain && j < r) plain[m * r + j] = v;
-  if (scaled) scaled[m * 64 + j] = bf16_bits_rn(v * scale);
+  if (scaled) {  // [M, 128]: bf16 hi | bf16 lo of scale * v
+    const float sv = v * scale;
+    const uint16_t hi = bf16_bits_rn(sv);
+    scaled[m * 128 + j] = hi;
+    scaled[m * 128 + 64 + j] = bf16_bits_rn(sv - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+  }
   if (hilo) {
     const uint16_t hi = bf16_bits_rn(v);
     const float hv = __uint_as_float(static_cast<uint32_t>(hi) << 16);
@@ -510,6 +519,11 @@ SplitPlan plan_split(int64_t rows, int64_t contraction) {
   p.tiles = (rows + 127) / 128;
   p.rows_pad = p.tiles * 128;
   p.steps_total = static_cast<int>((contraction + kBK - 1) / kBK);
+  if (p.steps_total == 0 || p.tiles == 0) {  // empty operand: one (idle) split
+    p.splits = 1;
+    p.steps_per = p.steps_total > 0 ? p.steps_total : 1;
+    return p;
+  }
   const int64_t target = 2LL * num_sms();
   int64_t want = (target + p.tiles - 1) / p.tiles;
   want = std::max<int64_t>(1, std::min<int64_t>(want, (p.steps_total + 1) / 2));
@@ -586,7 +600,7 @@ struct Carve {
 size_t fwd_layout(const LinearShape& s, void* ws, float** part, uint16_t** ts) {
   Carve c(ws);
   *part = c.take<float>(partial_floats(s.M, s.K, 64));
-  *ts = c.take<uint16_t>(static_cast<size_t>(s.M) * 64);
+  *ts = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
   return c.off + 256;
 }
 
@@ -598,7 +612,7 @@ size_t bwd_layout(const LinearShape& s, void* ws, float** part, uint16_t** gs, u
   pf = std::max(pf, partial_floats(s.K, s.M, 128));            // dA
   pf = std::max(pf, partial_floats(s.N, s.M, 128));            // dB
   *part = c.take<float>(pf);
-  *gs = c.take<uint16_t>(static_cast<size_t>(s.M) * 64);
+  *gs = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
   *ghl = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
   *thl = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
   *t = c.take<float>(static_cast<size_t>(s.M) * s.r);
@@ -658,7 +672,7 @@ qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const ui
          CU_TENSOR_MAP_SWIZZLE_NONE);
   QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 256, kSW128);
   QL_MAP(&tw, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);   // B [r, N], MN-major chunks
-  QL_MAP(&tx, kBF16, ts, 64, s.M, 128, 64, 256, kSW128);      // bf16(scale T) [M, 64]
+  QL_MAP(&tx, kBF16, ts, 128, s.M, 256, 64, 256, kSW128);     // scale T, bf16 hi | lo
   FusedArgs a;
   a.c2 = w.c2;
   a.c1 = w.c1;
@@ -711,7 +725,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
            CU_TENSOR_MAP_SWIZZLE_NONE);
     QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 256, kSW128);
     QL_MAP(&tw, kBF16, A, s.r, s.K, s.r * 2, 64, 128, kSW128);   // A [K, r] K-major
-    QL_MAP(&tx, kBF16, gs, 64, s.M, 128, 64, 256, kSW128);       // bf16(scale G) [M, 64]
+    QL_MAP(&tx, kBF16, gs, 128, s.M, 256, 64, 256, kSW128);      // scale G, bf16 hi | lo
     FusedArgs a;
     a.c2 = w.c2;
     a.c1 = w.c1;

@@ -81,6 +81,7 @@ def test_codes_at_every_threshold_window():
     probes = np.concatenate([probes, O.nf4_levels(), np.array([0.0, -0.0], np.float32)])
     per = 63
     nblk = -(-probes.size // per)
+    nblk = -(-nblk // 10) * 10             # whole rows of 640 weights
     probes = np.concatenate([probes, np.zeros(nblk * per - probes.size, np.float32)])
     W = np.concatenate([np.ones((nblk, 1), np.float32), probes.reshape(nblk, per)], axis=1)
     W = W.reshape(-1, 640)[: (nblk * 64) // 640]
