@@ -17,6 +17,8 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdio>
+#include <mutex>
 
 #include "internal.h"
 #include "nf4_device.cuh"
@@ -306,3 +308,135 @@ qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const 
 }
 
 }  // namespace qlora
+
+// ============================================================================
+// Allocation-free variant of the decode forward.
+//
+// Some callers cannot call cudaMalloc when they run the layer: a runtime that plans
+// all device memory once at start-up and forbids later allocation, or a decode loop
+// that must not pay cudaMalloc's implicit device synchronisation on every token.
+// They cannot hand over a workspace either. For them, qlora_linear_fwd_decode_static
+// keeps the split partial sums in the fixed array below, which every GPU that loads
+// this library holds until the process exits.
+namespace qlora {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t{4} << 20;  // 4 MiB per device
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_decode_scratch on the current device. In host code the name
+// g_decode_scratch is only a host-side stand-in, so the address is looked up once
+// per device with that device current, and cached.
+qlora_status scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= kMaxScratchDevices) {
+    set_last_error("device index out of range for the static scratch table");
+    return QLORA_ERR_INVALID_ARG;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return QLORA_OK;
+}
+
+bool aligned16_ptr(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+}  // namespace qlora
+
+extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_t M,
+                                                       qlora_nf4_weight w, const uint16_t* A,
+                                                       const uint16_t* B, int r, float scale,
+                                                       uint16_t* Y, float* T_save, void* stream) {
+  using namespace qlora;
+  if (!w.codes || !w.c2 || !w.c1 || !w.mean) return QLORA_ERR_INVALID_ARG;
+  if (w.n_out < 1 || w.k_in < 64 || w.k_in % 64 != 0 || w.n_out % 8 != 0 ||
+      w.n_out > (int64_t{1} << 31) || w.k_in > (int64_t{1} << 31))
+    return QLORA_ERR_SHAPE;
+  if (M < 0 || M > kDecodeMaxM) {
+    set_last_error("qlora_linear_fwd_decode_static serves 0 <= M <= 16 tokens");
+    return QLORA_ERR_SHAPE;
+  }
+  if (r < 8 || r > 64 || r % 8 != 0) return QLORA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16_ptr(w.codes) || !aligned16_ptr(w.c2) || !aligned16_ptr(w.c1) ||
+      !aligned16_ptr(w.mean))
+    return QLORA_ERR_ALIGN;
+  if (M == 0) return QLORA_OK;
+  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16_ptr(X) || !aligned16_ptr(A) || !aligned16_ptr(B) || !aligned16_ptr(Y) ||
+      (T_save && !aligned16_ptr(T_save)))
+    return QLORA_ERR_ALIGN;
+
+  const LinearShape s{M, w.n_out, w.k_in, r, scale};
+  DecodePlan p = plan_decode(s);
+  // Fewer K splits when the planned partial sums would not fit the static array.
+  const size_t per_split = static_cast<size_t>(M) * (s.N + s.r) * 4;
+  const size_t fit = (kStaticScratchBytes - 512) / per_split;
+  if (fit < 1) {
+    char msg[200];
+    std::snprintf(msg, sizeof(msg),
+                  "qlora_linear_fwd_decode_static: M * (N + r) * 4 = %zu bytes exceeds the "
+                  "%zu-byte static scratch",
+                  per_split, kStaticScratchBytes);
+    set_last_error(msg);
+    return QLORA_ERR_WORKSPACE;
+  }
+  if (static_cast<size_t>(p.splits) > fit) {
+    p.units_per = static_cast<int>((p.nunits + fit - 1) / fit);
+    p.splits = (p.nunits + p.units_per - 1) / p.units_per;
+  }
+  void* scratch = nullptr;
+  qlora_status q = scratch_address(&scratch);
+  if (q != QLORA_OK) return q;
+
+  DecodeArgs a;
+  a.codes = w.codes;
+  a.c2 = w.c2;
+  a.c1 = w.c1;
+  a.mean = w.mean;
+  a.X = X;
+  a.A = A;
+  a.M = s.M;
+  a.N = s.N;
+  a.K = s.K;
+  a.r = s.r;
+  a.splits = p.splits;
+  a.units_per = p.units_per;
+  a.nunits = p.nunits;
+  a.row_groups = p.row_groups;
+  a.t_groups = p.t_groups;
+  // Every partial sum below is written by the GEMV before the finalize kernel reads
+  // it, so nothing left in the array by an earlier call needs clearing.
+  char* base = static_cast<char*>(scratch);
+  a.part = reinterpret_cast<float*>(base);
+  a.tpart = reinterpret_cast<float*>(
+      base + align_up(static_cast<size_t>(p.splits) * s.M * s.N * 4, 256));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t warps = static_cast<int64_t>(p.row_groups + p.t_groups) * p.splits;
+  const unsigned ctas = static_cast<unsigned>((warps + 7) / 8);
+  if (s.M > 8)
+    k_decode_gemv<true><<<ctas, kDecThreads, 0, st>>>(a);
+  else
+    k_decode_gemv<false><<<ctas, kDecThreads, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e);
+  k_decode_finalize<<<static_cast<unsigned>((s.N + 255) / 256), 256, 0, st>>>(
+      a.part, a.tpart, p.splits, s.M, s.N, s.r, s.scale, B, Y, T_save);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e);
+  return QLORA_OK;
+}
+

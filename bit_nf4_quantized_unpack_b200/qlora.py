@@ -54,6 +54,8 @@ _SIGNATURES = {
     "qlora_dequant": (_i32, [CNF4Weight, _vp, _vp]),
     "qlora_linear_fwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
     "qlora_linear_fwd": (_i32, [_vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_linear_fwd_decode_static": (_i32, [_vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp,
+                                              _vp, _vp]),
     "qlora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
     "qlora_linear_bwd": (_i32, [_vp, _vp, _vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp,
                                 _vp, _vp, _sz, _vp]),

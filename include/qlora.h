@@ -179,6 +179,31 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, qlora_nf4_weight w,
                               uint16_t *Y, float *T_save, void *workspace,
                               size_t workspace_bytes, void *stream);
 
+/*
+ * qlora_linear_fwd_decode_static: the decode forward (0 <= M <= 16 tokens) of
+ * qlora_linear_fwd, for callers that cannot allocate device memory when they run the
+ * layer: a runtime that plans all device memory once at start-up and forbids later
+ * allocation, or a token-by-token decode loop that must not pay the implicit device
+ * synchronisation of cudaMalloc. It takes no workspace. The method's pages have no
+ * counterpart of this entry point; it is a deployment convenience.
+ *   Arguments, layouts and results are those of qlora_linear_fwd with M <= 16.
+ *   Scratch: a fixed 4 MiB array in device memory inside this library, which every
+ *   GPU that loads the library holds until the process exits. It must hold
+ *   M * (N + r) * 4 bytes for at least one split of K; larger problems are rejected
+ *   with QLORA_ERR_WORKSPACE (qlora_last_error() gives the sizes), M > 16 with
+ *   QLORA_ERR_SHAPE. When the usual number of K splits does not fit, fewer are used.
+ *   The first call on each device looks up the array's device address (with that
+ *   device current) and caches it; make that first call before any stream capture.
+ *   Every call uses the same array and overwrites what it needs, so calls whose
+ *   kernels overlap on the GPU (different streams, or different host threads on
+ *   one device) race on it: issue them in order on one stream.
+ *   The function itself allocates nothing (no cudaMalloc, no cudaFree).
+ */
+qlora_status qlora_linear_fwd_decode_static(const uint16_t *X, int64_t M, qlora_nf4_weight w,
+                                            const uint16_t *A, const uint16_t *B, int r,
+                                            float scale, uint16_t *Y, float *T_save,
+                                            void *stream);
+
 /* Device bytes of workspace qlora_linear_bwd needs. */
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
 
