@@ -348,6 +348,22 @@ def profile_linear(device, scale, warmup, steps):
         raise RuntimeError("a kernel reported a timed-out wait")
 
 
+def profile_decode(device, warmup, steps, n=8192, k=28672, M=1, r=16, alpha=32.0):
+    """M-token forward (decode kernels) on one n x k weight, for ncu captures."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(6)
+    W = (torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    q = qlora.qlora_quantize_nf4_dq(W)
+    del W
+    A = (torch.randn(k, r, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    B = (torch.randn(r, n, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    X = torch.randn(M, k, generator=g, device=device).to(torch.bfloat16)
+    for _ in range(warmup + steps):
+        qlora.qlora_linear_fwd(X, q, A, B, alpha / r, save_T=False)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -356,6 +372,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-decode", action="store_true",
+                    help="only run the M=1 forward of an 8192x28672 weight --steps times "
+                         "(no graph): a small, self-contained case for profiler captures")
     ap.add_argument("--profile-linear", action="store_true",
                     help="only run forward + backward of the gate linear (11008x4096, M=4096) "
                          "--steps times: a small, self-contained case for profiler captures")
@@ -379,6 +398,9 @@ def main():
     scale = ALPHA / RANK_R
     if args.profile_linear:
         profile_linear(device, scale, args.warmup, args.steps)
+        return
+    if args.profile_decode:
+        profile_decode(device, args.warmup, args.steps)
         return
     L = build_layer(device, seed=3 + 1000 * rank)
     flops = layer_flops(inputs.LLAMA7B_LINEARS, M_TOKENS, RANK_R)

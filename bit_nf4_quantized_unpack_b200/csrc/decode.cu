@@ -26,7 +26,7 @@
 namespace qlora {
 namespace {
 
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 128;
 constexpr int kRowsPerWarp = 32;
 constexpr int kUnitK = 256;  // K covered by one warp step (4 lanes x 64)
 
@@ -39,10 +39,11 @@ struct DecodeArgs {
   const uint16_t* A;
   int64_t M, N, K;
   int r;
-  int splits, units_per, nunits;
-  int row_groups, t_groups;
-  float* part;   // [splits][M][N]
-  float* tpart;  // [splits][M][r]
+  int splits, units_per, nunits;  // K is cut into `splits` ranges of `units_per` 256-units
+  int row_groups;                 // 32-row groups of W
+  int t_groups;                   // 8-column groups of A (for T = X A)
+  float* part;   // [splits][M][N]   partial sums of X W_hat^T
+  float* tpart;  // [splits][M][r]   partial sums of T = X A
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
@@ -83,161 +84,213 @@ __device__ __forceinline__ void load_x64(const uint16_t* X, int64_t K, int64_t r
   }
 }
 
-template <bool kTall>  // kTall: M > 8 (tokens 8..15 live in the upper fragment rows)
-__global__ void __launch_bounds__(kDecThreads, kTall ? 1 : 2) k_decode_gemv(const DecodeArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int task = blockIdx.x * (kDecThreads / 32) + warp;
-  const int ngroups = a.row_groups + a.t_groups;
-  if (task >= ngroups * a.splits) return;
-  const int group = task % ngroups;
-  const int split = task / ngroups;
-  const bool is_t = group >= a.row_groups;
+// Fragment mapping of the weight tasks: mma.m16n8k16 with the dequantized weight as the
+// A operand (16 weight rows) and X as the B operand (8 token columns). Lane (g = lane/4,
+// t = lane%4) owns K columns kb .. kb + 63 (kb = unit * 256 + 64 t) of weight rows g
+// and g + 8 of each 16-row group; MMA number j (0..15) of a unit takes from every lane
+// the four columns kb + 4j .. kb + 4j + 3: A pairs (rows g and g + 8), B pairs (token
+// g). Summation order over K does not matter, so this relabelling of the MMA's k index
+// is free, and the unpacked pairs land directly in the A operand registers.
+constexpr int kGroups = 2;  // 16-row groups per warp (32 weight rows)
+
+__device__ __forceinline__ int64_t lmin(int64_t x, int64_t y) { return x < y ? x : y; }
+
+template <bool kTall>
+__device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, int split,
+                                                   int lane, const float* t8) {
   const int g = lane >> 2, t = lane & 3;
   const int u0 = split * a.units_per;
   const int u1 = min(a.nunits, u0 + a.units_per);
-  const int64_t bpr = a.K / 64;
+  const int64_t K = a.K, N = a.N;
+  const int64_t bpr = K / 64;
   const float mean = *a.mean;
-  const int64_t rbase = static_cast<int64_t>(is_t ? group - a.row_groups : group) * kRowsPerWarp;
-  const int64_t rlimit = is_t ? a.r : a.N;
-
-  float acc[4][4];
+  const int64_t rbase = static_cast<int64_t>(rg) * kRowsPerWarp;
+  // token rows this lane feeds to the B operand; tokens >= M compute columns nobody stores
+  const int64_t xr0 = lmin(g, a.M - 1);
+  const int64_t xr1 = lmin(g + 8, a.M - 1);
+  float acc[kGroups][kTall ? 2 : 1][4];
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int q = 0; q < kGroups; ++q)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
+    for (int h = 0; h < (kTall ? 2 : 1); ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[q][h][i] = 0.f;
 
   for (int u = u0; u < u1; ++u) {
-    const int64_t kb = static_cast<int64_t>(u) * kUnitK + 64 * t;
-    const bool kv = kb < a.K;
-    if (!is_t) {
-      uint32_t xa[32], xb[32];
-      load_x64(a.X, a.K, g, kv && g < a.M, kb, xa);
-      if (kTall) load_x64(a.X, a.K, g + 8, kv && g + 8 < a.M, kb, xb);
-      // issue the code and constant loads of all four row groups before any math
-      uint4 cq[4][2];
-      uint32_t e2[4];
-      float e1[4];
+    const int64_t kraw = static_cast<int64_t>(u) * kUnitK + 64 * t;
+    const bool kv = kraw < K;
+    const int64_t kb = kv ? kraw : K - 64;  // clamped: the scale below is zero then
+    // every load of this unit is issued before any math; rows beyond N are clamped and
+    // get a zero scale
+    uint4 cq[kGroups][2][2];
+    uint32_t e2[kGroups][2];
+    float e1[kGroups][2];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int64_t row = rbase + q * 8 + g;
-        cq[q][0] = cq[q][1] = make_uint4(0, 0, 0, 0);
-        e2[q] = 0u;
-        e1[q] = 0.f;
-        if (kv && row < rlimit) {
-          const uint8_t* p = a.codes + row * (a.K / 2) + kb / 2;
-          cq[q][0] = ldg_stream(p);
-          cq[q][1] = ldg_stream(p + 16);
-          const int64_t j = row * bpr + kb / 64;
-          e2[q] = __ldg(a.c2 + j);
-          e1[q] = __ldg(a.c1 + (j >> 8));
-        }
+    for (int q = 0; q < kGroups; ++q)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = lmin(rbase + q * 16 + g + 8 * h, N - 1);
+        const uint8_t* p = a.codes + row * (K / 2) + kb / 2;
+        cq[q][h][0] = ldg_stream(p);
+        cq[q][h][1] = ldg_stream(p + 16);
+        const int64_t j = row * bpr + kb / 64;
+        e2[q][h] = __ldg(a.c2 + j);
+        e1[q][h] = __ldg(a.c1 + (j >> 8));
+      }
+    uint32_t xa[32], xb[32];
+    load_x64(a.X, K, xr0, true, kb, xa);
+    if (kTall) load_x64(a.X, K, xr1, true, kb, xb);
+#pragma unroll
+    for (int q = 0; q < kGroups; ++q) {
+      Nf4Lut lut[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const bool live = kv && (rbase + q * 16 + g + 8 * h) < N;
+        build_lut(live ? block_scale_tab(t8, e2[q][h], e1[q][h], mean) : 0.f, lut[h]);
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (rbase + q * 8 >= rlimit) continue;  // warp-uniform
-        const int64_t row = rbase + q * 8 + g;
-        const float sc = (kv && row < rlimit) ? block_scale(e2[q], e1[q], mean) : 0.f;
-        Nf4Lut lut;
-        build_lut(sc, lut);
-        const uint32_t words[8] = {cq[q][0].x, cq[q][0].y, cq[q][0].z, cq[q][0].w,
-                                   cq[q][1].x, cq[q][1].y, cq[q][1].z, cq[q][1].w};
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          uint32_t o[4];
-          lut_decode8(words[w], lut, o);
-          mma_bf16_16816(acc[q], xa[4 * w], kTall ? xb[4 * w] : 0u,
-                         xa[4 * w + 1], kTall ? xb[4 * w + 1] : 0u, o[0],
-                         o[1]);
-          mma_bf16_16816(acc[q], xa[4 * w + 2], kTall ? xb[4 * w + 2] : 0u,
-                         xa[4 * w + 3], kTall ? xb[4 * w + 3] : 0u, o[2],
-                         o[3]);
+      for (int w = 0; w < 8; ++w) {
+        uint32_t o0[4], o1[4];
+        lut_decode8(w < 4 ? (&cq[q][0][0].x)[w] : (&cq[q][0][1].x)[w - 4], lut[0], o0);
+        lut_decode8(w < 4 ? (&cq[q][1][0].x)[w] : (&cq[q][1][1].x)[w - 4], lut[1], o1);
+        mma_bf16_16816(acc[q][0], o0[0], o1[0], o0[1], o1[1], xa[4 * w], xa[4 * w + 1]);
+        mma_bf16_16816(acc[q][0], o0[2], o1[2], o0[3], o1[3], xa[4 * w + 2], xa[4 * w + 3]);
+        if (kTall) {
+          mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[0], o1[0], o0[1], o1[1], xb[4 * w],
+                         xb[4 * w + 1]);
+          mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[2], o1[2], o0[3], o1[3], xb[4 * w + 2],
+                         xb[4 * w + 3]);
         }
-      }
-    } else {
-      // A [K, r] column `row` plays the weight: strided bf16 loads, pairs along k
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        if (rbase + q * 8 >= rlimit) continue;  // warp-uniform
-        const int64_t row = rbase + q * 8 + g;
-        const bool live = kv && row < rlimit;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-        for (int j = 0; j < 16; ++j) {
-          uint32_t b[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t lo = 0, hi = 0;
-            if (live) {
-              lo = __ldg(a.A + (kb + 4 * j + 2 * h) * a.r + row);
-              hi = __ldg(a.A + (kb + 4 * j + 2 * h + 1) * a.r + row);
-            }
-            b[h] = lo | (hi << 16);
-          }
-          // the X pairs of this k group, re-read from L1 to keep registers free
-          const uint32_t* xr = reinterpret_cast<const uint32_t*>(a.X + g * a.K + kb + 4 * j);
-          const uint32_t* xr8 = reinterpret_cast<const uint32_t*>(a.X + (g + 8) * a.K + kb + 4 * j);
-          const bool lg = kv && g < a.M, lg8 = kv && g + 8 < a.M;
-          mma_bf16_16816(d, lg ? __ldg(xr) : 0u, lg8 ? __ldg(xr8) : 0u, lg ? __ldg(xr + 1) : 0u,
-                         lg8 ? __ldg(xr8 + 1) : 0u, b[0], b[1]);
-        }
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq)
-          if (qq == q)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[qq][i] += d[i];
       }
     }
   }
-  // C fragment: acc[q][0..1] = (token g, rows 2t, 2t+1), acc[q][2..3] = (token g+8, ...)
+  // C fragment: c0,c1 = (weight row g, tokens 2t, 2t+1), c2,c3 = (row g + 8, same tokens);
+  // the second accumulator (M > 8) holds tokens 8 + 2t, 8 + 2t + 1.
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < kGroups; ++q)
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t m = g + 8 * h;
-      if (m >= a.M) continue;
+    for (int hm = 0; hm < (kTall ? 2 : 1); ++hm)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int64_t row = rbase + q * 8 + 2 * t + e;
-        if (row >= rlimit) continue;
-        if (is_t)
-          a.tpart[(static_cast<int64_t>(split) * a.M + m) * a.r + row] = acc[q][2 * h + e];
-        else
-          a.part[(static_cast<int64_t>(split) * a.M + m) * a.N + row] = acc[q][2 * h + e];
+      for (int i = 0; i < 4; ++i) {
+        const int64_t row = rbase + q * 16 + g + 8 * (i >> 1);
+        const int64_t m = 8 * hm + 2 * t + (i & 1);
+        if (row < N && m < a.M)
+          a.part[(static_cast<int64_t>(split) * a.M + m) * N + row] = acc[q][hm][i];
       }
+}
+
+// T partials over the K range of `split` for A columns tg*8 .. tg*8+7 (A [K, r] plays
+// the weight: its column is gathered with strided bf16 loads).
+template <bool kTall>
+__device__ __forceinline__ void decode_t_task(const DecodeArgs& a, int idx, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int tg = idx % a.t_groups;
+  const int split = idx / a.t_groups;
+  const int u0 = split * a.units_per;
+  const int u1 = min(a.nunits, u0 + a.units_per);
+  const int col = tg * 8 + g;
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int u = u0; u < u1; ++u) {
+    const int64_t kb = static_cast<int64_t>(u) * kUnitK + 64 * t;
+    const bool kv = kb < a.K;
+    const bool live = kv && col < a.r;
+    uint32_t bw[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      uint32_t lo = 0, hi = 0;
+      if (live) {
+        lo = __ldg(a.A + (kb + 2 * i) * a.r + col);
+        hi = __ldg(a.A + (kb + 2 * i + 1) * a.r + col);
+      }
+      bw[i] = lo | (hi << 16);
+    }
+    uint32_t xa[32], xb[32];
+    load_x64(a.X, a.K, g, kv && g < a.M, kb, xa);
+    if (kTall) load_x64(a.X, a.K, g + 8, kv && g + 8 < a.M, kb, xb);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      mma_bf16_16816(d, xa[2 * j], kTall ? xb[2 * j] : 0u, xa[2 * j + 1],
+                     kTall ? xb[2 * j + 1] : 0u, bw[2 * j], bw[2 * j + 1]);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t m = g + 8 * h;
+    if (m >= a.M) continue;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = tg * 8 + 2 * t + e;
+      if (c < a.r) a.tpart[(static_cast<int64_t>(split) * a.M + m) * a.r + c] = d[2 * h + e];
     }
   }
 }
 
+template <bool kTall>  // kTall: M > 8 (tokens 8..15 live in the upper fragment rows)
+__global__ void __launch_bounds__(kDecThreads, kTall ? 2 : 3) k_decode_gemv(const DecodeArgs a) {
+  // the finalize kernel may be scheduled now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float t8[256];  // T8 by E4M3 code
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int task = blockIdx.x * (kDecThreads / 32) + warp;
+  const int wtasks = a.row_groups * a.splits;
+  if (task < wtasks)
+    decode_weight_task<kTall>(a, task % a.row_groups, task / a.row_groups, lane, t8);
+  else if (task < wtasks + a.t_groups * a.splits)
+    decode_t_task<kTall>(a, task - wtasks, lane);
+}
+
+// One CTA per 32 output columns: T = sum of its split partials (lanes over splits,
+// warp shuffles), the Y partials summed by 8 groups of splits then combined through
+// shared memory, plus scale * T B, rounded to bf16.
+constexpr int kFinCols = 32;
 __global__ void __launch_bounds__(256)
     k_decode_finalize(const float* __restrict__ part, const float* __restrict__ tpart,
                       int splits, int64_t M, int64_t N, int r, float scale,
                       const uint16_t* __restrict__ B, uint16_t* __restrict__ Y,
                       float* __restrict__ T_save) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the GEMV's partial sums are complete
   __shared__ float T[16 * 64];
-  for (int i = threadIdx.x; i < M * r; i += blockDim.x) {
+  __shared__ float red[8][16][kFinCols];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mr = static_cast<int>(M) * r;
+  for (int e = warp; e < mr; e += 8) {
     float v = 0.f;
-    for (int s = 0; s < splits; ++s) v += tpart[static_cast<int64_t>(s) * M * r + i];
-    T[i] = v;
-    if (T_save && blockIdx.x == 0) T_save[i] = v;
+    for (int s = lane; s < splits; s += 32) v += tpart[static_cast<int64_t>(s) * mr + e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if (lane == 0) {
+      T[e] = v;
+      if (T_save && blockIdx.x == 0) T_save[e] = v;
+    }
   }
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kFinCols;
+  const int64_t n = n0 + lane;
+  float acc[16];
+#pragma unroll
+  for (int m = 0; m < 16; ++m) acc[m] = 0.f;
+  if (n < N) {
+    for (int s = warp; s < splits; s += 8) {
+#pragma unroll
+      for (int m = 0; m < 16; ++m)
+        if (m < M) acc[m] += part[(static_cast<int64_t>(s) * M + m) * N + n];
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 16; ++m)
+    if (m < M) red[warp][m][lane] = acc[m];
   __syncthreads();
-  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  float lora[16];
-#pragma unroll
-  for (int m = 0; m < 16; ++m) lora[m] = 0.f;
-  for (int j = 0; j < r; ++j) {
-    const float bj = __uint_as_float(static_cast<uint32_t>(__ldg(B + j * N + n)) << 16);
-#pragma unroll
-    for (int m = 0; m < 16; ++m)
-      if (m < M) lora[m] += T[m * r + j] * bj;
-  }
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    if (m >= M) break;
+  for (int idx = threadIdx.x; idx < static_cast<int>(M) * kFinCols; idx += blockDim.x) {
+    const int m = idx / kFinCols, c = idx % kFinCols;
+    const int64_t nn = n0 + c;
+    if (nn >= N) continue;
     float y = 0.f;
-    for (int s = 0; s < splits; ++s) y += part[(static_cast<int64_t>(s) * M + m) * N + n];
-    Y[m * N + n] = bf16_bits_rn(y + scale * lora[m]);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) y += red[w][m][c];
+    float lora = 0.f;
+    for (int j = 0; j < r; ++j)
+      lora += T[m * r + j] * __uint_as_float(static_cast<uint32_t>(__ldg(B + j * N + nn)) << 16);
+    Y[m * N + nn] = bf16_bits_rn(y + scale * lora);
   }
 }
 
@@ -249,29 +302,27 @@ DecodePlan plan_decode(const LinearShape& s) {
   DecodePlan p;
   p.nunits = static_cast<int>((s.K + kUnitK - 1) / kUnitK);
   p.row_groups = static_cast<int>((s.N + kRowsPerWarp - 1) / kRowsPerWarp);
-  p.t_groups = (s.r + kRowsPerWarp - 1) / kRowsPerWarp;
-  const int64_t target_warps = static_cast<int64_t>(num_sms()) * 16;
-  int64_t want = (target_warps + p.row_groups - 1) / p.row_groups;
-  // keep the fp32 partials small next to the weight bytes
-  want = std::min<int64_t>(want, std::max<int64_t>(1, s.K / (64 * std::max<int64_t>(1, s.M))));
-  want = std::max<int64_t>(1, std::min<int64_t>(want, p.nunits));
+  p.t_groups = (s.r + 7) / 8;
+  // As many K splits as keep the fp32 partial sums (splits * M * N * 4 bytes) to a few
+  // percent of the weight bytes (N * K / 2): splits <= K / (128 M).
+  int64_t want = std::max<int64_t>(1, s.K / (128 * std::max<int64_t>(1, s.M)));
+  want = std::min<int64_t>(want, p.nunits);
   p.units_per = static_cast<int>((p.nunits + want - 1) / want);
   p.splits = (p.nunits + p.units_per - 1) / p.units_per;
   return p;
 }
 
-}  // namespace
-
-size_t decode_workspace(const LinearShape& s) {
-  const DecodePlan p = plan_decode(s);
-  return align_up(static_cast<size_t>(p.splits) * s.M * s.N * 4, 256) +
-         align_up(static_cast<size_t>(p.splits) * s.M * s.r * 4, 256) + 256;
+size_t part_bytes(const DecodePlan& p, const LinearShape& s) {
+  return align_up(static_cast<size_t>(p.splits) * s.M * s.N * 4, 256);
+}
+size_t tpart_bytes(const DecodePlan& p, const LinearShape& s) {
+  return align_up(static_cast<size_t>(p.splits) * s.M * s.r * 4, 256);
 }
 
-qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
-                            const uint16_t* B, const LinearShape& s, uint16_t* Y,
-                            float* T_save, void* ws, cudaStream_t st) {
-  const DecodePlan p = plan_decode(s);
+// The GEMV grid, then the finalize kernel with programmatic dependent launch.
+qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
+                           const uint16_t* B, const LinearShape& s, const DecodePlan& p,
+                           uint16_t* Y, float* T_save, char* scratch, cudaStream_t st) {
   DecodeArgs a;
   a.codes = w.codes;
   a.c2 = w.c2;
@@ -288,23 +339,44 @@ qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const 
   a.nunits = p.nunits;
   a.row_groups = p.row_groups;
   a.t_groups = p.t_groups;
-  char* base = static_cast<char*>(ws);
-  a.part = reinterpret_cast<float*>(base);
-  a.tpart = reinterpret_cast<float*>(
-      base + align_up(static_cast<size_t>(p.splits) * s.M * s.N * 4, 256));
+  a.part = reinterpret_cast<float*>(scratch);
+  a.tpart = reinterpret_cast<float*>(scratch + part_bytes(p, s));
   const int64_t warps = static_cast<int64_t>(p.row_groups + p.t_groups) * p.splits;
-  const unsigned ctas = static_cast<unsigned>((warps + 7) / 8);
+  const unsigned ctas = static_cast<unsigned>((warps + kDecThreads / 32 - 1) / (kDecThreads / 32));
   if (s.M > 8)
     k_decode_gemv<true><<<ctas, kDecThreads, 0, st>>>(a);
   else
     k_decode_gemv<false><<<ctas, kDecThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e);
-  k_decode_finalize<<<static_cast<unsigned>((s.N + 255) / 256), 256, 0, st>>>(
-      a.part, a.tpart, p.splits, s.M, s.N, s.r, s.scale, B, Y, T_save);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((s.N + kFinCols - 1) / kFinCols));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_decode_finalize, static_cast<const float*>(a.part),
+                         static_cast<const float*>(a.tpart), p.splits, s.M, s.N, s.r, s.scale, B,
+                         Y, T_save);
   if (e != cudaSuccess) return cuda_status(e);
   return QLORA_OK;
+}
+
+}  // namespace
+
+size_t decode_workspace(const LinearShape& s) {
+  const DecodePlan p = plan_decode(s);
+  return part_bytes(p, s) + tpart_bytes(p, s) + 256;
+}
+
+qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
+                            const uint16_t* B, const LinearShape& s, uint16_t* Y,
+                            float* T_save, void* ws, cudaStream_t st) {
+  return launch_decode(X, w, A, B, s, plan_decode(s), Y, T_save, static_cast<char*>(ws), st);
 }
 
 }  // namespace qlora
@@ -382,15 +454,16 @@ extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_
 
   const LinearShape s{M, w.n_out, w.k_in, r, scale};
   DecodePlan p = plan_decode(s);
-  // Fewer K splits when the planned partial sums would not fit the static array.
-  const size_t per_split = static_cast<size_t>(M) * (s.N + s.r) * 4;
-  const size_t fit = (kStaticScratchBytes - 512) / per_split;
+  // Fewer K splits when the planned partial sums do not fit the static array.
+  const size_t per_split = static_cast<size_t>(M) * s.N * 4;
+  const size_t fixed = tpart_bytes(p, s) + 512;
+  const size_t fit = fixed < kStaticScratchBytes ? (kStaticScratchBytes - fixed) / per_split : 0;
   if (fit < 1) {
     char msg[200];
     std::snprintf(msg, sizeof(msg),
-                  "qlora_linear_fwd_decode_static: M * (N + r) * 4 = %zu bytes exceeds the "
-                  "%zu-byte static scratch",
-                  per_split, kStaticScratchBytes);
+                  "qlora_linear_fwd_decode_static: needs more than %zu bytes of partial sums; "
+                  "the static scratch holds %zu bytes",
+                  per_split + fixed, kStaticScratchBytes);
     set_last_error(msg);
     return QLORA_ERR_WORKSPACE;
   }
@@ -401,42 +474,9 @@ extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_
   void* scratch = nullptr;
   qlora_status q = scratch_address(&scratch);
   if (q != QLORA_OK) return q;
-
-  DecodeArgs a;
-  a.codes = w.codes;
-  a.c2 = w.c2;
-  a.c1 = w.c1;
-  a.mean = w.mean;
-  a.X = X;
-  a.A = A;
-  a.M = s.M;
-  a.N = s.N;
-  a.K = s.K;
-  a.r = s.r;
-  a.splits = p.splits;
-  a.units_per = p.units_per;
-  a.nunits = p.nunits;
-  a.row_groups = p.row_groups;
-  a.t_groups = p.t_groups;
-  // Every partial sum below is written by the GEMV before the finalize kernel reads
-  // it, so nothing left in the array by an earlier call needs clearing.
-  char* base = static_cast<char*>(scratch);
-  a.part = reinterpret_cast<float*>(base);
-  a.tpart = reinterpret_cast<float*>(
-      base + align_up(static_cast<size_t>(p.splits) * s.M * s.N * 4, 256));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t warps = static_cast<int64_t>(p.row_groups + p.t_groups) * p.splits;
-  const unsigned ctas = static_cast<unsigned>((warps + 7) / 8);
-  if (s.M > 8)
-    k_decode_gemv<true><<<ctas, kDecThreads, 0, st>>>(a);
-  else
-    k_decode_gemv<false><<<ctas, kDecThreads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_status(e);
-  k_decode_finalize<<<static_cast<unsigned>((s.N + 255) / 256), 256, 0, st>>>(
-      a.part, a.tpart, p.splits, s.M, s.N, s.r, s.scale, B, Y, T_save);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_status(e);
-  return QLORA_OK;
+  // Every partial sum the finalize kernel reads is written by the GEMV first, so
+  // nothing left in the array by an earlier call needs clearing.
+  return launch_decode(X, w, A, B, s, p, Y, T_save, static_cast<char*>(scratch),
+                       static_cast<cudaStream_t>(stream));
 }
 

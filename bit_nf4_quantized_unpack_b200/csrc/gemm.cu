@@ -35,22 +35,39 @@ namespace {
 // ================================================================== fused NF4 GEMM
 enum class Mode { kForward, kDgrad };
 
-constexpr int kFusedThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 dequant + epilogue
-constexpr int kStages = 4;
-constexpr int kTileRows = 128;  // D rows on the weight side (n forward, k dgrad) = TMEM lanes
-constexpr int kTileCols = 256;  // D columns on the token side (m) = TMEM columns
-constexpr int kBK = 64;         // contraction per pipeline step
+// Warp roles of the persistent fused kernel:
+//   warp 0      TMA producer of the token-side operand (and the LoRA operands)
+//   warp 1      MMA issuer (one thread), owner of the TMEM allocation
+//   warp 2      TMA producer of the packed codes (its own, deeper ring)
+//   warp 3      idle
+//   warps 4-7   epilogue: TMEM -> registers -> bf16 -> global, one TMEM lane quarter each
+//   warps 8-..  dequantization, kDeqGroups warpgroups taking code steps in turn
+constexpr int kDeqGroups = 3;
+constexpr int kFusedThreads = 256 + 128 * kDeqGroups;
+constexpr int kEpiWarp0 = 4;
+constexpr int kDeqWarp0 = 8;
+constexpr int kStages = 4;       // token-side operand (32 KB each)
+constexpr int kWStages = 4;      // weight-side operand: dequantized tile or LoRA operand (16 KB)
+constexpr int kCodeStages = 8;   // packed codes (4 KB each)
+constexpr int kCodePrefetch = 16;  // code steps fetched into L2 ahead of their TMA load
+constexpr int kActPrefetch = 4;    // token-side steps fetched into L2 ahead
+constexpr int kTileRows = 128;   // D rows on the weight side (n forward, k dgrad) = TMEM lanes
+constexpr int kTileCols = 256;   // D columns on the token side (m) = TMEM columns per buffer
+constexpr int kBK = 64;          // contraction per pipeline step
 constexpr uint32_t kActBytes = kTileCols * kBK * 2;   // 32 KB
 constexpr uint32_t kWBytes = kTileRows * kBK * 2;     // 16 KB
 constexpr uint32_t kCodeBytes = kTileRows * kBK / 2;  // 4 KB
-constexpr uint32_t kFusedSmem = kStages * (kActBytes + kWBytes + kCodeBytes) + 1024 + 256;
+constexpr uint32_t kFusedSmem =
+    kStages * kActBytes + kWStages * kWBytes + kCodeStages * kCodeBytes + 1024 + 512 + 1024;
 
 struct FusedArgs {
   const uint8_t* c2;
   const float* c1;
   const float* mean;
   int64_t N, K, M;    // W is N x K, M tokens
-  int ext_mmas;       // 16-wide MMAs of the LoRA step (0: no LoRA step)
+  int ext_mmas;       // 16-wide MMAs per LoRA step (0: no LoRA steps)
+  int row_tiles;      // tiles along the D rows (weight side)
+  int num_tiles;      // row_tiles x token tiles
   uint16_t* out;      // [M, out_ld] bf16
   int64_t out_ld;     // N (forward) or K (dgrad)
   int64_t out_rows;   // valid D rows: N (forward) or K (dgrad)
@@ -69,6 +86,11 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
     if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
 }
 
+__device__ __forceinline__ void mbar_arrive_count(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
 template <Mode MODE>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     k_fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_codes,
@@ -78,167 +100,334 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* act_s = smem;                           // [kStages][kActBytes]  token-side operand
-  uint8_t* w_s = act_s + kStages * kActBytes;      // [kStages][kWBytes]    weight-side operand
-  uint8_t* code_s = w_s + kStages * kWBytes;       // [kStages][kCodeBytes] packed codes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(code_s + kStages * kCodeBytes);
-  uint64_t* full = bars;                 // TMA data of the stage landed
-  uint64_t* deq = bars + kStages;        // dequantized weight tile of the stage written
-  uint64_t* empty = bars + 2 * kStages;  // MMAs reading the stage completed
-  uint64_t* acc_full = bars + 3 * kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+  uint8_t* act_s = smem;                           // [kStages][kActBytes]   token-side operand
+  uint8_t* w_s = act_s + kStages * kActBytes;      // [kWStages][kWBytes]    weight-side operand
+  uint8_t* code_s = w_s + kWStages * kWBytes;      // [kCodeStages][kCodeBytes] packed codes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(code_s + kCodeStages * kCodeBytes);
+  uint64_t* act_full = bars;                      // [kStages] token-side tile landed
+  uint64_t* stage_empty = act_full + kStages;     // [kStages] MMAs reading the act slot done
+  uint64_t* deq_full = stage_empty + kStages;     // [kWStages] weight-side tile ready
+  uint64_t* w_empty = deq_full + kWStages;        // [kWStages] MMAs reading the W slot done
+  uint64_t* code_full = w_empty + kWStages;       // [kCodeStages] codes landed
+  uint64_t* code_empty = code_full + kCodeStages; // [kCodeStages] codes read by dequant
+  uint64_t* acc_full = code_empty + kCodeStages;  // [2] accumulator buffer complete
+  uint64_t* acc_empty = acc_full + 2;             // [2] accumulator buffer read out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* t8 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);  // [256]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileRows;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kTileCols;
+  if (threadIdx.x < 256) t8[threadIdx.x] = t8_value(threadIdx.x);
   const int64_t contraction = (MODE == Mode::kForward) ? args.K : args.N;
   const int ksteps = static_cast<int>((contraction + kBK - 1) / kBK);
   // the LoRA product enters as two steps: bf16 hi part, then bf16 lo part of scale*T
   const int total = ksteps + (args.ext_mmas > 0 ? 2 : 0);
+  const int my_tiles = (static_cast<int>(blockIdx.x) < args.num_tiles)
+                           ? (args.num_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                           : 0;
+  auto tile_coords = [&](int i, int64_t& row0, int64_t& m0) {
+    const int tile = blockIdx.x + i * gridDim.x;
+    row0 = static_cast<int64_t>(tile % args.row_tiles) * kTileRows;
+    m0 = static_cast<int64_t>(tile / args.row_tiles) * kTileCols;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&deq[s], 4);
-      mbar_init(&empty[s], 1);
+      mbar_init(&act_full[s], 1);
+      mbar_init(&stage_empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(&deq_full[s], 4);
+      mbar_init(&w_empty[s], 1);
+    }
+    for (int s = 0; s < kCodeStages; ++s) {
+      mbar_init(&code_full[s], 1);
+      mbar_init(&code_empty[s], 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_codes);
-    tma_prefetch_desc(&tm_act);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTileCols);
+    tmem_alloc(tmem_slot, 2 * kTileCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_d = *tmem_slot;
+  const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA: token-side operand, LoRA steps
     if (lane == 0) {
+      tma_prefetch_desc(&tm_act);
       int issued = 0;
-      for (int step = 0; step < total; ++step) {
-        const int s = step % kStages;
-        const uint32_t use = step / kStages;
-        if (step >= kStages && !mbar_wait(&empty[s], (use - 1) & 1u, abort_flag)) {
-          record_error(args.err, abort_flag, kErrTimeoutProducer);
-          break;
+      // L2 prefetch cursor over the main steps, kActPrefetch steps ahead of the loads
+      int pf_i = 0, pf_t = 0;
+      int64_t pf_row0 = 0, pf_m0 = 0;
+      if (my_tiles > 0) tile_coords(0, pf_row0, pf_m0);
+      auto prefetch_act = [&]() {
+        if (pf_i >= my_tiles) return;
+        tma_prefetch_l2_2d(&tm_act, pf_t * kBK, static_cast<int>(pf_m0));
+        if (++pf_t == ksteps) {
+          pf_t = 0;
+          if (++pf_i < my_tiles) tile_coords(pf_i, pf_row0, pf_m0);
         }
-        if (step < ksteps) {
-          mbar_arrive_expect_tx(&full[s], kActBytes + kCodeBytes);
+      };
+      for (int p = 0; p < kActPrefetch; ++p) prefetch_act();
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+        int64_t row0, m0;
+        tile_coords(i, row0, m0);
+        for (int step = 0; step < total; ++step) {
+          const int g = i * total + step;
+          const int s = g % kStages;
+          if (step < ksteps) prefetch_act();
+          if (g >= kStages && !mbar_wait(&stage_empty[s], ((g / kStages) - 1) & 1u, abort_flag)) {
+            record_error(args.err, abort_flag, kErrTimeoutProducer);
+            break;
+          }
+          if (step < ksteps) {
+            mbar_arrive_expect_tx(&act_full[s], kActBytes);
+            tma_load_2d(act_s + s * kActBytes, &tm_act, &act_full[s], step * kBK,
+                        static_cast<int>(m0));
+          } else {
+            const int ws = g % kWStages;
+            if (g >= kWStages &&
+                !mbar_wait(&w_empty[ws], ((g / kWStages) - 1) & 1u, abort_flag)) {
+              record_error(args.err, abort_flag, kErrTimeoutProducer);
+              break;
+            }
+            mbar_arrive_expect_tx(&act_full[s], kWBytes + kActBytes);
+            if (MODE == Mode::kForward) {
+              // B [r, N] as an MN-major operand: two 64-wide chunks of n, rows j >= r are 0
+              tma_load_2d(w_s + ws * kWBytes, &tm_ext_w, &act_full[s], static_cast<int>(row0), 0);
+              tma_load_2d(w_s + ws * kWBytes + 8192, &tm_ext_w, &act_full[s],
+                          static_cast<int>(row0) + 64, 0);
+            } else {
+              // A [K, r] as a K-major operand (columns j >= r are 0)
+              tma_load_2d(w_s + ws * kWBytes, &tm_ext_w, &act_full[s], 0, static_cast<int>(row0));
+            }
+            tma_load_2d(act_s + s * kActBytes, &tm_ext_act, &act_full[s], (step - ksteps) * 64,
+                        static_cast<int>(m0));
+            mbar_arrive_count(&deq_full[ws], 4);  // no dequantization in a LoRA step
+          }
+          ++issued;
+        }
+      }
+      if (*abort_flag)  // let copies already in flight land before the CTA exits
+        for (int g = (issued > kStages ? issued - kStages : 0); g < issued; ++g)
+          mbar_wait_drain(&act_full[g % kStages], (g / kStages) & 1u);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ TMA: packed codes
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_codes);
+      int issued = 0;
+      // L2 prefetch cursor, kCodePrefetch code steps ahead of the loads
+      int pf_i = 0, pf_t = 0;
+      int64_t pf_row0 = 0, pf_m0 = 0;
+      if (my_tiles > 0) tile_coords(0, pf_row0, pf_m0);
+      auto prefetch_codes = [&]() {
+        if (pf_i >= my_tiles) return;
+        if (MODE == Mode::kForward)
+          tma_prefetch_l2_2d(&tm_codes, pf_t * (kBK / 2), static_cast<int>(pf_row0));
+        else
+          tma_prefetch_l2_2d(&tm_codes, static_cast<int>(pf_row0 / 2), pf_t * kBK);
+        if (++pf_t == ksteps) {
+          pf_t = 0;
+          if (++pf_i < my_tiles) tile_coords(pf_i, pf_row0, pf_m0);
+        }
+      };
+      for (int p = 0; p < kCodePrefetch; ++p) prefetch_codes();
+      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+        int64_t row0, m0;
+        tile_coords(i, row0, m0);
+        for (int step = 0; step < ksteps; ++step) {
+          const int c = i * ksteps + step;
+          const int s = c % kCodeStages;
+          prefetch_codes();
+          if (c >= kCodeStages &&
+              !mbar_wait(&code_empty[s], ((c / kCodeStages) - 1) & 1u, abort_flag)) {
+            record_error(args.err, abort_flag, kErrTimeoutProducer);
+            break;
+          }
+          mbar_arrive_expect_tx(&code_full[s], kCodeBytes);
           if (MODE == Mode::kForward)
-            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &full[s], step * (kBK / 2),
+            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &code_full[s], step * (kBK / 2),
                         static_cast<int>(row0));
           else
-            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &full[s],
+            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &code_full[s],
                         static_cast<int>(row0 / 2), step * kBK);
-          tma_load_2d(act_s + s * kActBytes, &tm_act, &full[s], step * kBK,
-                      static_cast<int>(m0));
-        } else {
-          mbar_arrive_expect_tx(&full[s], kWBytes + kActBytes);
-          if (MODE == Mode::kForward) {
-            // B [r, N] as an MN-major operand: two 64-wide chunks of n, rows j >= r are 0
-            tma_load_2d(w_s + s * kWBytes, &tm_ext_w, &full[s], static_cast<int>(row0), 0);
-            tma_load_2d(w_s + s * kWBytes + 8192, &tm_ext_w, &full[s],
-                        static_cast<int>(row0) + 64, 0);
-          } else {
-            // A [K, r] as a K-major operand (columns j >= r are 0)
-            tma_load_2d(w_s + s * kWBytes, &tm_ext_w, &full[s], 0, static_cast<int>(row0));
-          }
-          tma_load_2d(act_s + s * kActBytes, &tm_ext_act, &full[s], (step - ksteps) * 64,
-                      static_cast<int>(m0));
+          ++issued;
         }
-        ++issued;
       }
-      if (*abort_flag) {  // let copies already in flight land before the CTA exits
-        for (int step = std::max(0, issued - kStages); step < issued; ++step)
-          mbar_wait_drain(&full[step % kStages], (step / kStages) & 1u);
-      }
+      if (*abort_flag)
+        for (int c = (issued > kCodeStages ? issued - kCodeStages : 0); c < issued; ++c)
+          mbar_wait_drain(&code_full[c % kCodeStages], (c / kCodeStages) & 1u);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_main =
           idesc_bf16_f32(kTileRows, kTileCols, MODE == Mode::kDgrad, false);
       constexpr uint32_t idesc_ext =
           idesc_bf16_f32(kTileRows, kTileCols, MODE == Mode::kForward, false);
       bool ok = true;
-      for (int step = 0; step < total && ok; ++step) {
-        const int s = step % kStages;
-        const uint32_t par = (step / kStages) & 1u;
-        if (!mbar_wait(&full[s], par, abort_flag) ||
-            (step < ksteps && !mbar_wait(&deq[s], par, abort_flag))) {
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int buf = i & 1;
+        const uint32_t tmem_d = tmem_base + buf * kTileCols;
+        if (i >= 2 && !mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1u, abort_flag)) {
           record_error(args.err, abort_flag, kErrTimeoutMma);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(w_s + s * kWBytes);
-        const uint32_t b0 = smem_u32(act_s + s * kActBytes);
-        if (step < ksteps) {
+        for (int step = 0; step < total; ++step) {
+          const int g = i * total + step;
+          const int s = g % kStages;
+          const int ws = g % kWStages;
+          if (!mbar_wait(&act_full[s], (g / kStages) & 1u, abort_flag) ||
+              !mbar_wait(&deq_full[ws], (g / kWStages) & 1u, abort_flag)) {
+            record_error(args.err, abort_flag, kErrTimeoutMma);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(w_s + ws * kWBytes);
+          const uint32_t b0 = smem_u32(act_s + s * kActBytes);
+          if (step < ksteps) {
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = (MODE == Mode::kForward)
-                                    ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
-                                    : smem_desc_sw128(a0 + kk * 4096, 1024, 2048);
-            const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-            umma_bf16(tmem_d, ad, bd, idesc_main, (step | kk) != 0);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = (MODE == Mode::kForward)
+                                      ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
+                                      : smem_desc_sw128(a0 + kk * 4096, 1024, 2048);
+              const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+              umma_bf16(tmem_d, ad, bd, idesc_main, (step | kk) != 0);
+            }
+          } else {
+            for (int kk = 0; kk < args.ext_mmas; ++kk) {
+              const uint64_t ad = (MODE == Mode::kForward)
+                                      ? smem_desc_sw128(a0 + kk * 2048, 8192, 1024)
+                                      : smem_desc_sw128(a0 + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+              umma_bf16(tmem_d, ad, bd, idesc_ext, 1u);
+            }
           }
-        } else {
-          for (int kk = 0; kk < args.ext_mmas; ++kk) {
-            const uint64_t ad = (MODE == Mode::kForward)
-                                    ? smem_desc_sw128(a0 + kk * 2048, 8192, 1024)
-                                    : smem_desc_sw128(a0 + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-            umma_bf16(tmem_d, ad, bd, idesc_ext, 1u);
-          }
+          umma_commit(&stage_empty[s]);
+          umma_commit(&w_empty[ws]);
         }
-        umma_commit(&empty[s]);
+        if (ok) umma_commit(&acc_full[buf]);
       }
-      umma_commit(acc_full);
-      if (!ok) mbar_wait_drain(acc_full, 0);  // MMAs in flight finish before TMEM is freed
+      if (!ok) {  // MMAs in flight finish before TMEM is freed
+        umma_commit(&acc_full[0]);
+        mbar_wait_drain(&acc_full[0], 0);
+      }
+      // The commits of the last steps arrive asynchronously on barriers nobody else
+      // waits for any more: let them land before the CTA (and its shared memory) goes.
+      const int steps_done = my_tiles * total;
+      for (int s = 0; s < kStages; ++s) {
+        const int last = steps_done - 1 - ((steps_done - 1 - s) % kStages + kStages) % kStages;
+        if (last >= 0 && last < steps_done) mbar_wait_drain(&stage_empty[s], (last / kStages) & 1u);
+      }
+      for (int s = 0; s < kWStages; ++s) {
+        const int last = steps_done - 1 - ((steps_done - 1 - s) % kWStages + kWStages) % kWStages;
+        if (last >= 0 && last < steps_done) mbar_wait_drain(&w_empty[s], (last / kWStages) & 1u);
+      }
     }
-  } else {
-    // ------------------------------------------------------------ dequant warps
-    const int dw = warp - 2;
-    const int wg = dw >> 2;                  // warpgroup: even / odd pipeline steps
+  } else if (warp >= kDeqWarp0) {
+    // ------------------------------------------------ dequantization
+    const int dw = warp - kDeqWarp0;
+    const int wg = dw >> 2;                  // warpgroup: code steps wg, wg + kDeqGroups, ...
     const int local = (dw & 3) * 32 + lane;  // 0..127
     const float mean = *args.mean;
     const int64_t bpr = args.K / 64;  // 64-blocks per weight row
-    for (int step = wg; step < ksteps; step += 2) {
-      const int s = step % kStages;
-      const uint32_t par = (step / kStages) & 1u;
-      int64_t n, kb;
+    const int ncodes = my_tiles * ksteps;
+    // Code step c = tile i * ksteps + step t; this warpgroup walks c = wg, wg + kDeqGroups, ...
+    // (i, t) and the tile origin are advanced incrementally (no divisions per step).
+    struct Cursor {
+      int i, t;
+      int64_t row0, m0;
+    };
+    auto advance = [&](Cursor& k, int by) {
+      k.t += by;
+      while (k.t >= ksteps) {
+        k.t -= ksteps;
+        ++k.i;
+      }
+    };
+    auto set_tile = [&](Cursor& k) { tile_coords(k.i, k.row0, k.m0); };
+    // (row n, 64-block kb) of this thread at a cursor; false outside W
+    auto block_of = [&](const Cursor& k, int64_t& n, int64_t& kb) {
       if (MODE == Mode::kForward) {
-        n = row0 + local;
-        kb = step;
+        n = k.row0 + local;
+        kb = k.t;
       } else {
-        n = static_cast<int64_t>(step) * kBK + (local >> 1);
-        kb = row0 / 64 + (local & 1);
+        n = static_cast<int64_t>(k.t) * kBK + (local >> 1);
+        kb = k.row0 / 64 + (local & 1);
       }
-      float sc = 0.f;  // rows / blocks outside W dequantize to zeros
-      if (n < args.N && kb < bpr) {
+      return n < args.N && kb < bpr;
+    };
+    Cursor cur{0, 0, 0, 0};
+    advance(cur, wg);
+    set_tile(cur);
+    Cursor nxt = cur;  // the next step of this warpgroup, for the prefetch
+    advance(nxt, kDeqGroups);
+    if (nxt.i < my_tiles) set_tile(nxt);
+    // the block constants of this warpgroup's next step are loaded one step ahead
+    uint32_t e2_next = 0u;
+    float e1_next = 0.f;
+    {
+      int64_t n, kb;
+      if (wg < ncodes && block_of(cur, n, kb)) {
         const int64_t j = n * bpr + kb;
-        sc = block_scale(__ldg(args.c2 + j), __ldg(args.c1 + (j >> 8)), mean);
+        e2_next = __ldg(args.c2 + j);
+        e1_next = __ldg(args.c1 + (j >> 8));
       }
-      if (!mbar_wait(&full[s], par, abort_flag)) {
+    }
+    for (int c = wg; c < ncodes; c += kDeqGroups) {
+      int64_t n, kb;
+      const bool valid = block_of(cur, n, kb);
+      const uint32_t e2 = e2_next;
+      const float e1 = e1_next;
+      if (c + kDeqGroups < ncodes) {
+        int64_t n2, kb2;
+        if (block_of(nxt, n2, kb2)) {
+          const int64_t j = n2 * bpr + kb2;
+          e2_next = __ldg(args.c2 + j);
+          e1_next = __ldg(args.c1 + (j >> 8));
+        }
+      }
+      const float sc = valid ? block_scale_tab(t8, e2, e1, mean) : 0.f;  // zeros outside W
+      Nf4Lut lut;
+      build_lut(sc, lut);
+      // stage of the pipeline this code step feeds
+      const int g = cur.i * total + cur.t;
+      const int ws = g % kWStages;
+      const int cs = c % kCodeStages;
+      // move both cursors two steps on
+      cur = nxt;
+      advance(nxt, kDeqGroups);
+      if (nxt.i != cur.i && nxt.i < my_tiles) set_tile(nxt);
+      if (!mbar_wait(&code_full[cs], (c / kCodeStages) & 1u, abort_flag)) {
         record_error(args.err, abort_flag, kErrTimeoutDequant);
         break;
       }
       const uint8_t* src = (MODE == Mode::kForward)
-                               ? code_s + s * kCodeBytes + local * 32
-                               : code_s + s * kCodeBytes + (local >> 1) * 64 + (local & 1) * 32;
+                               ? code_s + cs * kCodeBytes + local * 32
+                               : code_s + cs * kCodeBytes + (local >> 1) * 64 + (local & 1) * 32;
       const uint4 q0 = *reinterpret_cast<const uint4*>(src);
       const uint4 q1 = *reinterpret_cast<const uint4*>(src + 16);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&code_empty[cs]);  // codes are in registers now
+      if (g >= kWStages && !mbar_wait(&w_empty[ws], ((g / kWStages) - 1) & 1u, abort_flag)) {
+        record_error(args.err, abort_flag, kErrTimeoutDequant);
+        break;
+      }
       const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      Nf4Lut lut;
-      build_lut(sc, lut);
-      uint8_t* dst = w_s + s * kWBytes;
+      uint8_t* dst = w_s + ws * kWBytes;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t o[4];
@@ -255,37 +444,45 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&deq[s]);
+      if (lane == 0) mbar_arrive(&deq_full[ws]);
     }
-    // ------------------------------------------------------------ epilogue
-    if (mbar_wait(acc_full, 0, abort_flag) && !*abort_flag) {
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    for (int i = 0; i < my_tiles; ++i) {
+      const int buf = i & 1;
+      if (!mbar_wait(&acc_full[buf], (i >> 1) & 1u, abort_flag)) {
+        if (!*abort_flag) record_error(args.err, abort_flag, kErrTimeoutEpilogue);
+        break;
+      }
       tc_fence_after();
-      const int quarter = warp & 3;  // TMEM lanes this warp may read
+      int64_t row0, m0;
+      tile_coords(i, row0, m0);
       const int64_t orow = row0 + quarter * 32 + lane;
-      const int colbase = wg * (kTileCols / 2);
+      const uint32_t taddr = tmem_base + buf * kTileCols + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < kTileCols / 2 / 32; ++c) {
+      for (int c = 0; c < kTileCols / 32; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(quarter * 32) << 16) + colbase + c * 32,
-                           v);
+        tmem_ld_32x32b_x32(taddr + c * 32, v);
         tmem_ld_wait();
         if (orow < args.out_rows) {
-          const int64_t mb = m0 + colbase + c * 32;
+          const int64_t mb = m0 + c * 32;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (mb + i < args.M)
-              args.out[(mb + i) * args.out_ld + orow] = bf16_bits_rn(__uint_as_float(v[i]));
+          for (int k = 0; k < 32; ++k)
+            if (mb + k < args.M)
+              args.out[(mb + k) * args.out_ld + orow] = bf16_bits_rn(__uint_as_float(v[k]));
         }
       }
-    } else if (!*abort_flag) {
-      record_error(args.err, abort_flag, kErrTimeoutEpilogue);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_d, kTileCols);
+    tmem_dealloc(tmem_base, 2 * kTileCols);
   }
 }
 
@@ -406,6 +603,12 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
       }
       umma_commit(acc_full);
       if (!ok) mbar_wait_drain(acc_full, 0);
+      // let the last commits arrive before the CTA's shared memory is released
+      for (int s = 0; s < kLoraStages; ++s) {
+        const int last = nsteps - 1 - ((nsteps - 1 - s) % kLoraStages + kLoraStages) % kLoraStages;
+        if (ok && last >= 0 && last < nsteps) mbar_wait_drain(&empty[s], (last / kLoraStages) & 1u);
+      }
+      mbar_wait_drain(acc_full, 0);
     }
   } else {
     const bool have = nsteps > 0;
@@ -483,26 +686,34 @@ __global__ void k_hilo_from_plain(const float* __restrict__ t, int64_t M, int r,
 }
 
 // grad[row, j] (or its transpose) = scale * sum_s (P[s][row][j] + P[s][row][64 + j]).
-__global__ void k_finalize_grad(const float* __restrict__ part, int splits, int64_t rows_pad,
-                                int64_t rows, int r, float scale, bool transpose,
-                                float* __restrict__ out) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= rows * r) return;
-  int64_t row;
-  int j;
-  if (transpose) {  // out [r, rows]: consecutive threads walk rows (coalesced store)
-    j = static_cast<int>(i / rows);
-    row = i % rows;
-  } else {          // out [rows, r]
-    row = i / r;
-    j = static_cast<int>(i % r);
+// One block per 32 rows: coalesced reads of the partials, a shared-memory tile, and
+// coalesced writes in either output orientation.
+__global__ void __launch_bounds__(256)
+    k_finalize_grad(const float* __restrict__ part, int splits, int64_t rows_pad, int64_t rows,
+                    int r, float scale, bool transpose, float* __restrict__ out) {
+  __shared__ float tile[32][65];
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32;
+  for (int idx = threadIdx.x; idx < 32 * 64; idx += blockDim.x) {
+    const int rl = idx >> 6, j = idx & 63;
+    float v = 0.f;
+    if (j < r && row0 + rl < rows) {
+      for (int s = 0; s < splits; ++s) {
+        const float* p = part + (s * rows_pad + row0 + rl) * 128;
+        v += p[j] + p[64 + j];
+      }
+    }
+    tile[rl][j] = scale * v;
   }
-  float v = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* p = part + (s * rows_pad + row) * 128;
-    v += p[j] + p[64 + j];
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 32 * r; idx += blockDim.x) {
+    if (transpose) {  // out [r, rows]
+      const int j = idx >> 5, rl = idx & 31;
+      if (row0 + rl < rows) out[static_cast<int64_t>(j) * rows + row0 + rl] = tile[rl][j];
+    } else {          // out [rows, r]
+      const int rl = idx / r, j = idx % r;
+      if (row0 + rl < rows) out[(row0 + rl) * r + j] = tile[rl][j];
+    }
   }
-  out[transpose ? (static_cast<int64_t>(j) * rows + row) : (row * r + j)] = scale * v;
 }
 
 // ================================================================== host side
@@ -561,14 +772,15 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
 
 template <Mode MODE>
 cudaError_t run_fused(const CUtensorMap& tc, const CUtensorMap& ta, const CUtensorMap& tw,
-                      const CUtensorMap& tx, const FusedArgs& args, cudaStream_t st) {
+                      const CUtensorMap& tx, FusedArgs args, cudaStream_t st) {
   auto kern = k_fused_nf4_gemm<MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
   if (e != cudaSuccess) return e;
   const int64_t rows = (MODE == Mode::kForward) ? args.N : args.K;
-  dim3 grid(static_cast<unsigned>((rows + kTileRows - 1) / kTileRows),
-            static_cast<unsigned>((args.M + kTileCols - 1) / kTileCols));
+  args.row_tiles = static_cast<int>((rows + kTileRows - 1) / kTileRows);
+  args.num_tiles = args.row_tiles * static_cast<int>((args.M + kTileCols - 1) / kTileCols);
+  const int grid = std::min(args.num_tiles, num_sms());  // persistent: one CTA per SM
   cudaEvent_t before, after;
   profile_events(&before, &after);
   if (before) {
@@ -746,7 +958,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 64, kSW128);    // X as MN-major (k inner)
     QL_MAP(&tb, kBF16, ghl, 128, s.M, 256, 64, 64, kSW128);      // G hi/lo MN-major
     QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits)));
-    k_finalize_grad<<<blocks_for(s.K * s.r, 256), 256, 0, st>>>(
+    k_finalize_grad<<<blocks_for(s.K, 32), 256, 0, st>>>(
         part, splits, plan_split(s.K, s.M).rows_pad, s.K, s.r, s.scale, false, dA);
     QL_TRY(cudaGetLastError());
   }
@@ -756,7 +968,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);   // dY as MN-major (n inner)
     QL_MAP(&tb, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);      // T hi/lo MN-major
     QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.N, s.M, part, st, &splits)));
-    k_finalize_grad<<<blocks_for(s.N * s.r, 256), 256, 0, st>>>(
+    k_finalize_grad<<<blocks_for(s.N, 32), 256, 0, st>>>(
         part, splits, plan_split(s.N, s.M).rows_pad, s.N, s.r, s.scale, true, dB);
     QL_TRY(cudaGetLastError());
   }

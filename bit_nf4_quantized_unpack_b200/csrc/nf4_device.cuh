@@ -29,10 +29,20 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
   return (b & 0x80u) ? -v : v;
 }
 
+// T8 entry of an E4M3 code: fl32(e4m3 / 448) (IEEE division).
+__device__ __forceinline__ float t8_value(uint32_t c2) {
+  return __fdiv_rn(e4m3_value(c2), 448.0f);
+}
+
 // Reconstructed absmax of one 64-block from its double-quantized constants.
 __device__ __forceinline__ float block_scale(uint32_t c2, float c1, float mean) {
-  const float t8 = __fdiv_rn(e4m3_value(c2), 448.0f);
-  return __fadd_rn(__fmul_rn(t8, c1), mean);
+  return __fadd_rn(__fmul_rn(t8_value(c2), c1), mean);
+}
+
+// The same with T8 read from a 256-entry table (t8[e] = t8_value(e)).
+__device__ __forceinline__ float block_scale_tab(const float* t8, uint32_t c2, float c1,
+                                                 float mean) {
+  return __fadd_rn(__fmul_rn(t8[c2], c1), mean);
 }
 
 // 16-entry bf16 table {bf16(NF4[i] * s)} split into byte planes for prmt lookups:

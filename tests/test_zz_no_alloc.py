@@ -50,8 +50,8 @@ def test_static_scratch_decode_matches_workspace_path(M, N, K, r):
 
 
 def test_static_scratch_with_fewer_k_splits():
-    """N = 16384 at M = 16: the planned five K splits of partial sums do not fit the
-    4 MiB array, so the entry point uses three; results must not change."""
+    """N = 16384 at M = 16: the planned K splits of fp32 partial sums do not all fit
+    the 4 MiB array, so the entry point uses fewer; results must not change."""
     need_gpu()
     g = torch.Generator(device="cuda")
     g.manual_seed(7)
