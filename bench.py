@@ -38,6 +38,9 @@ M_TOKENS, RANK_R, ALPHA = 4096, 64, 16.0
 INPUT_OF = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out",
             "gate": "mlp_in", "up": "mlp_in", "down": "mlp_act"}
 KERNELS_PER_LINEAR_STEP = 3 + 8   # forward 3 launches, backward 8 launches
+# dram__bytes_read.sum + dram__bytes_write.sum per FLOP of k_fused_nf4_gemm, from one ncu
+# capture of the current kernel (forward + dX of the 11008 x 4096 linear at M = 4096)
+FUSED_DRAM_BYTES_PER_FLOP = (118.8e6 + 145.2e6) / (3.751e11 + 3.715e11)
 
 
 def layer_flops(linears, M, r):
@@ -228,8 +231,23 @@ def layer_step(L, scale, world, events=None, pool=None):
                                workspace=L["ws_b"])
     if events is not None:
         qlora.qlora_profile_events(None, None)
+    allreduce_lora_grads(L["grads"], world)
+
+
+def allreduce_lora_grads(grads, world):
+    """Data-parallel exchange of one step: the LoRA gradients of all linears live in one
+    flat fp32 buffer, summed over the ranks with a single all-reduce."""
     if world > 1:
-        torch.distributed.all_reduce(L["grads"])   # data-parallel LoRA gradient exchange
+        torch.distributed.all_reduce(grads)
+
+
+def max_over_ranks(value, world, device):
+    """The slowest rank's time (every rank takes part)."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 def time_steps(fn, steps, world):
@@ -244,12 +262,7 @@ def time_steps(fn, steps, world):
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms = start.elapsed_time(stop) / steps
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(start.elapsed_time(stop) / steps, world, "cuda")
 
 
 def decode_bandwidth(device, M=1, iters=40):
@@ -300,6 +313,49 @@ def decode_bandwidth(device, M=1, iters=40):
                            "GBps": algo / us / 1e3, "weight_copies": copies}
         del graph, qs, q0
         torch.cuda.empty_cache()
+    return out
+
+
+def codec_bandwidth(device, reps=5):
+    """HBM throughput of quantization (bf16 in) and double dequantization (bf16 out) over
+    the three Llama-7B weight shapes, cycled so that no pass finds its data in L2 (the
+    three matrices hold 107M parameters, 267 MB per pass)."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(1)
+    shapes = [(4096, 4096), (4096, 11008), (11008, 4096)]
+    Ws, Qs, Outs, wss = [], [], [], []
+    for n, k in shapes:
+        W = torch.randn(n, k, generator=g, device=device) * 0.02
+        mask = torch.rand(n, k, generator=g, device=device) < 1e-3   # 0.1 % outliers x10
+        W = torch.where(mask, W * 10, W).to(torch.bfloat16)
+        Ws.append(W)
+        Qs.append(qlora.NF4Weight.empty(n, k, device))
+        Outs.append(torch.empty(n, k, dtype=torch.bfloat16, device=device))
+        wss.append(torch.empty(qlora.qlora_quantize_workspace_size(n, k), dtype=torch.uint8,
+                               device=device))
+    params = sum(n * k for n, k in shapes)
+    per_param = 2.0 + 0.515869140625
+    out = {}
+    for name in ("quantize", "dequant"):
+        def one_pass():
+            for W, q, o, ws in zip(Ws, Qs, Outs, wss):
+                if name == "quantize":
+                    qlora.qlora_quantize_nf4_dq(W, out=q, workspace=ws)
+                else:
+                    qlora.qlora_dequant(q, out=o)
+        one_pass()
+        one_pass()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            one_pass()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / reps
+        out[name] = {"us_per_pass": us, "params": params, "bytes_per_param": per_param,
+                     "GBps": params * per_param / us / 1e3}
     return out
 
 
@@ -434,17 +490,22 @@ def main():
         fused_flops += 2 * M_TOKENS * lin["n"] * lin["k"] + 2 * M_TOKENS * RANK_R * other
     peaks, peaks_src = load_peaks()
     achieved = fused_flops / (fused_ms / 1e3) / 1e12
+    # DRAM bytes per FLOP of the fused kernel from its ncu capture (gate linear, forward and
+    # dX; profiles/k_fused_nf4_gemm_gate_11008x4096_m4096.md), scaled to this step's
+    # average launch
+    traffic = FUSED_DRAM_BYTES_PER_FLOP * fused_flops / len(events)
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     roofline = {"bound": "tensor", "kernel": "k_fused_nf4_gemm (forward + dX)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_source": f"{peaks_src} bf16_tflops_sustained",
-                "fused_share_of_step": fused_ms / args.steps / ms, "traffic": None}
+                "fused_share_of_step": fused_ms / args.steps / ms, "traffic": traffic,
+                "traffic_unit": "bytes per launch (scaled from the ncu capture)"}
 
     e2e_ms, h2d, d2h = e2e_steps(L, scale, world, max(2, args.steps // 2))
     e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    decode = None
+    decode = codec = None
     if not args.no_decode and rank == 0:
         del L
         torch.cuda.empty_cache()
@@ -454,6 +515,11 @@ def main():
             v["frac_of_hbm"] = v["GBps"] / hbm
         decode["hbm_peak_GBps"] = hbm
         decode["hbm_peak_source"] = f"{peaks_src} hbm_gbs"
+        codec = codec_bandwidth(device)
+        for v in codec.values():
+            v["frac_of_hbm"] = v["GBps"] / hbm
+        codec["workload"] = ("bf16 weights 4096x4096, 4096x11008, 11008x4096 ~N(0,0.02), "
+                             "0.1% x10 outliers; NF4 block 64, double-quant block 256")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -473,7 +539,7 @@ def main():
                            "l2": "inputs larger than L2 (weights + activations ~1.3 GB per step)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": KERNELS_PER_LINEAR_STEP * len(inputs.LLAMA7B_LINEARS) * args.steps,
-                "clocks": clk, "decode": decode}
+                "clocks": clk, "decode": decode, "codec": codec}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -12,18 +12,18 @@ namespace {
 constexpr int kQuantThreads = 256;
 constexpr int kMaxQuantCtas = 148 * 8;
 
-// NF4 code of x in [-1, 1]: the number of thresholds <= x, by a 4-level bisection in
-// registers (thresholds are kernel parameters).
-__device__ __forceinline__ uint32_t nf4_code(float x, const Nf4Thresholds& th) {
-  uint32_t c = (x >= th.t[7]) ? 8u : 0u;
-  const float t1 = c ? th.t[11] : th.t[3];
+// NF4 code of x in [-1, 1]: the number of thresholds <= x, by a 4-level bisection over
+// thresholds held in registers.
+__device__ __forceinline__ uint32_t nf4_code(float x, const float (&t)[15]) {
+  uint32_t c = (x >= t[7]) ? 8u : 0u;
+  const float t1 = c ? t[11] : t[3];
   c += (x >= t1) ? 4u : 0u;
-  const float t2 = (c & 8u) ? ((c & 4u) ? th.t[13] : th.t[9]) : ((c & 4u) ? th.t[5] : th.t[1]);
+  const float t2 = (c & 8u) ? ((c & 4u) ? t[13] : t[9]) : ((c & 4u) ? t[5] : t[1]);
   c += (x >= t2) ? 2u : 0u;
-  const float a0 = (c & 4u) ? th.t[4] : th.t[0];
-  const float a1 = (c & 4u) ? th.t[6] : th.t[2];
-  const float b0 = (c & 4u) ? th.t[12] : th.t[8];
-  const float b1 = (c & 4u) ? th.t[14] : th.t[10];
+  const float a0 = (c & 4u) ? t[4] : t[0];
+  const float a1 = (c & 4u) ? t[6] : t[2];
+  const float b0 = (c & 4u) ? t[12] : t[8];
+  const float b1 = (c & 4u) ? t[14] : t[10];
   const float lo = (c & 2u) ? a1 : a0;
   const float hi = (c & 2u) ? b1 : b0;
   const float t3 = (c & 8u) ? hi : lo;
@@ -58,6 +58,14 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int sub = lane & 7;
   const unsigned gmask = 0xFFu << (lane & 24);
   const int64_t per_cta = kQuantThreads / 8;
+  // thresholds through shared memory into registers (kept out of the constant bank,
+  // which the bisection would otherwise index)
+  __shared__ float sth[15];
+  if (threadIdx.x < 15) sth[threadIdx.x] = th.t[threadIdx.x];
+  __syncthreads();
+  float t[15];
+#pragma unroll
+  for (int i = 0; i < 15; ++i) t[i] = sth[i];
   double acc = 0.0;
   for (int64_t b = blockIdx.x * per_cta + threadIdx.x / 8; b < nblocks;
        b += static_cast<int64_t>(gridDim.x) * per_cta) {
@@ -73,7 +81,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float x = (m > 0.f) ? __fdiv_rn(v[i], m) : 0.f;
-      packed |= nf4_code(x, th) << (4 * i);
+      packed |= nf4_code(x, t) << (4 * i);
     }
     reinterpret_cast<uint32_t*>(codes + b * 32)[sub] = packed;
     if (sub == 0) {
@@ -165,13 +173,15 @@ __global__ void __launch_bounds__(256)
               const float* __restrict__ c1, const float* __restrict__ mean_p, int64_t nwords,
               uint4* __restrict__ out) {
   __shared__ float lut[16];
+  __shared__ float t8[256];  // T8 by E4M3 code
   if (threadIdx.x < 16) lut[threadIdx.x] = nf4_level(threadIdx.x);
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) t8[e] = t8_value(e);
   __syncthreads();
   const float mean = *mean_p;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t j = i >> 3;  // 64-block of this word
-    const float s = block_scale(c2[j], c1[j >> 8], mean);
+    const float s = block_scale_tab(t8, c2[j], c1[j >> 8], mean);
     const uint32_t w = __ldg(codes + i);
     uint32_t o[4];
 #pragma unroll

@@ -49,8 +49,6 @@ constexpr int kDeqWarp0 = 8;
 constexpr int kStages = 4;       // token-side operand (32 KB each)
 constexpr int kWStages = 4;      // weight-side operand: dequantized tile or LoRA operand (16 KB)
 constexpr int kCodeStages = 8;   // packed codes (4 KB each)
-constexpr int kCodePrefetch = 16;  // code steps fetched into L2 ahead of their TMA load
-constexpr int kActPrefetch = 4;    // token-side steps fetched into L2 ahead
 constexpr int kTileRows = 128;   // D rows on the weight side (n forward, k dgrad) = TMEM lanes
 constexpr int kTileCols = 256;   // D columns on the token side (m) = TMEM columns per buffer
 constexpr int kBK = 64;          // contraction per pipeline step
@@ -112,7 +110,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   uint64_t* code_empty = code_full + kCodeStages; // [kCodeStages] codes read by dequant
   uint64_t* acc_full = code_empty + kCodeStages;  // [2] accumulator buffer complete
   uint64_t* acc_empty = acc_full + 2;             // [2] accumulator buffer read out
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* mma_drain = acc_empty + 2;            // all MMAs of the CTA completed (exit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* t8 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);  // [256]
 
@@ -148,6 +147,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);
     }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -165,26 +165,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_act);
       int issued = 0;
-      // L2 prefetch cursor over the main steps, kActPrefetch steps ahead of the loads
-      int pf_i = 0, pf_t = 0;
-      int64_t pf_row0 = 0, pf_m0 = 0;
-      if (my_tiles > 0) tile_coords(0, pf_row0, pf_m0);
-      auto prefetch_act = [&]() {
-        if (pf_i >= my_tiles) return;
-        tma_prefetch_l2_2d(&tm_act, pf_t * kBK, static_cast<int>(pf_m0));
-        if (++pf_t == ksteps) {
-          pf_t = 0;
-          if (++pf_i < my_tiles) tile_coords(pf_i, pf_row0, pf_m0);
-        }
-      };
-      for (int p = 0; p < kActPrefetch; ++p) prefetch_act();
       for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
         int64_t row0, m0;
         tile_coords(i, row0, m0);
         for (int step = 0; step < total; ++step) {
           const int g = i * total + step;
           const int s = g % kStages;
-          if (step < ksteps) prefetch_act();
           if (g >= kStages && !mbar_wait(&stage_empty[s], ((g / kStages) - 1) & 1u, abort_flag)) {
             record_error(args.err, abort_flag, kErrTimeoutProducer);
             break;
@@ -226,29 +212,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_codes);
       int issued = 0;
-      // L2 prefetch cursor, kCodePrefetch code steps ahead of the loads
-      int pf_i = 0, pf_t = 0;
-      int64_t pf_row0 = 0, pf_m0 = 0;
-      if (my_tiles > 0) tile_coords(0, pf_row0, pf_m0);
-      auto prefetch_codes = [&]() {
-        if (pf_i >= my_tiles) return;
-        if (MODE == Mode::kForward)
-          tma_prefetch_l2_2d(&tm_codes, pf_t * (kBK / 2), static_cast<int>(pf_row0));
-        else
-          tma_prefetch_l2_2d(&tm_codes, static_cast<int>(pf_row0 / 2), pf_t * kBK);
-        if (++pf_t == ksteps) {
-          pf_t = 0;
-          if (++pf_i < my_tiles) tile_coords(pf_i, pf_row0, pf_m0);
-        }
-      };
-      for (int p = 0; p < kCodePrefetch; ++p) prefetch_codes();
       for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
         int64_t row0, m0;
         tile_coords(i, row0, m0);
         for (int step = 0; step < ksteps; ++step) {
           const int c = i * ksteps + step;
           const int s = c % kCodeStages;
-          prefetch_codes();
           if (c >= kCodeStages &&
               !mbar_wait(&code_empty[s], ((c / kCodeStages) - 1) & 1u, abort_flag)) {
             record_error(args.err, abort_flag, kErrTimeoutProducer);
@@ -321,10 +290,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
         if (ok) umma_commit(&acc_full[buf]);
       }
-      if (!ok) {  // MMAs in flight finish before TMEM is freed
-        umma_commit(&acc_full[0]);
-        mbar_wait_drain(&acc_full[0], 0);
-      }
+      // every MMA this thread issued has completed before TMEM is freed (on the normal
+      // path and after an abort alike); the barrier is used for this one phase only
+      umma_commit(mma_drain);
+      mbar_wait_drain(mma_drain, 0);
       // The commits of the last steps arrive asynchronously on barriers nobody else
       // waits for any more: let them land before the CTA (and its shared memory) goes.
       const int steps_done = my_tiles * total;

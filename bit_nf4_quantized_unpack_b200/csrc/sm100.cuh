@@ -83,13 +83,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* map, uin
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
-// Bring one box of a 2D tensor into L2 ahead of its load (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const void* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
-}
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tcgen05.mma reads operands through it).
 __device__ __forceinline__ void fence_proxy_async_smem() {
