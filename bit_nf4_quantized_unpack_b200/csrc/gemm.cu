@@ -38,25 +38,35 @@ enum class Mode { kForward, kDgrad };
 // Warp roles of the persistent fused kernel:
 //   warp 0      TMA producer of the token-side operand (and the LoRA operands)
 //   warp 1      MMA issuer (one thread), owner of the TMEM allocation
-//   warp 2      TMA producer of the packed codes (its own, deeper ring)
+//   warp 2      TMA producer of the packed codes (its own ring)
 //   warp 3      idle
 //   warps 4-7   epilogue: TMEM -> registers -> bf16 -> global, one TMEM lane quarter each
 //   warps 8-..  dequantization, kDeqGroups warpgroups taking code steps in turn
+// A tile is 128 weight-side rows x 512 tokens held as two 256-column fp32 accumulators
+// (all 512 TMEM columns): every dequantized 128 x 64 weight tile feeds 8 MMAs.
 constexpr int kDeqGroups = 3;
 constexpr int kFusedThreads = 256 + 128 * kDeqGroups;
 constexpr int kEpiWarp0 = 4;
 constexpr int kDeqWarp0 = 8;
-constexpr int kStages = 4;       // token-side operand (32 KB each)
-constexpr int kWStages = 4;      // weight-side operand: dequantized tile or LoRA operand (16 KB)
-constexpr int kCodeStages = 8;   // packed codes (4 KB each)
 constexpr int kTileRows = 128;   // D rows on the weight side (n forward, k dgrad) = TMEM lanes
-constexpr int kTileCols = 256;   // D columns on the token side (m) = TMEM columns per buffer
+constexpr int kHalfCols = 256;   // tokens per MMA / per accumulator
+constexpr int kHalves = 2;       // accumulators per tile
+constexpr int kTileCols = kHalfCols * kHalves;  // tokens per tile
 constexpr int kBK = 64;          // contraction per pipeline step
-constexpr uint32_t kActBytes = kTileCols * kBK * 2;   // 32 KB
+constexpr int kHalfSlots = 4;    // ring of 256-token operand tiles (2 per step)
+// Rings that several dequant warpgroups touch are laid out so that every slot has a
+// single owner that uses it in order: code step c (c-th dequantized step of this CTA)
+// belongs to warpgroup c % kDeqGroups, which owns weight slot c % kDeqGroups and code
+// slots c % (kDeqGroups * kCodesPerGroup). An mbarrier parity wait is only meaningful
+// when the waiter is at most one phase ahead; with these owners it never is.
+constexpr int kCodesPerGroup = 2;
+constexpr int kCodeSlots = kDeqGroups * kCodesPerGroup;
+constexpr uint32_t kHalfBytes = kHalfCols * kBK * 2;  // 32 KB
 constexpr uint32_t kWBytes = kTileRows * kBK * 2;     // 16 KB
 constexpr uint32_t kCodeBytes = kTileRows * kBK / 2;  // 4 KB
-constexpr uint32_t kFusedSmem =
-    kStages * kActBytes + kWStages * kWBytes + kCodeStages * kCodeBytes + 1024 + 512 + 1024;
+constexpr uint32_t kEpiBytes = 4 * 32 * 32 * 2;        // per epilogue warp: 32 tokens x 32 rows
+constexpr uint32_t kFusedSmem = kHalfSlots * kHalfBytes + (kDeqGroups + 1) * kWBytes +
+                                kCodeSlots * kCodeBytes + kEpiBytes + 1024 + 512 + 1024;
 
 struct FusedArgs {
   const uint8_t* c2;
@@ -69,6 +79,7 @@ struct FusedArgs {
   uint16_t* out;      // [M, out_ld] bf16
   int64_t out_ld;     // N (forward) or K (dgrad)
   int64_t out_rows;   // valid D rows: N (forward) or K (dgrad)
+  int vec_store;      // out 16-byte aligned and out_ld % 8 == 0: 8 rows per vector store
   int* err;
 };
 
@@ -77,16 +88,20 @@ __device__ __forceinline__ void record_error(int* err, volatile int* abort, int 
   *abort = 1;
 }
 
-// Wait bounded by time only (used while draining after an abort).
+// Wait bounded by time only (used while draining).
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity))
     if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
 }
 
-__device__ __forceinline__ void mbar_arrive_count(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
+// Phase parity of the last use of slot s in a ring of `slots` after `uses` uses in all
+// (returns false when the slot was never used).
+__device__ __forceinline__ bool last_use(int uses, int slots, int s, uint32_t& parity) {
+  if (uses <= s) return false;
+  const int last = uses - 1 - ((uses - 1 - s) % slots);
+  parity = static_cast<uint32_t>(last / slots) & 1u;
+  return true;
 }
 
 template <Mode MODE>
@@ -98,19 +113,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* act_s = smem;                           // [kStages][kActBytes]   token-side operand
-  uint8_t* w_s = act_s + kStages * kActBytes;      // [kWStages][kWBytes]    weight-side operand
-  uint8_t* code_s = w_s + kWStages * kWBytes;      // [kCodeStages][kCodeBytes] packed codes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(code_s + kCodeStages * kCodeBytes);
-  uint64_t* act_full = bars;                      // [kStages] token-side tile landed
-  uint64_t* stage_empty = act_full + kStages;     // [kStages] MMAs reading the act slot done
-  uint64_t* deq_full = stage_empty + kStages;     // [kWStages] weight-side tile ready
-  uint64_t* w_empty = deq_full + kWStages;        // [kWStages] MMAs reading the W slot done
-  uint64_t* code_full = w_empty + kWStages;       // [kCodeStages] codes landed
-  uint64_t* code_empty = code_full + kCodeStages; // [kCodeStages] codes read by dequant
-  uint64_t* acc_full = code_empty + kCodeStages;  // [2] accumulator buffer complete
-  uint64_t* acc_empty = acc_full + 2;             // [2] accumulator buffer read out
-  uint64_t* mma_drain = acc_empty + 2;            // all MMAs of the CTA completed (exit)
+  uint8_t* act_s = smem;                             // [kHalfSlots][kHalfBytes] token side
+  uint8_t* w_s = act_s + kHalfSlots * kHalfBytes;    // [kDeqGroups][kWBytes] dequantized
+  uint8_t* wext_s = w_s + kDeqGroups * kWBytes;      // [kWBytes] LoRA weight-side operand
+  uint8_t* code_s = wext_s + kWBytes;                // [kCodeSlots][kCodeBytes] packed codes
+  uint16_t* epi_s = reinterpret_cast<uint16_t*>(code_s + kCodeSlots * kCodeBytes);  // [4][32][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(code_s + kCodeSlots * kCodeBytes + kEpiBytes);
+  uint64_t* half_full = bars;                       // [kHalfSlots] token tile landed
+  uint64_t* half_empty = half_full + kHalfSlots;    // [kHalfSlots] MMAs reading it done
+  uint64_t* deq_full = half_empty + kHalfSlots;     // [kDeqGroups] dequantized tile ready
+  uint64_t* w_empty = deq_full + kDeqGroups;        // [kDeqGroups] MMAs reading it done
+  uint64_t* code_full = w_empty + kDeqGroups;       // [kCodeSlots] codes landed
+  uint64_t* code_empty = code_full + kCodeSlots;    // [kCodeSlots] codes read by dequant
+  uint64_t* ext_empty = code_empty + kCodeSlots;    // LoRA operand slot read out
+  uint64_t* acc_full = ext_empty + 1;               // [kHalves] accumulator complete
+  uint64_t* acc_empty = acc_full + kHalves;         // [kHalves] accumulator read out
+  uint64_t* mma_drain = acc_empty + kHalves;        // all MMAs of the CTA completed (exit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* t8 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);  // [256]
@@ -120,10 +138,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const int64_t contraction = (MODE == Mode::kForward) ? args.K : args.N;
   const int ksteps = static_cast<int>((contraction + kBK - 1) / kBK);
   // the LoRA product enters as two steps: bf16 hi part, then bf16 lo part of scale*T
-  const int total = ksteps + (args.ext_mmas > 0 ? 2 : 0);
+  const bool has_ext = args.ext_mmas > 0;
+  const int total = ksteps + (has_ext ? 2 : 0);
   const int my_tiles = (static_cast<int>(blockIdx.x) < args.num_tiles)
                            ? (args.num_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
                            : 0;
+  // a tile whose second 256 tokens lie past M runs one accumulator only
+  auto halves_in = [&](int64_t m0) { return (args.M - m0 > kHalfCols) ? kHalves : 1; };
   auto tile_coords = [&](int i, int64_t& row0, int64_t& m0) {
     const int tile = blockIdx.x + i * gridDim.x;
     row0 = static_cast<int64_t>(tile % args.row_tiles) * kTileRows;
@@ -131,28 +152,29 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&act_full[s], 1);
-      mbar_init(&stage_empty[s], 1);
+    for (int s = 0; s < kHalfSlots; ++s) {
+      mbar_init(&half_full[s], 1);
+      mbar_init(&half_empty[s], 1);
     }
-    for (int s = 0; s < kWStages; ++s) {
+    for (int s = 0; s < kDeqGroups; ++s) {
       mbar_init(&deq_full[s], 4);
       mbar_init(&w_empty[s], 1);
     }
-    for (int s = 0; s < kCodeStages; ++s) {
+    for (int s = 0; s < kCodeSlots; ++s) {
       mbar_init(&code_full[s], 1);
       mbar_init(&code_empty[s], 4);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+    mbar_init(ext_empty, 1);
+    for (int h = 0; h < kHalves; ++h) {
+      mbar_init(&acc_full[h], 1);
+      mbar_init(&acc_empty[h], 4);
     }
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * kTileCols);
+    tmem_alloc(tmem_slot, kTileCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -164,63 +186,74 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     // ------------------------------------------------ TMA: token-side operand, LoRA steps
     if (lane == 0) {
       tma_prefetch_desc(&tm_act);
-      int issued = 0;
-      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+      int issued = 0;  // half tiles
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
         int64_t row0, m0;
         tile_coords(i, row0, m0);
-        for (int step = 0; step < total; ++step) {
-          const int g = i * total + step;
-          const int s = g % kStages;
-          if (g >= kStages && !mbar_wait(&stage_empty[s], ((g / kStages) - 1) & 1u, abort_flag)) {
+        const int nh = halves_in(m0);
+        for (int step = 0; step < total && ok; ++step) {
+          const bool ext = step >= ksteps;
+          const bool ext_w = ext && step == ksteps;  // this step also brings the LoRA operand
+          if (ext_w && i >= 1 && !mbar_wait(ext_empty, (i - 1) & 1u, abort_flag)) {
             record_error(args.err, abort_flag, kErrTimeoutProducer);
+            ok = false;
             break;
           }
-          if (step < ksteps) {
-            mbar_arrive_expect_tx(&act_full[s], kActBytes);
-            tma_load_2d(act_s + s * kActBytes, &tm_act, &act_full[s], step * kBK,
-                        static_cast<int>(m0));
-          } else {
-            const int ws = g % kWStages;
-            if (g >= kWStages &&
-                !mbar_wait(&w_empty[ws], ((g / kWStages) - 1) & 1u, abort_flag)) {
+          for (int h = 0; h < nh; ++h) {
+            const int hx = issued;
+            const int hs = hx % kHalfSlots;
+            if (hx >= kHalfSlots &&
+                !mbar_wait(&half_empty[hs], ((hx / kHalfSlots) - 1) & 1u, abort_flag)) {
               record_error(args.err, abort_flag, kErrTimeoutProducer);
+              ok = false;
               break;
             }
-            mbar_arrive_expect_tx(&act_full[s], kWBytes + kActBytes);
-            if (MODE == Mode::kForward) {
-              // B [r, N] as an MN-major operand: two 64-wide chunks of n, rows j >= r are 0
-              tma_load_2d(w_s + ws * kWBytes, &tm_ext_w, &act_full[s], static_cast<int>(row0), 0);
-              tma_load_2d(w_s + ws * kWBytes + 8192, &tm_ext_w, &act_full[s],
-                          static_cast<int>(row0) + 64, 0);
+            const int mh = static_cast<int>(m0) + h * kHalfCols;
+            if (!ext) {
+              mbar_arrive_expect_tx(&half_full[hs], kHalfBytes);
+              tma_load_2d(act_s + hs * kHalfBytes, &tm_act, &half_full[hs], step * kBK, mh);
             } else {
-              // A [K, r] as a K-major operand (columns j >= r are 0)
-              tma_load_2d(w_s + ws * kWBytes, &tm_ext_w, &act_full[s], 0, static_cast<int>(row0));
+              const bool with_w = ext_w && h == 0;
+              mbar_arrive_expect_tx(&half_full[hs], kHalfBytes + (with_w ? kWBytes : 0u));
+              if (with_w) {
+                if (MODE == Mode::kForward) {
+                  // B [r, N] as an MN-major operand: two 64-wide chunks of n, rows j >= r are 0
+                  tma_load_2d(wext_s, &tm_ext_w, &half_full[hs], static_cast<int>(row0), 0);
+                  tma_load_2d(wext_s + 8192, &tm_ext_w, &half_full[hs], static_cast<int>(row0) + 64,
+                              0);
+                } else {
+                  // A [K, r] as a K-major operand (columns j >= r are 0)
+                  tma_load_2d(wext_s, &tm_ext_w, &half_full[hs], 0, static_cast<int>(row0));
+                }
+              }
+              tma_load_2d(act_s + hs * kHalfBytes, &tm_ext_act, &half_full[hs],
+                          (step - ksteps) * 64, mh);
             }
-            tma_load_2d(act_s + s * kActBytes, &tm_ext_act, &act_full[s], (step - ksteps) * 64,
-                        static_cast<int>(m0));
-            mbar_arrive_count(&deq_full[ws], 4);  // no dequantization in a LoRA step
+            ++issued;
           }
-          ++issued;
         }
       }
       if (*abort_flag)  // let copies already in flight land before the CTA exits
-        for (int g = (issued > kStages ? issued - kStages : 0); g < issued; ++g)
-          mbar_wait_drain(&act_full[g % kStages], (g / kStages) & 1u);
+        for (int hx = (issued > kHalfSlots ? issued - kHalfSlots : 0); hx < issued; ++hx)
+          mbar_wait_drain(&half_full[hx % kHalfSlots], (hx / kHalfSlots) & 1u);
     }
   } else if (warp == 2) {
     // ------------------------------------------------ TMA: packed codes
     if (lane == 0) {
       tma_prefetch_desc(&tm_codes);
       int issued = 0;
-      for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
         int64_t row0, m0;
         tile_coords(i, row0, m0);
         for (int step = 0; step < ksteps; ++step) {
           const int c = i * ksteps + step;
-          const int s = c % kCodeStages;
-          if (c >= kCodeStages &&
-              !mbar_wait(&code_empty[s], ((c / kCodeStages) - 1) & 1u, abort_flag)) {
+          const int s = c % kCodeSlots;
+          if (c >= kCodeSlots &&
+              !mbar_wait(&code_empty[s], ((c / kCodeSlots) - 1) & 1u, abort_flag)) {
             record_error(args.err, abort_flag, kErrTimeoutProducer);
+            ok = false;
             break;
           }
           mbar_arrive_expect_tx(&code_full[s], kCodeBytes);
@@ -234,77 +267,105 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         }
       }
       if (*abort_flag)
-        for (int c = (issued > kCodeStages ? issued - kCodeStages : 0); c < issued; ++c)
-          mbar_wait_drain(&code_full[c % kCodeStages], (c / kCodeStages) & 1u);
+        for (int c = (issued > kCodeSlots ? issued - kCodeSlots : 0); c < issued; ++c)
+          mbar_wait_drain(&code_full[c % kCodeSlots], (c / kCodeSlots) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_main =
-          idesc_bf16_f32(kTileRows, kTileCols, MODE == Mode::kDgrad, false);
+          idesc_bf16_f32(kTileRows, kHalfCols, MODE == Mode::kDgrad, false);
       constexpr uint32_t idesc_ext =
-          idesc_bf16_f32(kTileRows, kTileCols, MODE == Mode::kForward, false);
+          idesc_bf16_f32(kTileRows, kHalfCols, MODE == Mode::kForward, false);
       bool ok = true;
+      int halves_done = 0, main_done = 0, ext_done = 0;
+      int acc_uses[kHalves] = {0, 0};  // tiles accumulated so far in each accumulator
       for (int i = 0; i < my_tiles && ok; ++i) {
-        const int buf = i & 1;
-        const uint32_t tmem_d = tmem_base + buf * kTileCols;
-        if (i >= 2 && !mbar_wait(&acc_empty[buf], ((i >> 1) - 1) & 1u, abort_flag)) {
-          record_error(args.err, abort_flag, kErrTimeoutMma);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int step = 0; step < total; ++step) {
-          const int g = i * total + step;
-          const int s = g % kStages;
-          const int ws = g % kWStages;
-          if (!mbar_wait(&act_full[s], (g / kStages) & 1u, abort_flag) ||
-              !mbar_wait(&deq_full[ws], (g / kWStages) & 1u, abort_flag)) {
-            record_error(args.err, abort_flag, kErrTimeoutMma);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(w_s + ws * kWBytes);
-          const uint32_t b0 = smem_u32(act_s + s * kActBytes);
-          if (step < ksteps) {
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t ad = (MODE == Mode::kForward)
-                                      ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
-                                      : smem_desc_sw128(a0 + kk * 4096, 1024, 2048);
-              const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-              umma_bf16(tmem_d, ad, bd, idesc_main, (step | kk) != 0);
+        int64_t row0, m0;
+        tile_coords(i, row0, m0);
+        const int nh = halves_in(m0);
+        for (int step = 0; step < total && ok; ++step) {
+          const bool main_step = step < ksteps;
+          const int c = i * ksteps + step;  // code step of a main step
+          uint32_t a0;
+          if (main_step) {
+            const int ws = c % kDeqGroups;
+            if (!mbar_wait(&deq_full[ws], (c / kDeqGroups) & 1u, abort_flag)) {
+              record_error(args.err, abort_flag, kErrTimeoutMma);
+              ok = false;
+              break;
             }
+            a0 = smem_u32(w_s + ws * kWBytes);
           } else {
-            for (int kk = 0; kk < args.ext_mmas; ++kk) {
-              const uint64_t ad = (MODE == Mode::kForward)
-                                      ? smem_desc_sw128(a0 + kk * 2048, 8192, 1024)
-                                      : smem_desc_sw128(a0 + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-              umma_bf16(tmem_d, ad, bd, idesc_ext, 1u);
+            a0 = smem_u32(wext_s);  // landed with the first half tile of the first LoRA step
+          }
+          for (int h = 0; h < nh; ++h) {
+            const int hx = halves_done;
+            const int hs = hx % kHalfSlots;
+            // the epilogue has read accumulator h of the previous tile out
+            if (step == 0 && acc_uses[h] >= 1 &&
+                !mbar_wait(&acc_empty[h], (acc_uses[h] - 1) & 1u, abort_flag)) {
+              record_error(args.err, abort_flag, kErrTimeoutMma);
+              ok = false;
+              break;
+            }
+            if (!mbar_wait(&half_full[hs], (hx / kHalfSlots) & 1u, abort_flag)) {
+              record_error(args.err, abort_flag, kErrTimeoutMma);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t tmem_d = tmem_base + h * kHalfCols;
+            const uint32_t b0 = smem_u32(act_s + hs * kHalfBytes);
+            if (main_step) {
+#pragma unroll
+              for (int kk = 0; kk < kBK / 16; ++kk) {
+                const uint64_t ad = (MODE == Mode::kForward)
+                                        ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
+                                        : smem_desc_sw128(a0 + kk * 4096, 1024, 2048);
+                const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+                umma_bf16(tmem_d, ad, bd, idesc_main, (step | kk) != 0);
+              }
+            } else {
+              for (int kk = 0; kk < args.ext_mmas; ++kk) {
+                const uint64_t ad = (MODE == Mode::kForward)
+                                        ? smem_desc_sw128(a0 + kk * 2048, 8192, 1024)
+                                        : smem_desc_sw128(a0 + kk * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+                umma_bf16(tmem_d, ad, bd, idesc_ext, 1u);
+              }
+            }
+            umma_commit(&half_empty[hs]);
+            ++halves_done;
+            if (step == total - 1) {  // accumulator h of this tile is complete
+              umma_commit(&acc_full[h]);
+              ++acc_uses[h];
             }
           }
-          umma_commit(&stage_empty[s]);
-          umma_commit(&w_empty[ws]);
+          if (!ok) break;
+          if (main_step) {
+            umma_commit(&w_empty[c % kDeqGroups]);
+            ++main_done;
+          } else if (step == total - 1) {
+            umma_commit(ext_empty);
+            ++ext_done;
+          }
         }
-        if (ok) umma_commit(&acc_full[buf]);
       }
       // every MMA this thread issued has completed before TMEM is freed (on the normal
       // path and after an abort alike); the barrier is used for this one phase only
       umma_commit(mma_drain);
       mbar_wait_drain(mma_drain, 0);
-      // The commits of the last steps arrive asynchronously on barriers nobody else
-      // waits for any more: let them land before the CTA (and its shared memory) goes.
-      const int steps_done = my_tiles * total;
-      for (int s = 0; s < kStages; ++s) {
-        const int last = steps_done - 1 - ((steps_done - 1 - s) % kStages + kStages) % kStages;
-        if (last >= 0 && last < steps_done) mbar_wait_drain(&stage_empty[s], (last / kStages) & 1u);
-      }
-      for (int s = 0; s < kWStages; ++s) {
-        const int last = steps_done - 1 - ((steps_done - 1 - s) % kWStages + kWStages) % kWStages;
-        if (last >= 0 && last < steps_done) mbar_wait_drain(&w_empty[s], (last / kWStages) & 1u);
-      }
+      // the commits of the last steps arrive asynchronously on barriers nobody else waits
+      // for any more: let them land before the CTA (and its shared memory) goes
+      uint32_t par;
+      for (int s = 0; s < kHalfSlots; ++s)
+        if (last_use(halves_done, kHalfSlots, s, par)) mbar_wait_drain(&half_empty[s], par);
+      for (int s = 0; s < kDeqGroups; ++s)
+        if (last_use(main_done, kDeqGroups, s, par)) mbar_wait_drain(&w_empty[s], par);
+      if (last_use(ext_done, 1, 0, par)) mbar_wait_drain(ext_empty, par);
+      for (int h = 0; h < kHalves; ++h)
+        if (acc_uses[h] >= 1) mbar_wait_drain(&acc_full[h], (acc_uses[h] - 1) & 1u);
     }
   } else if (warp >= kDeqWarp0) {
     // ------------------------------------------------ dequantization
@@ -314,6 +375,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const float mean = *args.mean;
     const int64_t bpr = args.K / 64;  // 64-blocks per weight row
     const int ncodes = my_tiles * ksteps;
+    uint8_t* dst = w_s + wg * kWBytes;  // this warpgroup's weight slot
     // Code step c = tile i * ksteps + step t; this warpgroup walks c = wg, wg + kDeqGroups, ...
     // (i, t) and the tile origin are advanced incrementally (no divisions per step).
     struct Cursor {
@@ -372,15 +434,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const float sc = valid ? block_scale_tab(t8, e2, e1, mean) : 0.f;  // zeros outside W
       Nf4Lut lut;
       build_lut(sc, lut);
-      // stage of the pipeline this code step feeds
-      const int g = cur.i * total + cur.t;
-      const int ws = g % kWStages;
-      const int cs = c % kCodeStages;
-      // move both cursors two steps on
+      const int cs = c % kCodeSlots;  // one of this warpgroup's code slots
       cur = nxt;
       advance(nxt, kDeqGroups);
       if (nxt.i != cur.i && nxt.i < my_tiles) set_tile(nxt);
-      if (!mbar_wait(&code_full[cs], (c / kCodeStages) & 1u, abort_flag)) {
+      if (!mbar_wait(&code_full[cs], (c / kCodeSlots) & 1u, abort_flag)) {
         record_error(args.err, abort_flag, kErrTimeoutDequant);
         break;
       }
@@ -391,12 +449,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       const uint4 q1 = *reinterpret_cast<const uint4*>(src + 16);
       __syncwarp();
       if (lane == 0) mbar_arrive(&code_empty[cs]);  // codes are in registers now
-      if (g >= kWStages && !mbar_wait(&w_empty[ws], ((g / kWStages) - 1) & 1u, abort_flag)) {
+      if (c >= kDeqGroups &&
+          !mbar_wait(&w_empty[wg], ((c / kDeqGroups) - 1) & 1u, abort_flag)) {
         record_error(args.err, abort_flag, kErrTimeoutDequant);
         break;
       }
       const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      uint8_t* dst = w_s + ws * kWBytes;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t o[4];
@@ -413,45 +471,76 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&deq_full[ws]);
+      if (lane == 0) mbar_arrive(&deq_full[wg]);
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------ epilogue
+    // TMEM lane = D row, column = token: each thread holds one D row of 32 tokens. The
+    // chunk is transposed through shared memory (stage[token][row]) so that every store
+    // to the token-major output writes 8 consecutive rows (16 bytes).
     const int quarter = warp & 3;  // TMEM lanes this warp may read
-    for (int i = 0; i < my_tiles; ++i) {
-      const int buf = i & 1;
-      if (!mbar_wait(&acc_full[buf], (i >> 1) & 1u, abort_flag)) {
-        if (!*abort_flag) record_error(args.err, abort_flag, kErrTimeoutEpilogue);
-        break;
-      }
-      tc_fence_after();
+    uint16_t* stage = epi_s + quarter * (32 * 32);
+    int uses[kHalves] = {0, 0};
+    bool ok = true;
+    for (int i = 0; i < my_tiles && ok; ++i) {
       int64_t row0, m0;
       tile_coords(i, row0, m0);
-      const int64_t orow = row0 + quarter * 32 + lane;
-      const uint32_t taddr = tmem_base + buf * kTileCols + (static_cast<uint32_t>(quarter * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < kTileCols / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, v);
-        tmem_ld_wait();
-        if (orow < args.out_rows) {
-          const int64_t mb = m0 + c * 32;
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (mb + k < args.M)
-              args.out[(mb + k) * args.out_ld + orow] = bf16_bits_rn(__uint_as_float(v[k]));
+      const int nh = halves_in(m0);
+      const int64_t obase = row0 + quarter * 32;  // first D row of this warp
+      for (int h = 0; h < nh; ++h) {
+        if (!mbar_wait(&acc_full[h], uses[h] & 1u, abort_flag)) {
+          if (!*abort_flag) record_error(args.err, abort_flag, kErrTimeoutEpilogue);
+          ok = false;
+          break;
         }
+        ++uses[h];
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + h * kHalfCols;
+#pragma unroll 1
+        for (int c = 0; c < kHalfCols / 32; ++c) {
+          const int64_t mb = m0 + h * kHalfCols + c * 32;
+          if (mb >= args.M) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const uint32_t pk = pack_bf16x2_rn(__uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+            stage[k * 32 + lane] = static_cast<uint16_t>(pk & 0xFFFFu);
+            stage[(k + 1) * 32 + lane] = static_cast<uint16_t>(pk >> 16);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int tr = (lane >> 2) + 8 * j;  // token inside the chunk
+            const int oc = (lane & 3) * 8;       // first of this thread's 8 rows
+            const int64_t tok = mb + tr;
+            const int64_t o = obase + oc;
+            const uint16_t* sv = stage + tr * 32 + oc;
+            if (tok < args.M) {
+              uint16_t* dst = args.out + tok * args.out_ld + o;
+              if (args.vec_store && o + 8 <= args.out_rows) {
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sv);
+              } else {
+                for (int e = 0; e < 8; ++e)
+                  if (o + e < args.out_rows) dst[e] = sv[e];
+              }
+            }
+          }
+          __syncwarp();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[h]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * kTileCols);
+    tmem_dealloc(tmem_base, kTileCols);
   }
 }
 
@@ -459,8 +548,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 constexpr int kLoraThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kLoraStages = 6;
 constexpr uint32_t kLoraABytes = 128 * kBK * 2;  // 16 KB
-constexpr uint32_t kLoraBMax = 128 * kBK * 2;    // 16 KB (NC = 128)
-constexpr uint32_t kLoraSmem = kLoraStages * (kLoraABytes + kLoraBMax) + 1024 + 256;
 
 struct LoraArgs {
   int64_t rows;      // D rows (128-row tiles)
@@ -749,6 +836,8 @@ cudaError_t run_fused(const CUtensorMap& tc, const CUtensorMap& ta, const CUtens
   const int64_t rows = (MODE == Mode::kForward) ? args.N : args.K;
   args.row_tiles = static_cast<int>((rows + kTileRows - 1) / kTileRows);
   args.num_tiles = args.row_tiles * static_cast<int>((args.M + kTileCols - 1) / kTileCols);
+  args.vec_store =
+      (args.out_ld % 8 == 0 && (reinterpret_cast<uintptr_t>(args.out) & 15u) == 0) ? 1 : 0;
   const int grid = std::min(args.num_tiles, num_sms());  // persistent: one CTA per SM
   cudaEvent_t before, after;
   profile_events(&before, &after);
