@@ -38,37 +38,49 @@ enum class Mode { kForward, kDgrad };
 // Warp roles of the persistent fused kernel:
 //   warp 0      TMA producer of the token-side operand (and the LoRA operands)
 //   warp 1      MMA issuer (one thread), owner of the TMEM allocation
-//   warp 2      TMA producer of the packed codes (its own ring)
-//   warp 3      idle
-//   warps 4-7   epilogue: TMEM -> registers -> bf16 -> global, one TMEM lane quarter each
-//   warps 8-..  dequantization, kDeqGroups warpgroups taking code steps in turn
+//   warps 2-5   epilogue: TMEM -> registers -> bf16 -> global, one TMEM lane quarter each
+//   warps 6-15  dequantization, two groups of four warps taking code steps in turn;
+//               warps 9 and 13 stay idle so that no dequantizing warp shares the MMA
+//               warp's scheduler (warp w issues from sub-partition w % 4): the single
+//               MMA thread then issues at full rate between its ALU-heavy neighbours.
 // A tile is 128 weight-side rows x 512 tokens held as two 256-column fp32 accumulators
 // (all 512 TMEM columns): every dequantized 128 x 64 weight tile feeds 8 MMAs.
-constexpr int kDeqGroups = 3;
-constexpr int kFusedThreads = 256 + 128 * kDeqGroups;
-constexpr int kEpiWarp0 = 4;
-constexpr int kDeqWarp0 = 8;
+//
+// Code step c (the c-th 64-wide contraction step of this CTA) belongs to warpgroup
+// c % kDeqGroups and is dequantized into weight slot c % kWSlots; every slot therefore
+// has one owner that uses it in order, so no mbarrier parity wait is ever more than one
+// phase ahead. The owner loads the packed codes and block constants of its next step
+// into registers and expands a step completely in registers before it waits for its
+// slot to be free: only the shared-memory stores remain on the path between the MMAs
+// of step c - kWSlots completing and step c being issued.
+constexpr int kDeqGroups = 2;
+constexpr int kWPerGroup = 2;
+constexpr int kWSlots = kDeqGroups * kWPerGroup;
+constexpr int kEpiWarp0 = 2;
+constexpr int kDeqWarp0 = 6;
+constexpr int kFusedThreads = 512;
+static_assert(kDeqGroups == 2, "dequant warp map below has eight entries");
+// position of a dequantizing warp in its groups (-1: not a dequantizing warp)
+__device__ __forceinline__ int deq_index(int warp) {
+  // warps 6 7 8 | 10 11 12 | 14 15  ->  0..7 ; 9, 13 (sub-partition 1) idle
+  if (warp < kDeqWarp0 || warp == 9 || warp == 13) return -1;
+  return warp - kDeqWarp0 - (warp > 9) - (warp > 13);
+}
 constexpr int kTileRows = 128;   // D rows on the weight side (n forward, k dgrad) = TMEM lanes
 constexpr int kHalfCols = 256;   // tokens per MMA / per accumulator
 constexpr int kHalves = 2;       // accumulators per tile
 constexpr int kTileCols = kHalfCols * kHalves;  // tokens per tile
 constexpr int kBK = 64;          // contraction per pipeline step
 constexpr int kHalfSlots = 4;    // ring of 256-token operand tiles (2 per step)
-// Rings that several dequant warpgroups touch are laid out so that every slot has a
-// single owner that uses it in order: code step c (c-th dequantized step of this CTA)
-// belongs to warpgroup c % kDeqGroups, which owns weight slot c % kDeqGroups and code
-// slots c % (kDeqGroups * kCodesPerGroup). An mbarrier parity wait is only meaningful
-// when the waiter is at most one phase ahead; with these owners it never is.
-constexpr int kCodesPerGroup = 2;
-constexpr int kCodeSlots = kDeqGroups * kCodesPerGroup;
 constexpr uint32_t kHalfBytes = kHalfCols * kBK * 2;  // 32 KB
 constexpr uint32_t kWBytes = kTileRows * kBK * 2;     // 16 KB
-constexpr uint32_t kCodeBytes = kTileRows * kBK / 2;  // 4 KB
 constexpr uint32_t kEpiBytes = 4 * 32 * 32 * 2;        // per epilogue warp: 32 tokens x 32 rows
-constexpr uint32_t kFusedSmem = kHalfSlots * kHalfBytes + (kDeqGroups + 1) * kWBytes +
-                                kCodeSlots * kCodeBytes + kEpiBytes + 1024 + 512 + 1024;
+constexpr uint32_t kFusedSmem = kHalfSlots * kHalfBytes + (kWSlots + 1) * kWBytes + kEpiBytes +
+                                1024 + 512 + 1024;
+static_assert(kFusedSmem <= 227 * 1024, "shared memory per CTA");
 
 struct FusedArgs {
+  const uint8_t* codes;  // [N][K/2] packed NF4 codes (16-byte aligned)
   const uint8_t* c2;
   const float* c1;
   const float* mean;
@@ -106,26 +118,22 @@ __device__ __forceinline__ bool last_use(int uses, int slots, int s, uint32_t& p
 
 template <Mode MODE>
 __global__ void __launch_bounds__(kFusedThreads, 1)
-    k_fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_codes,
-                     const __grid_constant__ CUtensorMap tm_act,
+    k_fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_act,
                      const __grid_constant__ CUtensorMap tm_ext_w,
                      const __grid_constant__ CUtensorMap tm_ext_act, const FusedArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* act_s = smem;                             // [kHalfSlots][kHalfBytes] token side
-  uint8_t* w_s = act_s + kHalfSlots * kHalfBytes;    // [kDeqGroups][kWBytes] dequantized
-  uint8_t* wext_s = w_s + kDeqGroups * kWBytes;      // [kWBytes] LoRA weight-side operand
-  uint8_t* code_s = wext_s + kWBytes;                // [kCodeSlots][kCodeBytes] packed codes
-  uint16_t* epi_s = reinterpret_cast<uint16_t*>(code_s + kCodeSlots * kCodeBytes);  // [4][32][32]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(code_s + kCodeSlots * kCodeBytes + kEpiBytes);
+  uint8_t* w_s = act_s + kHalfSlots * kHalfBytes;    // [kWSlots][kWBytes] dequantized
+  uint8_t* wext_s = w_s + kWSlots * kWBytes;         // [kWBytes] LoRA weight-side operand
+  uint16_t* epi_s = reinterpret_cast<uint16_t*>(wext_s + kWBytes);  // [4][32][32] staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wext_s + kWBytes + kEpiBytes);
   uint64_t* half_full = bars;                       // [kHalfSlots] token tile landed
   uint64_t* half_empty = half_full + kHalfSlots;    // [kHalfSlots] MMAs reading it done
-  uint64_t* deq_full = half_empty + kHalfSlots;     // [kDeqGroups] dequantized tile ready
-  uint64_t* w_empty = deq_full + kDeqGroups;        // [kDeqGroups] MMAs reading it done
-  uint64_t* code_full = w_empty + kDeqGroups;       // [kCodeSlots] codes landed
-  uint64_t* code_empty = code_full + kCodeSlots;    // [kCodeSlots] codes read by dequant
-  uint64_t* ext_empty = code_empty + kCodeSlots;    // LoRA operand slot read out
+  uint64_t* deq_full = half_empty + kHalfSlots;     // [kWSlots] dequantized tile ready
+  uint64_t* w_empty = deq_full + kWSlots;           // [kWSlots] MMAs reading it done
+  uint64_t* ext_empty = w_empty + kWSlots;          // LoRA operand slot read out
   uint64_t* acc_full = ext_empty + 1;               // [kHalves] accumulator complete
   uint64_t* acc_empty = acc_full + kHalves;         // [kHalves] accumulator read out
   uint64_t* mma_drain = acc_empty + kHalves;        // all MMAs of the CTA completed (exit)
@@ -156,13 +164,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       mbar_init(&half_full[s], 1);
       mbar_init(&half_empty[s], 1);
     }
-    for (int s = 0; s < kDeqGroups; ++s) {
+    for (int s = 0; s < kWSlots; ++s) {
       mbar_init(&deq_full[s], 4);
       mbar_init(&w_empty[s], 1);
-    }
-    for (int s = 0; s < kCodeSlots; ++s) {
-      mbar_init(&code_full[s], 1);
-      mbar_init(&code_empty[s], 4);
     }
     mbar_init(ext_empty, 1);
     for (int h = 0; h < kHalves; ++h) {
@@ -238,38 +242,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int hx = (issued > kHalfSlots ? issued - kHalfSlots : 0); hx < issued; ++hx)
           mbar_wait_drain(&half_full[hx % kHalfSlots], (hx / kHalfSlots) & 1u);
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------ TMA: packed codes
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_codes);
-      int issued = 0;
-      bool ok = true;
-      for (int i = 0; i < my_tiles && ok; ++i) {
-        int64_t row0, m0;
-        tile_coords(i, row0, m0);
-        for (int step = 0; step < ksteps; ++step) {
-          const int c = i * ksteps + step;
-          const int s = c % kCodeSlots;
-          if (c >= kCodeSlots &&
-              !mbar_wait(&code_empty[s], ((c / kCodeSlots) - 1) & 1u, abort_flag)) {
-            record_error(args.err, abort_flag, kErrTimeoutProducer);
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&code_full[s], kCodeBytes);
-          if (MODE == Mode::kForward)
-            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &code_full[s], step * (kBK / 2),
-                        static_cast<int>(row0));
-          else
-            tma_load_2d(code_s + s * kCodeBytes, &tm_codes, &code_full[s],
-                        static_cast<int>(row0 / 2), step * kBK);
-          ++issued;
-        }
-      }
-      if (*abort_flag)
-        for (int c = (issued > kCodeSlots ? issued - kCodeSlots : 0); c < issued; ++c)
-          mbar_wait_drain(&code_full[c % kCodeSlots], (c / kCodeSlots) & 1u);
-    }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -277,6 +249,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           idesc_bf16_f32(kTileRows, kHalfCols, MODE == Mode::kDgrad, false);
       constexpr uint32_t idesc_ext =
           idesc_bf16_f32(kTileRows, kHalfCols, MODE == Mode::kForward, false);
+      // Descriptor deltas per 16-wide K slice (start address field counts 16-byte units):
+      // K-major operands advance 32 bytes; the MN-major dequantized dgrad tile advances
+      // two 8-row groups (4096 bytes); the MN-major LoRA operand B [r, N] one 16-row
+      // slice of its 64-row chunk (2048 bytes).
+      constexpr uint32_t kDA = (MODE == Mode::kForward) ? 2u : 256u;
+      constexpr uint32_t kDX = (MODE == Mode::kForward) ? 128u : 2u;
+      const uint64_t desc_ext = (MODE == Mode::kForward)
+                                    ? smem_desc_sw128(smem_u32(wext_s), 8192, 1024)
+                                    : smem_desc_sw128(smem_u32(wext_s), 16, 1024);
       bool ok = true;
       int halves_done = 0, main_done = 0, ext_done = 0;
       int acc_uses[kHalves] = {0, 0};  // tiles accumulated so far in each accumulator
@@ -287,53 +268,46 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int step = 0; step < total && ok; ++step) {
           const bool main_step = step < ksteps;
           const int c = i * ksteps + step;  // code step of a main step
-          uint32_t a0;
+          uint64_t da;
           if (main_step) {
-            const int ws = c % kDeqGroups;
-            if (!mbar_wait(&deq_full[ws], (c / kDeqGroups) & 1u, abort_flag)) {
+            const int ws = c % kWSlots;
+            if (!mbar_wait(&deq_full[ws], (c / kWSlots) & 1u, abort_flag)) {
               record_error(args.err, abort_flag, kErrTimeoutMma);
               ok = false;
               break;
             }
-            a0 = smem_u32(w_s + ws * kWBytes);
+            da = (MODE == Mode::kForward) ? smem_desc_sw128(smem_u32(w_s + ws * kWBytes), 16, 1024)
+                                          : smem_desc_sw128(smem_u32(w_s + ws * kWBytes), 1024, 2048);
           } else {
-            a0 = smem_u32(wext_s);  // landed with the first half tile of the first LoRA step
+            da = desc_ext;  // landed with the first half tile of the first LoRA step
           }
           for (int h = 0; h < nh; ++h) {
             const int hx = halves_done;
             const int hs = hx % kHalfSlots;
             // the epilogue has read accumulator h of the previous tile out
-            if (step == 0 && acc_uses[h] >= 1 &&
-                !mbar_wait(&acc_empty[h], (acc_uses[h] - 1) & 1u, abort_flag)) {
-              record_error(args.err, abort_flag, kErrTimeoutMma);
-              ok = false;
-              break;
+            if (step == 0 && acc_uses[h] >= 1) {
+              if (!mbar_wait(&acc_empty[h], (acc_uses[h] - 1) & 1u, abort_flag)) {
+                record_error(args.err, abort_flag, kErrTimeoutMma);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
             if (!mbar_wait(&half_full[hs], (hx / kHalfSlots) & 1u, abort_flag)) {
               record_error(args.err, abort_flag, kErrTimeoutMma);
               ok = false;
               break;
             }
-            tc_fence_after();
             const uint32_t tmem_d = tmem_base + h * kHalfCols;
-            const uint32_t b0 = smem_u32(act_s + hs * kHalfBytes);
+            const uint64_t db = smem_desc_sw128(smem_u32(act_s + hs * kHalfBytes), 16, 1024);
             if (main_step) {
+              umma_bf16(tmem_d, da, db, idesc_main, step != 0);
 #pragma unroll
-              for (int kk = 0; kk < kBK / 16; ++kk) {
-                const uint64_t ad = (MODE == Mode::kForward)
-                                        ? smem_desc_sw128(a0 + kk * 32, 16, 1024)
-                                        : smem_desc_sw128(a0 + kk * 4096, 1024, 2048);
-                const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-                umma_bf16(tmem_d, ad, bd, idesc_main, (step | kk) != 0);
-              }
+              for (int kk = 1; kk < kBK / 16; ++kk)
+                umma_bf16(tmem_d, da + kk * kDA, db + kk * 2u, idesc_main, 1u);
             } else {
-              for (int kk = 0; kk < args.ext_mmas; ++kk) {
-                const uint64_t ad = (MODE == Mode::kForward)
-                                        ? smem_desc_sw128(a0 + kk * 2048, 8192, 1024)
-                                        : smem_desc_sw128(a0 + kk * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-                umma_bf16(tmem_d, ad, bd, idesc_ext, 1u);
-              }
+              for (int kk = 0; kk < args.ext_mmas; ++kk)
+                umma_bf16(tmem_d, da + kk * kDX, db + kk * 2u, idesc_ext, 1u);
             }
             umma_commit(&half_empty[hs]);
             ++halves_done;
@@ -344,7 +318,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           }
           if (!ok) break;
           if (main_step) {
-            umma_commit(&w_empty[c % kDeqGroups]);
+            umma_commit(&w_empty[c % kWSlots]);
             ++main_done;
           } else if (step == total - 1) {
             umma_commit(ext_empty);
@@ -361,23 +335,23 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       uint32_t par;
       for (int s = 0; s < kHalfSlots; ++s)
         if (last_use(halves_done, kHalfSlots, s, par)) mbar_wait_drain(&half_empty[s], par);
-      for (int s = 0; s < kDeqGroups; ++s)
-        if (last_use(main_done, kDeqGroups, s, par)) mbar_wait_drain(&w_empty[s], par);
+      for (int s = 0; s < kWSlots; ++s)
+        if (last_use(main_done, kWSlots, s, par)) mbar_wait_drain(&w_empty[s], par);
       if (last_use(ext_done, 1, 0, par)) mbar_wait_drain(ext_empty, par);
       for (int h = 0; h < kHalves; ++h)
         if (acc_uses[h] >= 1) mbar_wait_drain(&acc_full[h], (acc_uses[h] - 1) & 1u);
     }
-  } else if (warp >= kDeqWarp0) {
+  } else if (deq_index(warp) >= 0) {
     // ------------------------------------------------ dequantization
-    const int dw = warp - kDeqWarp0;
+    const int dw = deq_index(warp);
     const int wg = dw >> 2;                  // warpgroup: code steps wg, wg + kDeqGroups, ...
     const int local = (dw & 3) * 32 + lane;  // 0..127
     const float mean = *args.mean;
-    const int64_t bpr = args.K / 64;  // 64-blocks per weight row
+    const int64_t bpr = args.K / 64;     // 64-blocks per weight row
+    const int64_t code_ld = args.K / 2;  // bytes per weight row of codes
     const int ncodes = my_tiles * ksteps;
-    uint8_t* dst = w_s + wg * kWBytes;  // this warpgroup's weight slot
-    // Code step c = tile i * ksteps + step t; this warpgroup walks c = wg, wg + kDeqGroups, ...
-    // (i, t) and the tile origin are advanced incrementally (no divisions per step).
+    // Code step c = tile i * ksteps + step t; this warpgroup walks c = wg, wg + kDeqGroups,
+    // ... (i, t) and the tile origin are advanced incrementally (no divisions per step).
     struct Cursor {
       int i, t;
       int64_t row0, m0;
@@ -390,8 +364,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       }
     };
     auto set_tile = [&](Cursor& k) { tile_coords(k.i, k.row0, k.m0); };
-    // (row n, 64-block kb) of this thread at a cursor; false outside W
-    auto block_of = [&](const Cursor& k, int64_t& n, int64_t& kb) {
+    // This thread's 64-block at a cursor: weight row n, block kb along K. Forward: one
+    // block per D row; dgrad: two threads per contraction row n, 64 D rows (k) each.
+    // Loads its 32 code bytes and block constants; false outside W.
+    auto fetch = [&](const Cursor& k, uint4& a, uint4& b, uint32_t& e2, float& e1) {
+      int64_t n, kb;
       if (MODE == Mode::kForward) {
         n = k.row0 + local;
         kb = k.t;
@@ -399,66 +376,45 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         n = static_cast<int64_t>(k.t) * kBK + (local >> 1);
         kb = k.row0 / 64 + (local & 1);
       }
-      return n < args.N && kb < bpr;
+      if (n >= args.N || kb >= bpr) return false;
+      const uint4* src = reinterpret_cast<const uint4*>(args.codes + n * code_ld + kb * 32);
+      a = __ldg(src);
+      b = __ldg(src + 1);
+      const int64_t j = n * bpr + kb;
+      e2 = __ldg(args.c2 + j);
+      e1 = __ldg(args.c1 + (j >> 8));
+      return true;
     };
     Cursor cur{0, 0, 0, 0};
     advance(cur, wg);
     set_tile(cur);
-    Cursor nxt = cur;  // the next step of this warpgroup, for the prefetch
+    uint4 qa = make_uint4(0u, 0u, 0u, 0u), qb = qa;  // the next step's codes
+    uint32_t e2n = 0u;
+    float e1n = 0.f;
+    bool vn = (wg < ncodes) && fetch(cur, qa, qb, e2n, e1n);
+    Cursor nxt = cur;
     advance(nxt, kDeqGroups);
     if (nxt.i < my_tiles) set_tile(nxt);
-    // the block constants of this warpgroup's next step are loaded one step ahead
-    uint32_t e2_next = 0u;
-    float e1_next = 0.f;
-    {
-      int64_t n, kb;
-      if (wg < ncodes && block_of(cur, n, kb)) {
-        const int64_t j = n * bpr + kb;
-        e2_next = __ldg(args.c2 + j);
-        e1_next = __ldg(args.c1 + (j >> 8));
-      }
-    }
     for (int c = wg; c < ncodes; c += kDeqGroups) {
-      int64_t n, kb;
-      const bool valid = block_of(cur, n, kb);
-      const uint32_t e2 = e2_next;
-      const float e1 = e1_next;
-      if (c + kDeqGroups < ncodes) {
-        int64_t n2, kb2;
-        if (block_of(nxt, n2, kb2)) {
-          const int64_t j = n2 * bpr + kb2;
-          e2_next = __ldg(args.c2 + j);
-          e1_next = __ldg(args.c1 + (j >> 8));
-        }
-      }
-      const float sc = valid ? block_scale_tab(t8, e2, e1, mean) : 0.f;  // zeros outside W
-      Nf4Lut lut;
-      build_lut(sc, lut);
-      const int cs = c % kCodeSlots;  // one of this warpgroup's code slots
+      const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+      const float sc = vn ? block_scale_tab(t8, e2n, e1n, mean) : 0.f;  // zeros outside W
+      if (c + kDeqGroups < ncodes) vn = fetch(nxt, qa, qb, e2n, e1n);
       cur = nxt;
       advance(nxt, kDeqGroups);
       if (nxt.i != cur.i && nxt.i < my_tiles) set_tile(nxt);
-      if (!mbar_wait(&code_full[cs], (c / kCodeSlots) & 1u, abort_flag)) {
+      Nf4Lut lut;
+      build_lut(sc, lut);
+      uint32_t o[8][4];
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) lut_decode8(words[ch], lut, o[ch]);
+      const int ws = c % kWSlots;
+      if (c >= kWSlots && !mbar_wait(&w_empty[ws], ((c / kWSlots) - 1) & 1u, abort_flag)) {
         record_error(args.err, abort_flag, kErrTimeoutDequant);
         break;
       }
-      const uint8_t* src = (MODE == Mode::kForward)
-                               ? code_s + cs * kCodeBytes + local * 32
-                               : code_s + cs * kCodeBytes + (local >> 1) * 64 + (local & 1) * 32;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(src);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(src + 16);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&code_empty[cs]);  // codes are in registers now
-      if (c >= kDeqGroups &&
-          !mbar_wait(&w_empty[wg], ((c / kDeqGroups) - 1) & 1u, abort_flag)) {
-        record_error(args.err, abort_flag, kErrTimeoutDequant);
-        break;
-      }
-      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      uint8_t* dst = w_s + ws * kWBytes;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
-        uint32_t o[4];
-        lut_decode8(words[ch], lut, o);
         uint32_t off;
         if (MODE == Mode::kForward) {
           off = sw128_kmajor_offset(local, ch);
@@ -467,13 +423,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           off = (nr >> 3) * 2048u + (local & 1) * 1024u + (nr & 7u) * 128u +
                 ((ch ^ (nr & 7u)) << 4);
         }
-        *reinterpret_cast<uint4*>(dst + off) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(dst + off) = make_uint4(o[ch][0], o[ch][1], o[ch][2], o[ch][3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&deq_full[wg]);
+      if (lane == 0) mbar_arrive(&deq_full[ws]);
     }
-  } else if (warp >= kEpiWarp0) {
+  } else if (warp >= kEpiWarp0 && warp < kDeqWarp0) {
     // ------------------------------------------------ epilogue
     // TMEM lane = D row, column = token: each thread holds one D row of 32 tokens. The
     // chunk is transposed through shared memory (stage[token][row]) so that every store
@@ -546,25 +502,33 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
 // ================================================================== LoRA GEMMs
 constexpr int kLoraThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kLoraStages = 6;
 constexpr uint32_t kLoraABytes = 128 * kBK * 2;  // 16 KB
+// Pipeline depth: shared memory stays under 113 KB so that two CTAs share an SM.
+__host__ __device__ constexpr int lora_stages(int nc) { return nc == 128 ? 3 : 4; }
+__host__ __device__ constexpr uint32_t lora_smem(int nc) {
+  return lora_stages(nc) * (kLoraABytes + nc * kBK * 2) + 1024 + 256;
+}
+constexpr int kLoraCtasPerSm = 2;
+static_assert(lora_smem(128) <= 113 * 1024 && lora_smem(64) <= 113 * 1024, "two CTAs per SM");
 
 struct LoraArgs {
   int64_t rows;      // D rows (128-row tiles)
   int steps_total;   // 64-wide contraction steps
   int steps_per;     // steps per split
-  float* partial;    // [splits][rows_pad][NC] fp32
+  float* partial;    // [splits][rows_pad][64] fp32 (NC = 128: hi + lo columns summed)
   int64_t rows_pad;
   int* err;
 };
 
 // D[128-row tile, NC] = sum over this CTA's contraction range of A^T B (both bf16,
-// K-major or MN-major 128B-swizzled tiles loaded by TMA).
+// K-major or MN-major 128B-swizzled tiles loaded by TMA). With NC = 128 the B operand is
+// a bf16 hi | lo pair and the partial written is D[:, j] + D[:, 64 + j].
 template <bool A_MN, bool B_MN, int NC>
 __global__ void __launch_bounds__(kLoraThreads, 1)
     k_lora_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const LoraArgs args) {
   constexpr uint32_t kB = NC * kBK * 2;
+  constexpr int kLoraStages = lora_stages(NC);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -672,13 +636,22 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
       tc_fence_after();
       const int quarter = warp & 3;
       const int64_t row = row0 + quarter * 32 + lane;
-      float* dst = args.partial + (static_cast<int64_t>(blockIdx.y) * args.rows_pad + row) * NC;
+      float* dst = args.partial + (static_cast<int64_t>(blockIdx.y) * args.rows_pad + row) * 64;
+      const uint32_t taddr = tmem_d + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < NC / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
         if (have) {
-          tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(quarter * 32) << 16) + c * 32, v);
+          tmem_ld_32x32b_x32(taddr + c * 32, v);
           tmem_ld_wait();
+          if (NC == 128) {  // add the lo half of the pair
+            uint32_t w[32];
+            tmem_ld_32x32b_x32(taddr + 64 + c * 32, w);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
+          }
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = 0u;
@@ -711,7 +684,18 @@ __global__ void k_finalize_rank(const float* __restrict__ part, int splits, int6
   const int64_t m = i >> 6;
   const int j = static_cast<int>(i & 63);
   float v = 0.f;
-  for (int s = 0; s < splits; ++s) v += part[(s * rows_pad + m) * 64 + j];
+  const float* p = part + m * 64 + j;
+  const int64_t stride = rows_pad * 64;
+  int sp = 0;
+  float v1 = 0.f, v2 = 0.f, v3 = 0.f;
+  for (; sp + 4 <= splits; sp += 4) {  // four independent loads in flight
+    v += p[sp * stride];
+    v1 += p[(sp + 1) * stride];
+    v2 += p[(sp + 2) * stride];
+    v3 += p[(sp + 3) * stride];
+  }
+  for (; sp < splits; ++sp) v += p[sp * stride];
+  v = (v + v1) + (v2 + v3);
   if (j >= r) v = 0.f;
   if (plain && j < r) plain[m * r + j] = v;
   if (scaled) {  // [M, 128]: bf16 hi | bf16 lo of scale * v
@@ -741,29 +725,32 @@ __global__ void k_hilo_from_plain(const float* __restrict__ t, int64_t M, int r,
   hilo[m * 128 + 64 + j] = bf16_bits_rn(v - __uint_as_float(static_cast<uint32_t>(hi) << 16));
 }
 
-// grad[row, j] (or its transpose) = scale * sum_s (P[s][row][j] + P[s][row][64 + j]).
-// One block per 32 rows: coalesced reads of the partials, a shared-memory tile, and
-// coalesced writes in either output orientation.
+// grad[row, j] (or its transpose) = scale * sum_s P[s][row][j].
+// One block per 16 rows, four (row, j) items per thread with their split loads
+// interleaved; a shared-memory tile gives coalesced writes in either orientation.
+constexpr int kGradRows = 16;
 __global__ void __launch_bounds__(256)
     k_finalize_grad(const float* __restrict__ part, int splits, int64_t rows_pad, int64_t rows,
                     int r, float scale, bool transpose, float* __restrict__ out) {
-  __shared__ float tile[32][65];
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32;
-  for (int idx = threadIdx.x; idx < 32 * 64; idx += blockDim.x) {
+  __shared__ float tile[kGradRows][65];
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kGradRows;
+  const int64_t stride = rows_pad * 64;
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  const float* p = part + row0 * 64 + threadIdx.x;  // item u: row0 * 64 + threadIdx.x + 256 u
+  for (int sp = 0; sp < splits; ++sp) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] += p[sp * stride + 256 * u];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int idx = threadIdx.x + 256 * u;
     const int rl = idx >> 6, j = idx & 63;
-    float v = 0.f;
-    if (j < r && row0 + rl < rows) {
-      for (int s = 0; s < splits; ++s) {
-        const float* p = part + (s * rows_pad + row0 + rl) * 128;
-        v += p[j] + p[64 + j];
-      }
-    }
-    tile[rl][j] = scale * v;
+    tile[rl][j] = (j < r && row0 + rl < rows) ? scale * v[u] : 0.f;
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < 32 * r; idx += blockDim.x) {
+  for (int idx = threadIdx.x; idx < kGradRows * r; idx += blockDim.x) {
     if (transpose) {  // out [r, rows]
-      const int j = idx >> 5, rl = idx & 31;
+      const int j = idx / kGradRows, rl = idx % kGradRows;
       if (row0 + rl < rows) out[static_cast<int64_t>(j) * rows + row0 + rl] = tile[rl][j];
     } else {          // out [rows, r]
       const int rl = idx / r, j = idx % r;
@@ -791,18 +778,30 @@ SplitPlan plan_split(int64_t rows, int64_t contraction) {
     p.steps_per = p.steps_total > 0 ? p.steps_total : 1;
     return p;
   }
-  const int64_t target = 2LL * num_sms();
-  int64_t want = (target + p.tiles - 1) / p.tiles;
-  want = std::max<int64_t>(1, std::min<int64_t>(want, (p.steps_total + 1) / 2));
-  p.steps_per = static_cast<int>((p.steps_total + want - 1) / want);
-  p.splits = (p.steps_total + p.steps_per - 1) / p.steps_per;
+  // choose the split count that minimises (rounds of CTAs) x (steps per CTA + a fixed
+  // per-CTA cost of about three steps)
+  const int64_t slots = static_cast<int64_t>(kLoraCtasPerSm) * num_sms();
+  int64_t best = -1;
+  for (int want = 1; want <= p.steps_total && want <= 64; ++want) {
+    const int per = (p.steps_total + want - 1) / want;
+    const int splits = (p.steps_total + per - 1) / per;
+    if (splits != want) continue;
+    const int64_t rounds = (p.tiles * splits + slots - 1) / slots;
+    const int64_t cost = rounds * (per + 3);
+    if (best < 0 || cost < best) {
+      best = cost;
+      p.steps_per = per;
+      p.splits = splits;
+    }
+  }
   return p;
 }
 
 // Largest partial buffer (floats) the plans of one call may need.
 size_t partial_floats(int64_t rows, int64_t contraction, int nc) {
   const SplitPlan p = plan_split(rows, contraction);
-  return static_cast<size_t>(p.splits) * p.rows_pad * nc;
+  (void)nc;
+  return static_cast<size_t>(p.splits) * p.rows_pad * 64;
 }
 
 template <bool A_MN, bool B_MN, int NC>
@@ -817,7 +816,7 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
   a.rows_pad = p.rows_pad;
   a.err = device_error_word();
   auto kern = k_lora_gemm<A_MN, B_MN, NC>;
-  const uint32_t smem = kLoraStages * (kLoraABytes + NC * kBK * 2) + 1024 + 256;
+  const uint32_t smem = lora_smem(NC);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(static_cast<unsigned>(p.tiles), static_cast<unsigned>(p.splits)), kLoraThreads, smem,
@@ -827,8 +826,8 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
 }
 
 template <Mode MODE>
-cudaError_t run_fused(const CUtensorMap& tc, const CUtensorMap& ta, const CUtensorMap& tw,
-                      const CUtensorMap& tx, FusedArgs args, cudaStream_t st) {
+cudaError_t run_fused(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& tx,
+                      FusedArgs args, cudaStream_t st) {
   auto kern = k_fused_nf4_gemm<MODE>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
@@ -845,7 +844,7 @@ cudaError_t run_fused(const CUtensorMap& tc, const CUtensorMap& ta, const CUtens
     e = cudaEventRecord(before, st);
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, kFusedThreads, kFusedSmem, st>>>(tc, ta, tw, tx, args);
+  kern<<<grid, kFusedThreads, kFusedSmem, st>>>(ta, tw, tx, args);
   e = cudaGetLastError();
   if (e == cudaSuccess && after) e = cudaEventRecord(after, st);
   return e;
@@ -937,13 +936,12 @@ qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const ui
   qlora_status q = lora_down_T(X, A, s, part, T_save, ts, st);
   if (q != QLORA_OK) return q;
 
-  CUtensorMap tc, ta, tw, tx;
-  QL_MAP(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, s.K / 2, s.N, s.K / 2, 32, 128,
-         CU_TENSOR_MAP_SWIZZLE_NONE);
+  CUtensorMap ta, tw, tx;
   QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 256, kSW128);
   QL_MAP(&tw, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);   // B [r, N], MN-major chunks
   QL_MAP(&tx, kBF16, ts, 128, s.M, 256, 64, 256, kSW128);     // scale T, bf16 hi | lo
   FusedArgs a;
+  a.codes = w.codes;
   a.c2 = w.c2;
   a.c1 = w.c1;
   a.mean = w.mean;
@@ -955,7 +953,7 @@ qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const ui
   a.out_ld = s.N;
   a.out_rows = s.N;
   a.err = device_error_word();
-  QL_TRY(run_fused<Mode::kForward>(tc, ta, tw, tx, a, st));
+  QL_TRY(run_fused<Mode::kForward>(ta, tw, tx, a, st));
   return QLORA_OK;
 }
 
@@ -990,13 +988,12 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
 
   // dX = dY W_hat + scale G A^T
   if (dX) {
-    CUtensorMap tc, ta, tw, tx;
-    QL_MAP(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, s.K / 2, s.N, s.K / 2, 64, 64,
-           CU_TENSOR_MAP_SWIZZLE_NONE);
+    CUtensorMap ta, tw, tx;
     QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 256, kSW128);
     QL_MAP(&tw, kBF16, A, s.r, s.K, s.r * 2, 64, 128, kSW128);   // A [K, r] K-major
     QL_MAP(&tx, kBF16, gs, 128, s.M, 256, 64, 256, kSW128);      // scale G, bf16 hi | lo
     FusedArgs a;
+    a.codes = w.codes;
     a.c2 = w.c2;
     a.c1 = w.c1;
     a.mean = w.mean;
@@ -1008,7 +1005,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     a.out_ld = s.K;
     a.out_rows = s.K;
     a.err = device_error_word();
-    QL_TRY(run_fused<Mode::kDgrad>(tc, ta, tw, tx, a, st));
+    QL_TRY(run_fused<Mode::kDgrad>(ta, tw, tx, a, st));
   }
   // dA = scale X^T G  (rows k, contraction over tokens)
   {
@@ -1016,7 +1013,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 64, kSW128);    // X as MN-major (k inner)
     QL_MAP(&tb, kBF16, ghl, 128, s.M, 256, 64, 64, kSW128);      // G hi/lo MN-major
     QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits)));
-    k_finalize_grad<<<blocks_for(s.K, 32), 256, 0, st>>>(
+    k_finalize_grad<<<blocks_for(s.K, kGradRows), 256, 0, st>>>(
         part, splits, plan_split(s.K, s.M).rows_pad, s.K, s.r, s.scale, false, dA);
     QL_TRY(cudaGetLastError());
   }
@@ -1026,7 +1023,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);   // dY as MN-major (n inner)
     QL_MAP(&tb, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);      // T hi/lo MN-major
     QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.N, s.M, part, st, &splits)));
-    k_finalize_grad<<<blocks_for(s.N, 32), 256, 0, st>>>(
+    k_finalize_grad<<<blocks_for(s.N, kGradRows), 256, 0, st>>>(
         part, splits, plan_split(s.N, s.M).rows_pad, s.N, s.r, s.scale, true, dB);
     QL_TRY(cudaGetLastError());
   }
