@@ -1,19 +1,21 @@
 // decode.cu -- the QLoRA linear forward for M <= 16 tokens (decode), which is bound by
-// the HBM read of the packed weight (0.516 B per parameter).
+// reading the packed weight (0.516 B per parameter) and by the integer work of
+// expanding it.
 //
 //   Y = bf16(X W_hat^T + scale (X A) B)    (page "QLoRA", itwiki.kr, section "계산 방식";
 //                                           alpha/r from page "quantization", minnong511)
 //
+// k_decode_lora_down: T = X A on one cluster of 8 CTAs that split K; the CTA partial sums
+//   meet through distributed shared memory. It also clears the GEMV's arrival counters.
 // k_decode_gemv: each warp owns 32 weight rows and a contiguous range of K. Lanes load
-// 32 bytes of packed codes of one row with 128-bit loads, double-dequantize them in
-// registers (16-entry bf16 table per 64-block, prmt lookups) straight into the B
-// fragments of mma.m16n8k16 (X is the A operand, tokens padded to 16 rows). The
-// dequantized weight never leaves registers. Extra warps compute the split partial
-// sums of T = X A the same way (A plays the weight). Partial sums go to a workspace.
-// k_decode_finalize: sums the K splits, adds scale * T B and rounds to bf16.
-//
-// On tensor cores the multiply-adds cost nothing next to the unpack; mma.sync takes its
-// operands from registers, which is exactly where the unpack leaves the weights.
+//   32 bytes of packed codes of one row with 128-bit loads (the next 256-wide unit while
+//   the current one is expanded), double-dequantize them in registers (16-entry bf16
+//   table per 64-block, prmt lookups) straight into the A fragments of mma.m16n8k16 (X is
+//   the B operand). The dequantized weight never leaves registers. Every warp stores its
+//   partial sums; the last warp of a 32-row group to finish adds them up, adds
+//   scale * T B and writes the bf16 outputs, so no second pass over the partial sums runs.
+// The GEMV is a programmatic dependent of the T kernel: it streams the weight at once and
+// reads T and its counters only after griddepcontrol.wait.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -29,6 +31,8 @@ namespace {
 constexpr int kDecThreads = 128;
 constexpr int kRowsPerWarp = 32;
 constexpr int kUnitK = 256;  // K covered by one warp step (4 lanes x 64)
+constexpr int kTCtas = 8;    // cluster of the T kernel
+constexpr int kTThreads = 256;
 
 struct DecodeArgs {
   const uint8_t* codes;
@@ -37,13 +41,17 @@ struct DecodeArgs {
   const float* mean;
   const uint16_t* X;
   const uint16_t* A;
+  const uint16_t* B;
   int64_t M, N, K;
   int r;
+  float scale;
   int splits, units_per, nunits;  // K is cut into `splits` ranges of `units_per` 256-units
   int row_groups;                 // 32-row groups of W
-  int t_groups;                   // 8-column groups of A (for T = X A)
-  float* part;   // [splits][M][N]   partial sums of X W_hat^T
-  float* tpart;  // [splits][M][r]   partial sums of T = X A
+  float* part;      // [splits][row_groups][M][32] partial sums of X W_hat^T
+  float* T;         // [M][r] T = X A
+  float* T_save;    // optional copy of T for the backward pass
+  int* counters;    // [row_groups] warps of the group that have stored their partials
+  uint16_t* Y;      // [M][N]
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
@@ -64,23 +72,113 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-// 64 consecutive bf16 of X row `row` starting at column k, as 32 packed pairs (zeros
-// when the row is padding).
-__device__ __forceinline__ void load_x64(const uint16_t* X, int64_t K, int64_t row, bool live,
-                                         int64_t k, uint32_t (&x)[32]) {
-  if (live) {
-    const uint4* p = reinterpret_cast<const uint4*>(X + row * K + k);
+__device__ __forceinline__ float bf16_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+__device__ __forceinline__ int64_t lmin(int64_t x, int64_t y) { return x < y ? x : y; }
+
+// ---------------------------------------------------------------- T = X A
+// Thread layout: 4 columns of A per thread (jq), k lanes (kl) striding over this CTA's
+// share of K; X rows are read for all M tokens at once. Warp shuffles, then shared
+// memory, then the cluster sum the partial products.
+__global__ void __cluster_dims__(kTCtas, 1, 1) __launch_bounds__(kTThreads)
+    k_decode_lora_down(const DecodeArgs a) {
+  // the GEMV may start streaming the weight now; it waits for this grid before it
+  // touches T or the counters
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float wred[kTThreads / 32][16 * 64];
+  __shared__ float cpart[16 * 64];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int r = a.r;
+  const int M = static_cast<int>(a.M);
+  for (int i = static_cast<int>(rank) * kTThreads + tid; i < a.row_groups; i += kTCtas * kTThreads)
+    a.counters[i] = 0;
+
+  int jqn = 1;  // threads per A row: a power of two, 4 columns each
+  while (jqn * 4 < r) jqn <<= 1;
+  const int jq = tid & (jqn - 1), kl = tid / jqn, kls = kTThreads / jqn;
+  const int j0 = jq * 4;
+  const bool jlive = j0 < r;  // r is a multiple of 8, so j0 + 3 < r as well
+  const int64_t kper = (a.K + 8 * kTCtas - 1) / (8 * kTCtas) * 8;  // K is a multiple of 64
+  const int64_t k0 = static_cast<int64_t>(rank) * kper;
+  const int64_t k1 = lmin(a.K, k0 + kper);
+  float acc[16][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint4 v = __ldg(p + i);
-      x[4 * i] = v.x;
-      x[4 * i + 1] = v.y;
-      x[4 * i + 2] = v.z;
-      x[4 * i + 3] = v.w;
+  for (int m = 0; m < 16; ++m)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[m][c] = 0.f;
+  if (jlive) {
+    // chunks of 8 consecutive k: every load of a chunk is issued before its math
+    for (int64_t kc = k0 + 8 * kl; kc < k1; kc += 8 * kls) {
+      float av[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.A + (kc + i) * r + j0));
+        av[i][0] = bf16_to_f32(v.x & 0xFFFFu);
+        av[i][1] = bf16_to_f32(v.x >> 16);
+        av[i][2] = bf16_to_f32(v.y & 0xFFFFu);
+        av[i][3] = bf16_to_f32(v.y >> 16);
+      }
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        if (m < M) {
+          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.X + m * a.K + kc));
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float x = bf16_to_f32((i & 1) ? (xw[i >> 1] >> 16) : (xw[i >> 1] & 0xFFFFu));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[m][c] = fmaf(x, av[i][c], acc[m][c]);
+          }
+        }
+      }
     }
-  } else {
+  }
+  // lanes that share jq hold partial sums of the same outputs
+  for (int o = jqn; o < 32; o <<= 1)
 #pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = 0u;
+    for (int m = 0; m < 16; ++m)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[m][c] += __shfl_xor_sync(0xFFFFFFFFu, acc[m][c], o);
+  if (lane < jqn && jlive)
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) wred[warp][m * 64 + j0 + c] = acc[m][c];
+  __syncthreads();
+  const int mr = M * r;
+  for (int e = tid; e < mr; e += kTThreads) {
+    const int m = e / r, j = e % r;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kTThreads / 32; ++w) v += wred[w][m * 64 + j];
+    cpart[e] = v;
+  }
+  cluster_sync_all();  // every CTA's partial sums are in its shared memory
+  if (rank == 0) {
+    for (int e = tid; e < mr; e += kTThreads) {
+      float v = 0.f;
+#pragma unroll
+      for (int q = 0; q < kTCtas; ++q) v += ld_cluster_f32(&cpart[e], static_cast<uint32_t>(q));
+      a.T[e] = v;
+      if (a.T_save) a.T_save[e] = v;
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while rank 0 still reads its shared memory
+}
+
+// ---------------------------------------------------------------- X W_hat^T
+// 64 consecutive bf16 of X row `row` starting at column k, as 32 packed pairs.
+__device__ __forceinline__ void load_x64(const uint16_t* X, int64_t K, int64_t row, int64_t k,
+                                         uint32_t (&x)[32]) {
+  const uint4* p = reinterpret_cast<const uint4*>(X + row * K + k);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 v = __ldg(p + i);
+    x[4 * i] = v.x;
+    x[4 * i + 1] = v.y;
+    x[4 * i + 2] = v.z;
+    x[4 * i + 3] = v.w;
   }
 }
 
@@ -93,7 +191,77 @@ __device__ __forceinline__ void load_x64(const uint16_t* X, int64_t K, int64_t r
 // is free, and the unpacked pairs land directly in the A operand registers.
 constexpr int kGroups = 2;  // 16-row groups per warp (32 weight rows)
 
-__device__ __forceinline__ int64_t lmin(int64_t x, int64_t y) { return x < y ? x : y; }
+// Packed codes and block constants of one unit for this lane (rows beyond N are clamped
+// and K beyond the matrix is clamped; their scale is forced to zero later).
+struct UnitCodes {
+  uint4 q[kGroups][2][2];
+  uint32_t e2[kGroups][2];
+  float e1[kGroups][2];
+};
+
+// This lane's four weight rows (clamped to the last row; their scale is forced to zero
+// later) as one base and 32-bit offsets from it, computed once per task.
+struct RowBases {
+  const uint8_t* code;           // codes of the first row
+  int64_t blk;                   // index of the first row's first 64-block
+  int coff[kGroups][2];          // code byte offset of each row from `code`
+  int boff[kGroups][2];          // block offset of each row from `blk`
+};
+
+__device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases& rb, int u, int t,
+                                          int bpr, UnitCodes& c) {
+  const int kbi = min(u * (kUnitK / 64) + t, bpr - 1);  // 64-block of this lane (clamped)
+  const uint8_t* base = rb.code + kbi * 32;
+  const int64_t jb = rb.blk + kbi;
+#pragma unroll
+  for (int q = 0; q < kGroups; ++q)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint8_t* p = base + rb.coff[q][h];
+      c.q[q][h][0] = ldg_stream(p);
+      c.q[q][h][1] = ldg_stream(p + 16);
+      const int64_t j = jb + rb.boff[q][h];
+      c.e2[q][h] = __ldg(a.c2 + j);
+      c.e1[q][h] = __ldg(a.c1 + (j >> 8));
+    }
+}
+
+template <bool kTall>
+__device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int g,
+                                             int t, const UnitCodes& c, const float* t8,
+                                             float mean, float (&acc)[kGroups][kTall ? 2 : 1][4]) {
+  const int64_t K = a.K;
+  const int64_t kraw = static_cast<int64_t>(u) * kUnitK + 64 * t;
+  const bool kv = kraw < K;
+  const int64_t kb = kv ? kraw : K - 64;
+  // token rows this lane feeds to the B operand; tokens >= M compute columns nobody stores
+  uint32_t xa[32], xb[32];
+  load_x64(a.X, K, lmin(g, a.M - 1), kb, xa);
+  if (kTall) load_x64(a.X, K, lmin(g + 8, a.M - 1), kb, xb);
+#pragma unroll
+  for (int q = 0; q < kGroups; ++q) {
+    Nf4Lut lut[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const bool live = kv && (rbase + q * 16 + g + 8 * h) < a.N;
+      build_lut(live ? block_scale_tab(t8, c.e2[q][h], c.e1[q][h], mean) : 0.f, lut[h]);
+    }
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      uint32_t o0[4], o1[4];
+      lut_decode8(w < 4 ? (&c.q[q][0][0].x)[w] : (&c.q[q][0][1].x)[w - 4], lut[0], o0);
+      lut_decode8(w < 4 ? (&c.q[q][1][0].x)[w] : (&c.q[q][1][1].x)[w - 4], lut[1], o1);
+      mma_bf16_16816(acc[q][0], o0[0], o1[0], o0[1], o1[1], xa[4 * w], xa[4 * w + 1]);
+      mma_bf16_16816(acc[q][0], o0[2], o1[2], o0[3], o1[3], xa[4 * w + 2], xa[4 * w + 3]);
+      if (kTall) {
+        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[0], o1[0], o0[1], o1[1], xb[4 * w],
+                       xb[4 * w + 1]);
+        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[2], o1[2], o0[3], o1[3], xb[4 * w + 2],
+                       xb[4 * w + 3]);
+      }
+    }
+  }
+}
 
 template <bool kTall>
 __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, int split,
@@ -101,13 +269,8 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   const int g = lane >> 2, t = lane & 3;
   const int u0 = split * a.units_per;
   const int u1 = min(a.nunits, u0 + a.units_per);
-  const int64_t K = a.K, N = a.N;
-  const int64_t bpr = K / 64;
   const float mean = *a.mean;
   const int64_t rbase = static_cast<int64_t>(rg) * kRowsPerWarp;
-  // token rows this lane feeds to the B operand; tokens >= M compute columns nobody stores
-  const int64_t xr0 = lmin(g, a.M - 1);
-  const int64_t xr1 = lmin(g + 8, a.M - 1);
   float acc[kGroups][kTall ? 2 : 1][4];
 #pragma unroll
   for (int q = 0; q < kGroups; ++q)
@@ -116,210 +279,133 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[q][h][i] = 0.f;
 
-  for (int u = u0; u < u1; ++u) {
-    const int64_t kraw = static_cast<int64_t>(u) * kUnitK + 64 * t;
-    const bool kv = kraw < K;
-    const int64_t kb = kv ? kraw : K - 64;  // clamped: the scale below is zero then
-    // every load of this unit is issued before any math; rows beyond N are clamped and
-    // get a zero scale
-    uint4 cq[kGroups][2][2];
-    uint32_t e2[kGroups][2];
-    float e1[kGroups][2];
+  const int bpr = static_cast<int>(a.K / 64);
+  RowBases rb;
+  const int64_t row_g = lmin(rbase + g, a.N - 1);
+  rb.code = a.codes + row_g * (a.K / 2);
+  rb.blk = row_g * bpr;
 #pragma unroll
-    for (int q = 0; q < kGroups; ++q)
+  for (int q = 0; q < kGroups; ++q)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t row = lmin(rbase + q * 16 + g + 8 * h, N - 1);
-        const uint8_t* p = a.codes + row * (K / 2) + kb / 2;
-        cq[q][h][0] = ldg_stream(p);
-        cq[q][h][1] = ldg_stream(p + 16);
-        const int64_t j = row * bpr + kb / 64;
-        e2[q][h] = __ldg(a.c2 + j);
-        e1[q][h] = __ldg(a.c1 + (j >> 8));
-      }
-    uint32_t xa[32], xb[32];
-    load_x64(a.X, K, xr0, true, kb, xa);
-    if (kTall) load_x64(a.X, K, xr1, true, kb, xb);
-#pragma unroll
-    for (int q = 0; q < kGroups; ++q) {
-      Nf4Lut lut[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const bool live = kv && (rbase + q * 16 + g + 8 * h) < N;
-        build_lut(live ? block_scale_tab(t8, e2[q][h], e1[q][h], mean) : 0.f, lut[h]);
-      }
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        uint32_t o0[4], o1[4];
-        lut_decode8(w < 4 ? (&cq[q][0][0].x)[w] : (&cq[q][0][1].x)[w - 4], lut[0], o0);
-        lut_decode8(w < 4 ? (&cq[q][1][0].x)[w] : (&cq[q][1][1].x)[w - 4], lut[1], o1);
-        mma_bf16_16816(acc[q][0], o0[0], o1[0], o0[1], o1[1], xa[4 * w], xa[4 * w + 1]);
-        mma_bf16_16816(acc[q][0], o0[2], o1[2], o0[3], o1[3], xa[4 * w + 2], xa[4 * w + 3]);
-        if (kTall) {
-          mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[0], o1[0], o0[1], o1[1], xb[4 * w],
-                         xb[4 * w + 1]);
-          mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[2], o1[2], o0[3], o1[3], xb[4 * w + 2],
-                         xb[4 * w + 3]);
-        }
-      }
+    for (int h = 0; h < 2; ++h) {
+      const int dr = static_cast<int>(lmin(rbase + q * 16 + g + 8 * h, a.N - 1) - row_g);
+      rb.coff[q][h] = dr * static_cast<int>(a.K / 2);
+      rb.boff[q][h] = dr * bpr;
+    }
+  // two code buffers: the loads of unit u + 1 are in flight while unit u is expanded
+  UnitCodes cb0, cb1;
+  if (u0 < u1) load_unit(a, rb, u0, t, bpr, cb0);
+  for (int u = u0; u < u1; u += 2) {
+    if (u + 1 < u1) load_unit(a, rb, u + 1, t, bpr, cb1);
+    compute_unit<kTall>(a, rbase, u, g, t, cb0, t8, mean, acc);
+    if (u + 1 < u1) {
+      if (u + 2 < u1) load_unit(a, rb, u + 2, t, bpr, cb0);
+      compute_unit<kTall>(a, rbase, u + 1, g, t, cb1, t8, mean, acc);
     }
   }
+
   // C fragment: c0,c1 = (weight row g, tokens 2t, 2t+1), c2,c3 = (row g + 8, same tokens);
   // the second accumulator (M > 8) holds tokens 8 + 2t, 8 + 2t + 1.
+  const int64_t M = a.M;
+  float* pp = a.part + (static_cast<int64_t>(split) * a.row_groups + rg) * M * 32;
 #pragma unroll
   for (int q = 0; q < kGroups; ++q)
 #pragma unroll
     for (int hm = 0; hm < (kTall ? 2 : 1); ++hm)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int64_t row = rbase + q * 16 + g + 8 * (i >> 1);
-        const int64_t m = 8 * hm + 2 * t + (i & 1);
-        if (row < N && m < a.M)
-          a.part[(static_cast<int64_t>(split) * a.M + m) * N + row] = acc[q][hm][i];
+        const int rl = q * 16 + g + 8 * (i >> 1);
+        const int m = 8 * hm + 2 * t + (i & 1);
+        if (m < M) pp[m * 32 + rl] = acc[q][hm][i];
       }
-}
 
-// T partials over the K range of `split` for A columns tg*8 .. tg*8+7 (A [K, r] plays
-// the weight: its column is gathered with strided bf16 loads).
-template <bool kTall>
-__device__ __forceinline__ void decode_t_task(const DecodeArgs& a, int idx, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  const int tg = idx % a.t_groups;
-  const int split = idx / a.t_groups;
-  const int u0 = split * a.units_per;
-  const int u1 = min(a.nunits, u0 + a.units_per);
-  const int col = tg * 8 + g;
-  float d[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int u = u0; u < u1; ++u) {
-    const int64_t kb = static_cast<int64_t>(u) * kUnitK + 64 * t;
-    const bool kv = kb < a.K;
-    const bool live = kv && col < a.r;
-    uint32_t bw[32];
+  // T and the cleared counters come from the T kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = atomicAdd(a.counters + rg, 1) == a.splits - 1;
+  last = __shfl_sync(0xFFFFFFFFu, last, 0);
+  if (!last) return;
+  __threadfence();  // the other warps' partial sums are visible from here on
+
+  const int64_t row = rbase + lane;
+  if (row >= a.N) return;
+  float y[16], lora[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      uint32_t lo = 0, hi = 0;
-      if (live) {
-        lo = __ldg(a.A + (kb + 2 * i) * a.r + col);
-        hi = __ldg(a.A + (kb + 2 * i + 1) * a.r + col);
+  for (int m = 0; m < 16; ++m) {
+    y[m] = 0.f;
+    lora[m] = 0.f;
+  }
+  const int64_t sstride = static_cast<int64_t>(a.row_groups) * M * 32;
+  const float* p0 = a.part + static_cast<int64_t>(rg) * M * 32 + lane;
+  for (int s = 0; s < a.splits; ++s) {
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+      if (m < M) y[m] += __ldcg(p0 + s * sstride + m * 32);
+  }
+  const int r = a.r;
+  for (int j = 0; j < r; j += 4) {
+    float bv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bv[i] = bf16_to_f32(__ldg(a.B + (j + i) * a.N + row));
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+      if (m < M) {
+        const float4 tv = __ldcg(reinterpret_cast<const float4*>(a.T + m * r + j));
+        lora[m] = fmaf(tv.x, bv[0], lora[m]);
+        lora[m] = fmaf(tv.y, bv[1], lora[m]);
+        lora[m] = fmaf(tv.z, bv[2], lora[m]);
+        lora[m] = fmaf(tv.w, bv[3], lora[m]);
       }
-      bw[i] = lo | (hi << 16);
-    }
-    uint32_t xa[32], xb[32];
-    load_x64(a.X, a.K, g, kv && g < a.M, kb, xa);
-    if (kTall) load_x64(a.X, a.K, g + 8, kv && g + 8 < a.M, kb, xb);
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      mma_bf16_16816(d, xa[2 * j], kTall ? xb[2 * j] : 0u, xa[2 * j + 1],
-                     kTall ? xb[2 * j + 1] : 0u, bw[2 * j], bw[2 * j + 1]);
   }
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t m = g + 8 * h;
-    if (m >= a.M) continue;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int c = tg * 8 + 2 * t + e;
-      if (c < a.r) a.tpart[(static_cast<int64_t>(split) * a.M + m) * a.r + c] = d[2 * h + e];
-    }
-  }
+  for (int m = 0; m < 16; ++m)
+    if (m < M) a.Y[m * a.N + row] = bf16_bits_rn(y[m] + a.scale * lora[m]);
 }
 
+// Two CTAs (8 warps) per SM: the two code buffers of the prefetch need the registers, and
+// measured faster than three CTAs with spills.
 template <bool kTall>  // kTall: M > 8 (tokens 8..15 live in the upper fragment rows)
-__global__ void __launch_bounds__(kDecThreads, kTall ? 2 : 3) k_decode_gemv(const DecodeArgs a) {
-  // the finalize kernel may be scheduled now; it waits for this grid's results
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+__global__ void __launch_bounds__(kDecThreads, 2) k_decode_gemv(const DecodeArgs a) {
   __shared__ float t8[256];  // T8 by E4M3 code
   for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int task = blockIdx.x * (kDecThreads / 32) + warp;
-  const int wtasks = a.row_groups * a.splits;
-  if (task < wtasks)
+  if (task < a.row_groups * a.splits)
     decode_weight_task<kTall>(a, task % a.row_groups, task / a.row_groups, lane, t8);
-  else if (task < wtasks + a.t_groups * a.splits)
-    decode_t_task<kTall>(a, task - wtasks, lane);
 }
 
-// One CTA per 32 output columns: T = sum of its split partials (lanes over splits,
-// warp shuffles), the Y partials summed by 8 groups of splits then combined through
-// shared memory, plus scale * T B, rounded to bf16.
-constexpr int kFinCols = 32;
-__global__ void __launch_bounds__(256)
-    k_decode_finalize(const float* __restrict__ part, const float* __restrict__ tpart,
-                      int splits, int64_t M, int64_t N, int r, float scale,
-                      const uint16_t* __restrict__ B, uint16_t* __restrict__ Y,
-                      float* __restrict__ T_save) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // the GEMV's partial sums are complete
-  __shared__ float T[16 * 64];
-  __shared__ float red[8][16][kFinCols];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mr = static_cast<int>(M) * r;
-  for (int e = warp; e < mr; e += 8) {
-    float v = 0.f;
-    for (int s = lane; s < splits; s += 32) v += tpart[static_cast<int64_t>(s) * mr + e];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (lane == 0) {
-      T[e] = v;
-      if (T_save && blockIdx.x == 0) T_save[e] = v;
-    }
-  }
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kFinCols;
-  const int64_t n = n0 + lane;
-  float acc[16];
-#pragma unroll
-  for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-  if (n < N) {
-    for (int s = warp; s < splits; s += 8) {
-#pragma unroll
-      for (int m = 0; m < 16; ++m)
-        if (m < M) acc[m] += part[(static_cast<int64_t>(s) * M + m) * N + n];
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < 16; ++m)
-    if (m < M) red[warp][m][lane] = acc[m];
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < static_cast<int>(M) * kFinCols; idx += blockDim.x) {
-    const int m = idx / kFinCols, c = idx % kFinCols;
-    const int64_t nn = n0 + c;
-    if (nn >= N) continue;
-    float y = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) y += red[w][m][c];
-    float lora = 0.f;
-    for (int j = 0; j < r; ++j)
-      lora += T[m * r + j] * __uint_as_float(static_cast<uint32_t>(__ldg(B + j * N + nn)) << 16);
-    Y[m * N + nn] = bf16_bits_rn(y + scale * lora);
-  }
-}
-
+// ---------------------------------------------------------------- host side
 struct DecodePlan {
-  int splits, units_per, nunits, row_groups, t_groups;
+  int splits, units_per, nunits, row_groups;
 };
 
+// K splits: enough warps for about two waves of the GEMV (8 resident warps per SM), but
+// no more than K / (16 M): the partial sums (split x M x 128 bytes per 32 rows, written
+// and read back through L2) stay at most half the code bytes.
 DecodePlan plan_decode(const LinearShape& s) {
   DecodePlan p;
   p.nunits = static_cast<int>((s.K + kUnitK - 1) / kUnitK);
   p.row_groups = static_cast<int>((s.N + kRowsPerWarp - 1) / kRowsPerWarp);
-  p.t_groups = (s.r + 7) / 8;
-  // As many K splits as keep the fp32 partial sums (splits * M * N * 4 bytes) to a few
-  // percent of the weight bytes (N * K / 2): splits <= K / (128 M).
-  int64_t want = std::max<int64_t>(1, s.K / (128 * std::max<int64_t>(1, s.M)));
-  want = std::min<int64_t>(want, p.nunits);
+  const int64_t per_sm = 8;
+  const int64_t target = 2 * per_sm * num_sms();
+  int64_t want = (target + p.row_groups - 1) / p.row_groups;
+  want = std::min<int64_t>(want, std::max<int64_t>(1, s.K / (16 * std::max<int64_t>(1, s.M))));
+  want = std::max<int64_t>(1, std::min<int64_t>(want, p.nunits));
   p.units_per = static_cast<int>((p.nunits + want - 1) / want);
   p.splits = (p.nunits + p.units_per - 1) / p.units_per;
   return p;
 }
 
 size_t part_bytes(const DecodePlan& p, const LinearShape& s) {
-  return align_up(static_cast<size_t>(p.splits) * s.M * s.N * 4, 256);
+  return align_up(static_cast<size_t>(p.splits) * p.row_groups * s.M * 32 * 4, 256);
 }
-size_t tpart_bytes(const DecodePlan& p, const LinearShape& s) {
-  return align_up(static_cast<size_t>(p.splits) * s.M * s.r * 4, 256);
-}
+size_t t_bytes(const LinearShape& s) { return align_up(static_cast<size_t>(s.M) * s.r * 4, 256); }
+size_t counter_bytes(const DecodePlan& p) { return align_up(static_cast<size_t>(p.row_groups) * 4, 256); }
 
-// The GEMV grid, then the finalize kernel with programmatic dependent launch.
+// The T kernel, then the GEMV as its programmatic dependent.
 qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
                            const uint16_t* B, const LinearShape& s, const DecodePlan& p,
                            uint16_t* Y, float* T_save, char* scratch, cudaStream_t st) {
@@ -330,28 +416,28 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   a.mean = w.mean;
   a.X = X;
   a.A = A;
+  a.B = B;
   a.M = s.M;
   a.N = s.N;
   a.K = s.K;
   a.r = s.r;
+  a.scale = s.scale;
   a.splits = p.splits;
   a.units_per = p.units_per;
   a.nunits = p.nunits;
   a.row_groups = p.row_groups;
-  a.t_groups = p.t_groups;
   a.part = reinterpret_cast<float*>(scratch);
-  a.tpart = reinterpret_cast<float*>(scratch + part_bytes(p, s));
-  const int64_t warps = static_cast<int64_t>(p.row_groups + p.t_groups) * p.splits;
-  const unsigned ctas = static_cast<unsigned>((warps + kDecThreads / 32 - 1) / (kDecThreads / 32));
-  if (s.M > 8)
-    k_decode_gemv<true><<<ctas, kDecThreads, 0, st>>>(a);
-  else
-    k_decode_gemv<false><<<ctas, kDecThreads, 0, st>>>(a);
+  a.T = reinterpret_cast<float*>(scratch + part_bytes(p, s));
+  a.counters = reinterpret_cast<int*>(scratch + part_bytes(p, s) + t_bytes(s));
+  a.T_save = T_save;
+  a.Y = Y;
+  k_decode_lora_down<<<kTCtas, kTThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e);
+  const int64_t warps = static_cast<int64_t>(p.row_groups) * p.splits;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((s.N + kFinCols - 1) / kFinCols));
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3(static_cast<unsigned>((warps + kDecThreads / 32 - 1) / (kDecThreads / 32)));
+  cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -359,18 +445,20 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, k_decode_finalize, static_cast<const float*>(a.part),
-                         static_cast<const float*>(a.tpart), p.splits, s.M, s.N, s.r, s.scale, B,
-                         Y, T_save);
+  e = s.M > 8 ? cudaLaunchKernelEx(&cfg, k_decode_gemv<true>, a)
+              : cudaLaunchKernelEx(&cfg, k_decode_gemv<false>, a);
   if (e != cudaSuccess) return cuda_status(e);
   return QLORA_OK;
+}
+
+size_t decode_scratch_bytes(const DecodePlan& p, const LinearShape& s) {
+  return part_bytes(p, s) + t_bytes(s) + counter_bytes(p);
 }
 
 }  // namespace
 
 size_t decode_workspace(const LinearShape& s) {
-  const DecodePlan p = plan_decode(s);
-  return part_bytes(p, s) + tpart_bytes(p, s) + 256;
+  return decode_scratch_bytes(plan_decode(s), s) + 256;
 }
 
 qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
@@ -455,8 +543,8 @@ extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_
   const LinearShape s{M, w.n_out, w.k_in, r, scale};
   DecodePlan p = plan_decode(s);
   // Fewer K splits when the planned partial sums do not fit the static array.
-  const size_t per_split = static_cast<size_t>(M) * s.N * 4;
-  const size_t fixed = tpart_bytes(p, s) + 512;
+  const size_t per_split = static_cast<size_t>(p.row_groups) * M * 32 * 4;
+  const size_t fixed = t_bytes(s) + counter_bytes(p) + 512;
   const size_t fit = fixed < kStaticScratchBytes ? (kStaticScratchBytes - fixed) / per_split : 0;
   if (fit < 1) {
     char msg[200];
@@ -474,8 +562,8 @@ extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_
   void* scratch = nullptr;
   qlora_status q = scratch_address(&scratch);
   if (q != QLORA_OK) return q;
-  // Every partial sum the finalize kernel reads is written by the GEMV first, so
-  // nothing left in the array by an earlier call needs clearing.
+  // Every partial sum is written by the GEMV before it is read, and the T kernel clears
+  // the arrival counters, so nothing left in the array by an earlier call matters.
   return launch_decode(X, w, A, B, s, p, Y, T_save, static_cast<char*>(scratch),
                        static_cast<cudaStream_t>(stream));
 }

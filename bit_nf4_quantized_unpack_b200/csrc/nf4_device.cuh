@@ -66,18 +66,21 @@ __device__ __forceinline__ void build_lut(float s, Nf4Lut& t) {
 
 // Eight 4-bit codes (nibble i of w = code of element i) -> four bf16x2 registers
 // o[i] = (element 2i in the low half, element 2i+1 in the high half).
-// Bits 0-2 of a code index a byte inside an 8-byte prmt window; bit 3 picks the
-// window (entries 0-7 or 8-15) through a byte mask.
+// The raw codes serve as prmt selectors: bits 0-2 index a byte of an 8-byte window
+// (entries 0-7, or entries 8-15 with bit 3 flipped), and a selector whose bit 3 is set
+// replicates a sign bit instead of copying, which only happens in the window that the
+// byte mask then discards. The mask itself is a sign replication too: byte j of w has
+// bit 3 of code 2j+1 as its sign bit, byte j of w << 4 that of code 2j.
 __device__ __forceinline__ void lut_decode8(uint32_t w, const Nf4Lut& t, uint32_t (&o)[4]) {
-  const uint32_t sel = w & 0x77777777u;
-  const uint32_t msel = ((w >> 3) & 0x11111111u) * 9u;  // nibble 9 -> 0xFF byte, 0 -> 0x00
+  const uint32_t w4 = w << 4;
+  const uint32_t wx = w ^ 0x88888888u;  // selectors into entries 8-15
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t s4 = h ? (sel >> 16) : sel;
-    const uint32_t m4 = h ? (msel >> 16) : msel;
-    const uint32_t mask = prmt(0x00008000u, 0u, m4);
-    const uint32_t lo = (prmt(t.lo[0], t.lo[1], s4) & ~mask) | (prmt(t.lo[2], t.lo[3], s4) & mask);
-    const uint32_t hi = (prmt(t.hi[0], t.hi[1], s4) & ~mask) | (prmt(t.hi[2], t.hi[3], s4) & mask);
+    const uint32_t s = h ? (w >> 16) : w;
+    const uint32_t sx = h ? (wx >> 16) : wx;
+    const uint32_t mask = prmt(w, w4, h ? 0xBFAEu : 0x9D8Cu);  // 0xFF where the code is >= 8
+    const uint32_t lo = (prmt(t.lo[0], t.lo[1], s) & ~mask) | (prmt(t.lo[2], t.lo[3], sx) & mask);
+    const uint32_t hi = (prmt(t.hi[0], t.hi[1], s) & ~mask) | (prmt(t.hi[2], t.hi[3], sx) & mask);
     o[2 * h] = prmt(lo, hi, 0x5140u);
     o[2 * h + 1] = prmt(lo, hi, 0x7362u);
   }

@@ -188,8 +188,9 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, qlora_nf4_weight w,
  * counterpart of this entry point; it is a deployment convenience.
  *   Arguments, layouts and results are those of qlora_linear_fwd with M <= 16.
  *   Scratch: a fixed 4 MiB array in device memory inside this library, which every
- *   GPU that loads the library holds until the process exits. It must hold
- *   M * (N + r) * 4 bytes for at least one split of K; larger problems are rejected
+ *   GPU that loads the library holds until the process exits. It must hold one
+ *   K split of fp32 partial sums (M * 32 * ceil(N / 32) * 4 bytes), T (M * r * 4
+ *   bytes) and one counter per 32 rows of W; larger problems are rejected
  *   with QLORA_ERR_WORKSPACE (qlora_last_error() gives the sizes), M > 16 with
  *   QLORA_ERR_SHAPE. When the usual number of K splits does not fit, fewer are used.
  *   The first call on each device looks up the array's device address (with that
