@@ -40,7 +40,7 @@ INPUT_OF = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out",
 KERNELS_PER_LINEAR_STEP = 3 + 8   # forward 3 launches, backward 8 launches
 # dram__bytes_read.sum + dram__bytes_write.sum per FLOP of k_fused_nf4_gemm, from one ncu
 # capture of the current kernel (forward + dX of the 11008 x 4096 linear at M = 4096)
-FUSED_DRAM_BYTES_PER_FLOP = (118.8e6 + 145.2e6) / (3.751e11 + 3.715e11)
+FUSED_DRAM_BYTES_PER_FLOP = (118.751e6 + 170.849e6) / (3.751e11 + 3.715e11)
 
 
 def layer_flops(linears, M, r):
@@ -60,55 +60,82 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons sampled through NVML every few
+    milliseconds, from start() to stop() only: the timed region of a step loop lasts tens
+    of milliseconds, far shorter than nvidia-smi's -lms sampling can resolve. Falls back
+    to one nvidia-smi query per sample when NVML is unavailable."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device, period_s=0.002):
+        self.device = device
+        self.period = period_s
+        self.samples = []  # (sm_mhz, reason bits)
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        self._nvml = None
+        self.source = "nvml"
+
+    def _open(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(self.device)
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nvml, self._handle = pynvml, h
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self._nvml = None
+            self.source = "nvidia-smi"
+
+    def _sample(self):
+        if self._nvml is not None:
+            n = self._nvml
+            mhz = float(n.nvmlDeviceGetClockInfo(self._handle, n.NVML_CLOCK_SM))
+            bits = int(n.nvmlDeviceGetCurrentClocksEventReasons(self._handle))
+            return mhz, bits
+        props = torch.cuda.get_device_properties(self.device)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        out = subprocess.run(
+            ["nvidia-smi", "-i", bus,
+             "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+             "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+        parts = [x.strip() for x in out.stdout.split(",")]
+        self.max_mhz = float(parts[1])
+        return float(parts[0]), int(parts[2], 16)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._sample())
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            threading.Thread(target=self._read, daemon=True).start()
-        except OSError:
-            self.proc = None
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+        self._open()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[3:7]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=10)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no clock samples"],
+                    "samples": 0, "source": self.source}
+        reasons = sorted({name for _, bits in self.samples for name, bit in self.REASONS
+                          if bits & bit})
+        mhz = [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(mhz),
+                "source": self.source}
 
 
 # ------------------------------------------------------------------ oracle (CPU) leg
@@ -468,7 +495,7 @@ def main():
     if qlora.qlora_device_error() != 0:
         raise RuntimeError("a kernel reported a timed-out wait")
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(device)
     clocks.start()
     ms = time_steps(step, args.steps, world)
     clk = clocks.stop()
