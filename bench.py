@@ -59,83 +59,88 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ clocks
+_SAMPLER = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+key = sys.argv[1]
+h = (pynvml.nvmlDeviceGetHandleByUUID(key) if key.startswith("GPU-")
+     else pynvml.nvmlDeviceGetHandleByPciBusId(key))
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    t = time.monotonic()
+    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+    print(t, mhz, bits, flush=True)
+    time.sleep(0.001)
+"""
+
+
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons sampled through NVML every few
-    milliseconds, from start() to stop() only: the timed region of a step loop lasts tens
-    of milliseconds, far shorter than nvidia-smi's -lms sampling can resolve. Falls back
-    to one nvidia-smi query per sample when NVML is unavailable."""
+    """SM clock and clock-event (throttle) reasons, polled through NVML about every
+    millisecond by a separate process (a thread of this one would compete for the GIL
+    with the launch loop), and kept only between mark() and stop(): the timed region of
+    a step loop lasts tens of milliseconds, far shorter than nvidia-smi's -lms sampling
+    can resolve."""
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
                ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, device, period_s=0.002):
+    def __init__(self, device):
         self.device = device
-        self.period = period_s
-        self.samples = []  # (sm_mhz, reason bits)
+        self.proc = None
+        self.lines = []
         self.max_mhz = None
-        self._stop = threading.Event()
-        self._thread = None
-        self._handle = None
-        self._nvml = None
-        self.source = "nvml"
-
-    def _open(self):
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            props = torch.cuda.get_device_properties(self.device)
-            try:
-                h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
-            except Exception:
-                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-            self._nvml, self._handle = pynvml, h
-            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
-        except Exception:
-            self._nvml = None
-            self.source = "nvidia-smi"
-
-    def _sample(self):
-        if self._nvml is not None:
-            n = self._nvml
-            mhz = float(n.nvmlDeviceGetClockInfo(self._handle, n.NVML_CLOCK_SM))
-            bits = int(n.nvmlDeviceGetCurrentClocksEventReasons(self._handle))
-            return mhz, bits
-        props = torch.cuda.get_device_properties(self.device)
-        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-        out = subprocess.run(
-            ["nvidia-smi", "-i", bus,
-             "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
-             "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-        parts = [x.strip() for x in out.stdout.split(",")]
-        self.max_mhz = float(parts[1])
-        return float(parts[0]), int(parts[2], 16)
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self.samples.append(self._sample())
-            except Exception:
-                pass
-            time.sleep(self.period)
+        self.t0 = None
+        self._ready = threading.Event()
 
     def start(self):
-        self._open()
-        self._thread = threading.Thread(target=self._run, daemon=True)
-        self._thread.start()
+        props = torch.cuda.get_device_properties(self.device)
+        key = "GPU-" + str(props.uuid)
+        try:
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER, key],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+        self._ready.wait(timeout=60)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = line.split()
+            if parts and parts[0] == "max":
+                self.max_mhz = float(parts[1])
+                self._ready.set()
+            elif len(parts) == 3:
+                self.lines.append((float(parts[0]), float(parts[1]), int(parts[2])))
+        self._ready.set()
+
+    def mark(self):
+        """Opens the window of kept samples (call right before the timed region)."""
+        self.t0 = time.monotonic()
 
     def stop(self):
-        self._stop.set()
-        if self._thread is not None:
-            self._thread.join(timeout=10)
-        if not self.samples:
+        t1 = time.monotonic()
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampler unavailable"],
+                    "samples": 0}
+        time.sleep(0.01)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        t0 = self.t0 if self.t0 is not None else 0.0
+        kept = [(m, b) for t, m, b in self.lines if t0 <= t <= t1]
+        if not kept:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no clock samples"],
-                    "samples": 0, "source": self.source}
-        reasons = sorted({name for _, bits in self.samples for name, bit in self.REASONS
-                          if bits & bit})
-        mhz = [m for m, _ in self.samples]
+                    "samples": 0, "source": "nvml"}
+        reasons = sorted({name for _, bits in kept for name, bit in self.REASONS if bits & bit})
+        mhz = [m for m, _ in kept]
         return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz),
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(mhz),
-                "source": self.source}
+                "source": "nvml"}
 
 
 # ------------------------------------------------------------------ oracle (CPU) leg
@@ -388,25 +393,93 @@ def codec_bandwidth(device, reps=5):
 
 def e2e_steps(L, scale, world, steps):
     """The same step through the public API with host-resident inputs: every step copies
-    the activations and upstream gradients from pinned host memory and reads the LoRA
-    gradients back."""
+    its activations and upstream gradients from pinned host memory and reads its LoRA
+    gradients back. The copies run on a stream of their own into two sets of device
+    buffers, so that step i + 1's inputs arrive, and step i's gradients leave, while step
+    i computes (a data loader's prefetch). The timed region spans all copies: it opens
+    before the first input copy and closes after the last gradient read."""
+    dev = L["grads"].device
     host_x = {k: v.cpu().pin_memory() for k, v in L["xs"].items()}
     host_dy = [lin["dY"].cpu().pin_memory() for lin in L["layer"]]
-    host_grads = torch.empty(L["grads"].shape, dtype=torch.float32).pin_memory()
+    host_grads = [torch.empty(L["grads"].shape, dtype=torch.float32).pin_memory()
+                  for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_x.values()) + \
         sum(t.numel() * t.element_size() for t in host_dy)
-    d2h = host_grads.numel() * 4
+    d2h = host_grads[0].numel() * 4
 
-    def step():
-        for k, v in host_x.items():
-            L["xs"][k].copy_(v, non_blocking=True)
-        for lin, h in zip(L["layer"], host_dy):
-            lin["dY"].copy_(h, non_blocking=True)
+    def make_set(first):
+        if first:
+            xs, dys, grads = L["xs"], [lin["dY"] for lin in L["layer"]], L["grads"]
+        else:
+            xs = {k: torch.empty_like(v) for k, v in L["xs"].items()}
+            dys = [torch.empty_like(lin["dY"]) for lin in L["layer"]]
+            grads = torch.empty_like(L["grads"])
+        views, off = [], 0
+        for lin in L["layer"]:
+            nA, nB = lin["k"] * RANK_R, RANK_R * lin["n"]
+            views.append((grads[off:off + nA].view(lin["k"], RANK_R),
+                          grads[off + nA:off + nA + nB].view(RANK_R, lin["n"])))
+            off += nA + nB
+        return dict(xs=xs, dys=dys, grads=grads, views=views)
+
+    sets = [make_set(True), make_set(False)]
+    compute = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    read_back = [torch.cuda.Event() for _ in range(2)]
+
+    def enqueue_inputs(i):
+        S = sets[i % 2]
+        with torch.cuda.stream(copy):
+            if i >= 2:
+                copy.wait_event(computed[i % 2])  # step i - 2 no longer reads this set
+            for k, v in host_x.items():
+                S["xs"][k].copy_(v, non_blocking=True)
+            for d, h in zip(S["dys"], host_dy):
+                d.copy_(h, non_blocking=True)
+            copied[i % 2].record(copy)
+
+    def run(i):
+        S = sets[i % 2]
+        compute.wait_event(copied[i % 2])
+        if i >= 2:
+            compute.wait_event(read_back[i % 2])  # step i - 2's gradients have left
+        L["xs"], L["grads"] = S["xs"], S["grads"]
+        for lin, d, (dA, dB) in zip(L["layer"], S["dys"], S["views"]):
+            lin["dY"], lin["dA"], lin["dB"] = d, dA, dB
         layer_step(L, scale, world)
-        host_grads.copy_(L["grads"], non_blocking=True)
+        computed[i % 2].record(compute)
+        with torch.cuda.stream(copy):
+            copy.wait_event(computed[i % 2])
+            host_grads[i % 2].copy_(S["grads"], non_blocking=True)
+            read_back[i % 2].record(copy)
 
-    step()
-    ms = time_steps(step, steps, world)
+    def timed(n):
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(compute)
+        copy.wait_event(start)
+        enqueue_inputs(0)
+        for i in range(n):
+            if i + 1 < n:
+                enqueue_inputs(i + 1)
+            run(i)
+        compute.wait_event(read_back[(n - 1) % 2])
+        stop.record(compute)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        return max_over_ranks(start.elapsed_time(stop) / n, world, "cuda")
+
+    timed(2)  # warm-up of both buffer sets
+    ms = timed(steps)
+    restore = sets[0]
+    L["xs"], L["grads"] = restore["xs"], restore["grads"]
+    for lin, d, (dA, dB) in zip(L["layer"], restore["dys"], restore["views"]):
+        lin["dY"], lin["dA"], lin["dB"] = d, dA, dB
     return ms, h2d, d2h
 
 
@@ -497,6 +570,7 @@ def main():
 
     clocks = ClockSampler(device)
     clocks.start()
+    clocks.mark()
     ms = time_steps(step, args.steps, world)
     clk = clocks.stop()
     value = world * flops / (ms / 1e3) / 1e12

@@ -453,13 +453,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         tc_fence_after();
         const uint32_t taddr =
             tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + h * kHalfCols;
-#pragma unroll 1
-        for (int c = 0; c < kHalfCols / 32; ++c) {
-          const int64_t mb = m0 + h * kHalfCols + c * 32;
-          if (mb >= args.M) break;  // warp-uniform
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, v);
-          tmem_ld_wait();
+        // one 32-token chunk: TMEM values -> bf16 -> stage[token][row] -> 16-byte stores
+        auto store_chunk = [&](const uint32_t (&v)[32], int64_t mb) {
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
             const uint32_t pk = pack_bf16x2_rn(__uint_as_float(v[k]), __uint_as_float(v[k + 1]));
@@ -485,6 +480,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             }
           }
           __syncwarp();
+        };
+        // two chunks per TMEM round trip: both loads are in flight before one wait
+#pragma unroll 1
+        for (int c = 0; c < kHalfCols / 32; c += 2) {
+          const int64_t mb = m0 + h * kHalfCols + c * 32;
+          if (mb >= args.M) break;  // warp-uniform
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, v0);
+          tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v1);
+          tmem_ld_wait();
+          store_chunk(v0, mb);
+          if (mb + 32 < args.M) store_chunk(v1, mb + 32);
         }
         tc_fence_before();
         __syncwarp();
