@@ -351,7 +351,7 @@ def decode_bandwidth(device, M=1, iters=40):
 def codec_bandwidth(device, reps=5):
     """HBM throughput of quantization (bf16 in) and double dequantization (bf16 out) over
     the three Llama-7B weight shapes, cycled so that no pass finds its data in L2 (the
-    three matrices hold 107M parameters, 267 MB per pass)."""
+    three matrices hold 107M parameters, 267 MB per pass); CUDA-graph timed."""
     from bit_nf4_quantized_unpack_b200 import qlora
     g = torch.Generator(device=device)
     g.manual_seed(1)
@@ -376,15 +376,23 @@ def codec_bandwidth(device, reps=5):
                     qlora.qlora_quantize_nf4_dq(W, out=q, workspace=ws)
                 else:
                     qlora.qlora_dequant(q, out=o)
-        one_pass()
-        one_pass()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
+        s = torch.cuda.Stream(device)
+        with torch.cuda.stream(s):
             one_pass()
-        e1.record()
-        torch.cuda.synchronize()
+            one_pass()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()  # the passes' kernels only, no host work between them
+            with torch.cuda.graph(graph, stream=s):
+                for _ in range(reps):
+                    one_pass()
+            graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            graph.replay()
+            e1.record(s)
+            torch.cuda.synchronize()
+        del graph
         us = e0.elapsed_time(e1) * 1000.0 / reps
         out[name] = {"us_per_pass": us, "params": params, "bytes_per_param": per_param,
                      "GBps": params * per_param / us / 1e3}

@@ -12,65 +12,82 @@ namespace {
 constexpr int kQuantThreads = 256;
 constexpr int kMaxQuantCtas = 148 * 8;
 
-// NF4 code of x in [-1, 1]: the number of thresholds <= x, by a 4-level bisection over
-// thresholds held in registers.
-__device__ __forceinline__ uint32_t nf4_code(float x, const float (&t)[15]) {
-  uint32_t c = (x >= t[7]) ? 8u : 0u;
-  const float t1 = c ? t[11] : t[3];
-  c += (x >= t1) ? 4u : 0u;
-  const float t2 = (c & 8u) ? ((c & 4u) ? t[13] : t[9]) : ((c & 4u) ? t[5] : t[1]);
-  c += (x >= t2) ? 2u : 0u;
-  const float a0 = (c & 4u) ? t[4] : t[0];
-  const float a1 = (c & 4u) ? t[6] : t[2];
-  const float b0 = (c & 4u) ? t[12] : t[8];
-  const float b1 = (c & 4u) ? t[14] : t[10];
-  const float lo = (c & 2u) ? a1 : a0;
-  const float hi = (c & 2u) ? b1 : b0;
-  const float t3 = (c & 8u) ? hi : lo;
-  c += (x >= t3) ? 1u : 0u;
-  return c;
-}
-
-__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void load8(const uint16_t* p, float (&v)[8]) {
-  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+// Eight consecutive weights as loaded (kept raw until they are used, so that a prefetch
+// does not wait for its data) and their fp32 values.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
   }
+  __device__ __forceinline__ void values(float (&v)[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+template <>
+struct Raw8<uint16_t> {  // bf16
+  uint4 a;
+  __device__ __forceinline__ void load(const uint16_t* p) { a = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void values(float (&v)[8]) const {
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+
+// NF4 code of x in [-1, 1] from the bucket table in shared memory (entries: threshold,
+// code as bits): bucket = round-half-even(512 x + 512), which the FMA leaves in the low
+// mantissa bits of a number in [2^23, 2^24).
+__device__ __forceinline__ uint32_t bucket_code(float x, const float2* sb) {
+  const uint32_t idx =
+      min(static_cast<uint32_t>(__float_as_int(__fmaf_rn(x, 512.0f, 12583424.0f)) - 0x4B400000),
+          static_cast<uint32_t>(kCodeBuckets - 1));
+  const float2 bk = sb[idx];
+  return __float_as_uint(bk.y) + (x >= bk.x ? 1u : 0u);
 }
 
 // Level 1: one 64-block per group of 8 lanes (8 elements per lane). Writes the packed
 // codes, the fp32 absmax of each block, and one fp64 partial sum of absmax per CTA.
+//
+// x = fl32(w / absmax) is computed with Markstein's correction step (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor", IBM J.
+// Res. Dev. 34, 1990): with r = RN(1/m), q = RN(w r) and e = w - m q (exact in an FMA),
+// RN(q + e r) is the correctly rounded quotient. For m >= 2^-64, 1/m is finite and the
+// residual stays exact for every |x| above 2^-36, far below the smallest threshold
+// magnitude (0.04); blocks with a smaller absmax take plain IEEE division.
+// The code of x comes from the 1025-bucket table (one shared-memory load and one compare).
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
-    k_quantize_blocks(const T* __restrict__ W, int64_t nblocks, const Nf4Thresholds th,
-                      uint8_t* __restrict__ codes, float* __restrict__ absmax,
-                      double* __restrict__ partial) {
+    k_quantize_blocks(const T* __restrict__ W, int64_t nblocks,
+                      const __grid_constant__ Nf4BucketTable tab, uint8_t* __restrict__ codes,
+                      float* __restrict__ absmax, double* __restrict__ partial) {
   const int lane = threadIdx.x & 31;
   const int sub = lane & 7;
   const unsigned gmask = 0xFFu << (lane & 24);
   const int64_t per_cta = kQuantThreads / 8;
-  // thresholds through shared memory into registers (kept out of the constant bank,
-  // which the bisection would otherwise index)
-  __shared__ float sth[15];
-  if (threadIdx.x < 15) sth[threadIdx.x] = th.t[threadIdx.x];
+  __shared__ float2 sb[kCodeBuckets];  // (threshold, code as bits)
+  for (int i = threadIdx.x; i < kCodeBuckets; i += blockDim.x)
+    sb[i] = make_float2(tab.thr[i], __uint_as_float(static_cast<uint32_t>(tab.code[i])));
   __syncthreads();
-  float t[15];
-#pragma unroll
-  for (int i = 0; i < 15; ++i) t[i] = sth[i];
   double acc = 0.0;
-  for (int64_t b = blockIdx.x * per_cta + threadIdx.x / 8; b < nblocks;
-       b += static_cast<int64_t>(gridDim.x) * per_cta) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * per_cta;
+  int64_t b = blockIdx.x * per_cta + threadIdx.x / 8;
+  // the next two blocks' elements are in flight while this one is coded
+  Raw8<T> n0, n1;
+  if (b < nblocks) n0.load(W + b * 64 + sub * 8);
+  if (b + stride < nblocks) n1.load(W + (b + stride) * 64 + sub * 8);
+  for (; b < nblocks; b += stride) {
     float v[8];
-    load8(W + b * 64 + sub * 8, v);
+    n0.values(v);
+    n0 = n1;
+    if (b + 2 * stride < nblocks) n1.load(W + (b + 2 * stride) * 64 + sub * 8);
     float m = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
@@ -78,10 +95,19 @@ __global__ void __launch_bounds__(kQuantThreads)
     m = fmaxf(m, __shfl_xor_sync(gmask, m, 2));
     m = fmaxf(m, __shfl_xor_sync(gmask, m, 4));
     uint32_t packed = 0;
+    if (m >= 0x1p-64f) {
+      const float r = __fdiv_rn(1.0f, m);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float x = (m > 0.f) ? __fdiv_rn(v[i], m) : 0.f;
-      packed |= nf4_code(x, t) << (4 * i);
+      for (int i = 0; i < 8; ++i) {
+        const float w = v[i];
+        const float q = __fmul_rn(w, r);
+        const float e = __fmaf_rn(-q, m, w);
+        packed |= bucket_code(__fmaf_rn(e, r, q), sb) << (4 * i);
+      }
+    } else {  // absmax zero or below 2^-64: plain IEEE division (x = 0 for a zero block)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        packed |= bucket_code(m > 0.f ? __fdiv_rn(v[i], m) : 0.f, sb) << (4 * i);
     }
     reinterpret_cast<uint32_t*>(codes + b * 32)[sub] = packed;
     if (sub == 0) {
@@ -216,10 +242,10 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, ui
   const int ctas = quant_ctas(nblocks);
   if (w_bf16)
     k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const uint16_t*>(W), nblocks, nf4_thresholds(), codes, absmax, partial);
+        static_cast<const uint16_t*>(W), nblocks, nf4_buckets(), codes, absmax, partial);
   else
     k_quantize_blocks<float><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const float*>(W), nblocks, nf4_thresholds(), codes, absmax, partial);
+        static_cast<const float*>(W), nblocks, nf4_buckets(), codes, absmax, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_constants_mean<<<1, 1024, 0, st>>>(partial, ctas, nblocks, mean);

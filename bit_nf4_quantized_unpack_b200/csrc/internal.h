@@ -16,6 +16,15 @@ namespace qlora {
 extern const uint32_t kNf4Bits[16];
 constexpr int kT8Size = 253;  // distinct finite E4M3 values
 struct Nf4Thresholds { float t[15]; };
+// NF4 codes by table: bucket b = round-half-even(512 x + 512) of x in [-1, 1] (1025
+// buckets); within bucket b the code is code[b] + (x >= thr[b]) (thr = +inf when no
+// threshold falls inside the bucket; no bucket holds two).
+constexpr int kCodeBuckets = 1025;
+struct Nf4BucketTable {
+  float thr[kCodeBuckets];
+  uint8_t code[kCodeBuckets + 3];
+};
+const Nf4BucketTable& nf4_buckets();
 struct T8Thresholds { float t[kT8Size - 1]; };
 const Nf4Thresholds& nf4_thresholds();
 const T8Thresholds& t8_thresholds();

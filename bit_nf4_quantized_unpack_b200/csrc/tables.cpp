@@ -18,7 +18,9 @@
 // i is the smallest fp32 x whose index exceeds i. They are found here by bisection
 // over the ordered fp32 bit patterns, evaluating the argmin rule itself.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
+#include <limits>
 #include <mutex>
 
 #include "internal.h"
@@ -90,6 +92,7 @@ float e4m3_value(uint32_t b) {
 
 struct Tables {
   Nf4Thresholds nf4;
+  Nf4BucketTable buckets;
   T8Thresholds t8;
   float t8_vals[kT8Size];
   uint8_t t8_code[kT8Size];
@@ -102,6 +105,28 @@ const Tables& tables() {
     float nf4[16];
     for (int i = 0; i < 16; ++i) nf4[i] = bits_to_float(kNf4Bits[i]);
     for (int i = 0; i < 15; ++i) tab.nf4.t[i] = first_above(nf4, 16, i);
+    // Bucket b holds the fp32 x with round-half-even(512 x + 512) == b: its edges are
+    // (2b -+ 1 - 1024) / 1024, each tie going to the even bucket.
+    for (int b = 0; b < kCodeBuckets; ++b) {
+      float xmin = static_cast<float>((2.0 * b - 1025.0) / 1024.0);
+      float xmax = static_cast<float>((2.0 * b - 1023.0) / 1024.0);
+      if (b & 1) {
+        xmin = std::nextafter(xmin, std::numeric_limits<float>::infinity());
+        xmax = std::nextafter(xmax, -std::numeric_limits<float>::infinity());
+      }
+      int code = 0;
+      for (int i = 0; i < 15; ++i) code += (xmin >= tab.nf4.t[i]) ? 1 : 0;
+      float thr = std::numeric_limits<float>::infinity();
+      int inside = 0;
+      for (int i = 0; i < 15; ++i)
+        if (tab.nf4.t[i] > xmin && tab.nf4.t[i] <= xmax) {
+          thr = tab.nf4.t[i];
+          ++inside;
+        }
+      if (inside > 1) std::abort();  // the table form needs at most one threshold per bucket
+      tab.buckets.thr[b] = thr;
+      tab.buckets.code[b] = static_cast<uint8_t>(code);
+    }
     // T8 in ascending order: -448 .. -min (0xFE .. 0x81), 0 (0x00), +min .. +448.
     int n = 0;
     for (int b = 0xFE; b >= 0x81; --b) tab.t8_code[n++] = static_cast<uint8_t>(b);
@@ -120,6 +145,7 @@ const Tables& tables() {
 }  // namespace
 
 const Nf4Thresholds& nf4_thresholds() { return tables().nf4; }
+const Nf4BucketTable& nf4_buckets() { return tables().buckets; }
 const T8Thresholds& t8_thresholds() { return tables().t8; }
 const float* t8_values() { return tables().t8_vals; }
 const uint8_t* t8_codes() { return tables().t8_code; }
@@ -135,6 +161,14 @@ extern "C" void qlora_nf4_thresholds(float* out15) {
   if (!out15) return;
   const auto& t = qlora::nf4_thresholds();
   for (int i = 0; i < 15; ++i) out15[i] = t.t[i];
+}
+
+extern "C" void qlora_nf4_code_buckets(float* thr1025, uint8_t* code1025) {
+  const auto& t = qlora::nf4_buckets();
+  for (int i = 0; i < qlora::kCodeBuckets; ++i) {
+    if (thr1025) thr1025[i] = t.thr[i];
+    if (code1025) code1025[i] = t.code[i];
+  }
 }
 
 extern "C" void qlora_fp8_thresholds(float* out252, float* t8_out253, uint8_t* codes_out253) {

@@ -48,6 +48,7 @@ _SIGNATURES = {
     "qlora_profile_events": (None, [_vp, _vp]),
     "qlora_nf4_table": (None, [_vp]),
     "qlora_nf4_thresholds": (None, [_vp]),
+    "qlora_nf4_code_buckets": (None, [_vp, _vp]),
     "qlora_fp8_thresholds": (None, [_vp, _vp, _vp]),
     "qlora_quantize_workspace_size": (_sz, [_i64, _i64]),
     "qlora_quantize_nf4_dq": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -135,6 +136,15 @@ def nf4_thresholds() -> torch.Tensor:
     out = (ctypes.c_float * 15)()
     lib().qlora_nf4_thresholds(ctypes.cast(out, ctypes.c_void_p))
     return torch.tensor(list(out), dtype=torch.float32)
+
+
+def nf4_code_buckets():
+    """(thr [1025] fp32, code [1025] uint8): the bucket table of the quantization kernel."""
+    thr = (ctypes.c_float * 1025)()
+    code = (ctypes.c_uint8 * 1025)()
+    lib().qlora_nf4_code_buckets(ctypes.cast(thr, ctypes.c_void_p), ctypes.cast(code, ctypes.c_void_p))
+    return (torch.tensor(list(thr), dtype=torch.float32),
+            torch.tensor(list(code), dtype=torch.uint8))
 
 
 def fp8_thresholds():

@@ -121,6 +121,15 @@ void qlora_nf4_table(float *out16);
 void qlora_nf4_thresholds(float *out15);
 
 /*
+ * qlora_nf4_code_buckets: the table form of the same code search that the
+ * quantization kernel uses, to host memory. For fp32 x in [-1, 1] let
+ * b = round-half-even(512 x + 512) (0 <= b <= 1024); then
+ * code(x) = code1025[b] + (x >= thr1025[b] ? 1 : 0), with thr1025[b] = +inf when no
+ * threshold lies in bucket b. Either pointer may be NULL. Host-only.
+ */
+void qlora_nf4_code_buckets(float *thr1025, uint8_t *code1025);
+
+/*
  * qlora_fp8_thresholds: the same for the 253-entry double-quantization table T8
  * (distinct finite E4M3 values / 448, ascending): 252 thresholds to host memory
  * `out252`; also writes T8 itself to `t8_out253` and the E4M3 bit pattern of each

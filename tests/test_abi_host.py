@@ -77,6 +77,28 @@ def test_nf4_thresholds_reproduce_argmin(L):
     assert np.array_equal(O.nearest_code(x, table), _count_leq(th, x))
 
 
+def test_nf4_code_buckets_reproduce_argmin(L):
+    """The quantization kernel's table form of the code search: bucket
+    b = round-half-even(512 x + 512), code = code[b] + (x >= thr[b]); checked against the
+    oracle's argmin on random x, around every threshold and level, and on both sides of
+    every bucket edge."""
+    thr, code = (t.numpy() for t in qlora.nf4_code_buckets())
+    table = O.nf4_levels()
+    th = qlora.nf4_thresholds().numpy()
+    xs = [np.random.default_rng(2).uniform(-1, 1, 1 << 18).astype(np.float32), table,
+          np.array([-1.0, 1.0, 0.0, -0.0], np.float32)]
+    for t in th:
+        xs.append(_ulp_window(t, 256))
+    edges = ((2.0 * np.arange(1026) - 1025.0) / 1024.0).astype(np.float32)
+    for e in edges:
+        xs.append(_ulp_window(e, 3))
+    x = np.concatenate(xs)
+    x = x[(x >= -1) & (x <= 1)]
+    b = np.rint(512.0 * x.astype(np.float64) + 512.0).astype(np.int64)  # rint: half to even
+    got = code[b].astype(np.int64) + (x >= thr[b]).astype(np.int64)
+    assert np.array_equal(O.nearest_code(x, table), got)
+
+
 def test_fp8_table_and_thresholds_match_oracle(L):
     th, vals, codes = (t.numpy() for t in qlora.fp8_thresholds())
     ovals, ocodes = O.fp8_table()

@@ -61,6 +61,17 @@ def test_edge_values():
     W[4] = 1e-30                               # tiny magnitudes
     W[5, :64] = -0.5                           # constant blocks
     W[6, 64:128] = np.float32(2.0 ** -20) * np.arange(64)
+    # absmax on both sides of 2^-64 (the quantizer's switch between its reciprocal-based
+    # and its plain division), subnormal elements, and a block of subnormals only
+    W[7, :64] = rng.normal(0, 1, 64) * 2.0 ** -62
+    W[7, 64:128] = rng.normal(0, 1, 64) * 2.0 ** -66
+    W[7, 128:192] = rng.normal(0, 1, 64) * 2.0 ** -66
+    W[7, 130] = 2.0 ** -64
+    W[7, 192:256] = rng.normal(0, 1, 64) * 2.0 ** -66
+    W[7, 200] = np.nextafter(np.float32(2.0 ** -64), np.float32(0))
+    W[8, :64] = rng.normal(0, 1, 64) * 1e-40
+    W[8, 64:128] = rng.normal(0, 1, 64) * 1e-40
+    W[8, 100] = 0.03
     compare_full(W, bf16=False)
 
 
