@@ -349,14 +349,15 @@ def decode_bandwidth(device, M=1, iters=40):
 
 
 def codec_bandwidth(device, reps=5):
-    """HBM throughput of quantization (bf16 in) and double dequantization (bf16 out) over
+    """HBM throughput of quantization (bf16 in), double dequantization (bf16 out) and
+    merge_and_unload (bf16 out, r = 64 adapter) over
     the three Llama-7B weight shapes, cycled so that no pass finds its data in L2 (the
     three matrices hold 107M parameters, 267 MB per pass); CUDA-graph timed."""
     from bit_nf4_quantized_unpack_b200 import qlora
     g = torch.Generator(device=device)
     g.manual_seed(1)
     shapes = [(4096, 4096), (4096, 11008), (11008, 4096)]
-    Ws, Qs, Outs, wss = [], [], [], []
+    Ws, Qs, Outs, wss, As, Bs = [], [], [], [], [], []
     for n, k in shapes:
         W = torch.randn(n, k, generator=g, device=device) * 0.02
         mask = torch.rand(n, k, generator=g, device=device) < 1e-3   # 0.1 % outliers x10
@@ -364,18 +365,22 @@ def codec_bandwidth(device, reps=5):
         Ws.append(W)
         Qs.append(qlora.NF4Weight.empty(n, k, device))
         Outs.append(torch.empty(n, k, dtype=torch.bfloat16, device=device))
+        As.append((torch.randn(k, RANK_R, generator=g, device=device) * 0.02).to(torch.bfloat16))
+        Bs.append((torch.randn(RANK_R, n, generator=g, device=device) * 0.02).to(torch.bfloat16))
         wss.append(torch.empty(qlora.qlora_quantize_workspace_size(n, k), dtype=torch.uint8,
                                device=device))
     params = sum(n * k for n, k in shapes)
     per_param = 2.0 + 0.515869140625
     out = {}
-    for name in ("quantize", "dequant"):
+    for name in ("quantize", "dequant", "merge"):
         def one_pass():
-            for W, q, o, ws in zip(Ws, Qs, Outs, wss):
+            for W, q, o, ws, A, B in zip(Ws, Qs, Outs, wss, As, Bs):
                 if name == "quantize":
                     qlora.qlora_quantize_nf4_dq(W, out=q, workspace=ws)
-                else:
+                elif name == "dequant":
                     qlora.qlora_dequant(q, out=o)
+                else:  # merge_and_unload with the rank-64 adapter (A, B reads are 0.3 % extra)
+                    qlora.qlora_merge_lora(q, A, B, ALPHA / RANK_R, out=o)
         s = torch.cuda.Stream(device)
         with torch.cuda.stream(s):
             one_pass()
@@ -528,6 +533,20 @@ def profile_decode(device, warmup, steps, n=8192, k=28672, M=1, r=16, alpha=32.0
     torch.cuda.synchronize()
 
 
+def profile_merge(device, warmup, steps, n=4096, k=11008, r=RANK_R):
+    """merge_and_unload of one n x k weight with a rank-r adapter, for ncu captures."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    W = (torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    q = qlora.qlora_quantize_nf4_dq(W)
+    A = (torch.randn(k, r, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    B = (torch.randn(r, n, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    for _ in range(warmup + steps):
+        qlora.qlora_merge_lora(q, A, B, ALPHA / r, out=W)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -539,6 +558,8 @@ def main():
     ap.add_argument("--profile-decode", action="store_true",
                     help="only run the M=1 forward of an 8192x28672 weight --steps times "
                          "(no graph): a small, self-contained case for profiler captures")
+    ap.add_argument("--profile-merge", action="store_true",
+                    help="only run merge_and_unload of a 4096x11008 weight (r=64) --steps times")
     ap.add_argument("--profile-linear", action="store_true",
                     help="only run forward + backward of the gate linear (11008x4096, M=4096) "
                          "--steps times: a small, self-contained case for profiler captures")
@@ -560,6 +581,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     scale = ALPHA / RANK_R
+    if args.profile_merge:
+        profile_merge(device, args.warmup, args.steps)
+        return
     if args.profile_linear:
         profile_linear(device, scale, args.warmup, args.steps)
         return

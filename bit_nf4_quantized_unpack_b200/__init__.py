@@ -4,8 +4,9 @@ The compute lives in the C-ABI library ``lib/libqlora.so`` (CUDA, built from
 ``csrc/`` by ``build.py``); ``qlora`` is its thin ctypes binding and ``inputs``
 draws seeded synthetic workloads.
 """
-from .qlora import (NF4Weight, QLoraError, fp8_thresholds, lib, nf4_table, nf4_thresholds,  # noqa: F401
-                    qlora_dequant, qlora_device_error, qlora_linear_bwd,
+from .qlora import (NF4Weight, QLoraError, fp8_thresholds, lib, nf4_code_buckets,  # noqa: F401
+                    nf4_table, nf4_thresholds, qlora_dequant, qlora_device_error,
+                    qlora_linear_bwd, qlora_merge_lora,
                     qlora_linear_bwd_workspace_size, qlora_linear_fwd,
                     qlora_linear_fwd_workspace_size, qlora_profile_events, qlora_quantize_nf4_dq,
                     qlora_quantize_workspace_size)

@@ -236,6 +236,17 @@ qlora_status qlora_dequant(qlora_nf4_weight w, uint16_t* W_out, void* stream) {
   return cuda_status(launch_dequant(w, W_out, static_cast<cudaStream_t>(stream)));
 }
 
+qlora_status qlora_merge_lora(qlora_nf4_weight w, const uint16_t* A, const uint16_t* B, int r,
+                              float scale, uint16_t* W_out, void* stream) {
+  qlora_status q = check_linear(0, w, r, scale);
+  if (q != QLORA_OK) return q;
+  if (!A || !B || !W_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(W_out)) return QLORA_ERR_ALIGN;
+  q = check_device();
+  if (q != QLORA_OK) return q;
+  return cuda_status(launch_merge_lora(w, A, B, r, scale, W_out, static_cast<cudaStream_t>(stream)));
+}
+
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out < 1 || k_in < 64 || r < 8 || r > 64) return 0;
   const LinearShape s{M, n_out, k_in, r, 1.f};

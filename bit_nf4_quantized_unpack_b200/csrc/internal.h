@@ -51,6 +51,8 @@ cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_
 
 // ---- launchers (gemm.cu) --------------------------------------------------------
 struct LinearShape { int64_t M, N, K; int r; float scale; };
+cudaError_t launch_merge_lora(const qlora_nf4_weight& w, const uint16_t* A, const uint16_t* B,
+                              int r, float scale, uint16_t* out, cudaStream_t st);
 size_t gemm_fwd_workspace(const LinearShape& s);
 size_t gemm_bwd_workspace(const LinearShape& s);
 qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,

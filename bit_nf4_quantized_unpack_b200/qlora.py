@@ -53,6 +53,7 @@ _SIGNATURES = {
     "qlora_quantize_workspace_size": (_sz, [_i64, _i64]),
     "qlora_quantize_nf4_dq": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qlora_dequant": (_i32, [CNF4Weight, _vp, _vp]),
+    "qlora_merge_lora": (_i32, [CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp]),
     "qlora_linear_fwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
     "qlora_linear_fwd": (_i32, [_vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_linear_fwd_decode_static": (_i32, [_vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp,
@@ -185,6 +186,17 @@ def qlora_dequant(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor
     y = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16,
                                                 device=w.codes.device)
     _check(lib().qlora_dequant(w.c_struct(), _ptr(_as_bits(y)), _stream()), "qlora_dequant")
+    return y
+
+
+def qlora_merge_lora(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, scale: float,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """merge_and_unload: bf16(W_hat + scale (A B)^T) [N, K]; A [K, r], B [r, N] bf16."""
+    r = int(A.shape[1])
+    y = out if out is not None else torch.empty(w.n_out, w.k_in, dtype=torch.bfloat16,
+                                                device=w.codes.device)
+    _check(lib().qlora_merge_lora(w.c_struct(), _ptr(_as_bits(A)), _ptr(_as_bits(B)), r,
+                                  float(scale), _ptr(_as_bits(y)), _stream()), "qlora_merge_lora")
     return y
 
 

@@ -168,6 +168,23 @@ qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, int64_t n
  */
 qlora_status qlora_dequant(qlora_nf4_weight w, uint16_t *W_out, void *stream);
 
+/*
+ * qlora_merge_lora (merge_and_unload): W_out [n_out, k_in] bf16 (device) =
+ * bf16(W_hat + scale (A B)^T), W_hat = doubleDequant(c1, c2, W_NF4). After training, the
+ * base is dequantized to BF16 and the LoRA term added with its alpha/r scale (blog
+ * "QLoRA", irregular6612, sections "학습 → 추론 파이프라인 (실무)" and
+ * "재양자화 시 주의사항"; itwiki "QLoRA", section "한계와 주의점").
+ *   A [k_in, r] bf16 device, B [r, n_out] bf16 device (the layout of qlora_linear_fwd).
+ * Arithmetic: (A B)^T in fp32 on the tensor cores, then fl32(scale x it + W_hat) in one
+ * fused multiply-add, rounded to bf16. It equals the exactly rounded sum except where that sum lies
+ * within the fp32 error of a bf16 rounding boundary (then it may differ by one bf16 ulp).
+ * Errors: as qlora_linear_fwd for the weight, r and scale (n_out % 8 == 0, r in
+ * {8, 16, ..., 64}); QLORA_ERR_ALIGN unless A, B and W_out are 16-byte aligned.
+ * No workspace.
+ */
+qlora_status qlora_merge_lora(qlora_nf4_weight w, const uint16_t *A, const uint16_t *B, int r,
+                              float scale, uint16_t *W_out, void *stream);
+
 /* Device bytes of workspace qlora_linear_fwd needs (0 < r <= 64, r % 8 == 0). */
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r);
 

@@ -23,6 +23,10 @@ bf16/fp32 inputs. Sources, by page title and section:
   its worked example), "QLoRA에서 학습은 어떻게 되는 걸까?" (y = Wx + (alpha/r) B A x)
   and "그런데 Base Model은 4bit인데 학습이 가능한 이유는?" (W frozen, gradients for
   A and B only).
+* "QLoRA" (irregular6612 blog), section "학습 → 추론 파이프라인 (실무)" -- after
+  training, merge_and_unload dequantizes the base to BF16 and adds the LoRA term, with
+  the alpha/r scale (section "재양자화 시 주의사항"); itwiki "QLoRA", section
+  "한계와 주의점", on merging the adapter into a 16-bit weight.
 
 Readings where the pages are silent (each pinned or flagged in the tests):
 * nibble order: byte b holds code 2b in its low nibble and code 2b+1 in its high
@@ -36,6 +40,8 @@ Readings where the pages are silent (each pinned or flagged in the tests):
 * nearest-level ties go to the lower index (NumPy ``argmin`` takes the first).
 * the LoRA term carries the alpha/r scale of the minnong511 page; the itwiki
   equation omits it. A is K x r, B is r x N, so the LoRA product is X A B.
+* merge_and_unload: W_merged = bf16(Ŵ + scale (A B)^T) with the sum exact and one
+  rounding to bf16 (the pages do not say in which precision the sum is formed).
 """
 from __future__ import annotations
 
@@ -286,6 +292,33 @@ def linear_forward(X, W_hat, A, B, scale):
     T = X @ np.asarray(A, np.float64)
     Y = X @ np.asarray(W_hat, np.float64).T + scale * (T @ np.asarray(B, np.float64))
     return Y, T
+
+
+def merge_lora(q: dict, A, B, scale) -> np.ndarray:
+    """merge_and_unload (blog "QLoRA", irregular6612, section on the training-to-inference
+    pipeline: dequantize the base to BF16, then add the LoRA term, with the alpha/r scale
+    of the section on re-quantization; itwiki "QLoRA", section "한계와 주의점"):
+    W_merged = bf16(Ŵ + scale (A B)^T) [N, K]. Reading: the sum is exact (fp64 from the
+    bf16 Ŵ and the bf16 A, B) and rounded once to bf16. Returns fp64 pre-rounding values
+    and the bf16 result (as fp32 holding bf16 values)."""
+    W_hat = double_dequant(q).astype(np.float64)
+    delta = (np.asarray(A, np.float64) @ np.asarray(B, np.float64)).T
+    exact = W_hat + float(scale) * delta
+    return exact, bf16_round_f64(exact)
+
+
+def bf16_round_f64(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to bf16 in one step (nearest, ties to even), returned as fp32
+    holding bf16 values. bf16 keeps 8 significant bits, so the spacing of bf16 values
+    around x is ulp = 2^(E - 8) for x = m 2^E with m in [0.5, 1), and never below the
+    subnormal spacing 2^-133; x / ulp and q * ulp are exact in fp64 (powers of two).
+    Rounding to fp32 first and then to bf16 could round twice."""
+    x = np.asarray(x, np.float64)
+    _, E = np.frexp(x)
+    ulp = np.ldexp(1.0, np.maximum(E - 8, -133))
+    q = np.rint(x / ulp) * ulp              # np.rint: half to even
+    q = np.where(np.abs(q) > 3.3895313892515355e38, np.copysign(np.inf, x), q)
+    return q.astype(np.float32)
 
 
 def linear_backward(dY, X, W_hat, A, B, scale, T=None):

@@ -151,6 +151,17 @@ def test_quantize_rejects_bad_arguments(L):
     assert call(wsb=ws - 1) == 4
 
 
+def test_merge_rejects_bad_arguments(L):
+    merge = L.qlora_merge_lora
+    assert merge(W(), None, P, 8, 2.0, P, None) == 1
+    assert merge(W(), P, P, 12, 2.0, P, None) == 1
+    assert merge(W(), P, P, 8, float("inf"), P, None) == 1
+    assert merge(W(k=1000), P, P, 8, 2.0, P, None) == 2
+    assert merge(W(n=500), P, P, 8, 2.0, P, None) == 2
+    assert merge(W(), P, P, 8, 2.0, Q, None) == 3
+    assert merge(W(codes=None), P, P, 8, 2.0, P, None) == 1
+
+
 def test_linear_rejects_bad_arguments(L):
     fwd = L.qlora_linear_fwd
     need = L.qlora_linear_fwd_workspace_size(64, 512, 1024, 8)

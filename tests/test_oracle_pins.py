@@ -290,3 +290,54 @@ def test_quantized_weight_error_is_small():
     assert np.mean(np.abs(What - W)) < 2e-3
     rows = np.array([0, 17, 63])
     np.testing.assert_array_equal(O.double_dequant_rows(q, rows), What[rows])
+
+
+# ---------------------------------------------------------------- merge_and_unload
+def test_bf16_round_f64_is_one_rounding():
+    """On fp32 inputs it agrees with the fp32 rounding (itself pinned against torch);
+    exact ties go to the even neighbour; a value just above a tie rounds up, which
+    rounding to fp32 first would turn into a tie and round down."""
+    rng = np.random.default_rng(30)
+    x = (rng.standard_normal(50000) * 10.0 ** rng.integers(-40, 30, 50000)).astype(np.float32)
+    assert np.array_equal(O.bf16_round_f64(x.astype(np.float64)).view(np.uint32),
+                          O.bf16_round(x).view(np.uint32))
+    u = 2.0 ** -7  # bf16 spacing in [1, 2)
+    assert list(O.bf16_round_f64(np.array([1 + u / 2, 1 + 3 * u / 2, -(1 + u / 2)]))) == \
+        [1.0, 1.0 + 2 * u, -1.0]
+    assert O.bf16_round_f64(np.array([1 + u / 2 + 2.0 ** -40]))[0] == np.float32(1 + u)
+    assert O.bf16_round(np.array([1 + u / 2 + 2.0 ** -40], np.float32))[0] == np.float32(1.0)
+
+
+def test_merge_special_cases():
+    """A = 0 leaves the dequantized weight unchanged bit for bit; an all-zero base
+    weight leaves bf16(scale (A B)^T), a plain matrix product."""
+    rng = np.random.default_rng(31)
+    N, K, r = 48, 192, 8
+    q = O.quantize_nf4_dq(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+    B = O.bf16_round(rng.normal(0, 0.02, (r, N)).astype(np.float32))
+    _, merged = O.merge_lora(q, np.zeros((K, r)), B, 2.0)
+    assert np.array_equal(merged.view(np.uint32), O.double_dequant(q).view(np.uint32))
+    q0 = O.quantize_nf4_dq(np.zeros((N, K), np.float32))
+    A = O.bf16_round(rng.normal(0, 0.02, (K, r)).astype(np.float32))
+    _, merged = O.merge_lora(q0, A, B, 2.0)
+    direct = np.einsum("kj,jn->nk", A.astype(np.float64), B.astype(np.float64)) * 2.0
+    assert np.array_equal(merged.view(np.uint32), O.bf16_round_f64(direct).view(np.uint32))
+
+
+def test_merged_weight_reproduces_the_layer_forward():
+    """X W_merged^T equals the adapter-augmented forward up to the bf16 rounding of the
+    merged weight (a transposed or unscaled LoRA product would not)."""
+    rng = np.random.default_rng(32)
+    M, N, K, r, scale = 6, 40, 128, 16, 0.5
+    q = O.quantize_nf4_dq(rng.normal(0, 0.02, (N, K)).astype(np.float32))
+    A = O.bf16_round(rng.normal(0, 0.05, (K, r)).astype(np.float32))
+    B = O.bf16_round(rng.normal(0, 0.05, (r, N)).astype(np.float32))
+    X = O.bf16_round(rng.normal(0, 1, (M, K)).astype(np.float32)).astype(np.float64)
+    _, merged = O.merge_lora(q, A, B, scale)
+    Y, _ = O.linear_forward(X, O.double_dequant(q), A, B, scale)
+    Ym = X @ merged.astype(np.float64).T
+    half_ulp = np.ldexp(1.0, np.frexp(merged.astype(np.float64))[1] - 9)  # bf16 half spacing
+    bound = np.abs(X) @ half_ulp.T + 1e-12
+    assert np.all(np.abs(Ym - Y) <= bound)
+    unmerged = X @ O.double_dequant(q).astype(np.float64).T  # the LoRA term left out
+    assert not np.all(np.abs(unmerged - Y) <= bound)
