@@ -357,13 +357,14 @@ def codec_bandwidth(device, reps=5):
     g = torch.Generator(device=device)
     g.manual_seed(1)
     shapes = [(4096, 4096), (4096, 11008), (11008, 4096)]
-    Ws, Qs, Outs, wss, As, Bs = [], [], [], [], [], []
+    Ws, Qs, Outs, wss, As, Bs, Qu = [], [], [], [], [], [], []
     for n, k in shapes:
         W = torch.randn(n, k, generator=g, device=device) * 0.02
         mask = torch.rand(n, k, generator=g, device=device) < 1e-3   # 0.1 % outliers x10
         W = torch.where(mask, W * 10, W).to(torch.bfloat16)
         Ws.append(W)
         Qs.append(qlora.NF4Weight.empty(n, k, device))
+        Qu.append(qlora.qlora_quantize_nf4_dq(W, codebook=qlora.CODEBOOK_UNIFORM4))
         Outs.append(torch.empty(n, k, dtype=torch.bfloat16, device=device))
         As.append((torch.randn(k, RANK_R, generator=g, device=device) * 0.02).to(torch.bfloat16))
         Bs.append((torch.randn(RANK_R, n, generator=g, device=device) * 0.02).to(torch.bfloat16))
@@ -372,13 +373,15 @@ def codec_bandwidth(device, reps=5):
     params = sum(n * k for n, k in shapes)
     per_param = 2.0 + 0.515869140625
     out = {}
-    for name in ("quantize", "dequant", "merge"):
+    for name in ("quantize", "dequant", "merge", "dequant_uniform4"):
         def one_pass():
-            for W, q, o, ws, A, B in zip(Ws, Qs, Outs, wss, As, Bs):
+            for W, q, o, ws, A, B, qu in zip(Ws, Qs, Outs, wss, As, Bs, Qu):
                 if name == "quantize":
                     qlora.qlora_quantize_nf4_dq(W, out=q, workspace=ws)
                 elif name == "dequant":
                     qlora.qlora_dequant(q, out=o)
+                elif name == "dequant_uniform4":  # the same kernel for the evenly spaced codebook
+                    qlora.qlora_dequant(qu, out=o)
                 else:  # merge_and_unload with the rank-64 adapter (A, B reads are 0.3 % extra)
                     qlora.qlora_merge_lora(q, A, B, ALPHA / RANK_R, out=o)
         s = torch.cuda.Stream(device)

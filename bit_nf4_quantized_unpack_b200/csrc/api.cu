@@ -72,6 +72,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Common checks of a quantized weight.
 qlora_status check_weight(const qlora_nf4_weight& w) {
   if (!w.codes || !w.c2 || !w.c1 || !w.mean) return QLORA_ERR_INVALID_ARG;
+  if (w.codebook < 0 || w.codebook >= kCodebooks) return QLORA_ERR_INVALID_ARG;
   if (w.n_out < 1 || w.k_in < 64 || w.k_in % 64 != 0) return QLORA_ERR_SHAPE;
   if (w.n_out > (int64_t{1} << 31) || w.k_in > (int64_t{1} << 31)) return QLORA_ERR_SHAPE;
   if (!aligned16(w.codes) || !aligned16(w.c2) || !aligned16(w.c1) || !aligned16(w.mean))
@@ -208,9 +209,10 @@ size_t qlora_quantize_workspace_size(int64_t n_out, int64_t k_in) {
   return quantize_workspace_bytes(n_out, k_in);
 }
 
-qlora_status qlora_quantize_nf4_dq(const void* W, qlora_dtype w_dtype, int64_t n_out, int64_t k_in,
-                                   uint8_t* codes, uint8_t* c2, float* c1, float* mean,
-                                   void* workspace, size_t workspace_bytes, void* stream) {
+qlora_status qlora_quantize_dq(const void* W, qlora_dtype w_dtype, int64_t n_out, int64_t k_in,
+                               int32_t codebook, uint8_t* codes, uint8_t* c2, float* c1,
+                               float* mean, void* workspace, size_t workspace_bytes, void* stream) {
+  if (codebook < 0 || codebook >= kCodebooks) return QLORA_ERR_INVALID_ARG;
   if (!W || !codes || !c2 || !c1 || !mean) return QLORA_ERR_INVALID_ARG;
   if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
   if (n_out < 1 || k_in < 64 || k_in % 64 != 0) return QLORA_ERR_SHAPE;
@@ -222,8 +224,15 @@ qlora_status qlora_quantize_nf4_dq(const void* W, qlora_dtype w_dtype, int64_t n
   if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
   qlora_status q = check_device();
   if (q != QLORA_OK) return q;
-  return cuda_status(launch_quantize(W, w_dtype == QLORA_BF16, n_out, k_in, codes, c2, c1, mean,
-                                     workspace, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_quantize(W, w_dtype == QLORA_BF16, n_out, k_in, codebook, codes, c2,
+                                     c1, mean, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_quantize_nf4_dq(const void* W, qlora_dtype w_dtype, int64_t n_out, int64_t k_in,
+                                   uint8_t* codes, uint8_t* c2, float* c1, float* mean,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  return qlora_quantize_dq(W, w_dtype, n_out, k_in, QLORA_CODEBOOK_NF4, codes, c2, c1, mean,
+                           workspace, workspace_bytes, stream);
 }
 
 qlora_status qlora_dequant(qlora_nf4_weight w, uint16_t* W_out, void* stream) {

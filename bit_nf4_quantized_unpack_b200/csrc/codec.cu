@@ -194,13 +194,14 @@ __global__ void __launch_bounds__(256)
 }
 
 // Standalone double dequantization: one thread per 8 codes (one 32-bit word).
+template <int CB>
 __global__ void __launch_bounds__(256)
     k_dequant(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ c2,
               const float* __restrict__ c1, const float* __restrict__ mean_p, int64_t nwords,
               uint4* __restrict__ out) {
   __shared__ float lut[16];
   __shared__ float t8[256];  // T8 by E4M3 code
-  if (threadIdx.x < 16) lut[threadIdx.x] = nf4_level(threadIdx.x);
+  if (threadIdx.x < 16) lut[threadIdx.x] = code_level<CB>(threadIdx.x);
   for (int e = threadIdx.x; e < 256; e += blockDim.x) t8[e] = t8_value(e);
   __syncthreads();
   const float mean = *mean_p;
@@ -233,8 +234,9 @@ size_t quantize_workspace_bytes(int64_t n, int64_t k) {
   return align_up(static_cast<size_t>(nblocks) * 4, 256) + kMaxQuantCtas * sizeof(double);
 }
 
-cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, uint8_t* codes,
-                            uint8_t* c2, float* c1, float* mean, void* ws, cudaStream_t st) {
+cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, int codebook,
+                            uint8_t* codes, uint8_t* c2, float* c1, float* mean, void* ws,
+                            cudaStream_t st) {
   const int64_t nblocks = n * k / 64;
   float* absmax = static_cast<float*>(ws);
   double* partial = reinterpret_cast<double*>(static_cast<char*>(ws) +
@@ -242,10 +244,10 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, ui
   const int ctas = quant_ctas(nblocks);
   if (w_bf16)
     k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const uint16_t*>(W), nblocks, nf4_buckets(), codes, absmax, partial);
+        static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
   else
     k_quantize_blocks<float><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const float*>(W), nblocks, nf4_buckets(), codes, absmax, partial);
+        static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_constants_mean<<<1, 1024, 0, st>>>(partial, ctas, nblocks, mean);
@@ -265,9 +267,9 @@ cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_
   int64_t g = (nwords + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
   if (g > cap) g = cap;
-  k_dequant<<<static_cast<int>(g), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(w.codes),
-                                                 w.c2, w.c1, w.mean, nwords,
-                                                 reinterpret_cast<uint4*>(out));
+  auto kern = w.codebook == 1 ? k_dequant<1> : k_dequant<0>;
+  kern<<<static_cast<int>(g), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(w.codes), w.c2,
+                                            w.c1, w.mean, nwords, reinterpret_cast<uint4*>(out));
   return cudaGetLastError();
 }
 

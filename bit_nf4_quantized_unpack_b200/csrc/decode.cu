@@ -226,7 +226,7 @@ __device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases& r
     }
 }
 
-template <bool kTall>
+template <bool kTall, int CB>
 __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int g,
                                              int t, const UnitCodes& c, const float* t8,
                                              float mean, float (&acc)[kGroups][kTall ? 2 : 1][4]) {
@@ -244,7 +244,7 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const bool live = kv && (rbase + q * 16 + g + 8 * h) < a.N;
-      build_lut(live ? block_scale_tab(t8, c.e2[q][h], c.e1[q][h], mean) : 0.f, lut[h]);
+      build_lut<CB>(live ? block_scale_tab(t8, c.e2[q][h], c.e1[q][h], mean) : 0.f, lut[h]);
     }
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
@@ -263,7 +263,7 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
   }
 }
 
-template <bool kTall>
+template <bool kTall, int CB>
 __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, int split,
                                                    int lane, const float* t8) {
   const int g = lane >> 2, t = lane & 3;
@@ -297,10 +297,10 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   if (u0 < u1) load_unit(a, rb, u0, t, bpr, cb0);
   for (int u = u0; u < u1; u += 2) {
     if (u + 1 < u1) load_unit(a, rb, u + 1, t, bpr, cb1);
-    compute_unit<kTall>(a, rbase, u, g, t, cb0, t8, mean, acc);
+    compute_unit<kTall, CB>(a, rbase, u, g, t, cb0, t8, mean, acc);
     if (u + 1 < u1) {
       if (u + 2 < u1) load_unit(a, rb, u + 2, t, bpr, cb0);
-      compute_unit<kTall>(a, rbase, u + 1, g, t, cb1, t8, mean, acc);
+      compute_unit<kTall, CB>(a, rbase, u + 1, g, t, cb1, t8, mean, acc);
     }
   }
 
@@ -366,7 +366,7 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
 
 // Two CTAs (8 warps) per SM: the two code buffers of the prefetch need the registers, and
 // measured faster than three CTAs with spills.
-template <bool kTall>  // kTall: M > 8 (tokens 8..15 live in the upper fragment rows)
+template <bool kTall, int CB>  // kTall: M > 8 (tokens 8..15 in the upper fragment rows); CB: codebook
 __global__ void __launch_bounds__(kDecThreads, 2) k_decode_gemv(const DecodeArgs a) {
   __shared__ float t8[256];  // T8 by E4M3 code
   for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_gemv(const DecodeArgs
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int task = blockIdx.x * (kDecThreads / 32) + warp;
   if (task < a.row_groups * a.splits)
-    decode_weight_task<kTall>(a, task % a.row_groups, task / a.row_groups, lane, t8);
+    decode_weight_task<kTall, CB>(a, task % a.row_groups, task / a.row_groups, lane, t8);
 }
 
 // ---------------------------------------------------------------- host side
@@ -445,8 +445,12 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = s.M > 8 ? cudaLaunchKernelEx(&cfg, k_decode_gemv<true>, a)
-              : cudaLaunchKernelEx(&cfg, k_decode_gemv<false>, a);
+  if (w.codebook == 1)
+    e = s.M > 8 ? cudaLaunchKernelEx(&cfg, k_decode_gemv<true, 1>, a)
+                : cudaLaunchKernelEx(&cfg, k_decode_gemv<false, 1>, a);
+  else
+    e = s.M > 8 ? cudaLaunchKernelEx(&cfg, k_decode_gemv<true, 0>, a)
+                : cudaLaunchKernelEx(&cfg, k_decode_gemv<false, 0>, a);
   if (e != cudaSuccess) return cuda_status(e);
   return QLORA_OK;
 }
@@ -522,6 +526,7 @@ extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_
                                                        uint16_t* Y, float* T_save, void* stream) {
   using namespace qlora;
   if (!w.codes || !w.c2 || !w.c1 || !w.mean) return QLORA_ERR_INVALID_ARG;
+  if (w.codebook < 0 || w.codebook >= kCodebooks) return QLORA_ERR_INVALID_ARG;
   if (w.n_out < 1 || w.k_in < 64 || w.k_in % 64 != 0 || w.n_out % 8 != 0 ||
       w.n_out > (int64_t{1} << 31) || w.k_in > (int64_t{1} << 31))
     return QLORA_ERR_SHAPE;

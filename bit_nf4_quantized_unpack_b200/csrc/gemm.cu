@@ -92,6 +92,7 @@ struct FusedArgs {
   int64_t out_ld;     // N (forward) or K (dgrad)
   int64_t out_rows;   // valid D rows: N (forward) or K (dgrad)
   int vec_store;      // out 16-byte aligned and out_ld % 8 == 0: 8 rows per vector store
+  int codebook;       // 4-bit codebook of the codes (0 NF4, 1 uniform)
   int* err;
 };
 
@@ -116,7 +117,7 @@ __device__ __forceinline__ bool last_use(int uses, int slots, int s, uint32_t& p
   return true;
 }
 
-template <Mode MODE>
+template <Mode MODE, int CB>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     k_fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_act,
                      const __grid_constant__ CUtensorMap tm_ext_w,
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       advance(nxt, kDeqGroups);
       if (nxt.i != cur.i && nxt.i < my_tiles) set_tile(nxt);
       Nf4Lut lut;
-      build_lut(sc, lut);
+      build_lut<CB>(sc, lut);
       uint32_t o[8][4];
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) lut_decode8(words[ch], lut, o[ch]);
@@ -835,7 +836,7 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
 template <Mode MODE>
 cudaError_t run_fused(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& tx,
                       FusedArgs args, cudaStream_t st) {
-  auto kern = k_fused_nf4_gemm<MODE>;
+  auto kern = args.codebook == 1 ? k_fused_nf4_gemm<MODE, 1> : k_fused_nf4_gemm<MODE, 0>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
   if (e != cudaSuccess) return e;
@@ -948,6 +949,7 @@ qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const ui
   QL_MAP(&tw, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);   // B [r, N], MN-major chunks
   QL_MAP(&tx, kBF16, ts, 128, s.M, 256, 64, 256, kSW128);     // scale T, bf16 hi | lo
   FusedArgs a;
+  a.codebook = w.codebook;
   a.codes = w.codes;
   a.c2 = w.c2;
   a.c1 = w.c1;
@@ -1000,6 +1002,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&tw, kBF16, A, s.r, s.K, s.r * 2, 64, 128, kSW128);   // A [K, r] K-major
     QL_MAP(&tx, kBF16, gs, 128, s.M, 256, 64, 256, kSW128);      // scale G, bf16 hi | lo
     FusedArgs a;
+    a.codebook = w.codebook;
     a.codes = w.codes;
     a.c2 = w.c2;
     a.c1 = w.c1;

@@ -24,7 +24,9 @@ struct Nf4BucketTable {
   float thr[kCodeBuckets];
   uint8_t code[kCodeBuckets + 3];
 };
-const Nf4BucketTable& nf4_buckets();
+constexpr int kCodebooks = 2;  // qlora_codebook: 0 NF4, 1 uniform 4-bit
+const Nf4BucketTable& code_buckets(int codebook);
+const float* codebook_levels(int codebook);
 struct T8Thresholds { float t[kT8Size - 1]; };
 const Nf4Thresholds& nf4_thresholds();
 const T8Thresholds& t8_thresholds();
@@ -45,8 +47,9 @@ void profile_events(cudaEvent_t* before, cudaEvent_t* after);
 
 // ---- launchers (codec.cu) -------------------------------------------------------
 size_t quantize_workspace_bytes(int64_t n, int64_t k);
-cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, uint8_t* codes,
-                            uint8_t* c2, float* c1, float* mean, void* ws, cudaStream_t st);
+cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, int codebook,
+                            uint8_t* codes, uint8_t* c2, float* c1, float* mean, void* ws,
+                            cudaStream_t st);
 cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t st);
 
 // ---- launchers (gemm.cu) --------------------------------------------------------

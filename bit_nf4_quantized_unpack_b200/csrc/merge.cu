@@ -57,6 +57,7 @@ struct MergeArgs {
 
 // grid: x = 64-row bands of W, y = groups of `ktiles` consecutive 64-column tiles. B's
 // band, the T8 table and the MMA fragments that come from B are staged once per CTA.
+template <int CB>
 __global__ void __launch_bounds__(kMergeThreads) k_merge_lora(const MergeArgs a, int ktiles) {
   __shared__ __align__(16) uint16_t bs[kMergeTile][kRowPad];  // B[j][n0 + i] (rows j >= r zero)
   __shared__ __align__(16) uint16_t as[kMergeTile][kRowPad];  // A[k0 + i][j] (cols j >= r zero)
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_merge_lora(const MergeArgs a,
   const float mean = *a.mean;
 
   for (int e = tid; e < 256; e += kMergeThreads) t8[e] = t8_value(e);
-  if (tid < 16) lut[tid] = nf4_level(tid);
+  if (tid < 16) lut[tid] = code_level<CB>(tid);
   for (int idx = tid; idx < r16 * 8; idx += kMergeThreads) {
     const int j = idx >> 3, c = idx & 7;  // chunk c of row j: columns n0 + 8c .. + 7
     const int64_t n = n0 + c * 8;
@@ -199,7 +200,8 @@ cudaError_t launch_merge_lora(const qlora_nf4_weight& w, const uint16_t* A, cons
   if ((kt_total + ktiles - 1) / ktiles > 65535) ktiles = (kt_total + 65534) / 65535;  // grid y
   const dim3 grid(static_cast<unsigned>(bands),
                   static_cast<unsigned>((kt_total + ktiles - 1) / ktiles));
-  k_merge_lora<<<grid, kMergeThreads, 0, st>>>(a, static_cast<int>(ktiles));
+  auto kern = w.codebook == 1 ? k_merge_lora<1> : k_merge_lora<0>;
+  kern<<<grid, kMergeThreads, 0, st>>>(a, static_cast<int>(ktiles));
   return cudaGetLastError();
 }
 

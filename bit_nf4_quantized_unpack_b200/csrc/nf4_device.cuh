@@ -1,5 +1,6 @@
 // nf4_device.cuh -- device-side pieces of the double dequantization shared by the
-// standalone dequant, the fused GEMM and the decode kernels:
+// standalone dequant, the fused GEMM, the decode and the merge kernels (NF4 is the
+// codebook L below unless a kernel is instantiated for the uniform one):
 //   s_j   = fl32(fl32(T8[c2_j] * c1[j / 256]) + mean)     (T8[e] = fl32(e4m3(e) / 448))
 //   W_hat = bf16_rn(fl32(NF4[code] * s_j))
 // (page "QLoRA", itwiki.kr: sections "4비트 NormalFloat(NF4)" and "이중 양자화", and
@@ -12,14 +13,21 @@
 
 namespace qlora {
 
-// NF4 level i as an fp32 constant (bit patterns of the table, ascending).
-__device__ __forceinline__ float nf4_level(int i) {
-  constexpr uint32_t bits[16] = {0xbf800000u, 0xbf3239b3u, 0xbf066b30u, 0xbeca32a0u,
-                                 0xbe91a24cu, 0xbe3d353fu, 0xbdba786bu, 0x00000000u,
-                                 0x3da2fb03u, 0x3e24cae1u, 0x3e7c04dcu, 0x3ead0338u,
-                                 0x3ee1a4b7u, 0x3f1007aau, 0x3f3913b1u, 0x3f800000u};
-  return __uint_as_float(bits[i]);
+// Level i of codebook CB as an fp32 constant (bit patterns, ascending): CB 0 is NF4,
+// CB 1 the evenly spaced comparison codebook of the same section (-1 + 2i/15).
+template <int CB>
+__device__ __forceinline__ float code_level(int i) {
+  constexpr uint32_t nf4[16] = {0xbf800000u, 0xbf3239b3u, 0xbf066b30u, 0xbeca32a0u,
+                                0xbe91a24cu, 0xbe3d353fu, 0xbdba786bu, 0x00000000u,
+                                0x3da2fb03u, 0x3e24cae1u, 0x3e7c04dcu, 0x3ead0338u,
+                                0x3ee1a4b7u, 0x3f1007aau, 0x3f3913b1u, 0x3f800000u};
+  constexpr uint32_t uni[16] = {0xbf800000u, 0xbf5ddddeu, 0xbf3bbbbcu, 0xbf19999au,
+                                0xbeeeeeefu, 0xbeaaaaabu, 0xbe4ccccdu, 0xbd888889u,
+                                0x3d888889u, 0x3e4ccccdu, 0x3eaaaaabu, 0x3eeeeeefu,
+                                0x3f19999au, 0x3f3bbbbcu, 0x3f5ddddeu, 0x3f800000u};
+  return __uint_as_float(CB == 0 ? nf4[i] : uni[i]);
 }
+__device__ __forceinline__ float nf4_level(int i) { return code_level<0>(i); }
 
 // Value of an OCP FP8 E4M3 bit pattern (exact in fp32).
 __device__ __forceinline__ float e4m3_value(uint32_t b) {
@@ -52,11 +60,12 @@ struct Nf4Lut {
   uint32_t hi[4];
 };
 
+template <int CB = 0>
 __device__ __forceinline__ void build_lut(float s, Nf4Lut& t) {
   uint32_t p[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    p[i] = pack_bf16x2_rn(__fmul_rn(nf4_level(2 * i), s), __fmul_rn(nf4_level(2 * i + 1), s));
+    p[i] = pack_bf16x2_rn(__fmul_rn(code_level<CB>(2 * i), s), __fmul_rn(code_level<CB>(2 * i + 1), s));
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     t.lo[q] = prmt(p[2 * q], p[2 * q + 1], 0x6420u);

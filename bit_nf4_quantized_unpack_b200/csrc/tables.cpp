@@ -32,6 +32,13 @@ const uint32_t kNf4Bits[16] = {
     0xbdba786bu, 0x00000000u, 0x3da2fb03u, 0x3e24cae1u, 0x3e7c04dcu, 0x3ead0338u,
     0x3ee1a4b7u, 0x3f1007aau, 0x3f3913b1u, 0x3f800000u};
 
+// The comparison codebook of the same section: 16 evenly spaced levels on [-1, 1]
+// (-1 + 2i/15 in double, the end point exact, rounded to fp32).
+const uint32_t kUniform4Bits[16] = {
+    0xbf800000u, 0xbf5ddddeu, 0xbf3bbbbcu, 0xbf19999au, 0xbeeeeeefu, 0xbeaaaaabu,
+    0xbe4ccccdu, 0xbd888889u, 0x3d888889u, 0x3e4ccccdu, 0x3eaaaaabu, 0x3eeeeeefu,
+    0x3f19999au, 0x3f3bbbbcu, 0x3f5ddddeu, 0x3f800000u};
+
 namespace {
 
 float bits_to_float(uint32_t u) {
@@ -90,9 +97,42 @@ float e4m3_value(uint32_t b) {
   return (b & 0x80u) ? -v : v;
 }
 
-struct Tables {
-  Nf4Thresholds nf4;
+struct CodebookTables {
+  float levels[16];
+  Nf4Thresholds thr;
   Nf4BucketTable buckets;
+};
+
+// Thresholds and the 1025-bucket table of one 16-level codebook.
+void build_codebook(const uint32_t (&bits)[16], CodebookTables& cb) {
+  for (int i = 0; i < 16; ++i) cb.levels[i] = bits_to_float(bits[i]);
+  for (int i = 0; i < 15; ++i) cb.thr.t[i] = first_above(cb.levels, 16, i);
+  // Bucket b holds the fp32 x with round-half-even(512 x + 512) == b: its edges are
+  // (2b -+ 1 - 1024) / 1024, each tie going to the even bucket.
+  for (int b = 0; b < kCodeBuckets; ++b) {
+    float xmin = static_cast<float>((2.0 * b - 1025.0) / 1024.0);
+    float xmax = static_cast<float>((2.0 * b - 1023.0) / 1024.0);
+    if (b & 1) {
+      xmin = std::nextafter(xmin, std::numeric_limits<float>::infinity());
+      xmax = std::nextafter(xmax, -std::numeric_limits<float>::infinity());
+    }
+    int code = 0;
+    for (int i = 0; i < 15; ++i) code += (xmin >= cb.thr.t[i]) ? 1 : 0;
+    float thr = std::numeric_limits<float>::infinity();
+    int inside = 0;
+    for (int i = 0; i < 15; ++i)
+      if (cb.thr.t[i] > xmin && cb.thr.t[i] <= xmax) {
+        thr = cb.thr.t[i];
+        ++inside;
+      }
+    if (inside > 1) std::abort();  // the table form needs at most one threshold per bucket
+    cb.buckets.thr[b] = thr;
+    cb.buckets.code[b] = static_cast<uint8_t>(code);
+  }
+}
+
+struct Tables {
+  CodebookTables cb[kCodebooks];
   T8Thresholds t8;
   float t8_vals[kT8Size];
   uint8_t t8_code[kT8Size];
@@ -102,31 +142,8 @@ const Tables& tables() {
   static Tables tab;
   static std::once_flag once;
   std::call_once(once, [] {
-    float nf4[16];
-    for (int i = 0; i < 16; ++i) nf4[i] = bits_to_float(kNf4Bits[i]);
-    for (int i = 0; i < 15; ++i) tab.nf4.t[i] = first_above(nf4, 16, i);
-    // Bucket b holds the fp32 x with round-half-even(512 x + 512) == b: its edges are
-    // (2b -+ 1 - 1024) / 1024, each tie going to the even bucket.
-    for (int b = 0; b < kCodeBuckets; ++b) {
-      float xmin = static_cast<float>((2.0 * b - 1025.0) / 1024.0);
-      float xmax = static_cast<float>((2.0 * b - 1023.0) / 1024.0);
-      if (b & 1) {
-        xmin = std::nextafter(xmin, std::numeric_limits<float>::infinity());
-        xmax = std::nextafter(xmax, -std::numeric_limits<float>::infinity());
-      }
-      int code = 0;
-      for (int i = 0; i < 15; ++i) code += (xmin >= tab.nf4.t[i]) ? 1 : 0;
-      float thr = std::numeric_limits<float>::infinity();
-      int inside = 0;
-      for (int i = 0; i < 15; ++i)
-        if (tab.nf4.t[i] > xmin && tab.nf4.t[i] <= xmax) {
-          thr = tab.nf4.t[i];
-          ++inside;
-        }
-      if (inside > 1) std::abort();  // the table form needs at most one threshold per bucket
-      tab.buckets.thr[b] = thr;
-      tab.buckets.code[b] = static_cast<uint8_t>(code);
-    }
+    build_codebook(kNf4Bits, tab.cb[0]);
+    build_codebook(kUniform4Bits, tab.cb[1]);
     // T8 in ascending order: -448 .. -min (0xFE .. 0x81), 0 (0x00), +min .. +448.
     int n = 0;
     for (int b = 0xFE; b >= 0x81; --b) tab.t8_code[n++] = static_cast<uint8_t>(b);
@@ -144,8 +161,9 @@ const Tables& tables() {
 
 }  // namespace
 
-const Nf4Thresholds& nf4_thresholds() { return tables().nf4; }
-const Nf4BucketTable& nf4_buckets() { return tables().buckets; }
+const Nf4Thresholds& nf4_thresholds() { return tables().cb[0].thr; }
+const Nf4BucketTable& code_buckets(int codebook) { return tables().cb[codebook].buckets; }
+const float* codebook_levels(int codebook) { return tables().cb[codebook].levels; }
 const T8Thresholds& t8_thresholds() { return tables().t8; }
 const float* t8_values() { return tables().t8_vals; }
 const uint8_t* t8_codes() { return tables().t8_code; }
@@ -164,7 +182,7 @@ extern "C" void qlora_nf4_thresholds(float* out15) {
 }
 
 extern "C" void qlora_nf4_code_buckets(float* thr1025, uint8_t* code1025) {
-  const auto& t = qlora::nf4_buckets();
+  const auto& t = qlora::code_buckets(0);
   for (int i = 0; i < qlora::kCodeBuckets; ++i) {
     if (thr1025) thr1025[i] = t.thr[i];
     if (code1025) code1025[i] = t.code[i];
@@ -179,4 +197,19 @@ extern "C" void qlora_fp8_thresholds(float* out252, float* t8_out253, uint8_t* c
     for (int i = 0; i < qlora::kT8Size; ++i) t8_out253[i] = qlora::t8_values()[i];
   if (codes_out253)
     for (int i = 0; i < qlora::kT8Size; ++i) codes_out253[i] = qlora::t8_codes()[i];
+}
+
+extern "C" int qlora_codebook_tables(int32_t codebook, float* levels16, float* thr15,
+                                     float* bucket_thr1025, uint8_t* bucket_code1025) {
+  if (codebook < 0 || codebook >= qlora::kCodebooks) return -1;
+  const auto& cb = qlora::tables().cb[codebook];
+  for (int i = 0; i < 16; ++i)
+    if (levels16) levels16[i] = cb.levels[i];
+  for (int i = 0; i < 15; ++i)
+    if (thr15) thr15[i] = cb.thr.t[i];
+  for (int i = 0; i < qlora::kCodeBuckets; ++i) {
+    if (bucket_thr1025) bucket_thr1025[i] = cb.buckets.thr[i];
+    if (bucket_code1025) bucket_code1025[i] = cb.buckets.code[i];
+  }
+  return 0;
 }

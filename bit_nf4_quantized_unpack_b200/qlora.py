@@ -34,7 +34,8 @@ class QLoraError(RuntimeError):
 
 class CNF4Weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p),
-                ("mean", ctypes.c_void_p), ("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64)]
+                ("mean", ctypes.c_void_p), ("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64),
+                ("codebook", ctypes.c_int32)]
 
 
 _lib = None
@@ -52,6 +53,8 @@ _SIGNATURES = {
     "qlora_fp8_thresholds": (None, [_vp, _vp, _vp]),
     "qlora_quantize_workspace_size": (_sz, [_i64, _i64]),
     "qlora_quantize_nf4_dq": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_quantize_dq": (_i32, [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_codebook_tables": (_i32, [_i32, _vp, _vp, _vp, _vp]),
     "qlora_dequant": (_i32, [CNF4Weight, _vp, _vp]),
     "qlora_merge_lora": (_i32, [CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp]),
     "qlora_linear_fwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
@@ -111,21 +114,41 @@ class NF4Weight:
     mean: torch.Tensor    # float32 [1]
     n_out: int
     k_in: int
+    codebook: int = 0     # CODEBOOK_NF4 or CODEBOOK_UNIFORM4
 
     def c_struct(self) -> CNF4Weight:
         return CNF4Weight(self.codes.data_ptr(), self.c2.data_ptr(), self.c1.data_ptr(),
-                          self.mean.data_ptr(), self.n_out, self.k_in)
+                          self.mean.data_ptr(), self.n_out, self.k_in, self.codebook)
 
     @staticmethod
-    def empty(n_out: int, k_in: int, device="cuda") -> "NF4Weight":
+    def empty(n_out: int, k_in: int, device="cuda", codebook: int = 0) -> "NF4Weight":
         nb = n_out * k_in // 64
         return NF4Weight(torch.empty(n_out * k_in // 2, dtype=torch.uint8, device=device),
                          torch.empty(nb, dtype=torch.uint8, device=device),
                          torch.empty((nb + 255) // 256, dtype=torch.float32, device=device),
-                         torch.empty(1, dtype=torch.float32, device=device), n_out, k_in)
+                         torch.empty(1, dtype=torch.float32, device=device), n_out, k_in,
+                         codebook)
 
 
 # ------------------------------------------------------------------ host-only tables
+
+CODEBOOK_NF4, CODEBOOK_UNIFORM4 = 0, 1
+
+
+def codebook_tables(codebook: int):
+    """(levels [16], thresholds [15], bucket thresholds [1025], bucket codes [1025]) of a
+    codebook, as the library builds them."""
+    lev, thr = (ctypes.c_float * 16)(), (ctypes.c_float * 15)()
+    bthr, bcode = (ctypes.c_float * 1025)(), (ctypes.c_uint8 * 1025)()
+    rc = lib().qlora_codebook_tables(codebook, ctypes.cast(lev, ctypes.c_void_p),
+                                     ctypes.cast(thr, ctypes.c_void_p),
+                                     ctypes.cast(bthr, ctypes.c_void_p),
+                                     ctypes.cast(bcode, ctypes.c_void_p))
+    if rc != 0:
+        raise ValueError(f"unknown codebook {codebook}")
+    return (torch.tensor(list(lev), dtype=torch.float32), torch.tensor(list(thr), dtype=torch.float32),
+            torch.tensor(list(bthr), dtype=torch.float32), torch.tensor(list(bcode), dtype=torch.uint8))
+
 
 def nf4_table() -> torch.Tensor:
     out = (ctypes.c_float * 16)()
@@ -163,21 +186,23 @@ def qlora_quantize_workspace_size(n_out: int, k_in: int) -> int:
 
 
 def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Weight | None = None,
-                          workspace: torch.Tensor | None = None) -> NF4Weight:
-    """NF4 + double quantization of W [N, K] (fp32 or bf16, CUDA, contiguous)."""
+                          workspace: torch.Tensor | None = None, codebook: int = 0) -> NF4Weight:
+    """4-bit (NF4 by default, or the uniform codebook) + double quantization of
+    W [N, K] (fp32 or bf16, CUDA, contiguous)."""
     if W.dim() != 2 or not W.is_cuda or not W.is_contiguous():
         raise ValueError("W must be a contiguous 2-D CUDA tensor")
     dtype = {torch.float32: F32, torch.bfloat16: BF16}.get(W.dtype)
     if dtype is None:
         raise TypeError(f"unsupported weight dtype {W.dtype}")
     n, k = W.shape
-    q = out if out is not None else NF4Weight.empty(n, k, W.device)
+    q = out if out is not None else NF4Weight.empty(n, k, W.device, codebook)
+    q.codebook = codebook
     need = qlora_quantize_workspace_size(n, k)
     ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8,
                                                              device=W.device)
-    _check(lib().qlora_quantize_nf4_dq(_ptr(W), dtype, n, k, _ptr(q.codes), _ptr(q.c2), _ptr(q.c1),
-                                       _ptr(q.mean), _ptr(ws), ws.numel(), _stream()),
-           "qlora_quantize_nf4_dq")
+    _check(lib().qlora_quantize_dq(_ptr(W), dtype, n, k, codebook, _ptr(q.codes), _ptr(q.c2),
+                                   _ptr(q.c1), _ptr(q.mean), _ptr(ws), ws.numel(), _stream()),
+           "qlora_quantize_dq")
     return q
 
 

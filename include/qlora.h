@@ -66,13 +66,22 @@ typedef enum {
 typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
 /* A quantized weight as produced by qlora_quantize_nf4_dq (device pointers). */
+/*
+ * The 4-bit codebook L of a stored weight. NF4 is the method's own; UNIFORM4 is the
+ * comparison codebook of the same itwiki section (16 evenly spaced levels on [-1, 1],
+ * "uniform 4-bit, same method"), which goes through the same blocking, nearest-level
+ * search, double quantization and kernels.
+ */
+typedef enum { QLORA_CODEBOOK_NF4 = 0, QLORA_CODEBOOK_UNIFORM4 = 1 } qlora_codebook;
+
 typedef struct {
   const uint8_t *codes;
   const uint8_t *c2;
   const float *c1;
   const float *mean;
-  int64_t n_out; /* N: rows (output features) */
-  int64_t k_in;  /* K: columns (input features), K % 64 == 0 */
+  int64_t n_out;    /* N: rows (output features) */
+  int64_t k_in;     /* K: columns (input features), K % 64 == 0 */
+  int32_t codebook; /* qlora_codebook of the codes (0 = NF4) */
 } qlora_nf4_weight;
 
 /* Human-readable name of a status code (static storage). */
@@ -130,6 +139,14 @@ void qlora_nf4_thresholds(float *out15);
 void qlora_nf4_code_buckets(float *thr1025, uint8_t *code1025);
 
 /*
+ * The same three tables for any codebook (qlora_codebook): its 16 levels (fp32,
+ * ascending), its 15 exact decision thresholds, and its 1025-bucket code table. Null
+ * output pointers are skipped. Returns 0, or -1 for an unknown codebook. Host-only.
+ */
+int qlora_codebook_tables(int32_t codebook, float *levels16, float *thr15, float *bucket_thr1025,
+                          uint8_t *bucket_code1025);
+
+/*
  * qlora_fp8_thresholds: the same for the 253-entry double-quantization table T8
  * (distinct finite E4M3 values / 448, ascending): 252 thresholds to host memory
  * `out252`; also writes T8 itself to `t8_out253` and the E4M3 bit pattern of each
@@ -162,8 +179,22 @@ qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, int64_t n
                                    void *stream);
 
 /*
+ * qlora_quantize_dq: qlora_quantize_nf4_dq with the 4-bit codebook chosen by `codebook`
+ * (qlora_codebook). The nearest-level search uses that codebook's levels; everything
+ * else (blocks, absmax, double quantization, storage) is the same. The weight it
+ * describes must carry the same codebook in qlora_nf4_weight.codebook.
+ * Errors: those of qlora_quantize_nf4_dq, and QLORA_ERR_INVALID_ARG for an unknown
+ * codebook.
+ */
+qlora_status qlora_quantize_dq(const void *W, qlora_dtype w_dtype, int64_t n_out, int64_t k_in,
+                               int32_t codebook, uint8_t *codes, uint8_t *c2, float *c1,
+                               float *mean, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/*
  * qlora_dequant: W_out [n_out, k_in] bf16 (device) = doubleDequant(c1, c2, W_NF4)
- * (itwiki "QLoRA", computation section; formula in the storage notes above).
+ * (itwiki "QLoRA", computation section; formula in the storage notes above), with the
+ * levels of the weight's codebook.
  * Bit-exact with the definition. No workspace.
  */
 qlora_status qlora_dequant(qlora_nf4_weight w, uint16_t *W_out, void *stream);

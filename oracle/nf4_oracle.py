@@ -246,15 +246,23 @@ def reconstruct_absmax(c2: np.ndarray, c1: np.ndarray, mean, dq_block: int = DQ_
 # The stored weight and doubleDequant (itwiki "QLoRA", computation section)
 # ---------------------------------------------------------------------------
 
-def quantize_nf4_dq(W: np.ndarray):
+def quantize_nf4_dq(W: np.ndarray, levels: np.ndarray | None = None):
     """W [N, K] (fp32, or bf16 values held in fp32), K % 64 == 0 ->
-    dict(codes packed uint8 [N*K/2], c2 uint8 [N*K/64], c1 fp32, mean fp32, absmax)."""
+    dict(codes packed uint8 [N*K/2], c2 uint8 [N*K/64], c1 fp32, mean fp32, absmax,
+    levels). ``levels`` is the 4-bit codebook: NF4 by default, or the evenly spaced
+    comparison codebook of the itwiki NF4 section (``uniform4_levels``), which goes
+    through the same blocking, search and double quantization."""
     W = np.asarray(W, np.float32)
     assert W.ndim == 2 and W.shape[1] % BLOCK == 0
-    codes, absmax = quantize_blocks(W, nf4_levels())
+    levels = nf4_levels() if levels is None else np.asarray(levels, np.float32)
+    codes, absmax = quantize_blocks(W, levels)
     c2, c1, mean = double_quantize(absmax)
     return {"codes": pack_nibbles(codes), "c2": c2, "c1": c1, "mean": mean,
-            "absmax": absmax, "shape": W.shape}
+            "absmax": absmax, "shape": W.shape, "levels": levels}
+
+
+def _levels_of(q: dict) -> np.ndarray:
+    return q["levels"] if "levels" in q else nf4_levels()
 
 
 def double_dequant(q: dict) -> np.ndarray:
@@ -263,7 +271,7 @@ def double_dequant(q: dict) -> np.ndarray:
     n, k = q["shape"]
     s = reconstruct_absmax(q["c2"], q["c1"], q["mean"])
     codes = unpack_nibbles(q["codes"]).reshape(-1, BLOCK)
-    vals = nf4_levels()[codes] * s[:, None]             # fp32 products
+    vals = _levels_of(q)[codes] * s[:, None]            # fp32 products
     return bf16_round(vals.astype(np.float32)).reshape(n, k)
 
 
@@ -276,7 +284,7 @@ def double_dequant_rows(q: dict, rows: np.ndarray) -> np.ndarray:
     s = reconstruct_absmax(q["c2"], q["c1"], q["mean"])[blk]
     packed = q["codes"].reshape(n, k // 2)[rows]
     codes = unpack_nibbles(packed.ravel()).reshape(-1, BLOCK)
-    vals = nf4_levels()[codes] * s[:, None]
+    vals = _levels_of(q)[codes] * s[:, None]
     return bf16_round(vals.astype(np.float32)).reshape(rows.size, k)
 
 

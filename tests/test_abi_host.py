@@ -99,6 +99,28 @@ def test_nf4_code_buckets_reproduce_argmin(L):
     assert np.array_equal(O.nearest_code(x, table), got)
 
 
+@pytest.mark.parametrize("codebook", [0, 1])
+def test_codebook_tables_reproduce_argmin(L, codebook):
+    """Each codebook's levels are the oracle's bit for bit, and its thresholds and
+    bucket table both reproduce the oracle's argmin around every threshold and level."""
+    lev, th, bthr, bcode = (t.numpy() for t in qlora.codebook_tables(codebook))
+    table = O.nf4_levels() if codebook == 0 else O.uniform4_levels()
+    assert np.array_equal(lev.view(np.uint32), table.view(np.uint32))
+    xs = [np.random.default_rng(3 + codebook).uniform(-1, 1, 1 << 17).astype(np.float32), table,
+          np.array([-1.0, 1.0, 0.0, -0.0], np.float32)]
+    for t in th:
+        xs.append(_ulp_window(t, 256))
+    for e in ((2.0 * np.arange(1026) - 1025.0) / 1024.0).astype(np.float32):
+        xs.append(_ulp_window(e, 2))
+    x = np.concatenate(xs)
+    x = x[(x >= -1) & (x <= 1)]
+    want = O.nearest_code(x, table)
+    assert np.array_equal(want, _count_leq(th, x))
+    b = np.rint(512.0 * x.astype(np.float64) + 512.0).astype(np.int64)
+    assert np.array_equal(want, bcode[b].astype(np.int64) + (x >= bthr[b]).astype(np.int64))
+    assert L.qlora_codebook_tables(2, None, None, None, None) == -1
+
+
 def test_fp8_table_and_thresholds_match_oracle(L):
     th, vals, codes = (t.numpy() for t in qlora.fp8_thresholds())
     ovals, ocodes = O.fp8_table()
@@ -126,8 +148,8 @@ P = 1 << 20          # 16-byte aligned fake pointer
 Q = (1 << 20) + 8    # misaligned fake pointer
 
 
-def W(codes=P, c2=P, c1=P, mean=P, n=512, k=1024):
-    return qlora.CNF4Weight(codes, c2, c1, mean, n, k)
+def W(codes=P, c2=P, c1=P, mean=P, n=512, k=1024, codebook=0):
+    return qlora.CNF4Weight(codes, c2, c1, mean, n, k, codebook)
 
 
 def test_quantize_rejects_bad_arguments(L):
@@ -160,6 +182,13 @@ def test_merge_rejects_bad_arguments(L):
     assert merge(W(n=500), P, P, 8, 2.0, P, None) == 2
     assert merge(W(), P, P, 8, 2.0, Q, None) == 3
     assert merge(W(codes=None), P, P, 8, 2.0, P, None) == 1
+
+
+def test_unknown_codebook_is_rejected(L):
+    assert L.qlora_dequant(W(codebook=2), P, None) == 1
+    assert L.qlora_merge_lora(W(codebook=-1), P, P, 8, 2.0, P, None) == 1
+    ws = L.qlora_quantize_workspace_size(512, 1024)
+    assert L.qlora_quantize_dq(P, 0, 512, 1024, 7, P, P, P, P, P, ws, None) == 1
 
 
 def test_linear_rejects_bad_arguments(L):

@@ -16,16 +16,16 @@ def _gpu():
     need_gpu()
 
 
-def run_case(case, w_bf16=True, check_T=True):
+def run_case(case, w_bf16=True, check_T=True, codebook=0):
     W, A, B, X, dY, r, scale = (case[k] for k in ("W", "A", "B", "X", "dY", "r", "scale"))
     Wt = torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
-    q = qlora.qlora_quantize_nf4_dq(Wt.to(torch.bfloat16) if w_bf16 else Wt)
+    q = qlora.qlora_quantize_nf4_dq(Wt.to(torch.bfloat16) if w_bf16 else Wt, codebook=codebook)
     Xd, Ad, Bd, dYd = to_dev_bf16(X), to_dev_bf16(A), to_dev_bf16(B), to_dev_bf16(dY)
     Y, T = qlora.qlora_linear_fwd(Xd, q, Ad, Bd, scale)
     dX, dA, dB = qlora.qlora_linear_bwd(dYd, Xd, T, q, Ad, Bd, scale)
     torch.cuda.synchronize()
     assert qlora.qlora_device_error() == 0
-    ref = O.quantize_nf4_dq(W)
+    ref = O.quantize_nf4_dq(W, O.uniform4_levels() if codebook == 1 else None)
     What = O.double_dequant(ref)
     Y64, T64 = O.linear_forward(X, What, A, B, scale)
     dX64, dA64, dB64 = O.linear_backward(dY, X, What, A, B, scale, T=T64)
