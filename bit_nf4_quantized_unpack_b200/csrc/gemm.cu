@@ -482,17 +482,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           }
           __syncwarp();
         };
-        // two chunks per TMEM round trip: both loads are in flight before one wait
 #pragma unroll 1
-        for (int c = 0; c < kHalfCols / 32; c += 2) {
+        for (int c = 0; c < kHalfCols / 32; ++c) {
           const int64_t mb = m0 + h * kHalfCols + c * 32;
           if (mb >= args.M) break;  // warp-uniform
-          uint32_t v0[32], v1[32];
+          uint32_t v0[32];
           tmem_ld_32x32b_x32(taddr + c * 32, v0);
-          tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v1);
           tmem_ld_wait();
           store_chunk(v0, mb);
-          if (mb + 32 < args.M) store_chunk(v1, mb + 32);
         }
         tc_fence_before();
         __syncwarp();
