@@ -517,21 +517,24 @@ constexpr int kLoraCtasPerSm = 2;
 static_assert(lora_smem(128) <= 113 * 1024 && lora_smem(64) <= 113 * 1024, "two CTAs per SM");
 
 struct LoraArgs {
-  int64_t rows;      // D rows (128-row tiles)
   int steps_total;   // 64-wide contraction steps
   int steps_per;     // steps per split
+  int tiles0;        // row tiles of the first problem; later tiles belong to the second
   float* partial;    // [splits][rows_pad][64] fp32 (NC = 128: hi + lo columns summed)
-  int64_t rows_pad;
+  int64_t rows_pad;  // the problems' row tiles stacked: 128 x (tiles0 + tiles of the second)
   int* err;
 };
 
 // D[128-row tile, NC] = sum over this CTA's contraction range of A^T B (both bf16,
 // K-major or MN-major 128B-swizzled tiles loaded by TMA). With NC = 128 the B operand is
 // a bf16 hi | lo pair and the partial written is D[:, j] + D[:, 64 + j].
+// One launch may run two problems with the same contraction (operands tm_a/tm_b for
+// the first tiles0 row tiles, tm_a1/tm_b1 after); their partial rows are stacked.
 template <bool A_MN, bool B_MN, int NC>
 __global__ void __launch_bounds__(kLoraThreads, 1)
     k_lora_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                const LoraArgs args) {
+                const __grid_constant__ CUtensorMap tm_a1,
+                const __grid_constant__ CUtensorMap tm_b1, const LoraArgs args) {
   constexpr uint32_t kB = NC * kBK * 2;
   constexpr int kLoraStages = lora_stages(NC);
   extern __shared__ uint8_t smem_raw[];
@@ -547,7 +550,12 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const bool second = static_cast<int>(blockIdx.x) >= args.tiles0;
+  const CUtensorMap* map_a = second ? &tm_a1 : &tm_a;
+  const CUtensorMap* map_b = second ? &tm_b1 : &tm_b;
+  // row of the operand (TMA coordinate) and of the stacked partial
+  const int64_t row0 = static_cast<int64_t>(second ? blockIdx.x - args.tiles0 : blockIdx.x) * 128;
+  const int64_t prow0 = static_cast<int64_t>(blockIdx.x) * 128;
   const int s_begin = blockIdx.y * args.steps_per;
   const int s_end = std::min(args.steps_total, s_begin + args.steps_per);
   const int nsteps = std::max(0, s_end - s_begin);
@@ -583,18 +591,18 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
         const int kc = (s_begin + i) * kBK;  // contraction coordinate
         mbar_arrive_expect_tx(&full[s], kLoraABytes + kB);
         if (A_MN) {
-          tma_load_2d(a_s + s * kLoraABytes, &tm_a, &full[s], static_cast<int>(row0), kc);
-          tma_load_2d(a_s + s * kLoraABytes + 8192, &tm_a, &full[s], static_cast<int>(row0) + 64,
+          tma_load_2d(a_s + s * kLoraABytes, map_a, &full[s], static_cast<int>(row0), kc);
+          tma_load_2d(a_s + s * kLoraABytes + 8192, map_a, &full[s], static_cast<int>(row0) + 64,
                       kc);
         } else {
-          tma_load_2d(a_s + s * kLoraABytes, &tm_a, &full[s], kc, static_cast<int>(row0));
+          tma_load_2d(a_s + s * kLoraABytes, map_a, &full[s], kc, static_cast<int>(row0));
         }
         if (B_MN) {
 #pragma unroll
           for (int c = 0; c < NC / 64; ++c)
-            tma_load_2d(b_s + s * kB + c * 8192, &tm_b, &full[s], c * 64, kc);
+            tma_load_2d(b_s + s * kB + c * 8192, map_b, &full[s], c * 64, kc);
         } else {
-          tma_load_2d(b_s + s * kB, &tm_b, &full[s], kc, 0);
+          tma_load_2d(b_s + s * kB, map_b, &full[s], kc, 0);
         }
         ++issued;
       }
@@ -640,7 +648,7 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
     if (!have || (mbar_wait(acc_full, 0, abort_flag) && !*abort_flag)) {
       tc_fence_after();
       const int quarter = warp & 3;
-      const int64_t row = row0 + quarter * 32 + lane;
+      const int64_t row = prow0 + quarter * 32 + lane;
       float* dst = args.partial + (static_cast<int64_t>(blockIdx.y) * args.rows_pad + row) * 64;
       const uint32_t taddr = tmem_d + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
@@ -681,9 +689,11 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
 // T (or G) = sum of split partials [S][rows_pad][64]. Writes, where asked:
 //   plain fp32 [M, r]; bf16 hi/lo of scale * v [M, 128] (the K-extension operand);
 //   bf16 hi/lo of v [M, 128] (operand of the LoRA gradients).
+//   With t_in, also the bf16 hi/lo pair [M, 128] of that fp32 [M, r] (into t_hilo).
 __global__ void k_finalize_rank(const float* __restrict__ part, int splits, int64_t rows_pad,
                                 int64_t M, int r, float scale, float* __restrict__ plain,
-                                uint16_t* __restrict__ scaled, uint16_t* __restrict__ hilo) {
+                                uint16_t* __restrict__ scaled, uint16_t* __restrict__ hilo,
+                                const float* __restrict__ t_in, uint16_t* __restrict__ t_hilo) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= M * 64) return;
   const int64_t m = i >> 6;
@@ -715,33 +725,34 @@ __global__ void k_finalize_rank(const float* __restrict__ part, int splits, int6
     hilo[m * 128 + j] = hi;
     hilo[m * 128 + 64 + j] = bf16_bits_rn(v - hv);
   }
+  if (t_hilo) {
+    const float tv = (j < r) ? t_in[m * r + j] : 0.f;
+    const uint16_t hi = bf16_bits_rn(tv);
+    t_hilo[m * 128 + j] = hi;
+    t_hilo[m * 128 + 64 + j] = bf16_bits_rn(tv - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+  }
 }
 
-// hi/lo bf16 pair [M, 128] from a saved fp32 T [M, r].
-__global__ void k_hilo_from_plain(const float* __restrict__ t, int64_t M, int r,
-                                  uint16_t* __restrict__ hilo) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= M * 64) return;
-  const int64_t m = i >> 6;
-  const int j = static_cast<int>(i & 63);
-  const float v = (j < r) ? t[m * r + j] : 0.f;
-  const uint16_t hi = bf16_bits_rn(v);
-  hilo[m * 128 + j] = hi;
-  hilo[m * 128 + 64 + j] = bf16_bits_rn(v - __uint_as_float(static_cast<uint32_t>(hi) << 16));
-}
-
-// grad[row, j] (or its transpose) = scale * sum_s P[s][row][j].
-// One block per 16 rows, four (row, j) items per thread with their split loads
+// Both LoRA gradients from the stacked partials of one grouped launch:
+//   rows [0, pad0) of P:  dA[k, j]   = scale * sum_s P[s][k][j]          ([rows0, r])
+//   rows [pad0, ...):     dB[j, n]   = scale * sum_s P[s][pad0 + n][j]   ([r, rows1])
+// One block per 16 stacked rows, four (row, j) items per thread with their split loads
 // interleaved; a shared-memory tile gives coalesced writes in either orientation.
 constexpr int kGradRows = 16;
+static_assert(128 % kGradRows == 0, "a block of rows never straddles the two problems");
 __global__ void __launch_bounds__(256)
-    k_finalize_grad(const float* __restrict__ part, int splits, int64_t rows_pad, int64_t rows,
-                    int r, float scale, bool transpose, float* __restrict__ out) {
+    k_finalize_grad(const float* __restrict__ part, int splits, int64_t rows_pad, int64_t pad0,
+                    int64_t rows0, float* __restrict__ out0, int64_t rows1,
+                    float* __restrict__ out1, int r, float scale) {
   __shared__ float tile[kGradRows][65];
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kGradRows;
+  const int64_t srow0 = static_cast<int64_t>(blockIdx.x) * kGradRows;  // stacked
+  const bool transpose = srow0 >= pad0;
+  const int64_t row0 = transpose ? srow0 - pad0 : srow0;
+  const int64_t rows = transpose ? rows1 : rows0;
+  float* __restrict__ out = transpose ? out1 : out0;
   const int64_t stride = rows_pad * 64;
   float v[4] = {0.f, 0.f, 0.f, 0.f};
-  const float* p = part + row0 * 64 + threadIdx.x;  // item u: row0 * 64 + threadIdx.x + 256 u
+  const float* p = part + srow0 * 64 + threadIdx.x;  // item u: srow0 * 64 + threadIdx.x + 256 u
   for (int sp = 0; sp < splits; ++sp) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) v[u] += p[sp * stride + 256 * u];
@@ -809,12 +820,20 @@ size_t partial_floats(int64_t rows, int64_t contraction, int nc) {
   return static_cast<size_t>(p.splits) * p.rows_pad * 64;
 }
 
+// Stacked rows of a grouped launch: the first problem padded to whole tiles, then the second.
+inline int64_t stacked_rows(int64_t rows0, int64_t rows1) { return align_up(rows0, 128) + rows1; }
+
+// One problem (ta, tb over `rows`), or two with the same contraction when ta1/tb1 are given
+// (rows0 = rows of the first, rows1 of the second; partial rows stacked).
 template <bool A_MN, bool B_MN, int NC>
-cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows,
-                          int64_t contraction, float* partial, cudaStream_t st, int* splits_out) {
+cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows0,
+                          int64_t contraction, float* partial, cudaStream_t st, int* splits_out,
+                          const CUtensorMap* ta1 = nullptr, const CUtensorMap* tb1 = nullptr,
+                          int64_t rows1 = 0) {
+  const int64_t rows = ta1 ? stacked_rows(rows0, rows1) : rows0;
   const SplitPlan p = plan_split(rows, contraction);
   LoraArgs a;
-  a.rows = rows;
+  a.tiles0 = ta1 ? static_cast<int>((rows0 + 127) / 128) : static_cast<int>(p.tiles);
   a.steps_total = p.steps_total;
   a.steps_per = p.steps_per;
   a.partial = partial;
@@ -825,7 +844,7 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(static_cast<unsigned>(p.tiles), static_cast<unsigned>(p.splits)), kLoraThreads, smem,
-         st>>>(ta, tb, a);
+         st>>>(ta, tb, ta1 ? *ta1 : ta, tb1 ? *tb1 : tb, a);
   *splits_out = p.splits;
   return cudaGetLastError();
 }
@@ -883,8 +902,7 @@ size_t bwd_layout(const LinearShape& s, void* ws, float** part, uint16_t** gs, u
   Carve c(ws);
   size_t pf = partial_floats(s.M, s.N, 64);                    // G = dY B^T
   pf = std::max(pf, partial_floats(s.M, s.K, 64));             // T = X A (recompute)
-  pf = std::max(pf, partial_floats(s.K, s.M, 128));            // dA
-  pf = std::max(pf, partial_floats(s.N, s.M, 128));            // dB
+  pf = std::max(pf, partial_floats(stacked_rows(s.K, s.N), s.M, 128));  // dA and dB
   *part = c.take<float>(pf);
   *gs = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
   *ghl = c.take<uint16_t>(static_cast<size_t>(s.M) * 128);
@@ -912,8 +930,8 @@ qlora_status lora_down_T(const uint16_t* X, const uint16_t* A, const LinearShape
   int splits = 0;
   QL_TRY((run_lora_gemm<false, true, 64>(ta, tb, s.M, s.K, part, st, &splits)));
   const int64_t rows_pad = plan_split(s.M, s.K).rows_pad;
-  k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(part, splits, rows_pad, s.M, s.r,
-                                                              s.scale, t_plain, t_scaled, nullptr);
+  k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
+      part, splits, rows_pad, s.M, s.r, s.scale, t_plain, t_scaled, nullptr, nullptr, nullptr);
   QL_TRY(cudaGetLastError());
   return QLORA_OK;
 }
@@ -972,25 +990,24 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
   bwd_layout(s, ws, &part, &gs, &ghl, &thl, &tbuf);
   int splits = 0;
 
-  // G = dY B^T -> bf16(scale G) for the dX extension, bf16 hi/lo for dA.
-  {
-    CUtensorMap ta, tb;
-    QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 128, kSW128);  // dY K-major (over n)
-    QL_MAP(&tb, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);    // B [r, N] K-major
-    QL_TRY((run_lora_gemm<false, false, 64>(ta, tb, s.M, s.N, part, st, &splits)));
-    k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
-        part, splits, plan_split(s.M, s.N).rows_pad, s.M, s.r, s.scale, nullptr, gs, ghl);
-    QL_TRY(cudaGetLastError());
-  }
-  // T (saved, or recomputed) -> bf16 hi/lo for dB.
+  // T (saved, or recomputed first: the partial buffer is then free again)
   const float* t = T_saved;
   if (!t) {
     qlora_status q = lora_down_T(X, A, s, part, tbuf, nullptr, st);
     if (q != QLORA_OK) return q;
     t = tbuf;
   }
-  k_hilo_from_plain<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(t, s.M, s.r, thl);
-  QL_TRY(cudaGetLastError());
+  // G = dY B^T -> bf16(scale G) for the dX extension, bf16 hi/lo of G for dA; the same
+  // launch turns T into its bf16 hi/lo pair for dB.
+  {
+    CUtensorMap ta, tb;
+    QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 128, kSW128);  // dY K-major (over n)
+    QL_MAP(&tb, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);    // B [r, N] K-major
+    QL_TRY((run_lora_gemm<false, false, 64>(ta, tb, s.M, s.N, part, st, &splits)));
+    k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
+        part, splits, plan_split(s.M, s.N).rows_pad, s.M, s.r, s.scale, nullptr, gs, ghl, t, thl);
+    QL_TRY(cudaGetLastError());
+  }
 
   // dX = dY W_hat + scale G A^T
   if (dX) {
@@ -1014,24 +1031,19 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     a.err = device_error_word();
     QL_TRY(run_fused<Mode::kDgrad>(ta, tw, tx, a, st));
   }
-  // dA = scale X^T G  (rows k, contraction over tokens)
+  // dA = scale X^T G (rows k) and dB = scale T^T dY (rows n, stored [r, N]): both contract
+  // over the tokens, so they run as one grouped launch and one finalize
   {
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, ta1, tb1;
     QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 64, kSW128);    // X as MN-major (k inner)
     QL_MAP(&tb, kBF16, ghl, 128, s.M, 256, 64, 64, kSW128);      // G hi/lo MN-major
-    QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits)));
-    k_finalize_grad<<<blocks_for(s.K, kGradRows), 256, 0, st>>>(
-        part, splits, plan_split(s.K, s.M).rows_pad, s.K, s.r, s.scale, false, dA);
-    QL_TRY(cudaGetLastError());
-  }
-  // dB = scale T^T dY  (rows n, contraction over tokens), stored [r, N]
-  {
-    CUtensorMap ta, tb;
-    QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);   // dY as MN-major (n inner)
-    QL_MAP(&tb, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);      // T hi/lo MN-major
-    QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.N, s.M, part, st, &splits)));
-    k_finalize_grad<<<blocks_for(s.N, kGradRows), 256, 0, st>>>(
-        part, splits, plan_split(s.N, s.M).rows_pad, s.N, s.r, s.scale, true, dB);
+    QL_MAP(&ta1, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);  // dY as MN-major (n inner)
+    QL_MAP(&tb1, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);     // T hi/lo MN-major
+    QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits, &ta1, &tb1, s.N)));
+    const int64_t stacked = stacked_rows(s.K, s.N);
+    k_finalize_grad<<<blocks_for(stacked, kGradRows), 256, 0, st>>>(
+        part, splits, plan_split(stacked, s.M).rows_pad, align_up(s.K, 128), s.K, dA, s.N, dB, s.r,
+        s.scale);
     QL_TRY(cudaGetLastError());
   }
   return QLORA_OK;

@@ -102,3 +102,72 @@ def test_empty_batch():
                            A, B, 1.0, need_dX=False, dA=dA, dB=dB)
     torch.cuda.synchronize()
     assert Y.shape == (0, 128) and torch.count_nonzero(dA) == 0 and torch.count_nonzero(dB) == 0
+
+
+def _tiles(rows, M):
+    return -(-rows // 128) * -(-M // 512)
+
+
+@pytest.mark.parametrize("M,N,K,r", [
+    (600, 10368, 512, 16),   # forward: 81 x 2 = 162 tiles, a second partial wave of CTAs
+    (600, 256, 10368, 16),   # dX: 81 x 2 tiles along K, 4 code steps per tile
+    (700, 9600, 256, 8),     # forward: 75 x 2 = 150 tiles, the second token tile one accumulator
+])
+def test_more_tiles_than_sms(M, N, K, r):
+    """More weight x token tiles than SMs, not a multiple of them: the persistent CTAs take
+    a second tile each until the tiles run out (full oracle comparison)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert max(_tiles(N, M), _tiles(K, M)) > sms
+    run_case(inputs.linear_case(300 + M + r, M, N, K, r, alpha=2 * r))
+
+
+def test_graph_replay_matches_eager():
+    """Forward and backward captured once in a CUDA graph and replayed on new inputs, with
+    workspaces that start as all-ones bytes: every replay equals the eager calls bit for bit."""
+    M, N, K, r = 600, 10368, 512, 16
+    case = inputs.linear_case(41, M, N, K, r, alpha=32)
+    q = qlora.qlora_quantize_nf4_dq(to_dev_bf16(case["W"]))
+    Ad, Bd = to_dev_bf16(case["A"]), to_dev_bf16(case["B"])
+    scale = case["scale"]
+    g = torch.Generator(device="cuda").manual_seed(5)
+    draws = [(torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16),
+              torch.randn(M, N, device="cuda", generator=g).to(torch.bfloat16)) for _ in range(3)]
+    eager = []
+    for Xd, dYd in draws:
+        Y, T = qlora.qlora_linear_fwd(Xd, q, Ad, Bd, scale)
+        dX, dA, dB = qlora.qlora_linear_bwd(dYd, Xd, T, q, Ad, Bd, scale)
+        eager.append((Y, dX, dA, dB))
+    # static buffers
+    Xs, dYs = draws[0][0].clone(), draws[0][1].clone()
+    Ys = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    Ts = torch.empty(M, r, dtype=torch.float32, device="cuda")
+    dXs = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dAs = torch.empty(K, r, dtype=torch.float32, device="cuda")
+    dBs = torch.empty(r, N, dtype=torch.float32, device="cuda")
+    wf = torch.full((qlora.qlora_linear_fwd_workspace_size(M, N, K, r),), 255, dtype=torch.uint8,
+                    device="cuda")
+    wb = torch.full((qlora.qlora_linear_bwd_workspace_size(M, N, K, r),), 255, dtype=torch.uint8,
+                    device="cuda")
+
+    def step():
+        qlora.qlora_linear_fwd(Xs, q, Ad, Bd, scale, Y=Ys, T=Ts, workspace=wf)
+        qlora.qlora_linear_bwd(dYs, Xs, Ts, q, Ad, Bd, scale, dX=dXs, dA=dAs, dB=dBs, workspace=wb)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        step()
+    for i, (Xd, dYd) in enumerate(draws):
+        Xs.copy_(Xd)
+        dYs.copy_(dYd)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert qlora.qlora_device_error() == 0
+        for got, want, name in zip((Ys, dXs, dAs, dBs), eager[i], ("Y", "dX", "dA", "dB")):
+            assert torch.equal(got, want), f"replay {i}: {name}"
+    del graph
