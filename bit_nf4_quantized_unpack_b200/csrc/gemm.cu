@@ -454,42 +454,51 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         tc_fence_after();
         const uint32_t taddr =
             tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + h * kHalfCols;
-        // one 32-token chunk: TMEM values -> bf16 -> stage[token][row] -> 16-byte stores
-        auto store_chunk = [&](const uint32_t (&v)[32], int64_t mb) {
+        // One 32-token chunk: two 16-lane TMEM loads in the accumulator-fragment layout,
+        // bf16 pairs, four transposing stmatrix into stage[token][row], then 16-byte
+        // stores of 8 consecutive output rows. A token's 64-byte stage row holds four
+        // 16-byte row groups, group g at slot g ^ ((token >> 1) & 3), so the eight rows
+        // of each stored matrix fall in distinct banks.
+        const uint32_t stage_s = smem_u32(stage);
+        auto slot_of = [](int tok, int g) { return static_cast<uint32_t>(tok * 64 + ((g ^ ((tok >> 1) & 3)) << 4)); };
+#pragma unroll 1
+        for (int c = 0; c < kHalfCols / 32; ++c) {
+          const int64_t mb = m0 + h * kHalfCols + c * 32;
+          if (mb >= args.M) break;  // warp-uniform
+          uint32_t a[16], b[16];
+          tmem_ld_16x256b_x4(taddr + c * 32, a);                 // rows 0-15 of the quarter
+          tmem_ld_16x256b_x4(taddr + (16u << 16) + c * 32, b);   // rows 16-31
+          tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const uint32_t pk = pack_bf16x2_rn(__uint_as_float(v[k]), __uint_as_float(v[k + 1]));
-            stage[k * 32 + lane] = static_cast<uint16_t>(pk & 0xFFFFu);
-            stage[(k + 1) * 32 + lane] = static_cast<uint16_t>(pk >> 16);
+          for (int j = 0; j < 4; ++j) {  // tokens 8j..8j+7 of the chunk
+            // matrix m = row group m (8 rows), its stored row i = token 8j + i
+            const int tok = 8 * j + (lane & 7);
+            stmatrix_x4_trans(stage_s + slot_of(tok, lane >> 3),
+                              pack_bf16x2_rn(__uint_as_float(a[4 * j]), __uint_as_float(a[4 * j + 1])),
+                              pack_bf16x2_rn(__uint_as_float(a[4 * j + 2]), __uint_as_float(a[4 * j + 3])),
+                              pack_bf16x2_rn(__uint_as_float(b[4 * j]), __uint_as_float(b[4 * j + 1])),
+                              pack_bf16x2_rn(__uint_as_float(b[4 * j + 2]), __uint_as_float(b[4 * j + 3])));
           }
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int tr = (lane >> 2) + 8 * j;  // token inside the chunk
-            const int oc = (lane & 3) * 8;       // first of this thread's 8 rows
+            const int g = lane & 3;              // this thread's group of 8 rows
             const int64_t tok = mb + tr;
-            const int64_t o = obase + oc;
-            const uint16_t* sv = stage + tr * 32 + oc;
+            const int64_t o = obase + g * 8;
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + slot_of(tr, g) / 2);
             if (tok < args.M) {
               uint16_t* dst = args.out + tok * args.out_ld + o;
               if (args.vec_store && o + 8 <= args.out_rows) {
-                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sv);
+                *reinterpret_cast<uint4*>(dst) = v;
               } else {
+                const uint16_t* sv = reinterpret_cast<const uint16_t*>(&v);
                 for (int e = 0; e < 8; ++e)
                   if (o + e < args.out_rows) dst[e] = sv[e];
               }
             }
           }
           __syncwarp();
-        };
-#pragma unroll 1
-        for (int c = 0; c < kHalfCols / 32; ++c) {
-          const int64_t mb = m0 + h * kHalfCols + c * 32;
-          if (mb >= args.M) break;  // warp-uniform
-          uint32_t v0[32];
-          tmem_ld_32x32b_x32(taddr + c * 32, v0);
-          tmem_ld_wait();
-          store_chunk(v0, mb);
         }
         tc_fence_before();
         __syncwarp();
