@@ -38,7 +38,8 @@ enum class Mode { kForward, kDgrad };
 // Warp roles of the persistent fused kernel:
 //   warp 0      TMA producer of the token-side operand (and the LoRA operands)
 //   warp 1      MMA issuer (one thread), owner of the TMEM allocation
-//   warps 2-5   epilogue: TMEM -> registers -> bf16 -> global, one TMEM lane quarter each
+//   warps 2-5   epilogue: TMEM -> registers -> bf16 -> shared -> TMA store, one TMEM lane
+//               quarter each
 //   warps 6-15  dequantization, two groups of four warps taking code steps in turn;
 //               warps 9 and 13 stay idle so that no dequantizing warp shares the MMA
 //               warp's scheduler (warp w issues from sub-partition w % 4): the single
@@ -74,7 +75,7 @@ constexpr int kBK = 64;          // contraction per pipeline step
 constexpr int kHalfSlots = 4;    // ring of 256-token operand tiles (2 per step)
 constexpr uint32_t kHalfBytes = kHalfCols * kBK * 2;  // 32 KB
 constexpr uint32_t kWBytes = kTileRows * kBK * 2;     // 16 KB
-constexpr uint32_t kEpiBytes = 4 * 32 * 32 * 2;        // per epilogue warp: 32 tokens x 32 rows
+constexpr uint32_t kEpiBytes = 4 * 2 * 32 * 32 * 2;    // per epilogue warp: 2 x (32 tokens x 32 rows)
 constexpr uint32_t kFusedSmem = kHalfSlots * kHalfBytes + (kWSlots + 1) * kWBytes + kEpiBytes +
                                 1024 + 512 + 1024;
 static_assert(kFusedSmem <= 227 * 1024, "shared memory per CTA");
@@ -91,7 +92,6 @@ struct FusedArgs {
   uint16_t* out;      // [M, out_ld] bf16
   int64_t out_ld;     // N (forward) or K (dgrad)
   int64_t out_rows;   // valid D rows: N (forward) or K (dgrad)
-  int vec_store;      // out 16-byte aligned and out_ld % 8 == 0: 8 rows per vector store
   int codebook;       // 4-bit codebook of the codes (0 NF4, 1 uniform)
   int* err;
 };
@@ -121,14 +121,15 @@ template <Mode MODE, int CB>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     k_fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_act,
                      const __grid_constant__ CUtensorMap tm_ext_w,
-                     const __grid_constant__ CUtensorMap tm_ext_act, const FusedArgs args) {
+                     const __grid_constant__ CUtensorMap tm_ext_act,
+                     const __grid_constant__ CUtensorMap tm_out, const FusedArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* act_s = smem;                             // [kHalfSlots][kHalfBytes] token side
   uint8_t* w_s = act_s + kHalfSlots * kHalfBytes;    // [kWSlots][kWBytes] dequantized
   uint8_t* wext_s = w_s + kWSlots * kWBytes;         // [kWBytes] LoRA weight-side operand
-  uint16_t* epi_s = reinterpret_cast<uint16_t*>(wext_s + kWBytes);  // [4][32][32] staging
+  uint16_t* epi_s = reinterpret_cast<uint16_t*>(wext_s + kWBytes);  // [4][2][32][32] staging
   uint64_t* bars = reinterpret_cast<uint64_t*>(wext_s + kWBytes + kEpiBytes);
   uint64_t* half_full = bars;                       // [kHalfSlots] token tile landed
   uint64_t* half_empty = half_full + kHalfSlots;    // [kHalfSlots] MMAs reading it done
@@ -432,11 +433,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
   } else if (warp >= kEpiWarp0 && warp < kDeqWarp0) {
     // ------------------------------------------------ epilogue
-    // TMEM lane = D row, column = token: each thread holds one D row of 32 tokens. The
-    // chunk is transposed through shared memory (stage[token][row]) so that every store
-    // to the token-major output writes 8 consecutive rows (16 bytes).
+    // TMEM lane = D row, column = token. Each 32 x 32 chunk is transposed through shared
+    // memory (stage[token][row]) into the token-major output's layout.
     const int quarter = warp & 3;  // TMEM lanes this warp may read
-    uint16_t* stage = epi_s + quarter * (32 * 32);
+    uint16_t* stage2 = epi_s + quarter * (2 * 32 * 32);  // two stage buffers, used in turn
+    int chunks = 0;                                      // chunks staged by this warp
+    if (lane == 0) tma_prefetch_desc(&tm_out);
     int uses[kHalves] = {0, 0};
     bool ok = true;
     for (int i = 0; i < my_tiles && ok; ++i) {
@@ -455,16 +457,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const uint32_t taddr =
             tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + h * kHalfCols;
         // One 32-token chunk: two 16-lane TMEM loads in the accumulator-fragment layout,
-        // bf16 pairs, four transposing stmatrix into stage[token][row], then 16-byte
-        // stores of 8 consecutive output rows. A token's 64-byte stage row holds four
-        // 16-byte row groups, group g at slot g ^ ((token >> 1) & 3), so the eight rows
-        // of each stored matrix fall in distinct banks.
-        const uint32_t stage_s = smem_u32(stage);
+        // bf16 pairs, four transposing stmatrix into stage[token][row], then one TMA tile
+        // store. A token's 64-byte stage row holds four 16-byte row groups, group g at
+        // slot g ^ ((token >> 1) & 3), so the eight rows of each stored matrix fall in
+        // distinct banks. The warp's two stage buffers alternate between chunks.
         auto slot_of = [](int tok, int g) { return static_cast<uint32_t>(tok * 64 + ((g ^ ((tok >> 1) & 3)) << 4)); };
 #pragma unroll 1
         for (int c = 0; c < kHalfCols / 32; ++c) {
           const int64_t mb = m0 + h * kHalfCols + c * 32;
           if (mb >= args.M) break;  // warp-uniform
+          uint16_t* stage = stage2 + (chunks & 1) * (32 * 32);
+          const uint32_t stage_s = smem_u32(stage);
+          // the tile store issued from this buffer two chunks ago has read it
+          if (chunks >= 2 && lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          ++chunks;
           uint32_t a[16], b[16];
           tmem_ld_16x256b_x4(taddr + c * 32, a);                 // rows 0-15 of the quarter
           tmem_ld_16x256b_x4(taddr + (16u << 16) + c * 32, b);   // rows 16-31
@@ -479,32 +486,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                               pack_bf16x2_rn(__uint_as_float(b[4 * j]), __uint_as_float(b[4 * j + 1])),
                               pack_bf16x2_rn(__uint_as_float(b[4 * j + 2]), __uint_as_float(b[4 * j + 3])));
           }
+          // the stage's 64-byte rows and their 16-byte group swizzle are the tensor map's
+          // box (32 rows x 32 tokens) and its 64-byte swizzle; rows and tokens outside
+          // the output are not written
+          fence_proxy_async_smem();
           __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int tr = (lane >> 2) + 8 * j;  // token inside the chunk
-            const int g = lane & 3;              // this thread's group of 8 rows
-            const int64_t tok = mb + tr;
-            const int64_t o = obase + g * 8;
-            const uint4 v = *reinterpret_cast<const uint4*>(stage + slot_of(tr, g) / 2);
-            if (tok < args.M) {
-              uint16_t* dst = args.out + tok * args.out_ld + o;
-              if (args.vec_store && o + 8 <= args.out_rows) {
-                *reinterpret_cast<uint4*>(dst) = v;
-              } else {
-                const uint16_t* sv = reinterpret_cast<const uint16_t*>(&v);
-                for (int e = 0; e < 8; ++e)
-                  if (o + e < args.out_rows) dst[e] = sv[e];
-              }
-            }
+          if (lane == 0 && obase < args.out_rows) {
+            tma_store_2d(&tm_out, stage, static_cast<int>(obase), static_cast<int>(mb));
+            bulk_commit_group();
           }
-          __syncwarp();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[h]);
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // tile stores done before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -860,7 +857,7 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
 
 template <Mode MODE>
 cudaError_t run_fused(const CUtensorMap& ta, const CUtensorMap& tw, const CUtensorMap& tx,
-                      FusedArgs args, cudaStream_t st) {
+                      const CUtensorMap& to, FusedArgs args, cudaStream_t st) {
   auto kern = args.codebook == 1 ? k_fused_nf4_gemm<MODE, 1> : k_fused_nf4_gemm<MODE, 0>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
@@ -868,8 +865,6 @@ cudaError_t run_fused(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
   const int64_t rows = (MODE == Mode::kForward) ? args.N : args.K;
   args.row_tiles = static_cast<int>((rows + kTileRows - 1) / kTileRows);
   args.num_tiles = args.row_tiles * static_cast<int>((args.M + kTileCols - 1) / kTileCols);
-  args.vec_store =
-      (args.out_ld % 8 == 0 && (reinterpret_cast<uintptr_t>(args.out) & 15u) == 0) ? 1 : 0;
   const int grid = std::min(args.num_tiles, num_sms());  // persistent: one CTA per SM
   cudaEvent_t before, after;
   profile_events(&before, &after);
@@ -877,7 +872,7 @@ cudaError_t run_fused(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
     e = cudaEventRecord(before, st);
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, kFusedThreads, kFusedSmem, st>>>(ta, tw, tx, args);
+  kern<<<grid, kFusedThreads, kFusedSmem, st>>>(ta, tw, tx, to, args);
   e = cudaGetLastError();
   if (e == cudaSuccess && after) e = cudaEventRecord(after, st);
   return e;
@@ -986,7 +981,10 @@ qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const ui
   a.out_ld = s.N;
   a.out_rows = s.N;
   a.err = device_error_word();
-  QL_TRY(run_fused<Mode::kForward>(ta, tw, tx, a, st));
+  // Y [M, N] for the tile stores: 32 x 32 boxes, 64-byte swizzle (N % 8 == 0, Y aligned)
+  CUtensorMap to;
+  QL_MAP(&to, kBF16, Y, s.N, s.M, s.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  QL_TRY(run_fused<Mode::kForward>(ta, tw, tx, to, a, st));
   return QLORA_OK;
 }
 
@@ -1038,7 +1036,9 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     a.out_ld = s.K;
     a.out_rows = s.K;
     a.err = device_error_word();
-    QL_TRY(run_fused<Mode::kDgrad>(ta, tw, tx, a, st));
+    CUtensorMap to;  // dX [M, K] for the tile stores
+    QL_MAP(&to, kBF16, dX, s.K, s.M, s.K * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    QL_TRY(run_fused<Mode::kDgrad>(ta, tw, tx, to, a, st));
   }
   // dA = scale X^T G (rows k) and dB = scale T^T dY (rows n, stored [r, N]): both contract
   // over the tokens, so they run as one grouped launch and one finalize
