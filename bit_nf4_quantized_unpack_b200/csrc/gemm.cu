@@ -462,10 +462,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // slot g ^ ((token >> 1) & 3), so the eight rows of each stored matrix fall in
         // distinct banks. The warp's two stage buffers alternate between chunks.
         auto slot_of = [](int tok, int g) { return static_cast<uint32_t>(tok * 64 + ((g ^ ((tok >> 1) & 3)) << 4)); };
+        // chunks of this half inside M; the accumulator is released right after the last
+        // one's TMEM load, before its conversion and store
+        const int64_t left = (args.M - m0 - h * kHalfCols + 31) / 32;
+        const int nchunks = left < kHalfCols / 32 ? static_cast<int>(left) : kHalfCols / 32;
 #pragma unroll 1
-        for (int c = 0; c < kHalfCols / 32; ++c) {
+        for (int c = 0; c < nchunks; ++c) {
           const int64_t mb = m0 + h * kHalfCols + c * 32;
-          if (mb >= args.M) break;  // warp-uniform
           uint16_t* stage = stage2 + (chunks & 1) * (32 * 32);
           const uint32_t stage_s = smem_u32(stage);
           // the tile store issued from this buffer two chunks ago has read it
@@ -476,6 +479,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           tmem_ld_16x256b_x4(taddr + c * 32, a);                 // rows 0-15 of the quarter
           tmem_ld_16x256b_x4(taddr + (16u << 16) + c * 32, b);   // rows 16-31
           tmem_ld_wait();
+          if (c == nchunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[h]);
+          }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {  // tokens 8j..8j+7 of the chunk
             // matrix m = row group m (8 rows), its stored row i = token 8j + i
@@ -496,9 +504,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             bulk_commit_group();
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[h]);
       }
     }
     if (lane == 0) bulk_wait_group_all();  // tile stores done before the CTA exits
