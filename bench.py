@@ -37,10 +37,9 @@ WORKLOAD = ("7B-shaped decoder layer training step: q,k,v,o 4096x4096, gate/up 4
 M_TOKENS, RANK_R, ALPHA = 4096, 64, 16.0
 INPUT_OF = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out",
             "gate": "mlp_in", "up": "mlp_in", "down": "mlp_act"}
-KERNELS_PER_LINEAR_STEP = 3 + 8   # forward 3 launches, backward 8 launches
 # dram__bytes_read.sum + dram__bytes_write.sum per FLOP of k_fused_nf4_gemm, from one ncu
 # capture of the current kernel (forward + dX of the 11008 x 4096 linear at M = 4096)
-FUSED_DRAM_BYTES_PER_FLOP = (118.751e6 + 170.849e6) / (3.751e11 + 3.715e11)
+FUSED_DRAM_BYTES_PER_FLOP = (123.030e6 + 169.254e6) / (3.751e11 + 3.715e11)
 
 
 def layer_flops(linears, M, r):
@@ -606,7 +605,9 @@ def main():
     clocks = ClockSampler(device)
     clocks.start()
     clocks.mark()
+    launches0 = qlora.qlora_launch_count()
     ms = time_steps(step, args.steps, world)
+    launches = qlora.qlora_launch_count() - launches0  # this library's kernels, timed region
     clk = clocks.stop()
     value = world * flops / (ms / 1e3) / 1e12
     print(f"[bench] layer step {ms:.3f} ms -> {value:.1f} TFLOP/s per {world} GPU(s)",
@@ -674,7 +675,7 @@ def main():
                            "flops_per_step_per_gpu": flops,
                            "l2": "inputs larger than L2 (weights + activations ~1.3 GB per step)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": KERNELS_PER_LINEAR_STEP * len(inputs.LLAMA7B_LINEARS) * args.steps,
+                "gpu_launches": launches,
                 "clocks": clk, "decode": decode, "codec": codec}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" entry points: host-side validation (nothing is launched
 // when an argument is rejected), dispatch to the kernels, and host utilities.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -14,6 +15,7 @@ namespace {
 thread_local char g_last_error[256] = "";
 thread_local cudaEvent_t g_prof_before = nullptr;
 thread_local cudaEvent_t g_prof_after = nullptr;
+std::atomic<unsigned long long> g_launches{0};
 
 // Per-device error word written by kernels whose bounded waits ran out.
 __device__ int g_device_error;
@@ -119,6 +121,8 @@ int num_sms() {
   return g_sms[dev] > 0 ? g_sms[dev] : 148;
 }
 
+void note_launches(int n) { g_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed); }
+
 void profile_events(cudaEvent_t* before, cudaEvent_t* after) {
   *before = g_prof_before;
   *after = g_prof_after;
@@ -178,6 +182,8 @@ const char* qlora_status_str(qlora_status s) {
 const char* qlora_last_error(void) { return g_last_error; }
 
 int qlora_version(void) { return 100; }
+
+unsigned long long qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 void qlora_profile_events(void* before, void* after) {
   g_prof_before = static_cast<cudaEvent_t>(before);

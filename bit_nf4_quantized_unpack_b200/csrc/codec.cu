@@ -242,6 +242,7 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   double* partial = reinterpret_cast<double*>(static_cast<char*>(ws) +
                                               align_up(static_cast<size_t>(nblocks) * 4, 256));
   const int ctas = quant_ctas(nblocks);
+  note_launches(3);  // blocks, mean, double quantization
   if (w_bf16)
     k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
         static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
@@ -268,6 +269,7 @@ cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_
   const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
   if (g > cap) g = cap;
   auto kern = w.codebook == 1 ? k_dequant<1> : k_dequant<0>;
+  note_launches(1);
   kern<<<static_cast<int>(g), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(w.codes), w.c2,
                                             w.c1, w.mean, nwords, reinterpret_cast<uint4*>(out));
   return cudaGetLastError();

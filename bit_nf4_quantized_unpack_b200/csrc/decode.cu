@@ -431,6 +431,7 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   a.counters = reinterpret_cast<int*>(scratch + part_bytes(p, s) + t_bytes(s));
   a.T_save = T_save;
   a.Y = Y;
+  note_launches(2);  // this kernel and the GEMV below
   k_decode_lora_down<<<kTCtas, kTThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e);

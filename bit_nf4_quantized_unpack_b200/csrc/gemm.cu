@@ -854,6 +854,7 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
   const uint32_t smem = lora_smem(NC);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  note_launches(1);
   kern<<<dim3(static_cast<unsigned>(p.tiles), static_cast<unsigned>(p.splits)), kLoraThreads, smem,
          st>>>(ta, tb, ta1 ? *ta1 : ta, tb1 ? *tb1 : tb, a);
   *splits_out = p.splits;
@@ -877,6 +878,7 @@ cudaError_t run_fused(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
     e = cudaEventRecord(before, st);
     if (e != cudaSuccess) return e;
   }
+  note_launches(1);
   kern<<<grid, kFusedThreads, kFusedSmem, st>>>(ta, tw, tx, to, args);
   e = cudaGetLastError();
   if (e == cudaSuccess && after) e = cudaEventRecord(after, st);
@@ -939,6 +941,7 @@ qlora_status lora_down_T(const uint16_t* X, const uint16_t* A, const LinearShape
   int splits = 0;
   QL_TRY((run_lora_gemm<false, true, 64>(ta, tb, s.M, s.K, part, st, &splits)));
   const int64_t rows_pad = plan_split(s.M, s.K).rows_pad;
+  note_launches(1);
   k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
       part, splits, rows_pad, s.M, s.r, s.scale, t_plain, t_scaled, nullptr, nullptr, nullptr);
   QL_TRY(cudaGetLastError());
@@ -1016,6 +1019,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 128, kSW128);  // dY K-major (over n)
     QL_MAP(&tb, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);    // B [r, N] K-major
     QL_TRY((run_lora_gemm<false, false, 64>(ta, tb, s.M, s.N, part, st, &splits)));
+    note_launches(1);
     k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
         part, splits, plan_split(s.M, s.N).rows_pad, s.M, s.r, s.scale, nullptr, gs, ghl, t, thl);
     QL_TRY(cudaGetLastError());
@@ -1055,6 +1059,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&tb1, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);     // T hi/lo MN-major
     QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits, &ta1, &tb1, s.N)));
     const int64_t stacked = stacked_rows(s.K, s.N);
+    note_launches(1);
     k_finalize_grad<<<blocks_for(stacked, kGradRows), 256, 0, st>>>(
         part, splits, plan_split(stacked, s.M).rows_pad, align_up(s.K, 128), s.K, dA, s.N, dB, s.r,
         s.scale);

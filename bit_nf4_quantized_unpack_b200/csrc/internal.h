@@ -44,6 +44,7 @@ int* device_error_word();                          // per-device error flag of t
 // CUDA events (or NULL) this thread asked to have recorded around each launch of the
 // fused NF4 GEMM kernel (qlora_profile_events).
 void profile_events(cudaEvent_t* before, cudaEvent_t* after);
+void note_launches(int n);                         // count kernels enqueued (qlora_launch_count)
 
 // ---- launchers (codec.cu) -------------------------------------------------------
 size_t quantize_workspace_bytes(int64_t n, int64_t k);

@@ -201,6 +201,7 @@ cudaError_t launch_merge_lora(const qlora_nf4_weight& w, const uint16_t* A, cons
   const dim3 grid(static_cast<unsigned>(bands),
                   static_cast<unsigned>((kt_total + ktiles - 1) / ktiles));
   auto kern = w.codebook == 1 ? k_merge_lora<1> : k_merge_lora<0>;
+  note_launches(1);
   kern<<<grid, kMergeThreads, 0, st>>>(a, static_cast<int>(ktiles));
   return cudaGetLastError();
 }

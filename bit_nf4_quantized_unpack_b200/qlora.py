@@ -47,6 +47,7 @@ _SIGNATURES = {
     "qlora_version": (_i32, []),
     "qlora_device_error": (_i32, [_i32]),
     "qlora_profile_events": (None, [_vp, _vp]),
+    "qlora_launch_count": (ctypes.c_ulonglong, []),
     "qlora_nf4_table": (None, [_vp]),
     "qlora_nf4_thresholds": (None, [_vp]),
     "qlora_nf4_code_buckets": (None, [_vp, _vp]),
@@ -278,6 +279,11 @@ def qlora_profile_events(before=None, after=None):
     """Record torch.cuda.Event pair (or None) around each fused-GEMM launch of this thread."""
     lib().qlora_profile_events(ctypes.c_void_p(before.cuda_event) if before is not None else None,
                                ctypes.c_void_p(after.cuda_event) if after is not None else None)
+
+
+def qlora_launch_count() -> int:
+    """Kernel launches this library has enqueued so far in this process."""
+    return int(lib().qlora_launch_count())
 
 
 def qlora_device_error(clear: bool = True) -> int:

@@ -113,6 +113,13 @@ qlora_status qlora_device_error(int clear);
 void qlora_profile_events(void *before, void *after);
 
 /*
+ * qlora_launch_count: number of kernel launches this library has issued in this
+ * process, on all streams and devices (each launch is counted when it is enqueued).
+ * The difference of two readings is the number of the library's kernels between them.
+ */
+unsigned long long qlora_launch_count(void);
+
+/*
  * qlora_nf4_table: writes the 16 NF4 levels (fp32, ascending, NF4[7] == 0) that the
  * kernels use, to host memory `out16`. Host-only, needs no GPU.
  * Definition: itwiki "QLoRA", section "4비트 NormalFloat(NF4)": N(0,1) quantiles at

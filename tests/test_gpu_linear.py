@@ -171,3 +171,21 @@ def test_graph_replay_matches_eager():
         for got, want, name in zip((Ys, dXs, dAs, dBs), eager[i], ("Y", "dX", "dA", "dB")):
             assert torch.equal(got, want), f"replay {i}: {name}"
     del graph
+
+
+def test_launch_count_per_call():
+    """The library counts its own kernels: 3 per GEMM-path forward (T, its finalize, the
+    fused GEMM), 5 per backward with T saved (G, its finalize, the fused dX GEMM, the
+    grouped dA/dB GEMM and its finalize), 2 per decode-path forward."""
+    case = inputs.linear_case(51, 300, 256, 512, 16, alpha=32)
+    q = qlora.qlora_quantize_nf4_dq(to_dev_bf16(case["W"]))
+    Xd, Ad, Bd, dYd = (to_dev_bf16(case[k]) for k in ("X", "A", "B", "dY"))
+    n0 = qlora.qlora_launch_count()
+    _, T = qlora.qlora_linear_fwd(Xd, q, Ad, Bd, case["scale"])
+    n1 = qlora.qlora_launch_count()
+    qlora.qlora_linear_bwd(dYd, Xd, T, q, Ad, Bd, case["scale"])
+    n2 = qlora.qlora_launch_count()
+    qlora.qlora_linear_fwd(Xd[:4].contiguous(), q, Ad, Bd, case["scale"])
+    n3 = qlora.qlora_launch_count()
+    torch.cuda.synchronize()
+    assert (n1 - n0, n2 - n1, n3 - n2) == (3, 5, 2)
