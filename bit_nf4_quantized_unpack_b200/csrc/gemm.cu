@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "internal.h"
 #include "nf4_device.cuh"
@@ -187,6 +188,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait_and_release();  // inputs of the previous kernel are complete from here on
 
   if (warp == 0) {
     // ------------------------------------------------ TMA: token-side operand, LoRA steps
@@ -588,6 +590,7 @@ __global__ void __launch_bounds__(kLoraThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  griddep_wait_and_release();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -705,6 +708,7 @@ __global__ void k_finalize_rank(const float* __restrict__ part, int splits, int6
                                 int64_t M, int r, float scale, float* __restrict__ plain,
                                 uint16_t* __restrict__ scaled, uint16_t* __restrict__ hilo,
                                 const float* __restrict__ t_in, uint16_t* __restrict__ t_hilo) {
+  griddep_wait_and_release();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= M * 64) return;
   const int64_t m = i >> 6;
@@ -755,6 +759,7 @@ __global__ void __launch_bounds__(256)
     k_finalize_grad(const float* __restrict__ part, int splits, int64_t rows_pad, int64_t pad0,
                     int64_t rows0, float* __restrict__ out0, int64_t rows1,
                     float* __restrict__ out1, int r, float scale) {
+  griddep_wait_and_release();
   __shared__ float tile[kGradRows][65];
   const int64_t srow0 = static_cast<int64_t>(blockIdx.x) * kGradRows;  // stacked
   const bool transpose = srow0 >= pad0;
@@ -831,6 +836,26 @@ size_t partial_floats(int64_t rows, int64_t contraction, int nc) {
   return static_cast<size_t>(p.splits) * p.rows_pad * 64;
 }
 
+// Launch on `st` with programmatic stream serialization: the kernel may begin (its
+// prologue) while the stream's previous kernel drains; every kernel of this file waits
+// for its predecessor with griddep_wait_and_release before it touches global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launches(1);
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Stacked rows of a grouped launch: the first problem padded to whole tiles, then the second.
 inline int64_t stacked_rows(int64_t rows0, int64_t rows1) { return align_up(rows0, 128) + rows1; }
 
@@ -854,11 +879,9 @@ cudaError_t run_lora_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t 
   const uint32_t smem = lora_smem(NC);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  note_launches(1);
-  kern<<<dim3(static_cast<unsigned>(p.tiles), static_cast<unsigned>(p.splits)), kLoraThreads, smem,
-         st>>>(ta, tb, ta1 ? *ta1 : ta, tb1 ? *tb1 : tb, a);
   *splits_out = p.splits;
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(p.tiles), static_cast<unsigned>(p.splits)),
+                    dim3(kLoraThreads), smem, st, ta, tb, ta1 ? *ta1 : ta, tb1 ? *tb1 : tb, a);
 }
 
 template <Mode MODE>
@@ -878,9 +901,7 @@ cudaError_t run_fused(const CUtensorMap& ta, const CUtensorMap& tw, const CUtens
     e = cudaEventRecord(before, st);
     if (e != cudaSuccess) return e;
   }
-  note_launches(1);
-  kern<<<grid, kFusedThreads, kFusedSmem, st>>>(ta, tw, tx, to, args);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, dim3(grid), dim3(kFusedThreads), kFusedSmem, st, ta, tw, tx, to, args);
   if (e == cudaSuccess && after) e = cudaEventRecord(after, st);
   return e;
 }
@@ -941,10 +962,9 @@ qlora_status lora_down_T(const uint16_t* X, const uint16_t* A, const LinearShape
   int splits = 0;
   QL_TRY((run_lora_gemm<false, true, 64>(ta, tb, s.M, s.K, part, st, &splits)));
   const int64_t rows_pad = plan_split(s.M, s.K).rows_pad;
-  note_launches(1);
-  k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
-      part, splits, rows_pad, s.M, s.r, s.scale, t_plain, t_scaled, nullptr, nullptr, nullptr);
-  QL_TRY(cudaGetLastError());
+  QL_TRY(launch_pdl(k_finalize_rank, dim3(blocks_for(s.M * 64, 256)), dim3(256), 0, st, part,
+                    splits, rows_pad, s.M, s.r, s.scale, t_plain, t_scaled, nullptr, nullptr,
+                    nullptr));
   return QLORA_OK;
 }
 
@@ -1019,10 +1039,9 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 128, kSW128);  // dY K-major (over n)
     QL_MAP(&tb, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);    // B [r, N] K-major
     QL_TRY((run_lora_gemm<false, false, 64>(ta, tb, s.M, s.N, part, st, &splits)));
-    note_launches(1);
-    k_finalize_rank<<<blocks_for(s.M * 64, 256), 256, 0, st>>>(
-        part, splits, plan_split(s.M, s.N).rows_pad, s.M, s.r, s.scale, nullptr, gs, ghl, t, thl);
-    QL_TRY(cudaGetLastError());
+    QL_TRY(launch_pdl(k_finalize_rank, dim3(blocks_for(s.M * 64, 256)), dim3(256), 0, st, part,
+                      splits, plan_split(s.M, s.N).rows_pad, s.M, s.r, s.scale, nullptr, gs, ghl,
+                      t, thl));
   }
 
   // dX = dY W_hat + scale G A^T
@@ -1059,11 +1078,9 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     QL_MAP(&tb1, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);     // T hi/lo MN-major
     QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits, &ta1, &tb1, s.N)));
     const int64_t stacked = stacked_rows(s.K, s.N);
-    note_launches(1);
-    k_finalize_grad<<<blocks_for(stacked, kGradRows), 256, 0, st>>>(
-        part, splits, plan_split(stacked, s.M).rows_pad, align_up(s.K, 128), s.K, dA, s.N, dB, s.r,
-        s.scale);
-    QL_TRY(cudaGetLastError());
+    QL_TRY(launch_pdl(k_finalize_grad, dim3(blocks_for(stacked, kGradRows)), dim3(256), 0, st,
+                      part, splits, plan_split(stacked, s.M).rows_pad,
+                      static_cast<int64_t>(align_up(s.K, 128)), s.K, dA, s.N, dB, s.r, s.scale));
   }
   return QLORA_OK;
 }

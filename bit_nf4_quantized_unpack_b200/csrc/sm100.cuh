@@ -219,6 +219,16 @@ __device__ __forceinline__ uint32_t sw128_kmajor_offset(uint32_t row, uint32_t c
   return (row >> 3) * 1024u + (row & 7u) * 128u + ((chunk16 ^ (row & 7u)) << 4);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels launched with programmatic stream serialization may start while the previous
+// kernel of the stream still runs: they set up shared memory and TMEM, then wait here for
+// that kernel (and so, transitively, every earlier one) to complete before touching
+// global memory, and let their own dependents start launching.
+__device__ __forceinline__ void griddep_wait_and_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- thread-block clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
