@@ -97,27 +97,6 @@ struct FusedArgs {
   int* err;
 };
 
-__device__ __forceinline__ void record_error(int* err, volatile int* abort, int code) {
-  atomicCAS(err, 0, code);
-  *abort = 1;
-}
-
-// Wait bounded by time only (used while draining).
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
-}
-
-// Phase parity of the last use of slot s in a ring of `slots` after `uses` uses in all
-// (returns false when the slot was never used).
-__device__ __forceinline__ bool last_use(int uses, int slots, int s, uint32_t& parity) {
-  if (uses <= s) return false;
-  const int last = uses - 1 - ((uses - 1 - s) % slots);
-  parity = static_cast<uint32_t>(last / slots) & 1u;
-  return true;
-}
-
 template <Mode MODE, int CB>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     k_fused_nf4_gemm(const __grid_constant__ CUtensorMap tm_act,

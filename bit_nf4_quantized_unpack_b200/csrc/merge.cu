@@ -3,14 +3,19 @@
 // base is dequantized to BF16 and the LoRA term added, with its alpha/r scale, section
 // "재양자화 시 주의사항"; itwiki "QLoRA", section "한계와 주의점".)
 //
-// A CTA owns a band of 64 rows n and walks consecutive 64 x 64 tiles (one 64-block of K
-// per row each) along K. The rank-r
-// product goes through mma.sync.m16n8k16 (bf16 in, fp32 accumulation) with ldmatrix
-// fragments from shared memory: at r = 64 it is 64 multiply-adds per output element, more
-// than the CUDA cores sustain at the 2.5 bytes of HBM traffic each element costs. Every
-// output element is then fma(scale, product, W_hat) in fp32 (W_hat the exact double
-// dequantization, a bf16 value), rounded to bf16, and the tile leaves through shared
-// memory in 16-byte stores.
+// Persistent tcgen05 kernel (two CTAs per SM) over tiles of 128 rows n x 128 columns k:
+//   warp 0      TMA: B's 128 columns n (B [r, N] as an MN-major operand, two 64-wide
+//               chunks) and A's 128 rows k (A [K, r], K-major over j), into one of two stages
+//   warp 1      MMA: ceil(r/16) tcgen05.mma of 128 x 128 x 16 into one of two 128-column
+//               TMEM buffers, D[n][k] = sum_j B[j][n] A[k][j] in fp32
+//   warps 2-9   epilogue, two per TMEM lane quarter (one 64-column block each): the row's
+//               64 codes and block constants are expanded exactly through a prmt table of
+//               the block's 16 bf16 levels, and every element becomes
+//               bf16(fma(scale, D, W_hat)); each 32 x 32 chunk is staged in shared memory
+//               (64-byte swizzle) and leaves with one TMA tile store
+// At r = 64 the rank-r product is 64 multiply-adds per output element, which the tensor
+// cores absorb; the next tile's product runs while the epilogue drains this one.
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -19,159 +24,250 @@
 namespace qlora {
 namespace {
 
-constexpr int kMergeTile = 64;
-constexpr int kMergeThreads = 256;  // 8 warps: 16 rows x 32 columns of the tile each
-constexpr int kRowPad = 72;         // shared rows of 64 bf16 + 8: 16-byte aligned, banks spread
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(p)));
-}
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                          uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
+constexpr int kMgRows = 128;                     // rows n of a tile (TMEM lanes)
+constexpr int kMgCols = 128;                     // columns k of a tile (TMEM columns)
+constexpr int kMgStages = 2;
+constexpr uint32_t kMgABytes = kMgCols * 64 * 2;  // A rows k x 64 j (zero past r)
+constexpr uint32_t kMgBBytes = kMgRows * 64 * 2;  // B columns n x 64 j, two MN-major chunks
+constexpr int kMgEpiWarps = 8;
+constexpr int kMgThreads = 32 * (2 + kMgEpiWarps);
+constexpr uint32_t kMgStageOut = 2 * 32 * 64;   // per epilogue warp: two 32 x 32 bf16 chunks
+constexpr uint32_t kMgSmem =
+    kMgStages * (kMgABytes + kMgBBytes) + kMgEpiWarps * kMgStageOut + 1024 + 256 + 1024;
+constexpr int kMgCtasPerSm = 2;  // TMEM: 2 x (2 x kMgCols) columns
 
 struct MergeArgs {
   const uint8_t* codes;
   const uint8_t* c2;
   const float* c1;
   const float* mean;
-  const uint16_t* A;  // [K, r]
-  const uint16_t* B;  // [r, N]
   int64_t N, K;
   int r;
   float scale;
-  uint16_t* out;      // [N, K]
+  uint16_t* out;   // [N, K]
+  int row_tiles;   // tiles along n
+  int num_tiles;   // row_tiles x tiles along k
+  int* err;
 };
 
-// grid: x = 64-row bands of W, y = groups of `ktiles` consecutive 64-column tiles. B's
-// band, the T8 table and the MMA fragments that come from B are staged once per CTA.
 template <int CB>
-__global__ void __launch_bounds__(kMergeThreads) k_merge_lora(const MergeArgs a, int ktiles) {
-  __shared__ __align__(16) uint16_t bs[kMergeTile][kRowPad];  // B[j][n0 + i] (rows j >= r zero)
-  __shared__ __align__(16) uint16_t as[kMergeTile][kRowPad];  // A[k0 + i][j] (cols j >= r zero)
-  __shared__ __align__(16) uint16_t os[kMergeTile][kRowPad];  // output tile [n][k]
-  __shared__ __align__(16) uint8_t cs[kMergeTile][32];        // codes of the tile's rows
-  __shared__ float srow[kMergeTile];                          // block scale of each row
-  __shared__ float lut[16];
-  __shared__ float t8[256];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wr = 16 * (warp & 3);   // first tile row of this warp
-  const int wc = 32 * (warp >> 2);  // first tile column of this warp
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kMergeTile;
-  const int64_t kt_total = a.K / kMergeTile;
-  const int64_t kt0 = static_cast<int64_t>(blockIdx.y) * ktiles;
-  const int64_t kt1 = kt0 + ktiles < kt_total ? kt0 + ktiles : kt_total;
-  const int r = a.r, r16 = (a.r + 15) & ~15;
-  const float mean = *a.mean;
+__global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
+    k_merge_lora(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_out, const MergeArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* a_s = smem;                                   // [stages][kMgABytes]
+  uint8_t* b_s = a_s + kMgStages * kMgABytes;            // [stages][kMgBBytes]
+  uint8_t* o_s = b_s + kMgStages * kMgBBytes;             // [epilogue warps][2][32][64 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(o_s + kMgEpiWarps * kMgStageOut);
+  uint64_t* full = bars;                    // [stages] operands landed
+  uint64_t* empty = full + kMgStages;       // [stages] MMAs reading them done
+  uint64_t* acc_full = empty + kMgStages;   // [2] product complete
+  uint64_t* acc_empty = acc_full + 2;       // [2] product read out
+  uint64_t* mma_drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* t8 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // [256]
 
-  for (int e = tid; e < 256; e += kMergeThreads) t8[e] = t8_value(e);
-  if (tid < 16) lut[tid] = code_level<CB>(tid);
-  for (int idx = tid; idx < r16 * 8; idx += kMergeThreads) {
-    const int j = idx >> 3, c = idx & 7;  // chunk c of row j: columns n0 + 8c .. + 7
-    const int64_t n = n0 + c * 8;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (j < r && n < a.N) v = __ldg(reinterpret_cast<const uint4*>(a.B + j * a.N + n));
-    *reinterpret_cast<uint4*>(&bs[j][c * 8]) = v;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) t8[e] = t8_value(e);
+  const int my_tiles = (static_cast<int>(blockIdx.x) < args.num_tiles)
+                           ? (args.num_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                           : 0;
+  // consecutive CTAs take consecutive row bands of the same columns (A tile shared in L2)
+  auto tile_coords = [&](int i, int64_t& n0, int64_t& k0) {
+    const int tile = blockIdx.x + i * gridDim.x;
+    n0 = static_cast<int64_t>(tile % args.row_tiles) * kMgRows;
+    k0 = static_cast<int64_t>(tile / args.row_tiles) * kMgCols;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMgStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kMgEpiWarps);
+    }
+    mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * kMgCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  // the math A operand of the rank-r product is B^T (rows n, columns j), read transposed
-  // from bs[j][n]: the same for every column tile, so it stays in registers
-  const int mat = lane >> 3, rr = lane & 7;
-  uint32_t af[4][4];
-#pragma unroll
-  for (int jb = 0; jb < 4; ++jb)
-    if (16 * jb < r16)
-      ldsm_x4_trans(af[jb], &bs[16 * jb + rr + ((mat >> 1) << 3)][wr + ((mat & 1) << 3)]);
-  const int g = lane >> 2, t = lane & 3;
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
 
-  for (int64_t kt = kt0; kt < kt1; ++kt) {
-    const int64_t k0 = kt * kMergeTile;
-    const uint16_t* arow = a.A + k0 * r;
-#pragma unroll
-    for (int it = 0; it < (kMergeTile * 8) / kMergeThreads; ++it) {
-      const int idx = tid + it * kMergeThreads;
-      const int i = idx >> 3, c = idx & 7;  // 8-wide chunk c of row k0 + i (zeros past r)
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (c * 8 < r) v = __ldg(reinterpret_cast<const uint4*>(arow + i * r + c * 8));
-      *reinterpret_cast<uint4*>(&as[i][c * 8]) = v;
-    }
-    if (tid < 2 * kMergeTile) {
-      const int i = tid >> 1, h = tid & 1;  // 16 code bytes of row n0 + i
-      const int64_t n = n0 + i;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (n < a.N)
-        v = __ldg(reinterpret_cast<const uint4*>(a.codes + n * (a.K / 2) + k0 / 2 + h * 16));
-      *reinterpret_cast<uint4*>(&cs[i][h * 16]) = v;
-    } else if (tid < 3 * kMergeTile) {
-      const int i = tid - 2 * kMergeTile;
-      const int64_t n = n0 + i;
-      float sv = 0.f;
-      if (n < a.N) {
-        const int64_t j = n * (a.K / 64) + kt;
-        sv = block_scale_tab(t8, __ldg(a.c2 + j), __ldg(a.c1 + (j >> 8)), mean);
+  if (warp == 0) {
+    // ------------------------------------------------ TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      int issued = 0;
+      for (int i = 0; i < my_tiles; ++i) {
+        const int s = i % kMgStages;
+        if (i >= kMgStages && !mbar_wait(&empty[s], ((i / kMgStages) - 1) & 1u, abort_flag)) {
+          record_error(args.err, abort_flag, kErrTimeoutProducer);
+          break;
+        }
+        int64_t n0, k0;
+        tile_coords(i, n0, k0);
+        mbar_arrive_expect_tx(&full[s], kMgABytes + kMgBBytes);
+        tma_load_2d(b_s + s * kMgBBytes, &tm_b, &full[s], static_cast<int>(n0), 0);
+        tma_load_2d(b_s + s * kMgBBytes + 8192, &tm_b, &full[s], static_cast<int>(n0) + 64, 0);
+        tma_load_2d(a_s + s * kMgABytes, &tm_a, &full[s], 0, static_cast<int>(k0));
+        ++issued;
       }
-      srow[i] = sv;
+      if (*abort_flag)  // copies in flight land before the CTA exits
+        for (int i = (issued > kMgStages ? issued - kMgStages : 0); i < issued; ++i)
+          mbar_wait_drain(&full[i % kMgStages], (i / kMgStages) & 1u);
     }
-    __syncthreads();
-
-    // (A B)^T for this warp's 16 rows and 32 columns: the math B operand (j x k) is A^T,
-    // whose columns are the rows of as
-    float acc[4][4];
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      // A operand: B^T (rows n, K = j) MN-major, 64-row chunks 8 KB apart; B operand: A's
+      // rows k, K-major. Per 16-wide j slice the MN-major operand advances 16 rows of
+      // 128 bytes (2048 B) and the K-major one 32 bytes.
+      constexpr uint32_t idesc = idesc_bf16_f32(kMgRows, kMgCols, true, false);
+      const int nk = (args.r + 15) / 16;
+      int done = 0;
+      for (int i = 0; i < my_tiles; ++i) {
+        const int s = i % kMgStages, b = i & 1;
+        if (!mbar_wait(&full[s], (i / kMgStages) & 1u, abort_flag)) {
+          record_error(args.err, abort_flag, kErrTimeoutMma);
+          break;
+        }
+        if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1u, abort_flag)) {
+          record_error(args.err, abort_flag, kErrTimeoutMma);
+          break;
+        }
+        tc_fence_after();
+        const uint64_t da = smem_desc_sw128(smem_u32(b_s + s * kMgBBytes), 8192, 1024);
+        const uint64_t db = smem_desc_sw128(smem_u32(a_s + s * kMgABytes), 16, 1024);
+        for (int kk = 0; kk < nk; ++kk)
+          umma_bf16(tmem_base + b * kMgCols, da + kk * 128u, db + kk * 2u, idesc, kk != 0);
+        umma_commit(&empty[s]);
+        umma_commit(&acc_full[b]);
+        ++done;
+      }
+      umma_commit(mma_drain);
+      mbar_wait_drain(mma_drain, 0);
+      uint32_t par;
+      for (int s = 0; s < kMgStages; ++s)
+        if (last_use(done, kMgStages, s, par)) mbar_wait_drain(&empty[s], par);
+      for (int b = 0; b < 2; ++b)
+        if (last_use(done, 2, b, par)) mbar_wait_drain(&acc_full[b], par);
+    }
+  } else {
+    // ------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int quarter = warp & 3;           // TMEM lanes this warp may read
+    const int col0 = (ew >> 2) * 64;        // its 64-column block of the tile
+    const float mean = *args.mean;
+    uint8_t* stage2 = o_s + ew * kMgStageOut;  // this warp's two chunk buffers
+    int chunks = 0;
+    if (lane == 0) tma_prefetch_desc(&tm_out);
+    const int64_t bpr = args.K / 64;        // 64-blocks per row
+    const int64_t code_ld = args.K / 2;
+    // the codes (2 x 16 bytes) and raw block constants of this thread's row in its block
+    // of tile i (the scale is formed when the block is used, so the loads stay in flight)
+    auto fetch = [&](int i, uint4& q0, uint4& q1, uint32_t& e2, float& e1, bool& live,
+                     int64_t& n, int64_t& kb) {
+      int64_t n0, k0;
+      tile_coords(i, n0, k0);
+      n = n0 + quarter * 32 + lane;
+      kb = k0 + col0;
+      q0 = q1 = make_uint4(0u, 0u, 0u, 0u);
+      e2 = 0u;
+      e1 = 0.f;
+      live = n < args.N && kb < args.K;
+      if (live) {
+        const uint4* src = reinterpret_cast<const uint4*>(args.codes + n * code_ld + kb / 2);
+        q0 = __ldg(src);
+        q1 = __ldg(src + 1);
+        const int64_t j = n * bpr + kb / 64;
+        e2 = __ldg(args.c2 + j);
+        e1 = __ldg(args.c1 + (j >> 8));
+      }
+    };
+    uint4 q0, q1;
+    uint32_t e2;
+    float e1;
+    bool live;
+    int64_t n, kb;
+    if (my_tiles > 0) fetch(0, q0, q1, e2, e1, live, n, kb);
+    for (int i = 0; i < my_tiles; ++i) {
+      const int b = i & 1;
+      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const float s_cur = live ? block_scale_tab(t8, e2, e1, mean) : 0.f;
+      const int64_t n_cur = n, kb_cur = kb;
+      if (i + 1 < my_tiles) fetch(i + 1, q0, q1, e2, e1, live, n, kb);  // one tile ahead
+      Nf4Lut lut;
+      build_lut<CB>(s_cur, lut);
+      if (!mbar_wait(&acc_full[b], (i >> 1) & 1u, abort_flag)) {
+        if (!*abort_flag) record_error(args.err, abort_flag, kErrTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after();
+      if (kb_cur < args.K) {  // warp-uniform
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+        for (int h = 0; h < 2; ++h) {  // 32-column chunks of the block
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * kMgCols +
+                                 col0 + h * 32,
+                             v);
+          tmem_ld_wait();
+          if (h == 1) {  // this warp's part of buffer b is in registers
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+          }
+          // stage row = this lane's row n, its 16-byte group w at slot w ^ ((lane >> 1) & 3)
+          uint8_t* stage = stage2 + (chunks & 1) * (32 * 64);
+          if (chunks >= 2 && lane == 0) bulk_wait_group_read<1>();  // its previous store read it
+          __syncwarp();
+          ++chunks;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
+          for (int w = 0; w < 4; ++w) {
+            uint32_t o[4], y[4];
+            lut_decode8(words[4 * h + w], lut, o);  // elements 8w .. 8w+7 of the chunk
 #pragma unroll
-    for (int jb = 0; jb < 4; ++jb) {
-      if (16 * jb >= r16) break;
-#pragma unroll
-      for (int kt2 = 0; kt2 < 2; ++kt2) {
-        uint32_t bf[4];
-        ldsm_x4(bf, &as[wc + 16 * kt2 + rr + ((mat >> 1) << 3)][16 * jb + ((mat & 1) << 3)]);
-        mma_16816(acc[2 * kt2], af[jb], bf[0], bf[1]);
-        mma_16816(acc[2 * kt2 + 1], af[jb], bf[2], bf[3]);
+            for (int p = 0; p < 4; ++p) {
+              const float w_lo = __uint_as_float(o[p] << 16);
+              const float w_hi = __uint_as_float(o[p] & 0xFFFF0000u);
+              const int e = 8 * w + 2 * p;
+              y[p] = pack_bf16x2_rn(__fmaf_rn(args.scale, __uint_as_float(v[e]), w_lo),
+                                    __fmaf_rn(args.scale, __uint_as_float(v[e + 1]), w_hi));
+            }
+            *reinterpret_cast<uint4*>(stage + lane * 64 + ((w ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(y[0], y[1], y[2], y[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0)  // rows past N are not written
+            tma_store_2d(&tm_out, stage, static_cast<int>(kb_cur + h * 32),
+                         static_cast<int>(n_cur - lane));
+          if (lane == 0) bulk_commit_group();
+        }
+      } else {  // block past K: nothing to read, release the buffer
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
       }
     }
-
-    // C fragment: (row g, columns 2t, 2t+1) and (row g + 8, same columns) of each 8-column tile
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int nl = wr + g + 8 * h;
-        const int kl = wc + 8 * q + 2 * t;
-        const uint32_t byte = cs[nl][kl >> 1];  // codes of columns kl (low nibble), kl + 1
-        const float sv = srow[nl];
-        const float w0 =
-            __uint_as_float(static_cast<uint32_t>(bf16_bits_rn(__fmul_rn(lut[byte & 15u], sv))) << 16);
-        const float w1 =
-            __uint_as_float(static_cast<uint32_t>(bf16_bits_rn(__fmul_rn(lut[byte >> 4], sv))) << 16);
-        const uint32_t y0 = bf16_bits_rn(__fmaf_rn(a.scale, acc[q][2 * h], w0));
-        const uint32_t y1 = bf16_bits_rn(__fmaf_rn(a.scale, acc[q][2 * h + 1], w1));
-        *reinterpret_cast<uint32_t*>(&os[nl][kl]) = y0 | (y1 << 16);
-      }
-    __syncthreads();  // os complete; as, cs and srow free for the next tile
-#pragma unroll
-    for (int i = 0; i < (kMergeTile * 8) / kMergeThreads; ++i) {
-      const int idx = tid + i * kMergeThreads;
-      const int row = idx >> 3, ch = idx & 7;
-      const int64_t n = n0 + row;
-      if (n < a.N)
-        *reinterpret_cast<uint4*>(a.out + n * a.K + k0 + ch * 8) =
-            *reinterpret_cast<const uint4*>(&os[row][ch * 8]);
-    }
+    if (lane == 0) bulk_wait_group_all();  // tile stores done before the CTA exits
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kMgCols);
   }
 }
 
@@ -184,25 +280,32 @@ cudaError_t launch_merge_lora(const qlora_nf4_weight& w, const uint16_t* A, cons
   a.c2 = w.c2;
   a.c1 = w.c1;
   a.mean = w.mean;
-  a.A = A;
-  a.B = B;
   a.N = w.n_out;
   a.K = w.k_in;
   a.r = r;
   a.scale = scale;
   a.out = out;
-  // enough CTAs for several waves, each walking at most 8 column tiles of its band
-  const int64_t bands = (w.n_out + kMergeTile - 1) / kMergeTile;
-  const int64_t kt_total = w.k_in / kMergeTile;
-  const int64_t want = static_cast<int64_t>(num_sms()) * 24;
-  int64_t ktiles = (bands * kt_total + want - 1) / want;
-  ktiles = ktiles < 1 ? 1 : (ktiles > 8 ? 8 : ktiles);
-  if ((kt_total + ktiles - 1) / ktiles > 65535) ktiles = (kt_total + 65534) / 65535;  // grid y
-  const dim3 grid(static_cast<unsigned>(bands),
-                  static_cast<unsigned>((kt_total + ktiles - 1) / ktiles));
+  a.row_tiles = static_cast<int>((w.n_out + kMgRows - 1) / kMgRows);
+  a.num_tiles = a.row_tiles * static_cast<int>((w.k_in + kMgCols - 1) / kMgCols);
+  a.err = device_error_word();
+  CUtensorMap ta, tb, to;
+  // A [K, r]: rows k, 64-wide j box (zero past r); B [r, N]: 64 x 64 boxes of (n, j)
+  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, w.k_in, static_cast<uint64_t>(r) * 2,
+                    64, kMgCols, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, w.n_out, r, w.n_out * 2, 64, 64,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      // out [N, K]: 32 x 32 boxes (k inner), 64-byte swizzle
+      !make_tmap_2d(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, w.k_in, w.n_out, w.k_in * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
   auto kern = w.codebook == 1 ? k_merge_lora<1> : k_merge_lora<0>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMgSmem);
+  if (e != cudaSuccess) return e;
+  const int slots = num_sms() * kMgCtasPerSm;
+  const int grid = a.num_tiles < slots ? a.num_tiles : slots;  // persistent
+  if (grid == 0) return cudaSuccess;
   note_launches(1);
-  kern<<<grid, kMergeThreads, 0, st>>>(a, static_cast<int>(ktiles));
+  kern<<<grid, kMgThreads, kMgSmem, st>>>(ta, tb, to, a);
   return cudaGetLastError();
 }
 

@@ -70,6 +70,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Record the first error code of the launch in the device error word and tell the CTA's
+// other roles to give up their waits.
+__device__ __forceinline__ void record_error(int* err, volatile int* abort, int code) {
+  atomicCAS(err, 0, code);
+  *abort = 1;
+}
+
+// Wait bounded by time only (used while draining).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
+}
+
+// Phase parity of the last use of slot s in a ring of `slots` after `uses` uses in all
+// (returns false when the slot was never used).
+__device__ __forceinline__ bool last_use(int uses, int slots, int s, uint32_t& parity) {
+  if (uses <= s) return false;
+  const int last = uses - 1 - ((uses - 1 - s) % slots);
+  parity = static_cast<uint32_t>(last / slots) & 1u;
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
