@@ -5,7 +5,8 @@
 //
 // Persistent tcgen05 kernel (two CTAs per SM) over tiles of 128 rows n x 128 columns k:
 //   warp 0      TMA: B's 128 columns n (B [r, N] as an MN-major operand, two 64-wide
-//               chunks) and A's 128 rows k (A [K, r], K-major over j), into one of two stages
+//               chunks), A's 128 rows k (A [K, r], K-major over j) and the tile's codes
+//               (128 rows x 64 bytes), into one of two stages
 //   warp 1      MMA: ceil(r/16) tcgen05.mma of 128 x 128 x 16 into one of two 128-column
 //               TMEM buffers, D[n][k] = sum_j B[j][n] A[k][j] in fp32
 //   warps 2-9   epilogue, two per TMEM lane quarter (one 64-column block each): the row's
@@ -31,13 +32,13 @@ constexpr uint32_t kMgABytes = kMgCols * 64 * 2;  // A rows k x 64 j (zero past 
 constexpr uint32_t kMgBBytes = kMgRows * 64 * 2;  // B columns n x 64 j, two MN-major chunks
 constexpr int kMgEpiWarps = 8;
 constexpr int kMgThreads = 32 * (2 + kMgEpiWarps);
-constexpr uint32_t kMgStageOut = 2 * 32 * 64;   // per epilogue warp: two 32 x 32 bf16 chunks
-constexpr uint32_t kMgSmem =
-    kMgStages * (kMgABytes + kMgBBytes) + kMgEpiWarps * kMgStageOut + 1024 + 256 + 1024;
+constexpr uint32_t kMgCBytes = kMgRows * kMgCols / 2;  // the tile's codes, 64-byte swizzle
+constexpr uint32_t kMgStageOut = 32 * 64;       // per epilogue warp: one 32 x 32 bf16 chunk
+constexpr uint32_t kMgSmem = kMgStages * (kMgABytes + kMgBBytes + kMgCBytes) +
+                             kMgEpiWarps * kMgStageOut + 1024 + 256 + 1024;
 constexpr int kMgCtasPerSm = 2;  // TMEM: 2 x (2 x kMgCols) columns
 
 struct MergeArgs {
-  const uint8_t* codes;
   const uint8_t* c2;
   const float* c1;
   const float* mean;
@@ -53,16 +54,18 @@ struct MergeArgs {
 template <int CB>
 __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
     k_merge_lora(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_codes,
                  const __grid_constant__ CUtensorMap tm_out, const MergeArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* a_s = smem;                                   // [stages][kMgABytes]
   uint8_t* b_s = a_s + kMgStages * kMgABytes;            // [stages][kMgBBytes]
-  uint8_t* o_s = b_s + kMgStages * kMgBBytes;             // [epilogue warps][2][32][64 B]
+  uint8_t* c_s = b_s + kMgStages * kMgBBytes;             // [stages][128 rows][64 B] codes
+  uint8_t* o_s = c_s + kMgStages * kMgCBytes;             // [epilogue warps][32][64 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(o_s + kMgEpiWarps * kMgStageOut);
   uint64_t* full = bars;                    // [stages] operands landed
-  uint64_t* empty = full + kMgStages;       // [stages] MMAs reading them done
+  uint64_t* empty = full + kMgStages;       // [stages] MMAs and epilogue warps done with them
   uint64_t* acc_full = empty + kMgStages;   // [2] product complete
   uint64_t* acc_empty = acc_full + 2;       // [2] product read out
   uint64_t* mma_drain = acc_empty + 2;
@@ -85,7 +88,7 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMgStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + kMgEpiWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -109,6 +112,7 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
     if (lane == 0) {
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
+      tma_prefetch_desc(&tm_codes);
       int issued = 0;
       for (int i = 0; i < my_tiles; ++i) {
         const int s = i % kMgStages;
@@ -118,7 +122,9 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
         }
         int64_t n0, k0;
         tile_coords(i, n0, k0);
-        mbar_arrive_expect_tx(&full[s], kMgABytes + kMgBBytes);
+        mbar_arrive_expect_tx(&full[s], kMgABytes + kMgBBytes + kMgCBytes);
+        tma_load_2d(c_s + s * kMgCBytes, &tm_codes, &full[s], static_cast<int>(k0 / 2),
+                    static_cast<int>(n0));
         tma_load_2d(b_s + s * kMgBBytes, &tm_b, &full[s], static_cast<int>(n0), 0);
         tma_load_2d(b_s + s * kMgBBytes + 8192, &tm_b, &full[s], static_cast<int>(n0) + 64, 0);
         tma_load_2d(a_s + s * kMgABytes, &tm_a, &full[s], 0, static_cast<int>(k0));
@@ -170,51 +176,58 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
     const int quarter = warp & 3;           // TMEM lanes this warp may read
     const int col0 = (ew >> 2) * 64;        // its 64-column block of the tile
     const float mean = *args.mean;
-    uint8_t* stage2 = o_s + ew * kMgStageOut;  // this warp's two chunk buffers
+    uint8_t* stage1 = o_s + ew * kMgStageOut;  // this warp's chunk buffer
     int chunks = 0;
     if (lane == 0) tma_prefetch_desc(&tm_out);
     const int64_t bpr = args.K / 64;        // 64-blocks per row
-    const int64_t code_ld = args.K / 2;
-    // the codes (2 x 16 bytes) and raw block constants of this thread's row in its block
-    // of tile i (the scale is formed when the block is used, so the loads stay in flight)
-    auto fetch = [&](int i, uint4& q0, uint4& q1, uint32_t& e2, float& e1, bool& live,
-                     int64_t& n, int64_t& kb) {
+    // the raw block constants of this thread's row in its block of tile i (the scale is
+    // formed when the block is used, so the loads stay in flight meanwhile)
+    auto fetch = [&](int i, uint32_t& e2, float& e1, bool& live, int64_t& n, int64_t& kb) {
       int64_t n0, k0;
       tile_coords(i, n0, k0);
       n = n0 + quarter * 32 + lane;
       kb = k0 + col0;
-      q0 = q1 = make_uint4(0u, 0u, 0u, 0u);
       e2 = 0u;
       e1 = 0.f;
       live = n < args.N && kb < args.K;
       if (live) {
-        const uint4* src = reinterpret_cast<const uint4*>(args.codes + n * code_ld + kb / 2);
-        q0 = __ldg(src);
-        q1 = __ldg(src + 1);
         const int64_t j = n * bpr + kb / 64;
         e2 = __ldg(args.c2 + j);
         e1 = __ldg(args.c1 + (j >> 8));
       }
     };
-    uint4 q0, q1;
+    // this lane's row of the staged codes: its 16-byte groups g at slot g ^ ((row >> 1) & 3)
+    const int crow = quarter * 32 + lane;
+    const int g0 = col0 / 32;  // first 16-byte group of this warp's block
     uint32_t e2;
     float e1;
     bool live;
     int64_t n, kb;
-    if (my_tiles > 0) fetch(0, q0, q1, e2, e1, live, n, kb);
+    if (my_tiles > 0) fetch(0, e2, e1, live, n, kb);
     for (int i = 0; i < my_tiles; ++i) {
-      const int b = i & 1;
-      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const int b = i & 1, s = i % kMgStages;
       const float s_cur = live ? block_scale_tab(t8, e2, e1, mean) : 0.f;
       const int64_t n_cur = n, kb_cur = kb;
-      if (i + 1 < my_tiles) fetch(i + 1, q0, q1, e2, e1, live, n, kb);  // one tile ahead
+      if (i + 1 < my_tiles) fetch(i + 1, e2, e1, live, n, kb);  // one tile ahead
       Nf4Lut lut;
       build_lut<CB>(s_cur, lut);
-      if (!mbar_wait(&acc_full[b], (i >> 1) & 1u, abort_flag)) {
+      // codes of stage s (landed before the MMA that completes acc_full ran)
+      if (!mbar_wait(&full[s], (i / kMgStages) & 1u, abort_flag) ||
+          !mbar_wait(&acc_full[b], (i >> 1) & 1u, abort_flag)) {
         if (!*abort_flag) record_error(args.err, abort_flag, kErrTimeoutEpilogue);
         break;
       }
       tc_fence_after();
+      uint32_t words[8];
+      {
+        const uint8_t* crow_s = c_s + s * kMgCBytes + crow * 64;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(crow_s + (((g0) ^ ((crow >> 1) & 3)) << 4));
+        const uint4 q1 = *reinterpret_cast<const uint4*>(crow_s + (((g0 + 1) ^ ((crow >> 1) & 3)) << 4));
+        words[0] = q0.x; words[1] = q0.y; words[2] = q0.z; words[3] = q0.w;
+        words[4] = q1.x; words[5] = q1.y; words[6] = q1.z; words[7] = q1.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // this warp's codes are in registers
       if (kb_cur < args.K) {  // warp-uniform
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // 32-column chunks of the block
@@ -229,8 +242,8 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
             if (lane == 0) mbar_arrive(&acc_empty[b]);
           }
           // stage row = this lane's row n, its 16-byte group w at slot w ^ ((lane >> 1) & 3)
-          uint8_t* stage = stage2 + (chunks & 1) * (32 * 64);
-          if (chunks >= 2 && lane == 0) bulk_wait_group_read<1>();  // its previous store read it
+          uint8_t* stage = stage1;
+          if (chunks >= 1 && lane == 0) bulk_wait_group_read<0>();  // the previous store read it
           __syncwarp();
           ++chunks;
 #pragma unroll
@@ -276,7 +289,6 @@ __global__ void __launch_bounds__(kMgThreads, kMgCtasPerSm)
 cudaError_t launch_merge_lora(const qlora_nf4_weight& w, const uint16_t* A, const uint16_t* B,
                               int r, float scale, uint16_t* out, cudaStream_t st) {
   MergeArgs a;
-  a.codes = w.codes;
   a.c2 = w.c2;
   a.c1 = w.c1;
   a.mean = w.mean;
@@ -288,12 +300,15 @@ cudaError_t launch_merge_lora(const qlora_nf4_weight& w, const uint16_t* A, cons
   a.row_tiles = static_cast<int>((w.n_out + kMgRows - 1) / kMgRows);
   a.num_tiles = a.row_tiles * static_cast<int>((w.k_in + kMgCols - 1) / kMgCols);
   a.err = device_error_word();
-  CUtensorMap ta, tb, to;
+  CUtensorMap ta, tb, tc, to;
   // A [K, r]: rows k, 64-wide j box (zero past r); B [r, N]: 64 x 64 boxes of (n, j)
   if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, w.k_in, static_cast<uint64_t>(r) * 2,
                     64, kMgCols, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, w.n_out, r, w.n_out * 2, 64, 64,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      // codes [N, K/2] bytes: 64-byte x 128-row boxes, 64-byte swizzle
+      !make_tmap_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.codes, w.k_in / 2, w.n_out, w.k_in / 2,
+                    kMgCols / 2, kMgRows, CU_TENSOR_MAP_SWIZZLE_64B) ||
       // out [N, K]: 32 x 32 boxes (k inner), 64-byte swizzle
       !make_tmap_2d(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, w.k_in, w.n_out, w.k_in * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B))
@@ -305,7 +320,7 @@ cudaError_t launch_merge_lora(const qlora_nf4_weight& w, const uint16_t* A, cons
   const int grid = a.num_tiles < slots ? a.num_tiles : slots;  // persistent
   if (grid == 0) return cudaSuccess;
   note_launches(1);
-  kern<<<grid, kMgThreads, kMgSmem, st>>>(ta, tb, to, a);
+  kern<<<grid, kMgThreads, kMgSmem, st>>>(ta, tb, tc, to, a);
   return cudaGetLastError();
 }
 
