@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(kQuantThreads)
   for (int i = threadIdx.x; i < kCodeBuckets; i += blockDim.x)
     sb[i] = make_float2(tab.thr[i], __uint_as_float(static_cast<uint32_t>(tab.code[i])));
   __syncthreads();
+  // the double quantization may be scheduled now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   double acc = 0.0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * per_cta;
   int64_t b = blockIdx.x * per_cta + threadIdx.x / 8;
@@ -127,38 +129,40 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
-// Level 2a: the one mean of all block constants (fp64 sum, one rounding to fp32).
-__global__ void __launch_bounds__(1024)
-    k_constants_mean(const double* __restrict__ partial, int nparts, int64_t nblocks,
-                     float* __restrict__ mean) {
-  __shared__ double red[32];
-  double acc = 0.0;
-  for (int i = threadIdx.x; i < nparts; i += blockDim.x) acc += partial[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double s = 0.0;
-    for (int i = 0; i < static_cast<int>(blockDim.x / 32); ++i) s += red[i];
-    mean[0] = __double2float_rn(s / static_cast<double>(nblocks));
-  }
-}
-
 // Index of entry i of T8 (ascending) -> its E4M3 bit pattern.
 __device__ __forceinline__ uint32_t t8_index_to_code(int i) {
   return (i < 126) ? (0xFEu - static_cast<uint32_t>(i)) : (i == 126 ? 0u : static_cast<uint32_t>(i - 126));
 }
 
-// Level 2b: one warp per 256-block of constants, 8 constants per lane.
+// Level 2: the one mean of all block constants, then one warp per 256-block of constants,
+// 8 constants per lane. Launched as the programmatic dependent of level 1: every CTA forms
+// the mean itself from level 1's per-CTA fp64 partial sums, in the same order (fp64 sum,
+// one rounding to fp32), and CTA 0 stores it.
 __global__ void __launch_bounds__(256)
     k_double_quantize(const float* __restrict__ absmax, int64_t nblocks,
-                      const float* __restrict__ mean_p, const T8Thresholds th,
-                      uint8_t* __restrict__ c2, float* __restrict__ c1) {
+                      const double* __restrict__ partial, int nparts, float* __restrict__ mean_out,
+                      const T8Thresholds th, uint8_t* __restrict__ c2, float* __restrict__ c1) {
   __shared__ float sth[kT8Size - 1];
+  __shared__ double red[256 / 32];
+  __shared__ float mean_s;
   for (int i = threadIdx.x; i < kT8Size - 1; i += blockDim.x) sth[i] = th.t[i];
-  __syncthreads();
-  const float mean = *mean_p;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // level 1's absmax and partial sums
+  {
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < nparts; i += blockDim.x) acc += partial[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double sum = 0.0;
+      for (int i = 0; i < 256 / 32; ++i) sum += red[i];
+      mean_s = __double2float_rn(sum / static_cast<double>(nblocks));
+      if (blockIdx.x == 0) mean_out[0] = mean_s;
+    }
+    __syncthreads();
+  }
+  const float mean = mean_s;
   const int lane = threadIdx.x & 31;
   const int64_t ndq = (nblocks + 255) / 256;
   for (int64_t b = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; b < ndq;
@@ -242,7 +246,7 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   double* partial = reinterpret_cast<double*>(static_cast<char*>(ws) +
                                               align_up(static_cast<size_t>(nblocks) * 4, 256));
   const int ctas = quant_ctas(nblocks);
-  note_launches(3);  // blocks, mean, double quantization
+  note_launches(2);  // blocks, then the mean and double quantization
   if (w_bf16)
     k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
         static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
@@ -251,16 +255,22 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
         static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_constants_mean<<<1, 1024, 0, st>>>(partial, ctas, nblocks, mean);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const int64_t ndq = (nblocks + 255) / 256;
   int64_t g = (ndq + 7) / 8;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (g > cap) g = cap;
-  k_double_quantize<<<static_cast<int>(g), 256, 0, st>>>(absmax, nblocks, mean, t8_thresholds(),
-                                                         c2, c1);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(g));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_double_quantize, static_cast<const float*>(absmax), nblocks,
+                            static_cast<const double*>(partial), ctas, mean, t8_thresholds(), c2,
+                            c1);
 }
 
 cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t st) {
