@@ -7,12 +7,12 @@
 //
 // k_decode_lora_down: T = X A on one cluster of 8 CTAs that split K; the CTA partial sums
 //   meet through distributed shared memory. It also clears the GEMV's arrival counters.
-// k_decode_gemv: each warp owns 32 weight rows and a contiguous range of K. Lanes load
+// k_decode_gemv: each warp owns 16 (M <= 8) or 32 weight rows and a range of K. Lanes load
 //   32 bytes of packed codes of one row with 128-bit loads (the next 256-wide unit while
 //   the current one is expanded), double-dequantize them in registers (16-entry bf16
 //   table per 64-block, prmt lookups) straight into the A fragments of mma.m16n8k16 (X is
 //   the B operand). The dequantized weight never leaves registers. Every warp stores its
-//   partial sums; the last warp of a 32-row group to finish adds them up, adds
+//   partial sums; the last warp of a row group to finish adds them up, adds
 //   scale * T B and writes the bf16 outputs, so no second pass over the partial sums runs.
 // The GEMV is a programmatic dependent of the T kernel: it streams the weight at once and
 // reads T and its counters only after griddepcontrol.wait.
@@ -29,7 +29,10 @@ namespace qlora {
 namespace {
 
 constexpr int kDecThreads = 128;
-constexpr int kRowsPerWarp = 32;
+// Weight rows per warp: one 16-row MMA group for M <= 8, two for M > 8 (the X fragments
+// of 16 tokens are then shared by twice the rows); CTAs per SM follow the registers.
+__host__ __device__ constexpr int rows_per_warp(bool tall) { return tall ? 32 : 16; }
+__host__ __device__ constexpr int dec_ctas_per_sm(bool tall) { return tall ? 2 : 4; }
 constexpr int kUnitK = 256;  // K covered by one warp step (4 lanes x 64)
 constexpr int kTCtas = 8;    // cluster of the T kernel
 constexpr int kTThreads = 256;
@@ -46,8 +49,8 @@ struct DecodeArgs {
   int r;
   float scale;
   int splits, units_per, nunits;  // K is cut into `splits` ranges of `units_per` 256-units
-  int row_groups;                 // 32-row groups of W
-  float* part;      // [splits][row_groups][M][32] partial sums of X W_hat^T
+  int row_groups;                 // groups of rows_per_warp(M > 8) rows of W
+  float* part;      // [splits][row_groups][M][rows per warp] partial sums of X W_hat^T
   float* T;         // [M][r] T = X A
   float* T_save;    // optional copy of T for the backward pass
   int* counters;    // [row_groups] warps of the group that have stored their partials
@@ -189,10 +192,10 @@ __device__ __forceinline__ void load_x64(const uint16_t* X, int64_t K, int64_t r
 // the four columns kb + 4j .. kb + 4j + 3: A pairs (rows g and g + 8), B pairs (token
 // g). Summation order over K does not matter, so this relabelling of the MMA's k index
 // is free, and the unpacked pairs land directly in the A operand registers.
-constexpr int kGroups = 2;  // 16-row groups per warp (32 weight rows)
 
 // Packed codes and block constants of one unit for this lane (rows beyond N are clamped
 // and K beyond the matrix is clamped; their scale is forced to zero later).
+template <int kGroups>
 struct UnitCodes {
   uint4 q[kGroups][2][2];
   uint32_t e2[kGroups][2];
@@ -201,6 +204,7 @@ struct UnitCodes {
 
 // This lane's four weight rows (clamped to the last row; their scale is forced to zero
 // later) as one base and 32-bit offsets from it, computed once per task.
+template <int kGroups>
 struct RowBases {
   const uint8_t* code;           // codes of the first row
   int64_t blk;                   // index of the first row's first 64-block
@@ -208,8 +212,9 @@ struct RowBases {
   int boff[kGroups][2];          // block offset of each row from `blk`
 };
 
-__device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases& rb, int u, int t,
-                                          int bpr, UnitCodes& c) {
+template <int kGroups>
+__device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases<kGroups>& rb, int u,
+                                          int t, int bpr, UnitCodes<kGroups>& c) {
   const int kbi = min(u * (kUnitK / 64) + t, bpr - 1);  // 64-block of this lane (clamped)
   const uint8_t* base = rb.code + kbi * 32;
   const int64_t jb = rb.blk + kbi;
@@ -226,9 +231,9 @@ __device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases& r
     }
 }
 
-template <bool kTall, int CB>
+template <bool kTall, int CB, int kGroups = kTall ? 2 : 1>
 __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int g,
-                                             int t, const UnitCodes& c, const float* t8,
+                                             int t, const UnitCodes<kGroups>& c, const float* t8,
                                              float mean, float (&acc)[kGroups][kTall ? 2 : 1][4]) {
   const int64_t K = a.K;
   const int64_t kraw = static_cast<int64_t>(u) * kUnitK + 64 * t;
@@ -266,6 +271,8 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
 template <bool kTall, int CB>
 __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, int split,
                                                    int lane, const float* t8) {
+  constexpr int kGroups = kTall ? 2 : 1;
+  constexpr int kRowsPerWarp = rows_per_warp(kTall);
   const int g = lane >> 2, t = lane & 3;
   const int u0 = split * a.units_per;
   const int u1 = min(a.nunits, u0 + a.units_per);
@@ -280,7 +287,7 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
       for (int i = 0; i < 4; ++i) acc[q][h][i] = 0.f;
 
   const int bpr = static_cast<int>(a.K / 64);
-  RowBases rb;
+  RowBases<kGroups> rb;
   const int64_t row_g = lmin(rbase + g, a.N - 1);
   rb.code = a.codes + row_g * (a.K / 2);
   rb.blk = row_g * bpr;
@@ -293,7 +300,7 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
       rb.boff[q][h] = dr * bpr;
     }
   // two code buffers: the loads of unit u + 1 are in flight while unit u is expanded
-  UnitCodes cb0, cb1;
+  UnitCodes<kGroups> cb0, cb1;
   if (u0 < u1) load_unit(a, rb, u0, t, bpr, cb0);
   for (int u = u0; u < u1; u += 2) {
     if (u + 1 < u1) load_unit(a, rb, u + 1, t, bpr, cb1);
@@ -307,7 +314,7 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   // C fragment: c0,c1 = (weight row g, tokens 2t, 2t+1), c2,c3 = (row g + 8, same tokens);
   // the second accumulator (M > 8) holds tokens 8 + 2t, 8 + 2t + 1.
   const int64_t M = a.M;
-  float* pp = a.part + (static_cast<int64_t>(split) * a.row_groups + rg) * M * 32;
+  float* pp = a.part + (static_cast<int64_t>(split) * a.row_groups + rg) * M * kRowsPerWarp;
 #pragma unroll
   for (int q = 0; q < kGroups; ++q)
 #pragma unroll
@@ -316,7 +323,7 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
       for (int i = 0; i < 4; ++i) {
         const int rl = q * 16 + g + 8 * (i >> 1);
         const int m = 8 * hm + 2 * t + (i & 1);
-        if (m < M) pp[m * 32 + rl] = acc[q][hm][i];
+        if (m < M) pp[m * kRowsPerWarp + rl] = acc[q][hm][i];
       }
 
   // T and the cleared counters come from the T kernel
@@ -330,19 +337,19 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   __threadfence();  // the other warps' partial sums are visible from here on
 
   const int64_t row = rbase + lane;
-  if (row >= a.N) return;
+  if (lane >= kRowsPerWarp || row >= a.N) return;
   float y[16], lora[16];
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
     y[m] = 0.f;
     lora[m] = 0.f;
   }
-  const int64_t sstride = static_cast<int64_t>(a.row_groups) * M * 32;
-  const float* p0 = a.part + static_cast<int64_t>(rg) * M * 32 + lane;
+  const int64_t sstride = static_cast<int64_t>(a.row_groups) * M * kRowsPerWarp;
+  const float* p0 = a.part + static_cast<int64_t>(rg) * M * kRowsPerWarp + lane;
   for (int s = 0; s < a.splits; ++s) {
 #pragma unroll
     for (int m = 0; m < 16; ++m)
-      if (m < M) y[m] += __ldcg(p0 + s * sstride + m * 32);
+      if (m < M) y[m] += __ldcg(p0 + s * sstride + m * kRowsPerWarp);
   }
   const int r = a.r;
   for (int j = 0; j < r; j += 4) {
@@ -364,10 +371,10 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
     if (m < M) a.Y[m * a.N + row] = bf16_bits_rn(y[m] + a.scale * lora[m]);
 }
 
-// Two CTAs (8 warps) per SM: the two code buffers of the prefetch need the registers, and
-// measured faster than three CTAs with spills.
+// The two code buffers of the prefetch set the occupancy: 16 warps per SM with 16 rows per
+// warp (M <= 8), 8 with 32 (M > 8), each without spills.
 template <bool kTall, int CB>  // kTall: M > 8 (tokens 8..15 in the upper fragment rows); CB: codebook
-__global__ void __launch_bounds__(kDecThreads, 2) k_decode_gemv(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm(kTall)) k_decode_gemv(const DecodeArgs a) {
   __shared__ float t8[256];  // T8 by E4M3 code
   for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
   __syncthreads();
@@ -382,14 +389,15 @@ struct DecodePlan {
   int splits, units_per, nunits, row_groups;
 };
 
-// K splits: enough warps for about two waves of the GEMV (8 resident warps per SM), but
-// no more than K / (16 M): the partial sums (split x M x 128 bytes per 32 rows, written
+// K splits: enough warps for about two waves of the GEMV (16 or 8 resident warps per SM),
+// but no more than K / (16 M): the partial sums (split x M x 4 bytes per row, written
 // and read back through L2) stay at most half the code bytes.
 DecodePlan plan_decode(const LinearShape& s) {
   DecodePlan p;
   p.nunits = static_cast<int>((s.K + kUnitK - 1) / kUnitK);
-  p.row_groups = static_cast<int>((s.N + kRowsPerWarp - 1) / kRowsPerWarp);
-  const int64_t per_sm = 8;
+  const int rows = rows_per_warp(s.M > 8);
+  p.row_groups = static_cast<int>((s.N + rows - 1) / rows);
+  const int64_t per_sm = dec_ctas_per_sm(s.M > 8) * (kDecThreads / 32);
   const int64_t target = 2 * per_sm * num_sms();
   int64_t want = (target + p.row_groups - 1) / p.row_groups;
   want = std::min<int64_t>(want, std::max<int64_t>(1, s.K / (16 * std::max<int64_t>(1, s.M))));
@@ -400,7 +408,8 @@ DecodePlan plan_decode(const LinearShape& s) {
 }
 
 size_t part_bytes(const DecodePlan& p, const LinearShape& s) {
-  return align_up(static_cast<size_t>(p.splits) * p.row_groups * s.M * 32 * 4, 256);
+  return align_up(static_cast<size_t>(p.splits) * p.row_groups * s.M * rows_per_warp(s.M > 8) * 4,
+                  256);
 }
 size_t t_bytes(const LinearShape& s) { return align_up(static_cast<size_t>(s.M) * s.r * 4, 256); }
 size_t counter_bytes(const DecodePlan& p) { return align_up(static_cast<size_t>(p.row_groups) * 4, 256); }
@@ -549,7 +558,7 @@ extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_
   const LinearShape s{M, w.n_out, w.k_in, r, scale};
   DecodePlan p = plan_decode(s);
   // Fewer K splits when the planned partial sums do not fit the static array.
-  const size_t per_split = static_cast<size_t>(p.row_groups) * M * 32 * 4;
+  const size_t per_split = static_cast<size_t>(p.row_groups) * M * rows_per_warp(M > 8) * 4;
   const size_t fixed = t_bytes(s) + counter_bytes(p) + 512;
   const size_t fit = fixed < kStaticScratchBytes ? (kStaticScratchBytes - fixed) / per_split : 0;
   if (fit < 1) {
