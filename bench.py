@@ -498,6 +498,75 @@ def e2e_steps(L, scale, world, steps):
     return ms, h2d, d2h
 
 
+def stack_65b(device, warmup, steps, layers=80, M=8192, r=RANK_R, alpha=ALPHA):
+    """The 65B-shaped stack: `layers` decoder layers of 8192 / 22016 linears, all NF4 with
+    double-quantized constants resident at once (about 33 GB for 80 layers), LoRA r on each;
+    one step is the forward and backward (dX, dA, dB) of every linear at M tokens. Inputs
+    and upstream gradients are synthetic and shared by the layers (one buffer per shape);
+    every linear has its own weight, adapter and gradient buffers. Prints one JSON line."""
+    from bit_nf4_quantized_unpack_b200 import inputs, qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(4)
+    scale = alpha / r
+    lins = []
+    packed = 0
+    for _ in range(layers):
+        for name, n, k in inputs.LLAMA65B_LINEARS:
+            W = (torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16)
+            q = qlora.qlora_quantize_nf4_dq(W)
+            del W
+            packed += q.codes.numel() + q.c2.numel() + 4 * q.c1.numel() + 4
+            A = (torch.randn(k, r, generator=g, device=device) * 0.02).to(torch.bfloat16)
+            B = (torch.randn(r, n, generator=g, device=device) * 0.02).to(torch.bfloat16)
+            lins.append(dict(name=name, n=n, k=k, q=q, A=A, B=B,
+                             dA=torch.empty(k, r, device=device),
+                             dB=torch.empty(r, n, device=device)))
+    xs, dys, ys, dxs, ts = {}, {}, {}, {}, {}
+    for lin in lins[:7]:
+        n, k = lin["n"], lin["k"]
+        key = INPUT_OF[lin["name"]]
+        if key not in xs:
+            xs[key] = torch.randn(M, k, generator=g, device=device).to(torch.bfloat16)
+        if n not in dys:
+            dys[n] = torch.randn(M, n, generator=g, device=device).to(torch.bfloat16)
+            ys[n] = torch.empty(M, n, dtype=torch.bfloat16, device=device)
+        if k not in dxs:
+            dxs[k] = torch.empty(M, k, dtype=torch.bfloat16, device=device)
+    T = torch.empty(M, r, device=device)
+    wf = torch.empty(max(qlora.qlora_linear_fwd_workspace_size(M, l["n"], l["k"], r) for l in lins[:7]),
+                     dtype=torch.uint8, device=device)
+    wb = torch.empty(max(qlora.qlora_linear_bwd_workspace_size(M, l["n"], l["k"], r) for l in lins[:7]),
+                     dtype=torch.uint8, device=device)
+
+    def step():
+        for lin in lins:  # forward of every linear, then its backward (T reused)
+            x = xs[INPUT_OF[lin["name"]]]
+            qlora.qlora_linear_fwd(x, lin["q"], lin["A"], lin["B"], scale, Y=ys[lin["n"]], T=T,
+                                   workspace=wf)
+            qlora.qlora_linear_bwd(dys[lin["n"]], x, T, lin["q"], lin["A"], lin["B"], scale,
+                                   dX=dxs[lin["k"]], dA=lin["dA"], dB=lin["dB"], workspace=wb)
+
+    for _ in range(max(1, warmup)):
+        step()
+    torch.cuda.synchronize()
+    if qlora.qlora_device_error() != 0:
+        raise RuntimeError("a kernel reported a timed-out wait")
+    launches0 = qlora.qlora_launch_count()
+    ms = time_steps(step, steps, 1)
+    launches = qlora.qlora_launch_count() - launches0
+    flops = layers * layer_flops(inputs.LLAMA65B_LINEARS, M, r)
+    print(json.dumps({"metric": "QLoRA 65B-shaped stack fwd+bwd TFLOP/s (M=8192)",
+                      "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
+                      "steps": steps, "warmup": warmup, "ms_per_step": ms,
+                      "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": f"{layers} layers x (q,k,v,o 8192x8192, gate/up "
+                                             f"8192->22016, down 22016->8192), NF4-DQ, LoRA "
+                                             f"r={r} alpha={alpha}; M={M} tokens",
+                                 "packed_weight_bytes": packed, "flops_per_step": flops,
+                                 "peak_mem_gb": torch.cuda.max_memory_allocated() / 1e9},
+                      "gpu_launches": launches}), flush=True)
+
+
 def profile_linear(device, scale, warmup, steps):
     """One linear (gate, 11008 x 4096) forward + backward at M=4096, for ncu captures."""
     from bit_nf4_quantized_unpack_b200 import qlora
@@ -562,6 +631,9 @@ def main():
                          "(no graph): a small, self-contained case for profiler captures")
     ap.add_argument("--profile-merge", action="store_true",
                     help="only run merge_and_unload of a 4096x11008 weight (r=64) --steps times")
+    ap.add_argument("--stack-65b", action="store_true",
+                    help="time the 65B-shaped stack (80 layers of 8192/22016 linears, ~33 GB of "
+                         "NF4 weights resident, M=8192): forward and backward of every linear")
     ap.add_argument("--profile-linear", action="store_true",
                     help="only run forward + backward of the gate linear (11008x4096, M=4096) "
                          "--steps times: a small, self-contained case for profiler captures")
@@ -585,6 +657,9 @@ def main():
     scale = ALPHA / RANK_R
     if args.profile_merge:
         profile_merge(device, args.warmup, args.steps)
+        return
+    if args.stack_65b:
+        stack_65b(device, args.warmup, args.steps)
         return
     if args.profile_linear:
         profile_linear(device, scale, args.warmup, args.steps)

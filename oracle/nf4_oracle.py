@@ -288,6 +288,20 @@ def double_dequant_rows(q: dict, rows: np.ndarray) -> np.ndarray:
     return bf16_round(vals.astype(np.float32)).reshape(rows.size, k)
 
 
+def double_dequant_cols(q: dict, cols: np.ndarray) -> np.ndarray:
+    """Ŵ for selected columns only, [N, len(cols)] (same arithmetic as ``double_dequant``):
+    the code of (n, k) is nibble k % 2 of byte k // 2 of row n (low nibble first), its
+    scale that of block k // 64 of row n."""
+    n, k = q["shape"]
+    cols = np.asarray(cols)
+    bpr = k // BLOCK
+    s = reconstruct_absmax(q["c2"], q["c1"], q["mean"]).reshape(n, bpr)[:, cols // BLOCK]
+    packed = q["codes"].reshape(n, k // 2)[:, cols // 2]
+    codes = np.where((cols % 2 == 0)[None, :], packed & 0xF, packed >> 4)
+    vals = _levels_of(q)[codes] * s
+    return bf16_round(vals.astype(np.float32))
+
+
 # ---------------------------------------------------------------------------
 # The QLoRA linear layer (itwiki "QLoRA" computation section; minnong511
 # "quantization": y = W x + (alpha / r) B A x, W frozen, grads for A and B)

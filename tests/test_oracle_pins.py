@@ -290,6 +290,8 @@ def test_quantized_weight_error_is_small():
     assert np.mean(np.abs(What - W)) < 2e-3
     rows = np.array([0, 17, 63])
     np.testing.assert_array_equal(O.double_dequant_rows(q, rows), What[rows])
+    cols = np.array([0, 1, 63, 64, 130, 255])  # both nibbles, block edges
+    np.testing.assert_array_equal(O.double_dequant_cols(q, cols), What[:, cols])
 
 
 # ---------------------------------------------------------------- merge_and_unload
