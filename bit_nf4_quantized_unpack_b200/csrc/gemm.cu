@@ -947,6 +947,38 @@ qlora_status lora_down_T(const uint16_t* X, const uint16_t* A, const LinearShape
   return QLORA_OK;
 }
 
+// A non-blocking side stream and two events per host thread and device, for the part of
+// the backward that runs beside the fused dX kernel (fork and join by events, which a
+// CUDA graph capture of the caller's stream follows).
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+// Null (and success) when `st` is being captured and the side stream does not exist yet:
+// streams and events cannot be created during a capture, and the caller then runs
+// everything in order on `st`.
+cudaError_t side_stream(cudaStream_t st, SideStream** out) {
+  thread_local SideStream side[16];
+  *out = nullptr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 16) return cudaSuccess;
+  SideStream& s = side[dev];
+  if (!s.st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(st, &cs);
+    if (e != cudaSuccess) return e;
+    if (cs != cudaStreamCaptureStatusNone) return cudaSuccess;
+    e = cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  *out = &s;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 size_t gemm_fwd_workspace(const LinearShape& s) {
@@ -1023,12 +1055,34 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
                       t, thl));
   }
 
-  // dX = dY W_hat + scale G A^T
+  // dX = dY W_hat + scale G A^T, and the grouped dA = scale X^T G (rows k) with
+  // dB = scale T^T dY (rows n, stored [r, N]). dA and dB need G and T, not dX: with dX
+  // requested they run on a side stream beside the fused dX kernel, whose persistent CTAs
+  // are enqueued first and hold the SMs; the side stream's CTAs take SMs as fused CTAs
+  // finish (the last, partial wave of tiles).
+  CUtensorMap xa, xw, xx, xo, ga, gb, ga1, gb1;
   if (dX) {
-    CUtensorMap ta, tw, tx;
-    QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 256, kSW128);
-    QL_MAP(&tw, kBF16, A, s.r, s.K, s.r * 2, 64, 128, kSW128);   // A [K, r] K-major
-    QL_MAP(&tx, kBF16, gs, 128, s.M, 256, 64, 256, kSW128);      // scale G, bf16 hi | lo
+    QL_MAP(&xa, kBF16, dY, s.N, s.M, s.N * 2, 64, 256, kSW128);
+    QL_MAP(&xw, kBF16, A, s.r, s.K, s.r * 2, 64, 128, kSW128);   // A [K, r] K-major
+    QL_MAP(&xx, kBF16, gs, 128, s.M, 256, 64, 256, kSW128);      // scale G, bf16 hi | lo
+    // dX [M, K] for the tile stores: 32 x 32 boxes, 64-byte swizzle
+    QL_MAP(&xo, kBF16, dX, s.K, s.M, s.K * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  QL_MAP(&ga, kBF16, X, s.K, s.M, s.K * 2, 64, 64, kSW128);    // X as MN-major (k inner)
+  QL_MAP(&gb, kBF16, ghl, 128, s.M, 256, 64, 64, kSW128);      // G hi/lo MN-major
+  QL_MAP(&ga1, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);  // dY as MN-major (n inner)
+  QL_MAP(&gb1, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);     // T hi/lo MN-major
+
+  SideStream* side = nullptr;
+  if (dX) QL_TRY(side_stream(st, &side));
+  cudaStream_t gst = st;
+  if (side) {
+    QL_TRY(cudaEventRecord(side->fork, st));
+    QL_TRY(cudaStreamWaitEvent(side->st, side->fork, 0));
+    gst = side->st;
+  }
+  cudaError_t e = cudaSuccess;
+  if (dX) {
     FusedArgs a;
     a.codebook = w.codebook;
     a.codes = w.codes;
@@ -1043,24 +1097,22 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     a.out_ld = s.K;
     a.out_rows = s.K;
     a.err = device_error_word();
-    CUtensorMap to;  // dX [M, K] for the tile stores
-    QL_MAP(&to, kBF16, dX, s.K, s.M, s.K * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
-    QL_TRY(run_fused<Mode::kDgrad>(ta, tw, tx, to, a, st));
+    e = run_fused<Mode::kDgrad>(xa, xw, xx, xo, a, st);
   }
-  // dA = scale X^T G (rows k) and dB = scale T^T dY (rows n, stored [r, N]): both contract
-  // over the tokens, so they run as one grouped launch and one finalize
-  {
-    CUtensorMap ta, tb, ta1, tb1;
-    QL_MAP(&ta, kBF16, X, s.K, s.M, s.K * 2, 64, 64, kSW128);    // X as MN-major (k inner)
-    QL_MAP(&tb, kBF16, ghl, 128, s.M, 256, 64, 64, kSW128);      // G hi/lo MN-major
-    QL_MAP(&ta1, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);  // dY as MN-major (n inner)
-    QL_MAP(&tb1, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);     // T hi/lo MN-major
-    QL_TRY((run_lora_gemm<true, true, 128>(ta, tb, s.K, s.M, part, st, &splits, &ta1, &tb1, s.N)));
+  if (e == cudaSuccess)
+    e = run_lora_gemm<true, true, 128>(ga, gb, s.K, s.M, part, gst, &splits, &ga1, &gb1, s.N);
+  if (e == cudaSuccess) {
     const int64_t stacked = stacked_rows(s.K, s.N);
-    QL_TRY(launch_pdl(k_finalize_grad, dim3(blocks_for(stacked, kGradRows)), dim3(256), 0, st,
-                      part, splits, plan_split(stacked, s.M).rows_pad,
-                      static_cast<int64_t>(align_up(s.K, 128)), s.K, dA, s.N, dB, s.r, s.scale));
+    e = launch_pdl(k_finalize_grad, dim3(blocks_for(stacked, kGradRows)), dim3(256), 0, gst,
+                   part, splits, plan_split(stacked, s.M).rows_pad,
+                   static_cast<int64_t>(align_up(s.K, 128)), s.K, dA, s.N, dB, s.r, s.scale);
   }
+  if (side) {  // the caller's stream continues once both branches are done (on every path)
+    cudaError_t ej = cudaEventRecord(side->join, side->st);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, side->join, 0);
+    if (e == cudaSuccess) e = ej;
+  }
+  QL_TRY(e);
   return QLORA_OK;
 }
 
