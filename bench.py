@@ -688,10 +688,13 @@ def main():
     print(f"[bench] layer step {ms:.3f} ms -> {value:.1f} TFLOP/s per {world} GPU(s)",
           file=sys.stderr, flush=True)
 
-    # dominant kernel: the fused NF4 GEMM, timed per launch with events on its stream
+    # dominant kernel: the fused NF4 GEMM, timed per launch with events on its stream in a
+    # pass of its own. The GPU first idles for a second: its clocks fall within ~100 ms of
+    # sustained load, and this pass should start from the same state as the timed steps.
     events = []
     pool = [event_pair() for _ in range(2 * len(L["layer"]) * args.steps)]
     torch.cuda.synchronize()
+    time.sleep(1.0)
     for _ in range(args.steps):
         layer_step(L, scale, world, events=events, pool=pool)
     torch.cuda.synchronize()
