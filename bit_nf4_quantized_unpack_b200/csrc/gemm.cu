@@ -73,7 +73,8 @@ constexpr int kHalfCols = 256;   // tokens per MMA / per accumulator
 constexpr int kHalves = 2;       // accumulators per tile
 constexpr int kTileCols = kHalfCols * kHalves;  // tokens per tile
 constexpr int kBK = 64;          // contraction per pipeline step
-constexpr int kHalfSlots = 4;    // ring of 256-token operand tiles (2 per step)
+constexpr int kHalfSlots = 4;    // 256-token operand tiles in the ring
+constexpr int kXSlots = kHalfSlots / 2;  // ring slots: the two half tiles of one step
 constexpr uint32_t kHalfBytes = kHalfCols * kBK * 2;  // 32 KB
 constexpr uint32_t kWBytes = kTileRows * kBK * 2;     // 16 KB
 constexpr uint32_t kEpiBytes = 4 * 2 * 32 * 32 * 2;    // per epilogue warp: 2 x (32 tokens x 32 rows)
@@ -106,14 +107,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* act_s = smem;                             // [kHalfSlots][kHalfBytes] token side
+  uint8_t* act_s = smem;                             // [kXSlots][2][kHalfBytes] token side
   uint8_t* w_s = act_s + kHalfSlots * kHalfBytes;    // [kWSlots][kWBytes] dequantized
   uint8_t* wext_s = w_s + kWSlots * kWBytes;         // [kWBytes] LoRA weight-side operand
   uint16_t* epi_s = reinterpret_cast<uint16_t*>(wext_s + kWBytes);  // [4][2][32][32] staging
   uint64_t* bars = reinterpret_cast<uint64_t*>(wext_s + kWBytes + kEpiBytes);
-  uint64_t* half_full = bars;                       // [kHalfSlots] token tile landed
-  uint64_t* half_empty = half_full + kHalfSlots;    // [kHalfSlots] MMAs reading it done
-  uint64_t* deq_full = half_empty + kHalfSlots;     // [kWSlots] dequantized tile ready
+  uint64_t* half_full = bars;                       // [kHalfSlots] a token tile landed
+  uint64_t* x_empty = half_full + kHalfSlots;       // [kXSlots] MMAs reading a step's tiles done
+  uint64_t* deq_full = x_empty + kXSlots;           // [kWSlots] dequantized tile ready
   uint64_t* w_empty = deq_full + kWSlots;           // [kWSlots] MMAs reading it done
   uint64_t* ext_empty = w_empty + kWSlots;          // LoRA operand slot read out
   uint64_t* acc_full = ext_empty + 1;               // [kHalves] accumulator complete
@@ -142,10 +143,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kHalfSlots; ++s) {
-      mbar_init(&half_full[s], 1);
-      mbar_init(&half_empty[s], 1);
-    }
+    for (int s = 0; s < kHalfSlots; ++s) mbar_init(&half_full[s], 1);
+    for (int s = 0; s < kXSlots; ++s) mbar_init(&x_empty[s], 1);
     for (int s = 0; s < kWSlots; ++s) {
       mbar_init(&deq_full[s], 4);
       mbar_init(&w_empty[s], 1);
@@ -173,7 +172,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     // ------------------------------------------------ TMA: token-side operand, LoRA steps
     if (lane == 0) {
       tma_prefetch_desc(&tm_act);
-      int issued = 0;  // half tiles
+      // step g fills slot g % kXSlots: half tile h in buffer 2 (g % kXSlots) + h, counted
+      // on that buffer's own barrier (a tile with one accumulator leaves buffer 1 unused)
+      int issued = 0;                  // steps; buffer 2 xs is loaded at every use of slot xs
+      int h1_uses0 = 0, h1_uses1 = 0;  // loads of buffer 1 and buffer 3 (second halves)
       bool ok = true;
       for (int i = 0; i < my_tiles && ok; ++i) {
         int64_t row0, m0;
@@ -187,16 +189,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             ok = false;
             break;
           }
+          const int xs = issued % kXSlots;
+          if (issued >= kXSlots &&
+              !mbar_wait(&x_empty[xs], ((issued / kXSlots) - 1) & 1u, abort_flag)) {
+            record_error(args.err, abort_flag, kErrTimeoutProducer);
+            ok = false;
+            break;
+          }
           for (int h = 0; h < nh; ++h) {
-            const int hx = issued;
-            const int hs = hx % kHalfSlots;
-            if (hx >= kHalfSlots &&
-                !mbar_wait(&half_empty[hs], ((hx / kHalfSlots) - 1) & 1u, abort_flag)) {
-              record_error(args.err, abort_flag, kErrTimeoutProducer);
-              ok = false;
-              break;
-            }
+            const int hs = 2 * xs + h;
             const int mh = static_cast<int>(m0) + h * kHalfCols;
+            if (h == 1) {
+              if (xs == 0) ++h1_uses0;
+              else ++h1_uses1;
+            }
             if (!ext) {
               mbar_arrive_expect_tx(&half_full[hs], kHalfBytes);
               tma_load_2d(act_s + hs * kHalfBytes, &tm_act, &half_full[hs], step * kBK, mh);
@@ -217,13 +223,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               tma_load_2d(act_s + hs * kHalfBytes, &tm_ext_act, &half_full[hs],
                           (step - ksteps) * 64, mh);
             }
-            ++issued;
           }
+          ++issued;
         }
       }
-      if (*abort_flag)  // let copies already in flight land before the CTA exits
-        for (int hx = (issued > kHalfSlots ? issued - kHalfSlots : 0); hx < issued; ++hx)
-          mbar_wait_drain(&half_full[hx % kHalfSlots], (hx / kHalfSlots) & 1u);
+      if (*abort_flag) {  // let copies already in flight land before the CTA exits
+        for (int xs = 0; xs < kXSlots; ++xs) {
+          const int u0 = issued / kXSlots + (xs < issued % kXSlots ? 1 : 0);  // buffer 2 xs
+          const int u1 = xs == 0 ? h1_uses0 : h1_uses1;                       // buffer 2 xs + 1
+          if (u0 > 0) mbar_wait_drain(&half_full[2 * xs], (u0 - 1) & 1u);
+          if (u1 > 0) mbar_wait_drain(&half_full[2 * xs + 1], (u1 - 1) & 1u);
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -242,7 +253,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                                     ? smem_desc_sw128(smem_u32(wext_s), 8192, 1024)
                                     : smem_desc_sw128(smem_u32(wext_s), 16, 1024);
       bool ok = true;
-      int halves_done = 0, main_done = 0, ext_done = 0;
+      int steps_done = 0, main_done = 0, ext_done = 0;
+      int h1_uses0 = 0, h1_uses1 = 0;  // loads consumed from buffers 1 and 3 (second halves)
       int acc_uses[kHalves] = {0, 0};  // tiles accumulated so far in each accumulator
       for (int i = 0; i < my_tiles && ok; ++i) {
         int64_t row0, m0;
@@ -264,9 +276,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           } else {
             da = desc_ext;  // landed with the first half tile of the first LoRA step
           }
+          const int xs = steps_done % kXSlots;
           for (int h = 0; h < nh; ++h) {
-            const int hx = halves_done;
-            const int hs = hx % kHalfSlots;
+            const int hs = 2 * xs + h;
             // the epilogue has read accumulator h of the previous tile out
             if (step == 0 && acc_uses[h] >= 1) {
               if (!mbar_wait(&acc_empty[h], (acc_uses[h] - 1) & 1u, abort_flag)) {
@@ -276,10 +288,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               }
               tc_fence_after();
             }
-            if (!mbar_wait(&half_full[hs], (hx / kHalfSlots) & 1u, abort_flag)) {
+            // buffer 2 xs is loaded at every use of slot xs; buffer 2 xs + 1 only when the
+            // tile has a second half
+            const int uses = h == 0 ? steps_done / kXSlots : (xs == 0 ? h1_uses0 : h1_uses1);
+            if (!mbar_wait(&half_full[hs], uses & 1u, abort_flag)) {
               record_error(args.err, abort_flag, kErrTimeoutMma);
               ok = false;
               break;
+            }
+            if (h == 1) {
+              if (xs == 0) ++h1_uses0;
+              else ++h1_uses1;
             }
             const uint32_t tmem_d = tmem_base + h * kHalfCols;
             const uint64_t db = smem_desc_sw128(smem_u32(act_s + hs * kHalfBytes), 16, 1024);
@@ -292,14 +311,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
               for (int kk = 0; kk < args.ext_mmas; ++kk)
                 umma_bf16(tmem_d, da + kk * kDX, db + kk * 2u, idesc_ext, 1u);
             }
-            umma_commit(&half_empty[hs]);
-            ++halves_done;
             if (step == total - 1) {  // accumulator h of this tile is complete
               umma_commit(&acc_full[h]);
               ++acc_uses[h];
             }
           }
           if (!ok) break;
+          umma_commit(&x_empty[xs]);  // the step's token tiles are read
+          ++steps_done;
           if (main_step) {
             umma_commit(&w_empty[c % kWSlots]);
             ++main_done;
@@ -316,8 +335,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       // the commits of the last steps arrive asynchronously on barriers nobody else waits
       // for any more: let them land before the CTA (and its shared memory) goes
       uint32_t par;
-      for (int s = 0; s < kHalfSlots; ++s)
-        if (last_use(halves_done, kHalfSlots, s, par)) mbar_wait_drain(&half_empty[s], par);
+      for (int s = 0; s < kXSlots; ++s)
+        if (last_use(steps_done, kXSlots, s, par)) mbar_wait_drain(&x_empty[s], par);
       for (int s = 0; s < kWSlots; ++s)
         if (last_use(main_done, kWSlots, s, par)) mbar_wait_drain(&w_empty[s], par);
       if (last_use(ext_done, 1, 0, par)) mbar_wait_drain(ext_empty, par);
