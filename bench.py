@@ -39,7 +39,7 @@ INPUT_OF = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out",
             "gate": "mlp_in", "up": "mlp_in", "down": "mlp_act"}
 # dram__bytes_read.sum + dram__bytes_write.sum per FLOP of k_fused_nf4_gemm, from one ncu
 # capture of the current kernel (forward + dX of the 11008 x 4096 linear at M = 4096)
-FUSED_DRAM_BYTES_PER_FLOP = (123.030e6 + 169.254e6) / (3.751e11 + 3.715e11)
+FUSED_DRAM_BYTES_PER_FLOP = (125.920e6 + 169.601e6) / (3.751e11 + 3.715e11)
 
 
 def layer_flops(linears, M, r):
