@@ -3,6 +3,8 @@
 // "이중 양자화"). All three kernels are HBM-bound streaming passes.
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "internal.h"
 #include "nf4_device.cuh"
 
@@ -42,76 +44,117 @@ struct Raw8<uint16_t> {  // bf16
   }
 };
 
-// NF4 code of x in [-1, 1] from the bucket table in shared memory (entries: threshold,
-// code as bits): bucket = round-half-even(512 x + 512), which the FMA leaves in the low
-// mantissa bits of a number in [2^23, 2^24).
-__device__ __forceinline__ uint32_t bucket_code(float x, const float2* sb) {
-  const uint32_t idx =
-      min(static_cast<uint32_t>(__float_as_int(__fmaf_rn(x, 512.0f, 12583424.0f)) - 0x4B400000),
-          static_cast<uint32_t>(kCodeBuckets - 1));
-  const float2 bk = sb[idx];
-  return __float_as_uint(bk.y) + (x >= bk.x ? 1u : 0u);
+// NF4 code of x in [-1, 1] from the bucket table in shared memory, given
+// bk = fl32(16 x + 16 + 1.5 * 2^23): that number lies in [2^23, 2^24), where the ulp is 1,
+// so its low mantissa bits hold the bucket round-half-even(16 x + 16). The table is two
+// arrays of 4-byte words (fp32 thresholds, codes) at a fixed distance, so that one address
+// serves both loads; 33 words occupy 32 banks, so the lanes of a warp rarely conflict.
+// The unsigned clamp keeps any bit pattern (a NaN from a non-finite input) inside the table.
+struct BucketSmem {
+  float thr[kCodeBuckets];
+  uint32_t code[kCodeBuckets];
+};
+constexpr float kBucketBias = 16.0f + 12582912.0f;  // S + 1.5 * 2^23
+__device__ __forceinline__ uint32_t bucket_code(float x, float bk, const BucketSmem& sb) {
+  const uint32_t idx = min(__float_as_uint(bk), 0x4B400000u + (kCodeBuckets - 1)) - 0x4B400000u;
+  return sb.code[idx] + (x >= sb.thr[idx] ? 1u : 0u);
+}
+__device__ __forceinline__ uint32_t bucket_code(float x, const BucketSmem& sb) {
+  return bucket_code(x, __fmaf_rn(x, static_cast<float>(kBucketScale), kBucketBias), sb);
 }
 
-// Level 1: one 64-block per group of 8 lanes (8 elements per lane). Writes the packed
-// codes, the fp32 absmax of each block, and one fp64 partial sum of absmax per CTA.
+// max(|a|, |b|, |c|) in one three-input max (sm_100).
+__device__ __forceinline__ float absmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
+}
+
+// Level 1: one 64-block per group of kQuantLanes = 4 lanes (16 elements per lane). Writes
+// the packed codes, the fp32 absmax of each block, and one fp64 partial sum of absmax per
+// CTA.
 //
 // x = fl32(w / absmax) is computed with Markstein's correction step (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000 processor", IBM J.
 // Res. Dev. 34, 1990): with r = RN(1/m), q = RN(w r) and e = w - m q (exact in an FMA),
-// RN(q + e r) is the correctly rounded quotient. For m >= 2^-64, 1/m is finite and the
+// RN(q + e r) is the correctly rounded quotient. Two weights go through each step at
+// once in the packed f32x2 form. For m >= 2^-64, 1/m is finite and the
 // residual stays exact for every |x| above 2^-36, far below the smallest threshold
 // magnitude (0.04); blocks with a smaller absmax take plain IEEE division.
-// The code of x comes from the 1025-bucket table (one shared-memory load and one compare).
+// The code of x comes from the 33-bucket table (two shared-memory loads and one compare).
+constexpr int kQuantLanes = 4;
+constexpr int kQuantPer = 64 / kQuantLanes;  // elements per lane
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
     k_quantize_blocks(const T* __restrict__ W, int64_t nblocks,
                       const __grid_constant__ Nf4BucketTable tab, uint8_t* __restrict__ codes,
                       float* __restrict__ absmax, double* __restrict__ partial) {
   const int lane = threadIdx.x & 31;
-  const int sub = lane & 7;
-  const unsigned gmask = 0xFFu << (lane & 24);
-  const int64_t per_cta = kQuantThreads / 8;
-  __shared__ float2 sb[kCodeBuckets];  // (threshold, code as bits)
-  for (int i = threadIdx.x; i < kCodeBuckets; i += blockDim.x)
-    sb[i] = make_float2(tab.thr[i], __uint_as_float(static_cast<uint32_t>(tab.code[i])));
+  const int sub = lane & (kQuantLanes - 1);
+  const unsigned gmask = ((1u << kQuantLanes) - 1u) << (lane & (32 - kQuantLanes));
+  const int64_t per_cta = kQuantThreads / kQuantLanes;
+  __shared__ BucketSmem sb;
+  for (int i = threadIdx.x; i < kCodeBuckets; i += blockDim.x) {
+    sb.thr[i] = tab.thr[i];
+    sb.code[i] = tab.code[i];
+  }
   __syncthreads();
   // the double quantization may be scheduled now; it waits for this grid's results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   double acc = 0.0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * per_cta;
-  int64_t b = blockIdx.x * per_cta + threadIdx.x / 8;
+  int64_t b = blockIdx.x * per_cta + threadIdx.x / kQuantLanes;
   // the next two blocks' elements are in flight while this one is coded
-  Raw8<T> n0, n1;
-  if (b < nblocks) n0.load(W + b * 64 + sub * 8);
-  if (b + stride < nblocks) n1.load(W + (b + stride) * 64 + sub * 8);
-  for (; b < nblocks; b += stride) {
-    float v[8];
-    n0.values(v);
-    n0 = n1;
-    if (b + 2 * stride < nblocks) n1.load(W + (b + 2 * stride) * 64 + sub * 8);
-    float m = 0.f;
+  Raw8<T> n0[2], n1[2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
-    m = fmaxf(m, __shfl_xor_sync(gmask, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(gmask, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(gmask, m, 4));
-    uint32_t packed = 0;
+  for (int h = 0; h < 2; ++h) {
+    if (b < nblocks) n0[h].load(W + b * 64 + sub * kQuantPer + h * 8);
+    if (b + stride < nblocks) n1[h].load(W + (b + stride) * 64 + sub * kQuantPer + h * 8);
+  }
+  for (; b < nblocks; b += stride) {
+    float v[16];
+    {
+      float (&v0)[8] = *reinterpret_cast<float(*)[8]>(v);
+      float (&v1)[8] = *reinterpret_cast<float(*)[8]>(v + 8);
+      n0[0].values(v0);
+      n0[1].values(v1);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      n0[h] = n1[h];
+      if (b + 2 * stride < nblocks) n1[h].load(W + (b + 2 * stride) * 64 + sub * kQuantPer + h * 8);
+    }
+    float m = fmaxf(fabsf(v[14]), fabsf(v[15]));
+#pragma unroll
+    for (int i = 0; i < 14; i += 2) m = absmax3(m, v[i], v[i + 1]);
+#pragma unroll
+    for (int o = 1; o < kQuantLanes; o <<= 1) m = fmaxf(m, __shfl_xor_sync(gmask, m, o));
+    uint32_t packed[2] = {0u, 0u};
     if (m >= 0x1p-64f) {
-      const float r = __fdiv_rn(1.0f, m);
+      // the steps below on pairs of weights (packed f32x2: per lane the same roundings)
+      const float r = __frcp_rn(m);
+      const uint64_t rr = f2_pack(r, r), nm = f2_pack(-m, -m);
+      const uint64_t kscale = f2_pack(kBucketScale, kBucketScale);
+      const uint64_t kbias = f2_pack(kBucketBias, kBucketBias);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float w = v[i];
-        const float q = __fmul_rn(w, r);
-        const float e = __fmaf_rn(-q, m, w);
-        packed |= bucket_code(__fmaf_rn(e, r, q), sb) << (4 * i);
+        const uint64_t w = f2_pack(v[2 * i], v[2 * i + 1]);
+        const uint64_t q = f2_mul(w, rr);
+        const uint64_t e = f2_fma(q, nm, w);  // w - q m, exact
+        const uint64_t x = f2_fma(e, rr, q);  // fl32(w / m)
+        const uint64_t bk = f2_fma(x, kscale, kbias);
+        float x0, x1, b0, b1;
+        f2_unpack(x, x0, x1);
+        f2_unpack(bk, b0, b1);
+        packed[i / 4] |= bucket_code(x0, b0, sb) << (8 * (i % 4));
+        packed[i / 4] |= bucket_code(x1, b1, sb) << (8 * (i % 4) + 4);
       }
     } else {  // absmax zero or below 2^-64: plain IEEE division (x = 0 for a zero block)
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        packed |= bucket_code(m > 0.f ? __fdiv_rn(v[i], m) : 0.f, sb) << (4 * i);
+      for (int i = 0; i < 16; ++i)
+        packed[i / 8] |= bucket_code(m > 0.f ? __fdiv_rn(v[i], m) : 0.f, sb) << (4 * (i % 8));
     }
-    reinterpret_cast<uint32_t*>(codes + b * 32)[sub] = packed;
+    reinterpret_cast<uint2*>(codes + b * 32)[sub] = make_uint2(packed[0], packed[1]);
     if (sub == 0) {
       absmax[b] = m;
       acc += static_cast<double>(m);
@@ -197,7 +240,10 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Standalone double dequantization: one thread per 8 codes (one 32-bit word).
+// Standalone double dequantization: one thread per 8 codes (one 32-bit word), four words
+// per thread and pass (kDqUnroll, a CTA's 256 threads apart so that every load and store
+// instruction is coalesced), their loads all issued before the first is used.
+constexpr int kDqUnroll = 4;
 template <int CB>
 __global__ void __launch_bounds__(256)
     k_dequant(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ c2,
@@ -209,26 +255,57 @@ __global__ void __launch_bounds__(256)
   for (int e = threadIdx.x; e < 256; e += blockDim.x) t8[e] = t8_value(e);
   __syncthreads();
   const float mean = *mean_p;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t j = i >> 3;  // 64-block of this word
-    const float s = block_scale_tab(t8, c2[j], c1[j >> 8], mean);
-    const uint32_t w = __ldg(codes + i);
-    uint32_t o[4];
+  const int64_t chunk = static_cast<int64_t>(blockDim.x) * kDqUnroll;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * chunk + threadIdx.x; base < nwords;
+       base += static_cast<int64_t>(gridDim.x) * chunk) {
+    uint32_t w[kDqUnroll], e[kDqUnroll];
+    float g[kDqUnroll];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float a = __fmul_rn(lut[(w >> (8 * p)) & 15u], s);
-      const float b = __fmul_rn(lut[(w >> (8 * p + 4)) & 15u], s);
-      o[p] = pack_bf16x2_rn(a, b);
+    for (int u = 0; u < kDqUnroll; ++u) {
+      const int64_t i = base + u * static_cast<int64_t>(blockDim.x);
+      if (i < nwords) {
+        w[u] = __ldg(codes + i);
+        e[u] = c2[i >> 3];   // 64-block of this word
+        g[u] = c1[i >> 11];  // its 256-block of constants
+      }
     }
-    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) {
+      const int64_t i = base + u * static_cast<int64_t>(blockDim.x);
+      if (i < nwords) {
+        const float s = block_scale_tab(t8, e[u], g[u], mean);
+        uint32_t o[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float a = __fmul_rn(lut[(w[u] >> (8 * p)) & 15u], s);
+          const float b = __fmul_rn(lut[(w[u] >> (8 * p + 4)) & 15u], s);
+          o[p] = pack_bf16x2_rn(a, b);
+        }
+        out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
   }
 }
 
-int quant_ctas(int64_t nblocks) {
-  const int64_t want = (nblocks + kQuantThreads / 8 - 1) / (kQuantThreads / 8);
-  const int cap = num_sms() * 8 < kMaxQuantCtas ? num_sms() * 8 : kMaxQuantCtas;
-  return static_cast<int>(want < cap ? (want < 1 ? 1 : want) : cap);
+// CTAs of level 1: enough for every block, at most one resident wave (so that all of
+// them run from the start) and at most kMaxQuantCtas (the partial sums' slots).
+template <typename T>
+cudaError_t quant_ctas(int64_t nblocks, int* ctas) {
+  static std::atomic<int> resident{0};  // CTAs per SM, looked up once per input type
+  int per_sm = resident.load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    cudaError_t e =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quantize_blocks<T>, kQuantThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    resident.store(per_sm, std::memory_order_relaxed);
+  }
+  const int64_t per = kQuantThreads / kQuantLanes;  // blocks per CTA and pass
+  const int64_t want = (nblocks + per - 1) / per;
+  const int64_t wave = static_cast<int64_t>(num_sms()) * per_sm;
+  const int64_t cap = wave < kMaxQuantCtas ? wave : kMaxQuantCtas;
+  *ctas = static_cast<int>(want < cap ? (want < 1 ? 1 : want) : cap);
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -245,7 +322,9 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   float* absmax = static_cast<float*>(ws);
   double* partial = reinterpret_cast<double*>(static_cast<char*>(ws) +
                                               align_up(static_cast<size_t>(nblocks) * 4, 256));
-  const int ctas = quant_ctas(nblocks);
+  int ctas = 0;
+  cudaError_t e = w_bf16 ? quant_ctas<uint16_t>(nblocks, &ctas) : quant_ctas<float>(nblocks, &ctas);
+  if (e != cudaSuccess) return e;
   note_launches(2);  // blocks, then the mean and double quantization
   if (w_bf16)
     k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
@@ -253,7 +332,7 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   else
     k_quantize_blocks<float><<<ctas, kQuantThreads, 0, st>>>(
         static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t ndq = (nblocks + 255) / 256;
   int64_t g = (ndq + 7) / 8;
@@ -275,10 +354,17 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
 
 cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t st) {
   const int64_t nwords = w.n_out * w.k_in / 8;
-  int64_t g = (nwords + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
-  if (g > cap) g = cap;
   auto kern = w.codebook == 1 ? k_dequant<1> : k_dequant<0>;
+  static std::atomic<int> resident[kCodebooks];  // CTAs per SM, looked up once
+  int per_sm = resident[w.codebook == 1].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+    if (e != cudaSuccess) return e;
+    resident[w.codebook == 1].store(per_sm, std::memory_order_relaxed);
+  }
+  int64_t g = (nwords + 256 * kDqUnroll - 1) / (256 * kDqUnroll);
+  const int64_t cap = static_cast<int64_t>(num_sms()) * (per_sm > 0 ? per_sm : 1);
+  if (g > cap) g = cap;
   note_launches(1);
   kern<<<static_cast<int>(g), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(w.codes), w.c2,
                                             w.c1, w.mean, nwords, reinterpret_cast<uint4*>(out));

@@ -16,10 +16,12 @@ namespace qlora {
 extern const uint32_t kNf4Bits[16];
 constexpr int kT8Size = 253;  // distinct finite E4M3 values
 struct Nf4Thresholds { float t[15]; };
-// NF4 codes by table: bucket b = round-half-even(512 x + 512) of x in [-1, 1] (1025
-// buckets); within bucket b the code is code[b] + (x >= thr[b]) (thr = +inf when no
-// threshold falls inside the bucket; no bucket holds two).
-constexpr int kCodeBuckets = 1025;
+// NF4 codes by table: bucket b = round-half-even(16 x + 16) of x in [-1, 1] (33
+// buckets of width 1/16, narrower than the smallest gap between two thresholds of either
+// codebook, 0.080); within bucket b the code is code[b] + (x >= thr[b]) (thr = +inf when
+// no threshold falls inside the bucket; no bucket holds two).
+constexpr int kBucketScale = 16;
+constexpr int kCodeBuckets = 2 * kBucketScale + 1;
 struct Nf4BucketTable {
   float thr[kCodeBuckets];
   uint8_t code[kCodeBuckets + 3];

@@ -103,15 +103,16 @@ struct CodebookTables {
   Nf4BucketTable buckets;
 };
 
-// Thresholds and the 1025-bucket table of one 16-level codebook.
+// Thresholds and the bucket table of one 16-level codebook.
 void build_codebook(const uint32_t (&bits)[16], CodebookTables& cb) {
   for (int i = 0; i < 16; ++i) cb.levels[i] = bits_to_float(bits[i]);
   for (int i = 0; i < 15; ++i) cb.thr.t[i] = first_above(cb.levels, 16, i);
-  // Bucket b holds the fp32 x with round-half-even(512 x + 512) == b: its edges are
-  // (2b -+ 1 - 1024) / 1024, each tie going to the even bucket.
+  // Bucket b holds the fp32 x with round-half-even(S x + S) == b (S = kBucketScale): its
+  // edges are (2b -+ 1 - 2S) / 2S, each tie going to the even bucket.
+  const double s2 = 2.0 * kBucketScale;
   for (int b = 0; b < kCodeBuckets; ++b) {
-    float xmin = static_cast<float>((2.0 * b - 1025.0) / 1024.0);
-    float xmax = static_cast<float>((2.0 * b - 1023.0) / 1024.0);
+    float xmin = static_cast<float>((2.0 * b - 1.0 - s2) / s2);
+    float xmax = static_cast<float>((2.0 * b + 1.0 - s2) / s2);
     if (b & 1) {
       xmin = std::nextafter(xmin, std::numeric_limits<float>::infinity());
       xmax = std::nextafter(xmax, -std::numeric_limits<float>::infinity());
@@ -181,11 +182,11 @@ extern "C" void qlora_nf4_thresholds(float* out15) {
   for (int i = 0; i < 15; ++i) out15[i] = t.t[i];
 }
 
-extern "C" void qlora_nf4_code_buckets(float* thr1025, uint8_t* code1025) {
+extern "C" void qlora_nf4_code_buckets(float* thr33, uint8_t* code33) {
   const auto& t = qlora::code_buckets(0);
   for (int i = 0; i < qlora::kCodeBuckets; ++i) {
-    if (thr1025) thr1025[i] = t.thr[i];
-    if (code1025) code1025[i] = t.code[i];
+    if (thr33) thr33[i] = t.thr[i];
+    if (code33) code33[i] = t.code[i];
   }
 }
 
@@ -200,7 +201,7 @@ extern "C" void qlora_fp8_thresholds(float* out252, float* t8_out253, uint8_t* c
 }
 
 extern "C" int qlora_codebook_tables(int32_t codebook, float* levels16, float* thr15,
-                                     float* bucket_thr1025, uint8_t* bucket_code1025) {
+                                     float* bucket_thr33, uint8_t* bucket_code33) {
   if (codebook < 0 || codebook >= qlora::kCodebooks) return -1;
   const auto& cb = qlora::tables().cb[codebook];
   for (int i = 0; i < 16; ++i)
@@ -208,8 +209,8 @@ extern "C" int qlora_codebook_tables(int32_t codebook, float* levels16, float* t
   for (int i = 0; i < 15; ++i)
     if (thr15) thr15[i] = cb.thr.t[i];
   for (int i = 0; i < qlora::kCodeBuckets; ++i) {
-    if (bucket_thr1025) bucket_thr1025[i] = cb.buckets.thr[i];
-    if (bucket_code1025) bucket_code1025[i] = cb.buckets.code[i];
+    if (bucket_thr33) bucket_thr33[i] = cb.buckets.thr[i];
+    if (bucket_code33) bucket_code33[i] = cb.buckets.code[i];
   }
   return 0;
 }

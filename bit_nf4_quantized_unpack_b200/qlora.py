@@ -134,13 +134,15 @@ class NF4Weight:
 # ------------------------------------------------------------------ host-only tables
 
 CODEBOOK_NF4, CODEBOOK_UNIFORM4 = 0, 1
+BUCKET_SCALE = 16                    # code-search buckets: round-half-even(16 x + 16)
+CODE_BUCKETS = 2 * BUCKET_SCALE + 1
 
 
 def codebook_tables(codebook: int):
-    """(levels [16], thresholds [15], bucket thresholds [1025], bucket codes [1025]) of a
+    """(levels [16], thresholds [15], bucket thresholds [33], bucket codes [33]) of a
     codebook, as the library builds them."""
     lev, thr = (ctypes.c_float * 16)(), (ctypes.c_float * 15)()
-    bthr, bcode = (ctypes.c_float * 1025)(), (ctypes.c_uint8 * 1025)()
+    bthr, bcode = (ctypes.c_float * CODE_BUCKETS)(), (ctypes.c_uint8 * CODE_BUCKETS)()
     rc = lib().qlora_codebook_tables(codebook, ctypes.cast(lev, ctypes.c_void_p),
                                      ctypes.cast(thr, ctypes.c_void_p),
                                      ctypes.cast(bthr, ctypes.c_void_p),
@@ -164,9 +166,10 @@ def nf4_thresholds() -> torch.Tensor:
 
 
 def nf4_code_buckets():
-    """(thr [1025] fp32, code [1025] uint8): the bucket table of the quantization kernel."""
-    thr = (ctypes.c_float * 1025)()
-    code = (ctypes.c_uint8 * 1025)()
+    """(thr [33] fp32, code [33] uint8): the bucket table of the quantization kernel
+    (bucket b = round-half-even(16 x + 16), code = code[b] + (x >= thr[b]))."""
+    thr = (ctypes.c_float * CODE_BUCKETS)()
+    code = (ctypes.c_uint8 * CODE_BUCKETS)()
     lib().qlora_nf4_code_buckets(ctypes.cast(thr, ctypes.c_void_p), ctypes.cast(code, ctypes.c_void_p))
     return (torch.tensor(list(thr), dtype=torch.float32),
             torch.tensor(list(code), dtype=torch.uint8))

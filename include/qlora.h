@@ -139,19 +139,20 @@ void qlora_nf4_thresholds(float *out15);
 /*
  * qlora_nf4_code_buckets: the table form of the same code search that the
  * quantization kernel uses, to host memory. For fp32 x in [-1, 1] let
- * b = round-half-even(512 x + 512) (0 <= b <= 1024); then
- * code(x) = code1025[b] + (x >= thr1025[b] ? 1 : 0), with thr1025[b] = +inf when no
+ * b = round-half-even(16 x + 16) (0 <= b <= 32: 33 buckets of width 1/16, each
+ * holding at most one threshold); then
+ * code(x) = code33[b] + (x >= thr33[b] ? 1 : 0), with thr33[b] = +inf when no
  * threshold lies in bucket b. Either pointer may be NULL. Host-only.
  */
-void qlora_nf4_code_buckets(float *thr1025, uint8_t *code1025);
+void qlora_nf4_code_buckets(float *thr33, uint8_t *code33);
 
 /*
  * The same three tables for any codebook (qlora_codebook): its 16 levels (fp32,
- * ascending), its 15 exact decision thresholds, and its 1025-bucket code table. Null
+ * ascending), its 15 exact decision thresholds, and its 33-bucket code table. Null
  * output pointers are skipped. Returns 0, or -1 for an unknown codebook. Host-only.
  */
-int qlora_codebook_tables(int32_t codebook, float *levels16, float *thr15, float *bucket_thr1025,
-                          uint8_t *bucket_code1025);
+int qlora_codebook_tables(int32_t codebook, float *levels16, float *thr15, float *bucket_thr33,
+                          uint8_t *bucket_code33);
 
 /*
  * qlora_fp8_thresholds: the same for the 253-entry double-quantization table T8

@@ -79,7 +79,7 @@ def test_nf4_thresholds_reproduce_argmin(L):
 
 def test_nf4_code_buckets_reproduce_argmin(L):
     """The quantization kernel's table form of the code search: bucket
-    b = round-half-even(512 x + 512), code = code[b] + (x >= thr[b]); checked against the
+    b = round-half-even(16 x + 16), code = code[b] + (x >= thr[b]); checked against the
     oracle's argmin on random x, around every threshold and level, and on both sides of
     every bucket edge."""
     thr, code = (t.numpy() for t in qlora.nf4_code_buckets())
@@ -89,12 +89,14 @@ def test_nf4_code_buckets_reproduce_argmin(L):
           np.array([-1.0, 1.0, 0.0, -0.0], np.float32)]
     for t in th:
         xs.append(_ulp_window(t, 256))
-    edges = ((2.0 * np.arange(1026) - 1025.0) / 1024.0).astype(np.float32)
+    S = qlora.BUCKET_SCALE
+    assert thr.shape == code.shape == (2 * S + 1,)
+    edges = ((2.0 * np.arange(2 * S + 2) - 2 * S - 1.0) / (2 * S)).astype(np.float32)
     for e in edges:
         xs.append(_ulp_window(e, 3))
     x = np.concatenate(xs)
     x = x[(x >= -1) & (x <= 1)]
-    b = np.rint(512.0 * x.astype(np.float64) + 512.0).astype(np.int64)  # rint: half to even
+    b = np.rint(S * x.astype(np.float64) + S).astype(np.int64)  # rint: half to even
     got = code[b].astype(np.int64) + (x >= thr[b]).astype(np.int64)
     assert np.array_equal(O.nearest_code(x, table), got)
 
@@ -110,13 +112,14 @@ def test_codebook_tables_reproduce_argmin(L, codebook):
           np.array([-1.0, 1.0, 0.0, -0.0], np.float32)]
     for t in th:
         xs.append(_ulp_window(t, 256))
-    for e in ((2.0 * np.arange(1026) - 1025.0) / 1024.0).astype(np.float32):
+    S = qlora.BUCKET_SCALE
+    for e in ((2.0 * np.arange(2 * S + 2) - 2 * S - 1.0) / (2 * S)).astype(np.float32):
         xs.append(_ulp_window(e, 2))
     x = np.concatenate(xs)
     x = x[(x >= -1) & (x <= 1)]
     want = O.nearest_code(x, table)
     assert np.array_equal(want, _count_leq(th, x))
-    b = np.rint(512.0 * x.astype(np.float64) + 512.0).astype(np.int64)
+    b = np.rint(S * x.astype(np.float64) + S).astype(np.int64)
     assert np.array_equal(want, bcode[b].astype(np.int64) + (x >= bthr[b]).astype(np.int64))
     assert L.qlora_codebook_tables(2, None, None, None, None) == -1
 
