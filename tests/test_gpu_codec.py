@@ -144,3 +144,32 @@ def test_dequant_of_handmade_constants():
     torch.cuda.synchronize()
     got = wd.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(got, O.bf16_bits(O.double_dequant(ref)))
+
+
+def test_double_quantization_at_every_t8_threshold():
+    """Block constants that put y = fl32(cc / c1) on the fp32 grid (step 2^-23) around
+    every decision boundary of the T8 search, on both signs. Each 256-block of constants
+    holds 0 and 2 (so c1 = 1) and pairs 1 + d, 1 - d; the fp64 sum is exact, so the mean
+    is exactly 1, cc = +-d exactly and y = +-d. Probes sit from two steps below to two
+    steps above each midpoint of consecutive non-negative T8 entries."""
+    t8_vals, _ = O.fp8_table()
+    pos = np.sort(t8_vals[t8_vals >= 0].astype(np.float64))
+    mids = (pos[:-1] + pos[1:]) / 2
+    step = 2.0 ** -23
+    d = np.unique(np.concatenate([(np.floor(mids / step) + j) * step for j in range(-2, 3)]))
+    d = d[(d > 0) & (d < 1)].astype(np.float32)
+    free = 127                                    # pairs per 256-block besides 0 and 2
+    nblk = -(-d.size // free)
+    d = np.concatenate([d, np.zeros(nblk * free - d.size, np.float32)])
+    a = []
+    for b in range(nblk):
+        seg = d[b * free:(b + 1) * free]
+        a.append(np.concatenate([[0.0, 2.0], 1.0 + seg, 1.0 - seg]).astype(np.float32))
+    a = np.concatenate(a)
+    assert np.array_equal((1.0 + d).astype(np.float32) - np.float32(1.0), d)  # exact grid
+    W = np.zeros((a.size, 64), np.float32)
+    W[:, 0] = a                                   # one weight per block carries its absmax
+    W = W.reshape(-1, 640)
+    ref = O.quantize_nf4_dq(W)
+    assert np.float32(ref["mean"]) == np.float32(1.0)
+    compare_full(W, bf16=False)
