@@ -406,6 +406,53 @@ def codec_bandwidth(device, reps=5):
     return out
 
 
+def optimizer_bandwidth(device, reps=5):
+    """HBM throughput of the paged AdamW step (qlora_adamw_step) over the LoRA parameters
+    of a 7B-shaped model: 32 layers of the seven linears at r = 64, 160M fp32 values in
+    one flat buffer (2.9 GB moved per 8-bit step, beyond L2). CUDA-graph timed, the
+    states in device memory. Algorithmic bytes per parameter: p read and written (8),
+    g read (4), the bf16 copy written (2), and the states read and written: 8-bit codes
+    (4) plus two fp32 absmax per 256 values (0.0625), or fp32 m and v (16)."""
+    from bit_nf4_quantized_unpack_b200 import inputs, qlora
+    n = 32 * sum(RANK_R * (k + nn) for _, nn, k in inputs.LLAMA7B_LINEARS)
+    g = torch.Generator(device=device)
+    g.manual_seed(9)
+    p = torch.randn(n, generator=g, device=device) * 0.02
+    grad = torch.randn(n, generator=g, device=device) * 1e-3
+    pb = torch.empty(n, dtype=torch.bfloat16, device=device)
+    out = {}
+    for bits, per_param in ((8, 18.0625), (32, 30.0)):
+        state = torch.zeros(qlora.qlora_adamw_state_bytes(n, bits), dtype=torch.uint8, device=device)
+        step = [0]
+
+        def one():
+            step[0] += 1
+            qlora.qlora_adamw_step(p, grad, state, 1 + step[0] % 1000, state_bits=bits, p_bf16=pb)
+        s = torch.cuda.Stream(device)
+        with torch.cuda.stream(s):
+            one()
+            one()
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=s):
+                for _ in range(reps):
+                    one()
+            graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            graph.replay()
+            e1.record(s)
+            torch.cuda.synchronize()
+        del graph, state
+        us = e0.elapsed_time(e1) * 1000.0 / reps
+        out[f"adamw_{bits}bit"] = {"us_per_step": us, "params": n, "bytes_per_param": per_param,
+                                   "GBps": n * per_param / us / 1e3}
+    out["workload"] = ("AdamW step over the LoRA parameters of a 7B-shaped model "
+                       f"(32 layers x 7 linears, r={RANK_R}): {n} fp32 values, bf16 copy written")
+    return out
+
+
 def e2e_steps(L, scale, world, steps):
     """The same step through the public API with host-resident inputs: every step copies
     its activations and upstream gradients from pinned host memory and reads its LoRA
@@ -618,6 +665,21 @@ def profile_merge(device, warmup, steps, n=4096, k=11008, r=RANK_R):
     torch.cuda.synchronize()
 
 
+def profile_optimizer(device, warmup, steps, n=40_000_000, state_bits=8):
+    """The paged AdamW step (8-bit states by default) on n LoRA-sized fp32 parameters, for
+    ncu captures (0.72 GB moved per 8-bit step, beyond L2)."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(10)
+    p = torch.randn(n, generator=g, device=device) * 0.02
+    grad = torch.randn(n, generator=g, device=device) * 1e-3
+    pb = torch.empty(n, dtype=torch.bfloat16, device=device)
+    state = torch.zeros(qlora.qlora_adamw_state_bytes(n, state_bits), dtype=torch.uint8, device=device)
+    for t in range(1, warmup + steps + 1):
+        qlora.qlora_adamw_step(p, grad, state, t, state_bits=state_bits, p_bf16=pb)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -629,6 +691,8 @@ def main():
     ap.add_argument("--profile-decode", action="store_true",
                     help="only run the M=1 forward of an 8192x28672 weight --steps times "
                          "(no graph): a small, self-contained case for profiler captures")
+    ap.add_argument("--profile-optimizer", action="store_true",
+                    help="only run the 8-bit AdamW step on 40M parameters (for ncu)")
     ap.add_argument("--profile-merge", action="store_true",
                     help="only run merge_and_unload of a 4096x11008 weight (r=64) --steps times")
     ap.add_argument("--stack-65b", action="store_true",
@@ -657,6 +721,9 @@ def main():
     scale = ALPHA / RANK_R
     if args.profile_merge:
         profile_merge(device, args.warmup, args.steps)
+        return
+    if args.profile_optimizer:
+        profile_optimizer(device, args.warmup, args.steps)
         return
     if args.stack_65b:
         stack_65b(device, args.warmup, args.steps)
@@ -720,7 +787,7 @@ def main():
     e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    decode = codec = None
+    decode = codec = optim = None
     if not args.no_decode and rank == 0:
         del L
         torch.cuda.empty_cache()
@@ -735,6 +802,10 @@ def main():
             v["frac_of_hbm"] = v["GBps"] / hbm
         codec["workload"] = ("bf16 weights 4096x4096, 4096x11008, 11008x4096 ~N(0,0.02), "
                              "0.1% x10 outliers; NF4 block 64, double-quant block 256")
+        optim = optimizer_bandwidth(device)
+        for k, v in optim.items():
+            if isinstance(v, dict):
+                v["frac_of_hbm"] = v["GBps"] / hbm
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -754,7 +825,7 @@ def main():
                            "l2": "inputs larger than L2 (weights + activations ~1.3 GB per step)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches,
-                "clocks": clk, "decode": decode, "codec": codec}
+                "clocks": clk, "decode": decode, "codec": codec, "optimizer": optim}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

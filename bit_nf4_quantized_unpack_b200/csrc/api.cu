@@ -324,4 +324,65 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   return gemm_backward(dY, X, T_saved, w, A, B, s, dX, dA, dB, workspace, st);
 }
 
+size_t qlora_adamw_state_bytes(int64_t n, int32_t state_bits) {
+  if (n < 0 || (state_bits != 8 && state_bits != 32)) return 0;
+  return adamw_state_layout(n, state_bits).total;
+}
+
+qlora_status qlora_adamw_step(float* p, uint16_t* p_bf16, const float* g, int64_t n,
+                              int32_t state_bits, void* state, size_t state_bytes,
+                              qlora_adamw_hparams hp, void* stream) {
+  if (n < 0 || (state_bits != 8 && state_bits != 32) || hp.step < 1) return QLORA_ERR_INVALID_ARG;
+  auto finite = [](float x) { return x == x && x < 3.5e38f && x > -3.5e38f; };
+  if (!finite(hp.lr) || !finite(hp.eps) || !finite(hp.weight_decay) || !finite(hp.beta1) ||
+      !finite(hp.beta2) || hp.lr < 0.f || !(hp.eps > 0.f) || hp.weight_decay < 0.f ||
+      hp.beta1 < 0.f || !(hp.beta1 < 1.f) || hp.beta2 < 0.f || !(hp.beta2 < 1.f))
+    return QLORA_ERR_INVALID_ARG;
+  if (n == 0) return QLORA_OK;
+  if (!p || !g || !state) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(p) || !aligned16(g) || !aligned16(state) || (p_bf16 && !aligned16(p_bf16)))
+    return QLORA_ERR_ALIGN;
+  if (state_bytes < adamw_state_layout(n, state_bits).total) return QLORA_ERR_WORKSPACE;
+  qlora_status q = check_device();
+  if (q != QLORA_OK) return q;
+  return cuda_status(launch_adamw(p, p_bf16, g, n, state_bits, state, hp,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_paged_alloc(void** out, size_t bytes) {
+  if (!out || bytes == 0) return QLORA_ERR_INVALID_ARG;
+  *out = nullptr;
+  void* ptr = nullptr;
+  cudaError_t e = cudaMallocManaged(&ptr, bytes, cudaMemAttachGlobal);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = cudaMemset(ptr, 0, bytes);  // a fresh optimizer state is all zeros
+  if (e != cudaSuccess) {
+    cudaFree(ptr);
+    return cuda_status(e);
+  }
+  e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    cudaFree(ptr);
+    return cuda_status(e);
+  }
+  *out = ptr;
+  return QLORA_OK;
+}
+
+qlora_status qlora_paged_free(void* ptr) {
+  if (!ptr) return QLORA_OK;
+  return cuda_status(cudaFree(ptr));
+}
+
+qlora_status qlora_paged_prefetch(const void* ptr, size_t bytes, int32_t to_device, void* stream) {
+  if (!ptr) return QLORA_ERR_INVALID_ARG;
+  if (bytes == 0) return QLORA_OK;
+  int dev = cudaCpuDeviceId;
+  if (to_device) {
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return cuda_status(cudaMemPrefetchAsync(ptr, bytes, dev, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

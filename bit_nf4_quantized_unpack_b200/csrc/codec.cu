@@ -11,6 +11,7 @@
 namespace qlora {
 namespace {
 
+static_assert(kT8Entries == kT8Size, "one T8 table size for the host and the device");
 constexpr int kQuantThreads = 256;
 constexpr int kMaxQuantCtas = 148 * 8;
 
@@ -172,32 +173,11 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
-// Index of entry i of T8 (ascending) -> its E4M3 bit pattern.
-__device__ __forceinline__ uint32_t t8_index_to_code(int i) {
-  return (i < 126) ? (0xFEu - static_cast<uint32_t>(i)) : (i == 126 ? 0u : static_cast<uint32_t>(i - 126));
-}
-// E4M3 bit pattern -> index of its value in T8 (both zeros -> the one zero entry, 126).
-__device__ __forceinline__ int t8_code_to_index(uint32_t e) {
-  return (e & 0x80u) ? static_cast<int>(0xFEu - e) : static_cast<int>(126u + e);
-}
-// E4M3 bit patterns of two fp32 values (hardware conversion, round to nearest even,
-// saturated at +-448): lo in bits 0-7, hi in bits 8-15.
-__device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
-  uint16_t d;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-
 // Level 2: the one mean of all block constants, then one warp per 256-block of constants,
 // 8 constants per lane. Launched as the programmatic dependent of level 1: every CTA forms
 // the mean itself from level 1's per-CTA fp64 partial sums, in the same order (fp64 sum,
 // one rounding to fp32), and CTA 0 stores it.
-//
-// The nearest T8 entry of y = fl32(cc / c1) (ties to the lower index) is the number of
-// T8 thresholds <= y. The hardware E4M3 conversion of fl32(448 y) gives a candidate entry
-// i: its rounding errors are below 2^-23 relative while neighbouring E4M3 values lie at
-// least 1/16 apart, so the answer is i - 1, i or i + 1, and one comparison with each of
-// the two thresholds around i decides it.
+// The E4M3 code of each y = fl32(cc / c1) comes from t8_nearest_codes2.
 __global__ void __launch_bounds__(256)
     k_double_quantize(const float* __restrict__ absmax, int64_t nblocks,
                       const double* __restrict__ partial, int nparts, float* __restrict__ mean_out,
@@ -240,18 +220,9 @@ __global__ void __launch_bounds__(256)
     uint32_t out[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-      float y[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) y[h] = (m > 0.f) ? __fdiv_rn(cc[i + h], m) : 0.f;
-      const uint32_t cand = e4m3x2_rn(__fmul_rn(y[0], 448.0f), __fmul_rn(y[1], 448.0f));
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int c = t8_code_to_index((cand >> (8 * h)) & 0xFFu);
-        const float up = sth[min(c, kT8Size - 2)];  // threshold between entries c and c + 1
-        const float dn = sth[max(c - 1, 0)];        // threshold between entries c - 1 and c
-        const int pos = c + ((c < kT8Size - 1 && y[h] >= up) ? 1 : 0) - ((c > 0 && y[h] < dn) ? 1 : 0);
-        out[(i + h) / 4] |= t8_index_to_code(pos) << (8 * ((i + h) % 4));
-      }
+      const float y0 = (m > 0.f) ? __fdiv_rn(cc[i], m) : 0.f;
+      const float y1 = (m > 0.f) ? __fdiv_rn(cc[i + 1], m) : 0.f;
+      out[i / 4] |= t8_nearest_codes2(y0, y1, sth) << (8 * (i % 4));
     }
     if (j0 + 8 <= nblocks) {
       reinterpret_cast<uint2*>(c2 + j0)[0] = make_uint2(out[0], out[1]);

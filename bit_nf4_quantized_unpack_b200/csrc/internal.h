@@ -78,4 +78,13 @@ qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const 
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// ---- launchers (optim.cu) -------------------------------------------------------
+// Byte offsets inside the optimizer-state buffer of n parameters (qlora_adamw_state_bytes):
+// 8-bit: m codes at 0, v codes at off_vc, m absmax at off_ma, v absmax at off_va;
+// 32-bit: m at 0, v at off_vc.
+struct AdamwStateLayout { size_t off_vc, off_ma, off_va, total; };
+AdamwStateLayout adamw_state_layout(int64_t n, int state_bits);
+cudaError_t launch_adamw(float* p, uint16_t* p_bf16, const float* g, int64_t n, int state_bits,
+                         void* state, const qlora_adamw_hparams& hp, cudaStream_t st);
+
 }  // namespace qlora

@@ -95,6 +95,48 @@ __device__ __forceinline__ void lut_decode8(uint32_t w, const Nf4Lut& t, uint32_
   }
 }
 
+// ---- T8, the 8-bit float code table of the double quantization: the 253 distinct finite
+// E4M3 values / 448 in ascending order (page "QLoRA", itwiki.kr, section "이중 양자화").
+constexpr int kT8Entries = 253;
+
+// Index of entry i of T8 -> its E4M3 bit pattern.
+__device__ __forceinline__ uint32_t t8_index_to_code(int i) {
+  return (i < 126) ? (0xFEu - static_cast<uint32_t>(i)) : (i == 126 ? 0u : static_cast<uint32_t>(i - 126));
+}
+// E4M3 bit pattern -> index of its value in T8 (both zeros -> the one zero entry, 126).
+__device__ __forceinline__ int t8_code_to_index(uint32_t e) {
+  return (e & 0x80u) ? static_cast<int>(0xFEu - e) : static_cast<int>(126u + e);
+}
+// E4M3 bit patterns of two fp32 values (hardware conversion, round to nearest even,
+// saturated at +-448): lo in bits 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// E4M3 codes of the nearest T8 entries (ties to the lower index) of y0 and y1 in [-1, 1]:
+// code of y0 in bits 0-7, of y1 in bits 8-15. sth holds the 252 exact decision thresholds
+// (sth[k] = the smallest fp32 whose nearest entry is k + 1), so the answer is the number
+// of thresholds <= y. The hardware E4M3 conversion of fl32(448 y) gives a candidate entry
+// i: its rounding errors are below 2^-23 relative while neighbouring E4M3 values lie at
+// least 1/16 apart, so the answer is i - 1, i or i + 1, and one comparison with each of
+// the two thresholds around i decides it.
+__device__ __forceinline__ uint32_t t8_nearest_codes2(float y0, float y1, const float* sth) {
+  const uint32_t cand = e4m3x2_rn(__fmul_rn(y0, 448.0f), __fmul_rn(y1, 448.0f));
+  uint32_t out = 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float y = h ? y1 : y0;
+    const int c = t8_code_to_index((cand >> (8 * h)) & 0xFFu);
+    const float up = sth[min(c, kT8Entries - 2)];  // threshold between entries c and c + 1
+    const float dn = sth[max(c - 1, 0)];           // threshold between entries c - 1 and c
+    const int pos = c + ((c < kT8Entries - 1 && y >= up) ? 1 : 0) - ((c > 0 && y < dn) ? 1 : 0);
+    out |= t8_index_to_code(pos) << (8 * h);
+  }
+  return out;
+}
+
 __device__ __forceinline__ uint16_t bf16_bits_rn(float x) {
   uint32_t d;
   asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(d) : "f"(x));

@@ -9,6 +9,7 @@ Names follow the C entry points:
     qlora_dequant(w)                                  -> W_hat bf16 [N, K]
     qlora_linear_fwd(X, w, A, B, scale)               -> (Y, T)
     qlora_linear_bwd(dY, X, T, w, A, B, scale)        -> (dX, dA, dB)
+    qlora_adamw_step(p, g, state, step, ...)          (in place; paged states: PagedBuffer)
 """
 from __future__ import annotations
 
@@ -38,6 +39,11 @@ class CNF4Weight(ctypes.Structure):
                 ("codebook", ctypes.c_int32)]
 
 
+class CAdamwHparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
+
+
 _lib = None
 _vp, _i64, _i32, _sz, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
 
@@ -65,6 +71,11 @@ _SIGNATURES = {
     "qlora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
     "qlora_linear_bwd": (_i32, [_vp, _vp, _vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp,
                                 _vp, _vp, _sz, _vp]),
+    "qlora_adamw_state_bytes": (_sz, [_i64, _i32]),
+    "qlora_adamw_step": (_i32, [_vp, _vp, _vp, _i64, _i32, _vp, _sz, CAdamwHparams, _vp]),
+    "qlora_paged_alloc": (_i32, [ctypes.POINTER(ctypes.c_void_p), _sz]),
+    "qlora_paged_free": (_i32, [_vp]),
+    "qlora_paged_prefetch": (_i32, [_vp, _sz, _i32, _vp]),
 }
 
 
@@ -292,3 +303,63 @@ def qlora_launch_count() -> int:
 def qlora_device_error(clear: bool = True) -> int:
     """Status of the device error word (QLORA_ERR_TIMEOUT after a timed-out wait)."""
     return int(lib().qlora_device_error(1 if clear else 0))
+
+
+# ---------------------------------------------------------------- optimizer step
+class PagedBuffer:
+    """Unified (managed) memory from qlora_paged_alloc, zero-filled: a paged optimizer
+    state. The driver moves its pages between host and device memory on demand;
+    prefetch() moves them ahead of use. Released by free() or when collected."""
+
+    def __init__(self, nbytes: int):
+        ptr = ctypes.c_void_p()
+        _check(lib().qlora_paged_alloc(ctypes.byref(ptr), nbytes), "qlora_paged_alloc")
+        self.ptr, self.nbytes = ptr.value, int(nbytes)
+
+    def prefetch(self, to_device: bool = True):
+        _check(lib().qlora_paged_prefetch(ctypes.c_void_p(self.ptr), self.nbytes,
+                                          1 if to_device else 0, _stream()), "qlora_paged_prefetch")
+
+    def host_bytes(self) -> bytes:
+        """A host copy of the contents (synchronise the device first)."""
+        return ctypes.string_at(self.ptr, self.nbytes)
+
+    def free(self):
+        if self.ptr:
+            _check(lib().qlora_paged_free(ctypes.c_void_p(self.ptr)), "qlora_paged_free")
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def qlora_adamw_state_bytes(n: int, state_bits: int = 8) -> int:
+    return int(lib().qlora_adamw_state_bytes(n, state_bits))
+
+
+def qlora_adamw_step(p: torch.Tensor, g: torch.Tensor, state, step: int, *, lr: float = 2e-4,
+                     beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                     weight_decay: float = 0.0, state_bits: int = 8,
+                     p_bf16: torch.Tensor | None = None) -> None:
+    """One AdamW update of the fp32 parameters p (in place) with gradient g; state is a
+    uint8 CUDA tensor or a PagedBuffer of qlora_adamw_state_bytes(p.numel(), state_bits)
+    bytes (zeros before the first step). p_bf16, when given, receives bf16(p)."""
+    for t, name in ((p, "p"), (g, "g")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous fp32 CUDA tensor")
+    if g.numel() != p.numel():
+        raise ValueError("p and g differ in size")
+    if p_bf16 is not None and (_as_bits(p_bf16).numel() != p.numel()):
+        raise ValueError("p_bf16 differs in size from p")
+    if isinstance(state, PagedBuffer):
+        sptr, sbytes = ctypes.c_void_p(state.ptr), state.nbytes
+    else:
+        if not state.is_cuda or not state.is_contiguous():
+            raise ValueError("state: expected a contiguous CUDA tensor")
+        sptr, sbytes = _ptr(state), state.numel() * state.element_size()
+    hp = CAdamwHparams(lr, beta1, beta2, eps, weight_decay, step)
+    _check(lib().qlora_adamw_step(_ptr(p), _ptr(p_bf16), _ptr(g), p.numel(), state_bits, sptr,
+                                  sbytes, hp, _stream()), "qlora_adamw_step")

@@ -290,6 +290,73 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
                               float *dA, float *dB, void *workspace,
                               size_t workspace_bytes, void *stream);
 
+/*
+ * ---- The optimizer step after the LoRA gradients (paged AdamW) ----
+ * itwiki "QLoRA", section on paged optimizers: the optimizer states live in unified
+ * memory, move to host memory when the GPU runs short and come back for the update;
+ * the training example of the computation section uses optim="paged_adamw_8bit" at
+ * learning rate 2e-4 and names paged_adamw_32bit beside it.
+ *
+ * Update of each parameter p with gradient g at step t >= 1 (AdamW: Adam with
+ * decoupled weight decay), every operation one IEEE fp32 rounding, in this order:
+ *   m = b1 m' + (1-b1) g          v = b2 v' + ((1-b2) g) g
+ *   mh = m / bc1                  vh = v / bc2          bc_i = fl32(1 - b_i^t) (fp64 pow)
+ *   p = p (1 - lr wd) - lr (mh / (sqrt(vh) + eps))
+ * with (1 - b1), (1 - b2) and (1 - lr wd) formed in fp32 on the host.
+ *
+ * State forms (state_bits):
+ *   32: m and v as fp32 arrays.
+ *   8:  per block of 256 consecutive parameters one fp32 absmax per state, and per
+ *       parameter one E4M3 code of the nearest entry of T8 (qlora_fp8_thresholds; ties
+ *       to the lower index) to fl32(x / absmax) (0 when absmax = 0); a stored value
+ *       reads back as fl32(T8[code] x absmax). The update itself uses the fp32 m and v.
+ *       (The pages attribute the 8-bit states to the authors' block-wise quantization
+ *       work without giving its format; this is the pages' own block-wise 8-bit float.)
+ * A zero-filled state buffer is the state before the first step.
+ */
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay;
+  int64_t step; /* t of this update, 1 for the first */
+} qlora_adamw_hparams;
+
+/* Bytes of the state buffer for n parameters (state_bits 8 or 32; 0 for other values or
+ * n < 0). Layout, each section starting on a 256-byte boundary: 8-bit: m codes [n],
+ * v codes [n], m absmax fp32 [ceil(n/256)], v absmax fp32 [ceil(n/256)]; 32-bit: m fp32
+ * [n], v fp32 [n]. */
+size_t qlora_adamw_state_bytes(int64_t n, int32_t state_bits);
+
+/*
+ * qlora_adamw_step: one AdamW update of n parameters, in place.
+ *   p      [n] fp32 device (or managed), the parameters (updated)
+ *   p_bf16 [n] bf16 device or NULL: receives bf16_rn(p) after the update (the LoRA operand
+ *          of the next forward)
+ *   g      [n] fp32 device, the gradient (for the LoRA parameters: dA and dB of
+ *          qlora_linear_bwd, flattened)
+ *   state  device or unified memory of at least qlora_adamw_state_bytes(n, state_bits)
+ *          bytes (updated)
+ * n == 0 enqueues nothing. Errors: QLORA_ERR_INVALID_ARG for a NULL pointer with n > 0,
+ * state_bits other than 8 or 32, step < 1, or lr, eps, weight_decay, beta outside
+ * (lr >= 0, eps > 0, weight_decay >= 0, 0 <= beta < 1, all finite);
+ * QLORA_ERR_WORKSPACE when state_bytes is too small; QLORA_ERR_ALIGN unless p, p_bf16,
+ * g and state are 16-byte aligned. Nothing is enqueued on an error.
+ */
+qlora_status qlora_adamw_step(float *p, uint16_t *p_bf16, const float *g, int64_t n,
+                              int32_t state_bits, void *state, size_t state_bytes,
+                              qlora_adamw_hparams hp, void *stream);
+
+/*
+ * Paged optimizer states (unified memory). qlora_paged_alloc allocates `bytes` of
+ * managed memory, visible to every device and the host, zero-filled (a fresh optimizer
+ * state), into *out; QLORA_ERR_CUDA if the allocation fails. qlora_paged_free releases
+ * it. qlora_paged_prefetch enqueues on `stream` a migration of [ptr, ptr + bytes) to the
+ * current device (to_device != 0) or to host memory (to_device == 0); without it the
+ * pages move on first touch. These are the only functions of the library that allocate
+ * memory; they are for optimizer states, not for the layer's hot path.
+ */
+qlora_status qlora_paged_alloc(void **out, size_t bytes);
+qlora_status qlora_paged_free(void *ptr);
+qlora_status qlora_paged_prefetch(const void *ptr, size_t bytes, int32_t to_device, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

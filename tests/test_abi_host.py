@@ -224,3 +224,39 @@ def test_linear_rejects_bad_arguments(L):
     assert bwd(P, P, Q, 64, W(), P, P, 8, 2.0, P, P, P, P, bneed, None) == 3
     assert L.qlora_dequant(W(k=100), P, None) == 2
     assert L.qlora_dequant(W(), None, None) == 1
+
+
+def test_adamw_rejects_bad_arguments(L):
+    """The optimizer step checks every argument before it touches a device."""
+    from bit_nf4_quantized_unpack_b200.qlora import CAdamwHparams
+    n = 1000
+    sb8, sb32 = L.qlora_adamw_state_bytes(n, 8), L.qlora_adamw_state_bytes(n, 32)
+    nblk = -(-n // 256)
+    assert sb8 == 2 * 1024 + 2 * 256 and sb8 >= 2 * n + 8 * nblk
+    assert sb32 == 2 * 4096
+    assert L.qlora_adamw_state_bytes(n, 16) == 0 and L.qlora_adamw_state_bytes(-1, 8) == 0
+
+    def hp(**kw):
+        a = dict(lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1)
+        a.update(kw)
+        return CAdamwHparams(a["lr"], a["beta1"], a["beta2"], a["eps"], a["weight_decay"], a["step"])
+
+    def call(p=P, pb=None, g=P, nn=n, bits=8, st=P, sbytes=sb8, **kw):
+        return L.qlora_adamw_step(p, pb, g, nn, bits, st, sbytes, hp(**kw), None)
+
+    assert call(p=None) == 1 and call(g=None) == 1 and call(st=None) == 1
+    assert call(bits=16) == 1 and call(nn=-1) == 1
+    assert call(step=0) == 1
+    assert call(lr=-1.0) == 1 and call(lr=float("nan")) == 1
+    assert call(eps=0.0) == 1 and call(weight_decay=-0.1) == 1
+    assert call(beta1=1.0) == 1 and call(beta2=-0.5) == 1 and call(beta2=float("inf")) == 1
+    assert call(p=Q) == 3 and call(g=Q) == 3 and call(st=Q) == 3 and call(pb=Q) == 3
+    assert call(sbytes=sb8 - 1) == 4
+    assert call(bits=32, sbytes=sb8) == 4
+    assert call(nn=0) == 0          # nothing to update, nothing launched
+    assert L.qlora_paged_free(None) == 0
+    assert L.qlora_paged_prefetch(None, 16, 1, None) == 1
+    import ctypes
+    out = ctypes.c_void_p()
+    assert L.qlora_paged_alloc(ctypes.byref(out), 0) == 1
+    assert L.qlora_paged_alloc(None, 16) == 1
