@@ -85,6 +85,7 @@ __device__ __forceinline__ float absmax3(float a, float b, float c) {
 // The code of x comes from the 33-bucket table (two shared-memory loads and one compare).
 constexpr int kQuantLanes = 4;
 constexpr int kQuantPer = 64 / kQuantLanes;  // elements per lane
+constexpr int kQuantChunks = kQuantPer / 8;  // 8-element loads (and 32-bit code words) per lane
 template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
     k_quantize_blocks(const T* __restrict__ W, int64_t nblocks,
@@ -106,31 +107,29 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int64_t stride = static_cast<int64_t>(gridDim.x) * per_cta;
   int64_t b = blockIdx.x * per_cta + threadIdx.x / kQuantLanes;
   // the next two blocks' elements are in flight while this one is coded
-  Raw8<T> n0[2], n1[2];
+  Raw8<T> n0[kQuantChunks], n1[kQuantChunks];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < kQuantChunks; ++h) {
     if (b < nblocks) n0[h].load(W + b * 64 + sub * kQuantPer + h * 8);
     if (b + stride < nblocks) n1[h].load(W + (b + stride) * 64 + sub * kQuantPer + h * 8);
   }
   for (; b < nblocks; b += stride) {
-    float v[16];
-    {
-      float (&v0)[8] = *reinterpret_cast<float(*)[8]>(v);
-      float (&v1)[8] = *reinterpret_cast<float(*)[8]>(v + 8);
-      n0[0].values(v0);
-      n0[1].values(v1);
-    }
+    float v[kQuantPer];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < kQuantChunks; ++h) n0[h].values(*reinterpret_cast<float(*)[8]>(v + 8 * h));
+#pragma unroll
+    for (int h = 0; h < kQuantChunks; ++h) {
       n0[h] = n1[h];
       if (b + 2 * stride < nblocks) n1[h].load(W + (b + 2 * stride) * 64 + sub * kQuantPer + h * 8);
     }
-    float m = fmaxf(fabsf(v[14]), fabsf(v[15]));
+    float m = fmaxf(fabsf(v[kQuantPer - 2]), fabsf(v[kQuantPer - 1]));
 #pragma unroll
-    for (int i = 0; i < 14; i += 2) m = absmax3(m, v[i], v[i + 1]);
+    for (int i = 0; i < kQuantPer - 2; i += 2) m = absmax3(m, v[i], v[i + 1]);
 #pragma unroll
     for (int o = 1; o < kQuantLanes; o <<= 1) m = fmaxf(m, __shfl_xor_sync(gmask, m, o));
-    uint32_t packed[2] = {0u, 0u};
+    uint32_t packed[kQuantChunks];
+#pragma unroll
+    for (int h = 0; h < kQuantChunks; ++h) packed[h] = 0u;
     if (m >= 0x1p-64f) {
       // the steps below on pairs of weights (packed f32x2: per lane the same roundings)
       const float r = __frcp_rn(m);
@@ -138,7 +137,7 @@ __global__ void __launch_bounds__(kQuantThreads)
       const uint64_t kscale = f2_pack(kBucketScale, kBucketScale);
       const uint64_t kbias = f2_pack(kBucketBias, kBucketBias);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kQuantPer / 2; ++i) {
         const uint64_t w = f2_pack(v[2 * i], v[2 * i + 1]);
         const uint64_t q = f2_mul(w, rr);
         const uint64_t e = f2_fma(q, nm, w);  // w - q m, exact
@@ -152,10 +151,14 @@ __global__ void __launch_bounds__(kQuantThreads)
       }
     } else {  // absmax zero or below 2^-64: plain IEEE division (x = 0 for a zero block)
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < kQuantPer; ++i)
         packed[i / 8] |= bucket_code(m > 0.f ? __fdiv_rn(v[i], m) : 0.f, sb) << (4 * (i % 8));
     }
-    reinterpret_cast<uint2*>(codes + b * 32)[sub] = make_uint2(packed[0], packed[1]);
+    if (kQuantChunks == 4)
+      reinterpret_cast<uint4*>(codes + b * 32)[sub] =
+          make_uint4(packed[0], packed[1 % kQuantChunks], packed[2 % kQuantChunks], packed[3 % kQuantChunks]);
+    else
+      reinterpret_cast<uint2*>(codes + b * 32)[sub] = make_uint2(packed[0], packed[1 % kQuantChunks]);
     if (sub == 0) {
       absmax[b] = m;
       acc += static_cast<double>(m);
