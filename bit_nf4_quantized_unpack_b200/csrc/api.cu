@@ -324,6 +324,12 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   return gemm_backward(dY, X, T_saved, w, A, B, s, dX, dA, dB, workspace, st);
 }
 
+qlora_status qlora_selftest_wait_timeout(void* stream) {
+  qlora_status q = check_device();
+  if (q != QLORA_OK) return q;
+  return cuda_status(launch_wait_selftest(static_cast<cudaStream_t>(stream)));
+}
+
 size_t qlora_adamw_state_bytes(int64_t n, int32_t state_bits) {
   if (n < 0 || (state_bits != 8 && state_bits != 32)) return 0;
   return adamw_state_layout(n, state_bits).total;

@@ -78,6 +78,9 @@ qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const 
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// ---- launchers (selftest.cu) ----------------------------------------------------
+cudaError_t launch_wait_selftest(cudaStream_t st);
+
 // ---- launchers (optim.cu) -------------------------------------------------------
 // Byte offsets inside the optimizer-state buffer of n parameters (qlora_adamw_state_bytes):
 // 8-bit: m codes at 0, v codes at off_vc, m absmax at off_ma, v absmax at off_va;

@@ -18,6 +18,7 @@ enum DeviceError : int {
   kErrTimeoutMma = 2,
   kErrTimeoutDequant = 3,
   kErrTimeoutEpilogue = 4,
+  kErrTimeoutSelfTest = 5,  // the wait of qlora_selftest_wait_timeout
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

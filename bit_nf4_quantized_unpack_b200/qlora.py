@@ -71,6 +71,7 @@ _SIGNATURES = {
     "qlora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
     "qlora_linear_bwd": (_i32, [_vp, _vp, _vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp,
                                 _vp, _vp, _sz, _vp]),
+    "qlora_selftest_wait_timeout": (_i32, [_vp]),
     "qlora_adamw_state_bytes": (_sz, [_i64, _i32]),
     "qlora_adamw_step": (_i32, [_vp, _vp, _vp, _i64, _i32, _vp, _sz, CAdamwHparams, _vp]),
     "qlora_paged_alloc": (_i32, [ctypes.POINTER(ctypes.c_void_p), _sz]),
@@ -298,6 +299,12 @@ def qlora_profile_events(before=None, after=None):
 def qlora_launch_count() -> int:
     """Kernel launches this library has enqueued so far in this process."""
     return int(lib().qlora_launch_count())
+
+
+def qlora_selftest_wait_timeout() -> None:
+    """Enqueue the failure-path self-test: one kernel whose wait runs out after 2 s and
+    records QLORA_ERR_TIMEOUT in the device error word (read it with qlora_device_error)."""
+    _check(lib().qlora_selftest_wait_timeout(_stream()), "qlora_selftest_wait_timeout")
 
 
 def qlora_device_error(clear: bool = True) -> int:

@@ -291,6 +291,16 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
                               size_t workspace_bytes, void *stream);
 
 /*
+ * qlora_selftest_wait_timeout: a test hook for the failure path that every kernel's
+ * bounded waits share (not part of the method). Enqueues on `stream` one small kernel
+ * whose only wait, on an mbarrier that nothing arrives at, runs out after the library's
+ * wait limit (2 s). The kernel records the timeout in the device error word and exits;
+ * after the stream completes, qlora_device_error returns QLORA_ERR_TIMEOUT, and the
+ * context stays usable. Errors: QLORA_ERR_DEVICE / QLORA_ERR_CUDA as the other calls.
+ */
+qlora_status qlora_selftest_wait_timeout(void *stream);
+
+/*
  * ---- The optimizer step after the LoRA gradients (paged AdamW) ----
  * itwiki "QLoRA", section on paged optimizers: the optimizer states live in unified
  * memory, move to host memory when the GPU runs short and come back for the update;
