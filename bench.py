@@ -688,6 +688,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-m", type=int, default=1,
+                    help="tokens of the --profile-decode forward (1..16)")
     ap.add_argument("--profile-decode", action="store_true",
                     help="only run the M=1 forward of an 8192x28672 weight --steps times "
                          "(no graph): a small, self-contained case for profiler captures")
@@ -732,7 +734,7 @@ def main():
         profile_linear(device, scale, args.warmup, args.steps)
         return
     if args.profile_decode:
-        profile_decode(device, args.warmup, args.steps)
+        profile_decode(device, args.warmup, args.steps, M=args.decode_m)
         return
     L = build_layer(device, seed=3 + 1000 * rank)
     flops = layer_flops(inputs.LLAMA7B_LINEARS, M_TOKENS, RANK_R)
