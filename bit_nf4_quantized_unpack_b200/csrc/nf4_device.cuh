@@ -115,13 +115,40 @@ __device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
   return d;
 }
 
+// The nearest-entry search over T8 by E4M3 code: for each code c the threshold just
+// above its entry (up), the one just below (dn), and the codes of the next and previous
+// entries and of the entry itself (moves: bits 0-7 next, 8-15 previous, 16-23 self; the
+// negative zero's self is the zero code). Built in shared memory by every CTA from the
+// 252 exact decision thresholds (build_t8_search).
+struct T8Search {
+  float up[256];
+  float dn[256];
+  uint32_t moves[256];
+};
+
+// Fill t from sth (sth[k] = the smallest fp32 whose nearest T8 entry is k + 1) with the
+// CTA's threads; the caller synchronises before use.
+__device__ __forceinline__ void build_t8_search(const float* sth, T8Search& t) {
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+    const uint32_t e = static_cast<uint32_t>(c);
+    const bool nan = (e & 0x7Fu) == 0x7Fu;  // never produced by a saturating conversion
+    const int i = nan ? 126 : t8_code_to_index(e);
+    t.up[c] = i < kT8Entries - 1 ? sth[i] : __int_as_float(0x7F800000);   // +inf
+    t.dn[c] = i > 0 ? sth[i - 1] : __int_as_float(0xFF800000);             // -inf
+    const uint32_t next = t8_index_to_code(i < kT8Entries - 1 ? i + 1 : i);
+    const uint32_t prev = t8_index_to_code(i > 0 ? i - 1 : i);
+    t.moves[c] = next | (prev << 8) | (t8_index_to_code(i) << 16);
+  }
+}
+
 // E4M3 codes of the nearest T8 entries (ties to the lower index) of y0 and y1 in [-1, 1]:
-// code of y0 in bits 0-7, of y1 in bits 8-15. sth holds the 252 exact decision thresholds
-// (sth[k] = the smallest fp32 whose nearest entry is k + 1), so the answer is the number
-// of thresholds <= y. The hardware E4M3 conversion of fl32(448 y) gives a candidate entry
-// i: its rounding errors are below 2^-23 relative while neighbouring E4M3 values lie at
-// least 1/16 apart, so the answer is i - 1, i or i + 1, and one comparison with each of
-// the two thresholds around i decides it.
+// code of y0 in bits 0-7, of y1 in bits 8-15. The answer is the number of decision
+// thresholds <= y. The hardware E4M3 conversion of fl32(448 y) gives a candidate entry:
+// its rounding errors are below 2^-23 relative while neighbouring E4M3 values lie at
+// least 1/16 apart, so the answer is the candidate or one of its two neighbours, and one
+// comparison with each of the two thresholds around the candidate decides it.
+// This form reads the 252 thresholds sth directly (no table to build: for kernels whose
+// CTAs code few values); the T8Search form below needs fewer instructions per value.
 __device__ __forceinline__ uint32_t t8_nearest_codes2(float y0, float y1, const float* sth) {
   const uint32_t cand = e4m3x2_rn(__fmul_rn(y0, 448.0f), __fmul_rn(y1, 448.0f));
   uint32_t out = 0u;
@@ -133,6 +160,19 @@ __device__ __forceinline__ uint32_t t8_nearest_codes2(float y0, float y1, const 
     const float dn = sth[max(c - 1, 0)];           // threshold between entries c - 1 and c
     const int pos = c + ((c < kT8Entries - 1 && y >= up) ? 1 : 0) - ((c > 0 && y < dn) ? 1 : 0);
     out |= t8_index_to_code(pos) << (8 * h);
+  }
+  return out;
+}
+__device__ __forceinline__ uint32_t t8_nearest_codes2(float y0, float y1, const T8Search& t) {
+  const uint32_t cand = e4m3x2_rn(__fmul_rn(y0, 448.0f), __fmul_rn(y1, 448.0f));
+  uint32_t out = 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float y = h ? y1 : y0;
+    const uint32_t c = (cand >> (8 * h)) & 0xFFu;
+    const uint32_t mv = t.moves[c];
+    const uint32_t sh = y >= t.up[c] ? 0u : (y < t.dn[c] ? 8u : 16u);
+    out |= ((mv >> sh) & 0xFFu) << (8 * h);
   }
   return out;
 }

@@ -118,9 +118,12 @@ __global__ void __launch_bounds__(kOptThreads, kOpt8CtasPerSm)
                  float* __restrict__ ma, float* __restrict__ va, const AdamwConsts c,
                  const T8Thresholds th) {
   __shared__ float sth[kT8Size - 1];
+  __shared__ T8Search search;
   __shared__ float t8[256];  // T8 by E4M3 code
   for (int i = threadIdx.x; i < kT8Size - 1; i += blockDim.x) sth[i] = th.t[i];
   for (int e = threadIdx.x; e < 256; e += blockDim.x) t8[e] = t8_value(e);
+  __syncthreads();
+  build_t8_search(sth, search);
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t nblk = (n + kStateBlock - 1) / kStateBlock;
@@ -158,8 +161,8 @@ __global__ void __launch_bounds__(kOptThreads, kOpt8CtasPerSm)
       const float ym1 = block_ratio(m[i + 1], mmax, rm);
       const float yv0 = block_ratio(v[i], vmax, rv);
       const float yv1 = block_ratio(v[i + 1], vmax, rv);
-      mo[i / 4] |= t8_nearest_codes2(ym0, ym1, sth) << (8 * (i % 4));
-      vo[i / 4] |= t8_nearest_codes2(yv0, yv1, sth) << (8 * (i % 4));
+      mo[i / 4] |= t8_nearest_codes2(ym0, ym1, search) << (8 * (i % 4));
+      vo[i / 4] |= t8_nearest_codes2(yv0, yv1, search) << (8 * (i % 4));
     }
     store8(p, j0, n, pv);
     if (p_bf16) store8_bf16(p_bf16, j0, n, pv);
