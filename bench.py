@@ -797,6 +797,10 @@ def main():
         hbm = float(peaks["hbm_gbs"])
         for v in decode.values():
             v["frac_of_hbm"] = v["GBps"] / hbm
+        for m in (4, 16):  # the other decode batch sizes, same shapes and timing
+            for key, v in decode_bandwidth(device, M=m).items():
+                v["frac_of_hbm"] = v["GBps"] / hbm
+                decode[f"{key}_m{m}"] = v
         decode["hbm_peak_GBps"] = hbm
         decode["hbm_peak_source"] = f"{peaks_src} hbm_gbs"
         codec = codec_bandwidth(device)
