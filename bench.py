@@ -665,6 +665,19 @@ def profile_merge(device, warmup, steps, n=4096, k=11008, r=RANK_R):
     torch.cuda.synchronize()
 
 
+def profile_dequant(device, warmup, steps, n=4096, k=11008):
+    """The standalone double dequantization of one n x k NF4 weight (bf16 out), for ncu
+    captures; the quantization launches come first."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(8)
+    W = (torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    q = qlora.qlora_quantize_nf4_dq(W)
+    for _ in range(warmup + steps):
+        qlora.qlora_dequant(q, out=W)
+    torch.cuda.synchronize()
+
+
 def profile_optimizer(device, warmup, steps, n=40_000_000, state_bits=8):
     """The paged AdamW step (8-bit states by default) on n LoRA-sized fp32 parameters, for
     ncu captures (0.72 GB moved per 8-bit step, beyond L2)."""
@@ -693,6 +706,8 @@ def main():
     ap.add_argument("--profile-decode", action="store_true",
                     help="only run the M=1 forward of an 8192x28672 weight --steps times "
                          "(no graph): a small, self-contained case for profiler captures")
+    ap.add_argument("--profile-dequant", action="store_true",
+                    help="only run the double dequantization of a 4096x11008 weight (for ncu)")
     ap.add_argument("--profile-optimizer", action="store_true",
                     help="only run the 8-bit AdamW step on 40M parameters (for ncu)")
     ap.add_argument("--profile-merge", action="store_true",
@@ -726,6 +741,9 @@ def main():
         return
     if args.profile_optimizer:
         profile_optimizer(device, args.warmup, args.steps)
+        return
+    if args.profile_dequant:
+        profile_dequant(device, args.warmup, args.steps)
         return
     if args.stack_65b:
         stack_65b(device, args.warmup, args.steps)
