@@ -69,7 +69,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+namespace {
+bool aligned16(const void* p) { return is_aligned16(p); }
 
 // Common checks of a quantized weight.
 qlora_status check_weight(const qlora_nf4_weight& w) {
@@ -81,6 +87,8 @@ qlora_status check_weight(const qlora_nf4_weight& w) {
     return QLORA_ERR_ALIGN;
   return QLORA_OK;
 }
+
+}  // namespace
 
 qlora_status check_device() {
   int dev = 0;
@@ -102,8 +110,6 @@ qlora_status check_linear(int64_t M, const qlora_nf4_weight& w, int r, float sca
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return QLORA_ERR_INVALID_ARG;
   return QLORA_OK;
 }
-
-}  // namespace
 
 void set_last_error(const char* msg) {
   std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg ? msg : "");
@@ -223,6 +229,7 @@ qlora_status qlora_quantize_dq(const void* W, qlora_dtype w_dtype, int64_t n_out
   if (w_dtype != QLORA_F32 && w_dtype != QLORA_BF16) return QLORA_ERR_INVALID_ARG;
   if (n_out < 1 || k_in < 64 || k_in % 64 != 0) return QLORA_ERR_SHAPE;
   if (n_out > (int64_t{1} << 31) || k_in > (int64_t{1} << 31)) return QLORA_ERR_SHAPE;
+  if (n_out * k_in / 64 > (int64_t{1} << 31)) return QLORA_ERR_SHAPE;  // the mean's exact sums
   if (!aligned16(W) || !aligned16(codes) || !aligned16(c2) || !aligned16(c1) || !aligned16(mean))
     return QLORA_ERR_ALIGN;
   if (!workspace || workspace_bytes < quantize_workspace_bytes(n_out, k_in))
@@ -265,7 +272,8 @@ qlora_status qlora_merge_lora(qlora_nf4_weight w, const uint16_t* A, const uint1
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {
   if (M < 0 || n_out < 1 || k_in < 64 || r < 8 || r > 64) return 0;
   const LinearShape s{M, n_out, k_in, r, 1.f};
-  return M <= kDecodeMaxM ? decode_workspace(s) : gemm_fwd_workspace(s);
+  const size_t dec = M <= kDecodeMaxM ? decode_workspace(s) : 0;
+  return dec ? dec : gemm_fwd_workspace(s);
 }
 
 qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, qlora_nf4_weight w, const uint16_t* A,
@@ -279,14 +287,16 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, qlora_nf4_weight w, 
       (T_save && !aligned16(T_save)))
     return QLORA_ERR_ALIGN;
   const LinearShape s{M, w.n_out, w.k_in, r, scale};
-  const size_t need = M <= kDecodeMaxM ? decode_workspace(s) : gemm_fwd_workspace(s);
+  // M <= 16 takes the decode kernels, unless they cannot run the shape
+  const size_t dec = M <= kDecodeMaxM ? decode_workspace(s) : 0;
+  const size_t need = dec ? dec : gemm_fwd_workspace(s);
   if (!workspace || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
   q = check_device();
   if (q != QLORA_OK) return q;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return M <= kDecodeMaxM ? decode_forward(X, w, A, B, s, Y, T_save, workspace, st)
-                          : gemm_forward(X, w, A, B, s, Y, T_save, workspace, st);
+  return dec ? decode_forward(X, w, A, B, s, Y, T_save, workspace, st)
+             : gemm_forward(X, w, A, B, s, Y, T_save, workspace, st);
 }
 
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, int r) {

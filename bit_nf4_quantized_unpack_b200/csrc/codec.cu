@@ -72,8 +72,13 @@ __device__ __forceinline__ float absmax3(float a, float b, float c) {
 }
 
 // Level 1: one 64-block per group of kQuantLanes = 4 lanes (16 elements per lane). Writes
-// the packed codes, the fp32 absmax of each block, and one fp64 partial sum of absmax per
-// CTA.
+// the packed codes and the fp32 absmax of each block, and adds every absmax, exactly, into
+// 256 integer bins (one per fp32 exponent) for the mean: absmax = sig * 2^(e - 150) with
+// sig its 24-bit significand and e its biased exponent (1 for subnormals), and bin e sums
+// the sig of its exponent as a 64-bit integer (at most 2^31 blocks of 2^24 each). The CTA
+// sums into shared bins, then adds its nonzero bins into the global ones (zeroed before
+// the launch). Integer sums do not depend on their order, so the mean is the same for
+// any schedule and any range of constants.
 //
 // x = fl32(w / absmax) is computed with Markstein's correction step (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000 processor", IBM J.
@@ -90,20 +95,21 @@ template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
     k_quantize_blocks(const T* __restrict__ W, int64_t nblocks,
                       const __grid_constant__ Nf4BucketTable tab, uint8_t* __restrict__ codes,
-                      float* __restrict__ absmax, double* __restrict__ partial) {
+                      float* __restrict__ absmax, unsigned long long* __restrict__ bins) {
   const int lane = threadIdx.x & 31;
   const int sub = lane & (kQuantLanes - 1);
   const unsigned gmask = ((1u << kQuantLanes) - 1u) << (lane & (32 - kQuantLanes));
   const int64_t per_cta = kQuantThreads / kQuantLanes;
   __shared__ BucketSmem sb;
+  __shared__ unsigned long long sbins[256];
   for (int i = threadIdx.x; i < kCodeBuckets; i += blockDim.x) {
     sb.thr[i] = tab.thr[i];
     sb.code[i] = tab.code[i];
   }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
   __syncthreads();
   // the double quantization may be scheduled now; it waits for this grid's results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  double acc = 0.0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * per_cta;
   int64_t b = blockIdx.x * per_cta + threadIdx.x / kQuantLanes;
   // the next two blocks' elements are in flight while this one is coded
@@ -161,50 +167,97 @@ __global__ void __launch_bounds__(kQuantThreads)
       reinterpret_cast<uint2*>(codes + b * 32)[sub] = make_uint2(packed[0], packed[1 % kQuantChunks]);
     if (sub == 0) {
       absmax[b] = m;
-      acc += static_cast<double>(m);
+      const uint32_t u = __float_as_uint(m);  // m >= 0
+      const uint32_t e = u >> 23;
+      const uint32_t sig = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+      if (sig) atomicAdd(&sbins[e ? e : 1u], static_cast<unsigned long long>(sig));
     }
   }
-  __shared__ double red[kQuantThreads / 32];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-  if (lane == 0) red[threadIdx.x / 32] = acc;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    double s = 0.0;
-    for (int i = 0; i < kQuantThreads / 32; ++i) s += red[i];
-    partial[blockIdx.x] = s;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+    if (sbins[i]) atomicAdd(bins + i, sbins[i]);
+}
+
+// fl32(S / n) (round to nearest, ties to even) for S = sum_e bins[e] * 2^(e - 150), the
+// exact sum of the block constants, and n >= 1 of them. One thread; exact integer
+// arithmetic: the 256 bins give a 320-bit integer A = S * 2^150, the quotient
+// q = floor(A * 2^64 / n) (448 bits, 32-bit digits, remainder kept) then holds S / n as
+// q * 2^-214 to at least 33 significant bits, and its bits below the kept 24 (or below
+// 2^-149 for a subnormal result) decide the rounding.
+__device__ float exact_mean_f32(const unsigned long long* bins, int64_t n) {
+  constexpr int kD = 14;  // 32-bit digits of A * 2^64 (A < 2^311)
+  uint32_t d[kD];
+#pragma unroll 1
+  for (int i = 0; i < kD; ++i) d[i] = 0u;
+#pragma unroll 1
+  for (int e = 1; e < 256; ++e) {
+    const unsigned long long v = bins[e];
+    if (!v) continue;
+    // add v * 2^(e + 64): digits from (e + 64) / 32 on, shifted by (e + 64) % 32
+    const int w = (e + 64) >> 5, sh = (e + 64) & 31;
+    uint64_t carry = 0;
+    const uint64_t parts[3] = {(v << sh) & 0xFFFFFFFFull, (v >> (32 - sh)) & 0xFFFFFFFFull,
+                               sh ? (v >> (64 - sh)) : 0ull};
+    for (int k = w; k < kD; ++k) {
+      const uint64_t add = (k - w < 3) ? parts[k - w] : 0ull;
+      if (add == 0 && carry == 0 && k - w >= 3) break;
+      const uint64_t t = static_cast<uint64_t>(d[k]) + add + carry;
+      d[k] = static_cast<uint32_t>(t);
+      carry = t >> 32;
+    }
   }
+  // q = d / n, long division from the most significant digit (n < 2^32)
+  const uint64_t nn = static_cast<uint64_t>(n);
+  uint64_t rem = 0;
+  for (int k = kD - 1; k >= 0; --k) {
+    const uint64_t cur = (rem << 32) | d[k];
+    d[k] = static_cast<uint32_t>(cur / nn);
+    rem = cur % nn;
+  }
+  int top = -1;  // index of the most significant set bit of q
+  for (int k = kD - 1; k >= 0 && top < 0; --k)
+    if (d[k]) top = 32 * k + 31 - __clz(d[k]);
+  if (top < 0) return 0.f;
+  auto bit = [&](int p) -> uint32_t { return p < 0 ? 0u : (d[p >> 5] >> (p & 31)) & 1u; };
+  // value = q * 2^-214; its binade 2^(top - 214); fp32 keeps 24 bits, and nothing below
+  // 2^-149 (bit 65 of q)
+  const int lsb = max(top - 23, 65);
+  uint32_t sig = 0;
+  for (int p = top; p >= lsb; --p) sig = (sig << 1) | bit(p);
+  const uint32_t guard = bit(lsb - 1);
+  uint32_t sticky = rem != 0 ? 1u : 0u;
+  for (int p = lsb - 2; p >= 0 && !sticky; --p) sticky |= bit(p);
+  if (guard && (sticky || (sig & 1u))) ++sig;
+  if (lsb == 65) return __uint_as_float(sig);  // subnormal (sig == 2^23: smallest normal)
+  int ebits = top - 214 + 127;                   // biased exponent of the binade
+  if (sig == 0x1000000u) {                       // rounding carried into the next binade
+    sig >>= 1;
+    ++ebits;
+  }
+  return __uint_as_float((static_cast<uint32_t>(ebits) << 23) | (sig & 0x7FFFFFu));
 }
 
 // Level 2: the one mean of all block constants, then one warp per 256-block of constants,
 // 8 constants per lane. Launched as the programmatic dependent of level 1: every CTA forms
-// the mean itself from level 1's per-CTA fp64 partial sums, in the same order (fp64 sum,
-// one rounding to fp32), and CTA 0 stores it.
+// the mean itself from level 1's exponent bins (exact sum, one rounding to fp32), and
+// CTA 0 stores it.
 // The E4M3 code of each y = fl32(cc / c1) comes from t8_nearest_codes2.
 __global__ void __launch_bounds__(256)
     k_double_quantize(const float* __restrict__ absmax, int64_t nblocks,
-                      const double* __restrict__ partial, int nparts, float* __restrict__ mean_out,
+                      const unsigned long long* __restrict__ bins, float* __restrict__ mean_out,
                       const T8Thresholds th, uint8_t* __restrict__ c2, float* __restrict__ c1) {
   __shared__ float sth[kT8Size - 1];
-  __shared__ double red[256 / 32];
+  __shared__ unsigned long long sbins[256];
   __shared__ float mean_s;
   for (int i = threadIdx.x; i < kT8Size - 1; i += blockDim.x) sth[i] = th.t[i];
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // level 1's absmax and partial sums
-  {
-    double acc = 0.0;
-    for (int i = threadIdx.x; i < nparts; i += blockDim.x) acc += partial[i];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = acc;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double sum = 0.0;
-      for (int i = 0; i < 256 / 32; ++i) sum += red[i];
-      mean_s = __double2float_rn(sum / static_cast<double>(nblocks));
-      if (blockIdx.x == 0) mean_out[0] = mean_s;
-    }
-    __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // level 1's absmax and bins
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = __ldcg(bins + i);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mean_s = exact_mean_f32(sbins, nblocks);
+    if (blockIdx.x == 0) mean_out[0] = mean_s;
   }
+  __syncthreads();
   const float mean = mean_s;
   const int lane = threadIdx.x & 31;
   const int64_t ndq = (nblocks + 255) / 256;
@@ -285,7 +338,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // CTAs of level 1: enough for every block, at most one resident wave (so that all of
-// them run from the start) and at most kMaxQuantCtas (the partial sums' slots).
+// them run from the start) and at most kMaxQuantCtas.
 template <typename T>
 cudaError_t quant_ctas(int64_t nblocks, int* ctas) {
   static std::atomic<int> resident{0};  // CTAs per SM, looked up once per input type
@@ -309,7 +362,7 @@ cudaError_t quant_ctas(int64_t nblocks, int* ctas) {
 
 size_t quantize_workspace_bytes(int64_t n, int64_t k) {
   const int64_t nblocks = n * k / 64;
-  return align_up(static_cast<size_t>(nblocks) * 4, 256) + kMaxQuantCtas * sizeof(double);
+  return align_up(static_cast<size_t>(nblocks) * 4, 256) + 256 * sizeof(unsigned long long);
 }
 
 cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, int codebook,
@@ -317,18 +370,20 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
                             cudaStream_t st) {
   const int64_t nblocks = n * k / 64;
   float* absmax = static_cast<float*>(ws);
-  double* partial = reinterpret_cast<double*>(static_cast<char*>(ws) +
-                                              align_up(static_cast<size_t>(nblocks) * 4, 256));
+  unsigned long long* bins = reinterpret_cast<unsigned long long*>(
+      static_cast<char*>(ws) + align_up(static_cast<size_t>(nblocks) * 4, 256));
   int ctas = 0;
   cudaError_t e = w_bf16 ? quant_ctas<uint16_t>(nblocks, &ctas) : quant_ctas<float>(nblocks, &ctas);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(bins, 0, 256 * sizeof(unsigned long long), st);
   if (e != cudaSuccess) return e;
   note_launches(2);  // blocks, then the mean and double quantization
   if (w_bf16)
     k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
+        static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, bins);
   else
     k_quantize_blocks<float><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, partial);
+        static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, bins);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t ndq = (nblocks + 255) / 256;
@@ -345,7 +400,7 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k_double_quantize, static_cast<const float*>(absmax), nblocks,
-                            static_cast<const double*>(partial), ctas, mean, t8_thresholds(), c2,
+                            static_cast<const unsigned long long*>(bins), mean, t8_thresholds(), c2,
                             c1);
 }
 

@@ -1,21 +1,25 @@
 // decode.cu -- the QLoRA linear forward for M <= 16 tokens (decode), which is bound by
-// reading the packed weight (0.516 B per parameter) and by the integer work of
-// expanding it.
+// reading the packed weight (0.516 B per parameter) and by the work of expanding it.
 //
 //   Y = bf16(X W_hat^T + scale (X A) B)    (page "QLoRA", itwiki.kr, section "계산 방식";
 //                                           alpha/r from page "quantization", minnong511)
 //
-// k_decode_lora_down: T = X A on one cluster of 8 CTAs that split K; the CTA partial sums
-//   meet through distributed shared memory. It also clears the GEMV's arrival counters.
-// k_decode_gemv: each warp owns 16 (M <= 8) or 32 weight rows and a range of K. Lanes load
-//   32 bytes of packed codes of one row with 128-bit loads (the next 256-wide unit while
-//   the current one is expanded), double-dequantize them in registers (16-entry bf16
-//   table per 64-block, prmt lookups) straight into the A fragments of mma.m16n8k16 (X is
-//   the B operand). The dequantized weight never leaves registers. Every warp stores its
-//   partial sums; the last warp of a row group to finish adds them up, adds
-//   scale * T B and writes the bf16 outputs, so no second pass over the partial sums runs.
-// The GEMV is a programmatic dependent of the T kernel: it streams the weight at once and
-// reads T and its counters only after griddepcontrol.wait.
+// Two launches per call:
+// k_decode_prep: zeroes T and the arrival counters of the call (one small CTA; it lets the
+//   main kernel launch at once).
+// k_decode_gemv (its programmatic dependent): one CTA per SM. CTA c owns one K split
+//   (split c % splits) and the row groups c / splits, + cps, ... of it. It stages the
+//   split's columns of X in shared memory once (padded so that the MMA operand loads are
+//   conflict-free), then
+//   * its weight warps each take one group of 16 (M <= 8) or 32 weight rows over the
+//     split: lanes stream 32 bytes of packed codes per row with 128-bit loads (the next
+//     256-wide unit while the current one is expanded), double-dequantize them straight
+//     into the A fragments of mma.m16n8k16 (X is the B operand; the dequantized weight
+//     never leaves registers) and store the split's partial sums; the last warp of a row
+//     group to finish adds the splits up, adds scale * T B and writes bf16 Y;
+//   * its last warp computes T = X A over its share of the split's rows from the staged X
+//     and adds it into T with fp32 atomics (so T's summation order varies from run to
+//     run, within fp32 rounding); the finishers wait, bounded, until every share is in.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -28,14 +32,23 @@
 namespace qlora {
 namespace {
 
-constexpr int kDecThreads = 128;
 // Weight rows per warp: one 16-row MMA group for M <= 8, two for M > 8 (the X fragments
-// of 16 tokens are then shared by twice the rows); CTAs per SM follow the registers.
+// of 16 tokens are then shared by twice the rows).
 __host__ __device__ constexpr int rows_per_warp(bool tall) { return tall ? 32 : 16; }
-__host__ __device__ constexpr int dec_ctas_per_sm(bool tall) { return tall ? 2 : 4; }
+// One CTA per SM: 16 warps at <= 128 registers (M <= 8) or 8 at <= 255 (M > 8); the last
+// warp of a CTA computes its share of T, the others take weight rows.
+__host__ __device__ constexpr int dec_threads(bool tall) { return tall ? 256 : 512; }
+__host__ __device__ constexpr int weight_warps(bool tall) { return dec_threads(tall) / 32 - 1; }
 constexpr int kUnitK = 256;  // K covered by one warp step (4 lanes x 64)
-constexpr int kTCtas = 8;    // cluster of the T kernel
-constexpr int kTThreads = 256;
+
+// X stage: each 64-column block of a token's row takes 128 bytes at a 144-byte stride,
+// and token rows are xs_tok bytes apart with xs_tok = 64 (mod 128). A B-fragment load
+// (lane (g, t) reads 16 bytes of block t of token g) then spreads over all eight 16-byte
+// bank groups.
+constexpr int kXBlkStride = 144;
+constexpr int kXStageMax = 48 * 1024;
+constexpr uint32_t kPairTabBytes = 65536;
+constexpr uint32_t kDecSmemMax = 2 * kPairTabBytes + kXStageMax + 1024;
 
 struct DecodeArgs {
   const uint8_t* codes;
@@ -50,10 +63,15 @@ struct DecodeArgs {
   float scale;
   int splits, units_per, nunits;  // K is cut into `splits` ranges of `units_per` 256-units
   int row_groups;                 // groups of rows_per_warp(M > 8) rows of W
+  int cps;                        // CTAs per split (grid = splits x cps)
+  int xs_tok;                     // bytes between token rows of the X stage
+  int xs_bytes;                   // bytes of the X stage (M x xs_tok)
   float* part;      // [splits][row_groups][M][rows per warp] partial sums of X W_hat^T
-  float* T;         // [M][r] T = X A
+  float* T;         // [M][r] T = X A (zeroed by k_decode_prep)
   float* T_save;    // optional copy of T for the backward pass
   int* counters;    // [row_groups] warps of the group that have stored their partials
+  int* t_count;     // T shares added so far
+  int* err;         // device error word
   uint16_t* Y;      // [M][N]
 };
 
@@ -67,131 +85,85 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ float bf16_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
 __device__ __forceinline__ int64_t lmin(int64_t x, int64_t y) { return x < y ? x : y; }
 
-// ---------------------------------------------------------------- T = X A
-// Thread layout: 4 columns of A per thread (jq), k lanes (kl) striding over this CTA's
-// share of K; X rows are read for all M tokens at once. Warp shuffles, then shared
-// memory, then the cluster sum the partial products.
-__global__ void __cluster_dims__(kTCtas, 1, 1) __launch_bounds__(kTThreads)
-    k_decode_lora_down(const DecodeArgs a) {
-  // the GEMV may start streaming the weight now; it waits for this grid before it
-  // touches T or the counters
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ float wred[kTThreads / 32][16 * 64];
-  __shared__ float cpart[16 * 64];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int r = a.r;
-  const int M = static_cast<int>(a.M);
-  for (int i = static_cast<int>(rank) * kTThreads + tid; i < a.row_groups; i += kTCtas * kTThreads)
-    a.counters[i] = 0;
+__device__ __forceinline__ uint64_t lds_b64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_b128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts_b128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
-  int jqn = 1;  // threads per A row: a power of two, 4 columns each
-  while (jqn * 4 < r) jqn <<= 1;
-  const int jq = tid & (jqn - 1), kl = tid / jqn, kls = kTThreads / jqn;
-  const int j0 = jq * 4;
-  const bool jlive = j0 < r;  // r is a multiple of 8, so j0 + 3 < r as well
-  const int64_t kper = (a.K + 8 * kTCtas - 1) / (8 * kTCtas) * 8;  // K is a multiple of 64
-  const int64_t k0 = static_cast<int64_t>(rank) * kper;
-  const int64_t k1 = lmin(a.K, k0 + kper);
-  float acc[16][4];
-#pragma unroll
-  for (int m = 0; m < 16; ++m)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[m][c] = 0.f;
-  if (jlive) {
-    // chunks of 8 consecutive k: every load of a chunk is issued before its math
-    for (int64_t kc = k0 + 8 * kl; kc < k1; kc += 8 * kls) {
-      float av[8][4];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.A + (kc + i) * r + j0));
-        av[i][0] = bf16_to_f32(v.x & 0xFFFFu);
-        av[i][1] = bf16_to_f32(v.x >> 16);
-        av[i][2] = bf16_to_f32(v.y & 0xFFFFu);
-        av[i][3] = bf16_to_f32(v.y >> 16);
-      }
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        if (m < M) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.X + m * a.K + kc));
-          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float x = bf16_to_f32((i & 1) ? (xw[i >> 1] >> 16) : (xw[i >> 1] & 0xFFFFu));
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[m][c] = fmaf(x, av[i][c], acc[m][c]);
-          }
-        }
-      }
-    }
-  }
-  // lanes that share jq hold partial sums of the same outputs
-  for (int o = jqn; o < 32; o <<= 1)
-#pragma unroll
-    for (int m = 0; m < 16; ++m)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[m][c] += __shfl_xor_sync(0xFFFFFFFFu, acc[m][c], o);
-  if (lane < jqn && jlive)
-#pragma unroll
-    for (int m = 0; m < 16; ++m)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) wred[warp][m * 64 + j0 + c] = acc[m][c];
-  __syncthreads();
-  const int mr = M * r;
-  for (int e = tid; e < mr; e += kTThreads) {
-    const int m = e / r, j = e % r;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kTThreads / 32; ++w) v += wred[w][m * 64 + j];
-    cpart[e] = v;
-  }
-  cluster_sync_all();  // every CTA's partial sums are in its shared memory
-  if (rank == 0) {
-    for (int e = tid; e < mr; e += kTThreads) {
-      float v = 0.f;
-#pragma unroll
-      for (int q = 0; q < kTCtas; ++q) v += ld_cluster_f32(&cpart[e], static_cast<uint32_t>(q));
-      a.T[e] = v;
-      if (a.T_save) a.T_save[e] = v;
-    }
-  }
-  cluster_sync_all();  // no CTA leaves while rank 0 still reads its shared memory
+// ---------------------------------------------------------------- call set-up
+__global__ void __launch_bounds__(256) k_decode_prep(float* T, int mr, int* counters, int nc,
+                                                     int* t_count) {
+  // the main kernel may launch now; it waits for this grid before it touches T or the
+  // counters
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int stride = gridDim.x * blockDim.x;
+  const int i0 = blockIdx.x * blockDim.x + threadIdx.x;
+  for (int i = i0; i < mr; i += stride) T[i] = 0.f;
+  for (int i = i0; i < nc; i += stride) counters[i] = 0;
+  if (i0 == 0) *t_count = 0;
 }
 
 // ---------------------------------------------------------------- X W_hat^T
-// 64 consecutive bf16 of X row `row` starting at column k, as 32 packed pairs.
-__device__ __forceinline__ void load_x64(const uint16_t* X, int64_t K, int64_t row, int64_t k,
-                                         uint32_t (&x)[32]) {
-  const uint4* p = reinterpret_cast<const uint4*>(X + row * K + k);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint4 v = __ldg(p + i);
-    x[4 * i] = v.x;
-    x[4 * i + 1] = v.y;
-    x[4 * i + 2] = v.z;
-    x[4 * i + 3] = v.w;
-  }
-}
-
 // Fragment mapping of the weight tasks: mma.m16n8k16 with the dequantized weight as the
 // A operand (16 weight rows) and X as the B operand (8 token columns). Lane (g = lane/4,
 // t = lane%4) owns K columns kb .. kb + 63 (kb = unit * 256 + 64 t) of weight rows g
 // and g + 8 of each 16-row group; MMA number j (0..15) of a unit takes from every lane
 // the four columns kb + 4j .. kb + 4j + 3: A pairs (rows g and g + 8), B pairs (token
 // g). Summation order over K does not matter, so this relabelling of the MMA's k index
-// is free, and the unpacked pairs land directly in the A operand registers.
+// is free, and the expanded pairs land directly in the A operand registers.
+//
+// Two ways to expand a 64-block of codes, both giving bf16_rn(fl32(L[code] * s)) bit for
+// bit; a warp uses both so that neither the integer ALU nor the shared-memory pipe
+// alone bounds it:
+//  * the pair table: every byte of codes (two weights) is the index of a shared-memory
+//    entry holding the two fp32 levels; one packed fp32 multiply by s and one bf16x2
+//    conversion give the operand pair. Per byte: one byte permute to form the address,
+//    one 8-byte shared load, one f32x2 multiply, one conversion.
+//  * the permute table (build_lut / lut_decode8 in nf4_device.cuh): a per-block
+//    16-entry bf16 table in registers, indexed by the codes through byte permutes.
+
+// Byte-pair level table: entry e (the code byte e: code e & 15 in its low nibble, e >> 4
+// in its high nibble) holds (L[e & 15], L[e >> 4]) as two fp32. Copy c (c = lane % 16)
+// of entry e lives at byte e * 256 + c * 8 of a 64 KB-aligned region, so the 16 lanes of
+// a half-warp read 16 distinct bank pairs whatever their bytes; the uniform codebook's
+// copies take bytes 128..255 of each 256-byte row. With the region 64 KB-aligned, one
+// byte permute builds the shared address from the code byte and a per-lane constant.
+
+// Eight codes (one word of packed codes) -> four bf16x2 operand registers through the
+// pair table (o[i] = elements 2i, 2i + 1); `lane_bits` holds the lane's copy offset in
+// byte 0 and byte 2 of the table's base in byte 2; s2 is the block scale in both halves.
+__device__ __forceinline__ void pair_decode8(uint32_t w, uint32_t lane_bits, uint64_t s2,
+                                             uint32_t (&o)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t addr = prmt(w, lane_bits, 0x7604u | (static_cast<uint32_t>(i) << 4));
+    float lo, hi;
+    f2_unpack(f2_mul(lds_b64(addr), s2), lo, hi);
+    o[i] = pack_bf16x2_rn(lo, hi);
+  }
+}
 
 // Packed codes and block constants of one unit for this lane (rows beyond N are clamped
 // and K beyond the matrix is clamped; their scale is forced to zero later).
@@ -202,8 +174,8 @@ struct UnitCodes {
   float e1[kGroups][2];
 };
 
-// This lane's four weight rows (clamped to the last row; their scale is forced to zero
-// later) as one base and 32-bit offsets from it, computed once per task.
+// This lane's weight rows (clamped to the last row; their scale is forced to zero later)
+// as one base and 32-bit offsets from it, computed once per task.
 template <int kGroups>
 struct RowBases {
   const uint8_t* code;           // codes of the first row
@@ -211,6 +183,16 @@ struct RowBases {
   int coff[kGroups][2];          // code byte offset of each row from `code`
   int boff[kGroups][2];          // block offset of each row from `blk`
 };
+
+// Streamed 16-byte load of packed codes that also asks L2 to fetch the whole 256-byte
+// segment (the next unit of the same row).
+__device__ __forceinline__ uint4 ldg_codes(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
 
 template <int kGroups>
 __device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases<kGroups>& rb, int u,
@@ -223,39 +205,67 @@ __device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases<kG
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const uint8_t* p = base + rb.coff[q][h];
-      c.q[q][h][0] = ldg_stream(p);
-      c.q[q][h][1] = ldg_stream(p + 16);
+      c.q[q][h][0] = ldg_codes(p);
+      c.q[q][h][1] = ldg_codes(p + 16);
       const int64_t j = jb + rb.boff[q][h];
       c.e2[q][h] = __ldg(a.c2 + j);
       c.e1[q][h] = __ldg(a.c1 + (j >> 8));
     }
 }
 
-template <bool kTall, int CB, int kGroups = kTall ? 2 : 1>
-__device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int g,
-                                             int t, const UnitCodes<kGroups>& c, const float* t8,
-                                             float mean, float (&acc)[kGroups][kTall ? 2 : 1][4]) {
-  const int64_t K = a.K;
-  const int64_t kraw = static_cast<int64_t>(u) * kUnitK + 64 * t;
-  const bool kv = kraw < K;
-  const int64_t kb = kv ? kraw : K - 64;
-  // token rows this lane feeds to the B operand; tokens >= M compute columns nobody stores
+// 64 bf16 of one token's row of the X stage (block `blk` of the split), as 32 pairs.
+__device__ __forceinline__ void lds_x64(uint32_t addr, uint32_t (&x)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 v = lds_b128(addr + 16 * i);
+    x[4 * i] = v.x;
+    x[4 * i + 1] = v.y;
+    x[4 * i + 2] = v.z;
+    x[4 * i + 3] = v.w;
+  }
+}
+
+// One unit: bit (2 q + h) of kPermMask selects the permute table for the row block of
+// rows (q, h); the others go through the pair table. xs0 / xs1: this lane's tokens' rows
+// of the X stage.
+template <bool kTall, int CB, uint32_t kPermMask, int kGroups = kTall ? 2 : 1>
+__device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int u0,
+                                             int nblk, int g, int t, const UnitCodes<kGroups>& c,
+                                             const float* t8, float mean, uint32_t lane_bits,
+                                             uint32_t xs0, uint32_t xs1,
+                                             float (&acc)[kGroups][kTall ? 2 : 1][4]) {
+  const int blk = (u - u0) * (kUnitK / 64) + t;  // block of the split
+  const bool kv = blk < nblk;                    // false past the end of K
+  const uint32_t xoff = static_cast<uint32_t>(min(blk, nblk - 1) * kXBlkStride);
   uint32_t xa[32], xb[32];
-  load_x64(a.X, K, lmin(g, a.M - 1), kb, xa);
-  if (kTall) load_x64(a.X, K, lmin(g + 8, a.M - 1), kb, xb);
+  lds_x64(xs0 + xoff, xa);
+  if (kTall) lds_x64(xs1 + xoff, xb);
 #pragma unroll
   for (int q = 0; q < kGroups; ++q) {
     Nf4Lut lut[2];
+    uint64_t s2[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const bool live = kv && (rbase + q * 16 + g + 8 * h) < a.N;
-      build_lut<CB>(live ? block_scale_tab(t8, c.e2[q][h], c.e1[q][h], mean) : 0.f, lut[h]);
+      const float s = live ? block_scale_tab(t8, c.e2[q][h], c.e1[q][h], mean) : 0.f;
+      if ((kPermMask >> (2 * q + h)) & 1u)
+        build_lut<CB>(s, lut[h]);
+      else
+        s2[h] = f2_pack(s, s);
     }
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       uint32_t o0[4], o1[4];
-      lut_decode8(w < 4 ? (&c.q[q][0][0].x)[w] : (&c.q[q][0][1].x)[w - 4], lut[0], o0);
-      lut_decode8(w < 4 ? (&c.q[q][1][0].x)[w] : (&c.q[q][1][1].x)[w - 4], lut[1], o1);
+      const uint32_t w0 = w < 4 ? (&c.q[q][0][0].x)[w] : (&c.q[q][0][1].x)[w - 4];
+      const uint32_t w1 = w < 4 ? (&c.q[q][1][0].x)[w] : (&c.q[q][1][1].x)[w - 4];
+      if ((kPermMask >> (2 * q)) & 1u)
+        lut_decode8(w0, lut[0], o0);
+      else
+        pair_decode8(w0, lane_bits, s2[0], o0);
+      if ((kPermMask >> (2 * q + 1)) & 1u)
+        lut_decode8(w1, lut[1], o1);
+      else
+        pair_decode8(w1, lane_bits, s2[1], o1);
       mma_bf16_16816(acc[q][0], o0[0], o1[0], o0[1], o1[1], xa[4 * w], xa[4 * w + 1]);
       mma_bf16_16816(acc[q][0], o0[2], o1[2], o0[3], o1[3], xa[4 * w + 2], xa[4 * w + 3]);
       if (kTall) {
@@ -268,9 +278,38 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
   }
 }
 
+// Which row blocks of a pair of units take the permute table: M <= 8, row g + 8 of every
+// unit (one half); M > 8, row g + 8 of the first 16-row group in even units and of the
+// second in odd ones (one quarter).
+template <bool kTall> struct PermMasks;
+template <> struct PermMasks<false> { static constexpr uint32_t even = 2u, odd = 2u; };
+template <> struct PermMasks<true> { static constexpr uint32_t even = 2u, odd = 8u; };
+
+// Bounded wait of a finisher for every T share of the call (lane 0 spins; false on
+// timeout, after recording it).
+__device__ __forceinline__ bool wait_t_complete(const DecodeArgs& a, int lane) {
+  int ok = 1;
+  if (lane == 0) {
+    const int need = a.splits * a.cps;
+    if (ld_acquire_gpu(a.t_count) < need) {
+      const uint64_t t0 = global_timer_ns();
+      for (uint32_t it = 0;; ++it) {
+        if (ld_acquire_gpu(a.t_count) >= need) break;
+        if ((it & 63) == 63 && global_timer_ns() - t0 > kWaitTimeoutNs) {
+          atomicCAS(a.err, 0, kErrTimeoutDecode);
+          ok = 0;
+          break;
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
 template <bool kTall, int CB>
 __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, int split,
-                                                   int lane, const float* t8) {
+                                                   int nblk, int lane, const float* t8,
+                                                   uint32_t lane_bits, uint32_t xs) {
   constexpr int kGroups = kTall ? 2 : 1;
   constexpr int kRowsPerWarp = rows_per_warp(kTall);
   const int g = lane >> 2, t = lane & 3;
@@ -278,6 +317,9 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   const int u1 = min(a.nunits, u0 + a.units_per);
   const float mean = *a.mean;
   const int64_t rbase = static_cast<int64_t>(rg) * kRowsPerWarp;
+  const uint32_t xs0 = xs + static_cast<uint32_t>(min(g, static_cast<int>(a.M) - 1) * a.xs_tok);
+  const uint32_t xs1 =
+      xs + static_cast<uint32_t>(min(g + 8, static_cast<int>(a.M) - 1) * a.xs_tok);
   float acc[kGroups][kTall ? 2 : 1][4];
 #pragma unroll
   for (int q = 0; q < kGroups; ++q)
@@ -304,10 +346,12 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   if (u0 < u1) load_unit(a, rb, u0, t, bpr, cb0);
   for (int u = u0; u < u1; u += 2) {
     if (u + 1 < u1) load_unit(a, rb, u + 1, t, bpr, cb1);
-    compute_unit<kTall, CB>(a, rbase, u, g, t, cb0, t8, mean, acc);
+    compute_unit<kTall, CB, PermMasks<kTall>::even>(a, rbase, u, u0, nblk, g, t, cb0, t8, mean,
+                                                     lane_bits, xs0, xs1, acc);
     if (u + 1 < u1) {
       if (u + 2 < u1) load_unit(a, rb, u + 2, t, bpr, cb0);
-      compute_unit<kTall, CB>(a, rbase, u + 1, g, t, cb1, t8, mean, acc);
+      compute_unit<kTall, CB, PermMasks<kTall>::odd>(a, rbase, u + 1, u0, nblk, g, t, cb1, t8,
+                                                      mean, lane_bits, xs0, xs1, acc);
     }
   }
 
@@ -326,7 +370,7 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
         if (m < M) pp[m * kRowsPerWarp + rl] = acc[q][hm][i];
       }
 
-  // T and the cleared counters come from the T kernel
+  // the counters come zeroed from k_decode_prep
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __threadfence();
   __syncwarp();
@@ -335,6 +379,7 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   last = __shfl_sync(0xFFFFFFFFu, last, 0);
   if (!last) return;
   __threadfence();  // the other warps' partial sums are visible from here on
+  if (!wait_t_complete(a, lane)) return;
 
   const int64_t row = rbase + lane;
   if (lane >= kRowsPerWarp || row >= a.N) return;
@@ -371,40 +416,135 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
     if (m < M) a.Y[m * a.N + row] = bf16_bits_rn(y[m] + a.scale * lora[m]);
 }
 
-// The two code buffers of the prefetch set the occupancy: 16 warps per SM with 16 rows per
-// warp (M <= 8), 8 with 32 (M > 8), each without spills.
+// ---------------------------------------------------------------- T = X A
+// The CTA's share of T: rows [k0, k1) of A (inside its split, so X comes from the stage).
+// Lane (jq, tg): columns 4 jq .. 4 jq + 3 of A, tokens tg, tg + tgn, ... (at most 8).
+__device__ __forceinline__ void decode_t_share(const uint16_t* __restrict__ A, float* T,
+                                               float* T_save, int* t_count, int shares, int r,
+                                               int M, int xs_tok, int64_t kbeg, int64_t k0,
+                                               int64_t k1, int lane, uint32_t xs) {
+  int jqn = 2;  // lanes per token: a power of two with 4 jqn >= r
+  while (jqn * 4 < r) jqn <<= 1;
+  const int tgn = 32 / jqn;  // token groups (>= 2)
+  const int jq = lane & (jqn - 1), tg = lane / jqn;
+  const int j0 = jq * 4;
+  const bool jlive = j0 < r;  // r is a multiple of 8, so j0 + 3 < r as well
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
+  if (jlive) {
+    for (int64_t k = k0; k < k1; k += 8) {  // k0, k1 are multiples of 8
+      float av[8][4];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(A + (k + e) * r + j0));
+        av[e][0] = bf16_to_f32(v.x & 0xFFFFu);
+        av[e][1] = bf16_to_f32(v.x >> 16);
+        av[e][2] = bf16_to_f32(v.y & 0xFFFFu);
+        av[e][3] = bf16_to_f32(v.y >> 16);
+      }
+      const int64_t kk = k - kbeg;
+      const uint32_t xo = static_cast<uint32_t>((kk >> 6) * kXBlkStride + (kk & 63) * 2);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int m = tg + i * tgn;
+        if (m < M) {
+          const uint4 xv = lds_b128(xs + static_cast<uint32_t>(m * xs_tok) + xo);
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x = bf16_to_f32((e & 1) ? (xw[e >> 1] >> 16) : (xw[e >> 1] & 0xFFFFu));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[i][c] = fmaf(x, av[e][c], acc[i][c]);
+          }
+        }
+      }
+    }
+  }
+  // T was zeroed by k_decode_prep
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (jlive && k0 < k1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int m = tg + i * tgn;
+      if (m < M)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) atomicAdd(T + m * r + j0 + c, acc[i][c]);
+    }
+  }
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = atomicAdd(t_count, 1) == shares - 1;
+  last = __shfl_sync(0xFFFFFFFFu, last, 0);
+  if (last && T_save) {
+    __threadfence();
+    for (int e = lane; e < M * r; e += 32) T_save[e] = __ldcg(T + e);
+  }
+}
+
+// ---------------------------------------------------------------- the main kernel
 template <bool kTall, int CB>  // kTall: M > 8 (tokens 8..15 in the upper fragment rows); CB: codebook
-__global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm(kTall)) k_decode_gemv(const DecodeArgs a) {
-  __shared__ float t8[256];  // T8 by E4M3 code
+__global__ void __launch_bounds__(dec_threads(kTall), 1) k_decode_gemv(const DecodeArgs a) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const uint32_t sbase = smem_u32(dsm);
+  const uint32_t tab = (sbase + kPairTabBytes - 1) & ~(kPairTabBytes - 1);
+  // the X stage and T8 go below the table when they fit there, else above it
+  const uint32_t need = static_cast<uint32_t>(a.xs_bytes) + 1024u;
+  const uint32_t xs_off = (tab - sbase >= need) ? 0u : (tab - sbase) + kPairTabBytes;
+  const uint32_t xs = sbase + xs_off;
+  float* t8 = reinterpret_cast<float*>(dsm + xs_off + a.xs_bytes);
+  uint8_t* tabp = dsm + (tab - sbase);
+  const int split = blockIdx.x % a.splits, cidx = blockIdx.x / a.splits;
+  const int u0 = split * a.units_per;
+  const int u1 = min(a.nunits, u0 + a.units_per);
+  const int64_t kbeg = static_cast<int64_t>(u0) * kUnitK;
+  const int64_t kend = lmin(a.K, static_cast<int64_t>(u1) * kUnitK);
+  const int nblk = static_cast<int>((kend - kbeg) / 64);  // K is a multiple of 64
+  const int M = static_cast<int>(a.M);
+
   for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
+  // 256 entries x 16 copies; thread i writes entry i / 16, copy i % 16
+  for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
+    const int e = i >> 4, cp = i & 15;
+    *reinterpret_cast<float2*>(tabp + e * 256 + CB * 128 + cp * 8) =
+        make_float2(code_level<CB>(e & 15), code_level<CB>(e >> 4));
+  }
+  // X columns [kbeg, kend) of every token, 16 bytes per thread and step
+  for (int i = threadIdx.x; i < M * nblk * 8; i += blockDim.x) {
+    const int m = i / (nblk * 8), rem = i - m * (nblk * 8);
+    const int b = rem >> 3, c = rem & 7;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.X + m * a.K + kbeg + b * 64 + c * 8));
+    sts_b128(xs + static_cast<uint32_t>(m * a.xs_tok + b * kXBlkStride + c * 16), v);
+  }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int task = blockIdx.x * (kDecThreads / 32) + warp;
-  if (task < a.row_groups * a.splits)
-    decode_weight_task<kTall, CB>(a, task % a.row_groups, task / a.row_groups, lane, t8);
+  constexpr int kW = weight_warps(kTall);
+  if (warp == kW) {
+    // this CTA's share of the split's rows of A
+    const int64_t share = ((kend - kbeg + a.cps - 1) / a.cps + 7) / 8 * 8;
+    const int64_t k0 = lmin(kend, kbeg + cidx * share);
+    const int64_t k1 = lmin(kend, k0 + share);
+    decode_t_share(a.A, a.T, a.T_save, a.t_count, a.splits * a.cps, a.r, M, a.xs_tok, kbeg, k0,
+                   k1, lane, xs);
+    return;
+  }
+  const uint32_t lane_bits =
+      static_cast<uint32_t>((lane & 15) * 8 + CB * 128) | (tab & 0x00FF0000u);
+  for (int rg = cidx + a.cps * warp; rg < a.row_groups; rg += a.cps * kW)
+    decode_weight_task<kTall, CB>(a, rg, split, nblk, lane, t8, lane_bits, xs);
 }
 
 // ---------------------------------------------------------------- host side
 struct DecodePlan {
-  int splits, units_per, nunits, row_groups;
+  int splits, units_per, nunits, row_groups, cps, xs_tok;
 };
 
-// K splits: enough warps for about two waves of the GEMV (16 or 8 resident warps per SM),
-// but no more than K / (16 M): the partial sums (split x M x 4 bytes per row, written
-// and read back through L2) stay at most half the code bytes.
-DecodePlan plan_decode(const LinearShape& s) {
-  DecodePlan p;
-  p.nunits = static_cast<int>((s.K + kUnitK - 1) / kUnitK);
-  const int rows = rows_per_warp(s.M > 8);
-  p.row_groups = static_cast<int>((s.N + rows - 1) / rows);
-  const int64_t per_sm = dec_ctas_per_sm(s.M > 8) * (kDecThreads / 32);
-  const int64_t target = 2 * per_sm * num_sms();
-  int64_t want = (target + p.row_groups - 1) / p.row_groups;
-  want = std::min<int64_t>(want, std::max<int64_t>(1, s.K / (16 * std::max<int64_t>(1, s.M))));
-  want = std::max<int64_t>(1, std::min<int64_t>(want, p.nunits));
-  p.units_per = static_cast<int>((p.nunits + want - 1) / want);
-  p.splits = (p.nunits + p.units_per - 1) / p.units_per;
-  return p;
+int x_stage_tok(int units_per) {
+  const int raw = units_per * (kUnitK / 64) * kXBlkStride;
+  return (raw + 63) / 128 * 128 + 64;  // >= raw, = 64 (mod 128)
 }
 
 size_t part_bytes(const DecodePlan& p, const LinearShape& s) {
@@ -412,9 +552,80 @@ size_t part_bytes(const DecodePlan& p, const LinearShape& s) {
                   256);
 }
 size_t t_bytes(const LinearShape& s) { return align_up(static_cast<size_t>(s.M) * s.r * 4, 256); }
-size_t counter_bytes(const DecodePlan& p) { return align_up(static_cast<size_t>(p.row_groups) * 4, 256); }
+size_t counter_bytes(const DecodePlan& p) {
+  return align_up(static_cast<size_t>(p.row_groups) * 4 + 4, 256);  // + the T count
+}
+size_t decode_scratch_bytes(const DecodePlan& p, const LinearShape& s) {
+  return part_bytes(p, s) + t_bytes(s) + counter_bytes(p);
+}
 
-// The T kernel, then the GEMV as its programmatic dependent.
+// K splits and CTAs per split. CTA c takes split c % splits and row groups c / splits,
+// + cps, ...; each of its weight warps one row group at a time over the whole split. The
+// choice minimises the units of the busiest warp (each task charged two extra units for
+// its pipeline fill and its partial-sum store, and a CTA with fewer than three quarters
+// of its weight warps busy charged for the bandwidth it leaves unused), subject to the X
+// stage fitting its shared-memory budget, at most K / (16 M) splits (the partial sums,
+// split x M x 4 bytes per row, stay at most half the code bytes) and the scratch fitting
+// `max_scratch`. Ties go to fewer splits. Returns splits = 0 when nothing fits.
+DecodePlan plan_decode(const LinearShape& s, size_t max_scratch = ~size_t{0}) {
+  DecodePlan p;
+  p.nunits = static_cast<int>((s.K + kUnitK - 1) / kUnitK);
+  const bool tall = s.M > 8;
+  const int rows = rows_per_warp(tall);
+  p.row_groups = static_cast<int>((s.N + rows - 1) / rows);
+  const int64_t W = weight_warps(tall);
+  const int64_t sms = num_sms();
+  const int64_t max_splits =
+      std::max<int64_t>(1, std::min<int64_t>(p.nunits, s.K / (16 * std::max<int64_t>(1, s.M))));
+  double best_cost = -1.0;
+  p.splits = 0;
+  p.units_per = p.nunits;
+  p.cps = 1;
+  p.xs_tok = x_stage_tok(p.nunits);
+  for (int up = p.nunits; up >= 1; --up) {
+    const int64_t splits = (p.nunits + up - 1) / up;
+    if (splits > max_splits || splits > sms) continue;
+    if (s.M * x_stage_tok(up) > kXStageMax) continue;
+    DecodePlan c = p;
+    c.splits = static_cast<int>(splits);
+    c.units_per = up;
+    if (decode_scratch_bytes(c, s) > max_scratch) continue;
+    const int64_t cps = std::max<int64_t>(1, std::min<int64_t>(sms / splits, p.row_groups));
+    const int64_t per_cta = (p.row_groups + cps - 1) / cps;
+    const int64_t tasks = (per_cta + W - 1) / W;
+    const int64_t busy = std::min<int64_t>(per_cta, W);
+    const double want = 0.75 * static_cast<double>(W);
+    const double cost = static_cast<double>(tasks * (up + 2)) *
+                        (static_cast<double>(busy) < want ? want / static_cast<double>(busy) : 1.0);
+    if (best_cost < 0.0 || cost < best_cost) {
+      best_cost = cost;
+      p.splits = static_cast<int>(splits);
+      p.units_per = up;
+      p.cps = static_cast<int>(cps);
+    }
+  }
+  p.xs_tok = x_stage_tok(p.units_per);
+  return p;
+}
+
+template <bool kTall, int CB>
+cudaError_t launch_gemv(cudaLaunchConfig_t& cfg, const DecodeArgs& a) {
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(k_decode_gemv<kTall, CB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kDecSmemMax));
+  });
+  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
+  return cudaLaunchKernelEx(&cfg, k_decode_gemv<kTall, CB>, a);
+}
+
+// The set-up kernel, then the main kernel as its programmatic dependent.
 qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
                            const uint16_t* B, const LinearShape& s, const DecodePlan& p,
                            uint16_t* Y, float* T_save, char* scratch, cudaStream_t st) {
@@ -435,20 +646,27 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   a.units_per = p.units_per;
   a.nunits = p.nunits;
   a.row_groups = p.row_groups;
+  a.cps = p.cps;
+  a.xs_tok = p.xs_tok;
+  a.xs_bytes = static_cast<int>(s.M) * p.xs_tok;
   a.part = reinterpret_cast<float*>(scratch);
   a.T = reinterpret_cast<float*>(scratch + part_bytes(p, s));
   a.counters = reinterpret_cast<int*>(scratch + part_bytes(p, s) + t_bytes(s));
+  a.t_count = a.counters + p.row_groups;
+  a.err = device_error_word();
   a.T_save = T_save;
   a.Y = Y;
-  note_launches(2);  // this kernel and the GEMV below
-  k_decode_lora_down<<<kTCtas, kTThreads, 0, st>>>(a);
+  if (!a.err) return QLORA_ERR_CUDA;
+  note_launches(2);  // the set-up kernel and the main kernel
+  const int mr = static_cast<int>(s.M) * s.r;
+  const int prep_ctas = std::max(1, std::min(num_sms(), (p.row_groups + 2047) / 2048));
+  k_decode_prep<<<prep_ctas, 256, 0, st>>>(a.T, mr, a.counters, p.row_groups, a.t_count);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e);
-  const int64_t warps = static_cast<int64_t>(p.row_groups) * p.splits;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((warps + kDecThreads / 32 - 1) / (kDecThreads / 32)));
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.gridDim = dim3(static_cast<unsigned>(p.splits * p.cps));
+  cfg.blockDim = dim3(dec_threads(s.M > 8));
+  cfg.dynamicSmemBytes = 2 * kPairTabBytes + static_cast<uint32_t>(a.xs_bytes) + 1024;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -456,23 +674,18 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (w.codebook == 1)
-    e = s.M > 8 ? cudaLaunchKernelEx(&cfg, k_decode_gemv<true, 1>, a)
-                : cudaLaunchKernelEx(&cfg, k_decode_gemv<false, 1>, a);
+    e = s.M > 8 ? launch_gemv<true, 1>(cfg, a) : launch_gemv<false, 1>(cfg, a);
   else
-    e = s.M > 8 ? cudaLaunchKernelEx(&cfg, k_decode_gemv<true, 0>, a)
-                : cudaLaunchKernelEx(&cfg, k_decode_gemv<false, 0>, a);
+    e = s.M > 8 ? launch_gemv<true, 0>(cfg, a) : launch_gemv<false, 0>(cfg, a);
   if (e != cudaSuccess) return cuda_status(e);
   return QLORA_OK;
-}
-
-size_t decode_scratch_bytes(const DecodePlan& p, const LinearShape& s) {
-  return part_bytes(p, s) + t_bytes(s) + counter_bytes(p);
 }
 
 }  // namespace
 
 size_t decode_workspace(const LinearShape& s) {
-  return decode_scratch_bytes(plan_decode(s), s) + 256;
+  const DecodePlan p = plan_decode(s);
+  return p.splits ? decode_scratch_bytes(p, s) + 256 : 0;
 }
 
 qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
@@ -490,8 +703,8 @@ qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const 
 // all device memory once at start-up and forbids later allocation, or a decode loop
 // that must not pay cudaMalloc's implicit device synchronisation on every token.
 // They cannot hand over a workspace either. For them, qlora_linear_fwd_decode_static
-// keeps the split partial sums in the fixed array below, which every GPU that loads
-// this library holds until the process exits.
+// keeps the split partial sums, T and the arrival counters in the fixed array below,
+// which every GPU that loads this library holds until the process exits.
 namespace qlora {
 namespace {
 
@@ -501,10 +714,28 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBy
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxScratchDevices] = {};
+CUcontext g_scratch_ctx[kMaxScratchDevices] = {};
+
+// The driver's cuCtxGetCurrent, to notice a new context on a device (after a device reset
+// the array lives at a new address).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 
 // Device address of g_decode_scratch on the current device. In host code the name
-// g_decode_scratch is only a host-side stand-in, so the address is looked up once
-// per device with that device current, and cached.
+// g_decode_scratch is only a host-side stand-in, so the address is looked up with the
+// device current, once per device and context, and cached.
 qlora_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -513,21 +744,21 @@ qlora_status scratch_address(void** out) {
     set_last_error("device index out of range for the static scratch table");
     return QLORA_ERR_INVALID_ARG;
   }
+  CUcontext ctx = nullptr;
+  if (auto fn = ctx_get_current()) fn(&ctx);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return cuda_status(e);
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_addr[dev];
   return QLORA_OK;
 }
 
-bool aligned16_ptr(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
-
 }  // namespace qlora
 
 extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_t M,
@@ -535,51 +766,38 @@ extern "C" qlora_status qlora_linear_fwd_decode_static(const uint16_t* X, int64_
                                                        const uint16_t* B, int r, float scale,
                                                        uint16_t* Y, float* T_save, void* stream) {
   using namespace qlora;
-  if (!w.codes || !w.c2 || !w.c1 || !w.mean) return QLORA_ERR_INVALID_ARG;
-  if (w.codebook < 0 || w.codebook >= kCodebooks) return QLORA_ERR_INVALID_ARG;
-  if (w.n_out < 1 || w.k_in < 64 || w.k_in % 64 != 0 || w.n_out % 8 != 0 ||
-      w.n_out > (int64_t{1} << 31) || w.k_in > (int64_t{1} << 31))
-    return QLORA_ERR_SHAPE;
-  if (M < 0 || M > kDecodeMaxM) {
+  // the argument checks of qlora_linear_fwd, in the same order
+  qlora_status q = check_linear(M, w, r, scale);
+  if (q != QLORA_OK) return q;
+  if (M > kDecodeMaxM) {
     set_last_error("qlora_linear_fwd_decode_static serves 0 <= M <= 16 tokens");
     return QLORA_ERR_SHAPE;
   }
-  if (r < 8 || r > 64 || r % 8 != 0) return QLORA_ERR_INVALID_ARG;
-  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16_ptr(w.codes) || !aligned16_ptr(w.c2) || !aligned16_ptr(w.c1) ||
-      !aligned16_ptr(w.mean))
-    return QLORA_ERR_ALIGN;
   if (M == 0) return QLORA_OK;
   if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16_ptr(X) || !aligned16_ptr(A) || !aligned16_ptr(B) || !aligned16_ptr(Y) ||
-      (T_save && !aligned16_ptr(T_save)))
+  if (!is_aligned16(X) || !is_aligned16(A) || !is_aligned16(B) || !is_aligned16(Y) ||
+      (T_save && !is_aligned16(T_save)))
     return QLORA_ERR_ALIGN;
-
   const LinearShape s{M, w.n_out, w.k_in, r, scale};
-  DecodePlan p = plan_decode(s);
-  // Fewer K splits when the planned partial sums do not fit the static array.
-  const size_t per_split = static_cast<size_t>(p.row_groups) * M * rows_per_warp(M > 8) * 4;
-  const size_t fixed = t_bytes(s) + counter_bytes(p) + 512;
-  const size_t fit = fixed < kStaticScratchBytes ? (kStaticScratchBytes - fixed) / per_split : 0;
-  if (fit < 1) {
+  const DecodePlan p = plan_decode(s, kStaticScratchBytes);
+  if (p.splits == 0) {
     char msg[200];
     std::snprintf(msg, sizeof(msg),
-                  "qlora_linear_fwd_decode_static: needs more than %zu bytes of partial sums; "
-                  "the static scratch holds %zu bytes",
-                  per_split + fixed, kStaticScratchBytes);
+                  "qlora_linear_fwd_decode_static: the partial sums of %lld x %lld at M = %lld "
+                  "need more than the %zu bytes of the static scratch",
+                  static_cast<long long>(w.n_out), static_cast<long long>(w.k_in),
+                  static_cast<long long>(M), kStaticScratchBytes);
     set_last_error(msg);
     return QLORA_ERR_WORKSPACE;
   }
-  if (static_cast<size_t>(p.splits) > fit) {
-    p.units_per = static_cast<int>((p.nunits + fit - 1) / fit);
-    p.splits = (p.nunits + p.units_per - 1) / p.units_per;
-  }
-  void* scratch = nullptr;
-  qlora_status q = scratch_address(&scratch);
+  q = check_device();
   if (q != QLORA_OK) return q;
-  // Every partial sum is written by the GEMV before it is read, and the T kernel clears
-  // the arrival counters, so nothing left in the array by an earlier call matters.
+  void* scratch = nullptr;
+  q = scratch_address(&scratch);
+  if (q != QLORA_OK) return q;
+  // Every partial sum is written before it is read, and the set-up kernel of the call
+  // clears T and the arrival counters, so nothing an earlier call left in the array
+  // matters.
   return launch_decode(X, w, A, B, s, p, Y, T_save, static_cast<char*>(scratch),
                        static_cast<cudaStream_t>(stream));
 }
-

@@ -43,6 +43,12 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                   uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
                   uint32_t box_outer, CUtensorMapSwizzle swizzle);
 int* device_error_word();                          // per-device error flag of the kernels
+bool is_aligned16(const void* p);
+// QLORA_ERR_DEVICE unless the current device is sm_100 class (QLORA_ERR_CUDA if it cannot
+// be queried)
+qlora_status check_device();
+// The argument checks shared by the linear entry points (weight, M, N % 8, r, scale).
+qlora_status check_linear(int64_t M, const qlora_nf4_weight& w, int r, float scale);
 // CUDA events (or NULL) this thread asked to have recorded around each launch of the
 // fused NF4 GEMM kernel (qlora_profile_events).
 void profile_events(cudaEvent_t* before, cudaEvent_t* after);
@@ -71,6 +77,8 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
 
 // ---- launchers (decode.cu) ------------------------------------------------------
 constexpr int64_t kDecodeMaxM = 16;
+// Workspace of the decode kernels, or 0 when they cannot run the shape (the fused GEMM
+// then serves it).
 size_t decode_workspace(const LinearShape& s);
 qlora_status decode_forward(const uint16_t* X, const qlora_nf4_weight& w, const uint16_t* A,
                             const uint16_t* B, const LinearShape& s, uint16_t* Y,

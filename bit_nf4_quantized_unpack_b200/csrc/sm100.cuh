@@ -19,6 +19,7 @@ enum DeviceError : int {
   kErrTimeoutDequant = 3,
   kErrTimeoutEpilogue = 4,
   kErrTimeoutSelfTest = 5,  // the wait of qlora_selftest_wait_timeout
+  kErrTimeoutDecode = 6,    // a decode finisher waiting for T = X A
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

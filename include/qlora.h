@@ -19,9 +19,12 @@
  *    Y is M x N, A is K x r, B is r x N.
  *  - bf16 data is passed as uint16_t bit patterns.
  *  - Every pointer argument named "device" is CUDA device memory owned by the
- *    caller; the library never allocates, frees or keeps device memory. Scratch
- *    space comes from the caller through (workspace, workspace_bytes); the
- *    matching *_workspace_size query says how much.
+ *    caller. The library allocates, frees and keeps no device memory, with two
+ *    exceptions declared below: the fixed static scratch array of
+ *    qlora_linear_fwd_decode_static, and qlora_paged_alloc, which exists to allocate
+ *    unified memory for optimizer states. Other scratch space comes from the caller
+ *    through (workspace, workspace_bytes); the matching *_workspace_size query says
+ *    how much.
  *  - Device pointers must be 16-byte aligned (QLORA_ERR_ALIGN otherwise).
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
  *    and runs asynchronously. Argument errors are detected on the host before
@@ -171,14 +174,19 @@ size_t qlora_quantize_workspace_size(int64_t n_out, int64_t k_in);
  * Steps (itwiki "QLoRA", NF4 and double-quantization sections):
  *   1. per 64-block absmax a_j = max |w|; x = fl32(w / a_j) (x = 0 when a_j = 0);
  *      code = nearest NF4 level (ties to the lower index); two codes per byte.
- *   2. mean = fl32(sum_j a_j / (N*K/64)) summed in fp64.
+ *   2. mean = the arithmetic mean of all a_j, formed exactly (integer sums of the
+ *      significands per exponent, so it does not depend on the summation order or
+ *      the range of the constants) and rounded once to fp32, to nearest, ties to even.
  *   3. per 256-block of centred constants cc_j = fl32(a_j - mean):
  *      c1 = max |cc|; y = fl32(cc_j / c1) (0 when c1 = 0); c2_j = E4M3 bit pattern
  *      of the nearest T8 entry (ties to the lower index).
  * Outputs (device): codes [N*K/2], c2 [N*K/64], c1 [ceil(N*K/16384)], mean [1].
  * Workspace: at least qlora_quantize_workspace_size(n_out, k_in) bytes (device).
- * Errors: QLORA_ERR_SHAPE unless n_out >= 1, k_in >= 64 and k_in % 64 == 0;
+ * Errors: QLORA_ERR_SHAPE unless n_out >= 1, k_in >= 64, k_in % 64 == 0 and
+ *         n_out * k_in <= 2^37 (at most 2^31 blocks);
  *         QLORA_ERR_INVALID_ARG for a NULL pointer or unknown dtype.
+ * The workspace also holds the 256 integer sums of the mean; the call clears them
+ * with cudaMemsetAsync on `stream` before the kernels run.
  * Inputs must be finite.
  */
 qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, int64_t n_out,
@@ -237,7 +245,10 @@ size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t n_out, int64_t k_in, i
  *          the backward.
  * M >= 0 (M == 0 enqueues nothing and X, Y may be NULL); r in {8, 16, ..., 64}. M <= 16 runs the decode
  * (GEMV) kernels, larger M the fused tensor-core GEMM; both dequantize W in
- * registers without writing it to memory.
+ * registers without writing it to memory. The decode kernels add the partial products
+ * of T = X A with fp32 atomics, so T (and through it Y) may differ in the last bits from
+ * run to run; shapes they cannot run (a split's columns of X must fit 48 KB of shared
+ * memory, at most 148 splits) go to the fused GEMM.
  */
 qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, qlora_nf4_weight w,
                               const uint16_t *A, const uint16_t *B, int r, float scale,
@@ -253,16 +264,25 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, qlora_nf4_weight w,
  * counterpart of this entry point; it is a deployment convenience.
  *   Arguments, layouts and results are those of qlora_linear_fwd with M <= 16.
  *   Scratch: a fixed 4 MiB array in device memory inside this library, which every
- *   GPU that loads the library holds until the process exits. It must hold one
- *   K split of fp32 partial sums (M * 32 * ceil(N / 32) * 4 bytes), T (M * r * 4
- *   bytes) and one counter per 32 rows of W; larger problems are rejected
- *   with QLORA_ERR_WORKSPACE (qlora_last_error() gives the sizes), M > 16 with
- *   QLORA_ERR_SHAPE. When the usual number of K splits does not fit, fewer are used.
- *   The first call on each device looks up the array's device address (with that
- *   device current) and caches it; make that first call before any stream capture.
- *   Every call uses the same array and overwrites what it needs, so calls whose
- *   kernels overlap on the GPU (different streams, or different host threads on
- *   one device) race on it: issue them in order on one stream.
+ *   GPU that loads the library holds until the process exits. A call splits K into
+ *   s ranges and needs
+ *       align256(s * ceil(N / R) * R * M * 4) + align256(M * r * 4)
+ *       + align256(4 * ceil(N / R) + 4)  bytes,   R = 16 rows (M <= 8) or 32 (M > 8),
+ *   for fp32 partial sums, T and the arrival counters. It takes the number of splits
+ *   its planner prefers when that fits, else the best that fits. The fewest splits it can
+ *   run is ceil(ceil(K / 256) / u) with u = 85, 42, 28, 21, 17, 14, 12, 10, 9, 8, 7, 7,
+ *   6, 5, 5, 5 for M = 1 .. 16 (a split's columns of X are staged in 48 KB of shared
+ *   memory); when even that does not fit the array, the call is rejected with
+ *   QLORA_ERR_WORKSPACE (qlora_last_error() gives the shape), and M > 16 with
+ *   QLORA_ERR_SHAPE. Argument errors are checked as in qlora_linear_fwd and give its
+ *   status codes.
+ *   The first call on each device, and the first after that device's context changes
+ *   (a cudaDeviceReset, for instance), looks up the array's device address with the
+ *   device current and caches it; make that first call before any stream capture.
+ *   Every call uses the same array: the set-up kernel of each call clears what must
+ *   start at zero, and the partial sums are written before they are read. Calls whose
+ *   kernels overlap on the GPU (different streams, or different host threads on one
+ *   device) race on it: issue them in order on one stream.
  *   The function itself allocates nothing (no cudaMalloc, no cudaFree).
  */
 qlora_status qlora_linear_fwd_decode_static(const uint16_t *X, int64_t M, qlora_nf4_weight w,

@@ -36,7 +36,8 @@ Readings where the pages are silent (each pinned or flagged in the tests):
 * the 8-bit float of the double quantization is OCP FP8 E4M3; its code table T8 is
   the 253 distinct finite E4M3 values divided by 448, rounded to fp32; a constant's
   code is the E4M3 bit pattern of its nearest T8 entry.
-* one mean per tensor (the only reading that gives exactly 0.127 bits/param).
+* one mean per tensor (the only reading that gives exactly 0.127 bits/param): the
+  arithmetic mean of the block constants taken exactly and rounded once to fp32.
 * nearest-level ties go to the lower index (NumPy ``argmin`` takes the first).
 * the LoRA term carries the alpha/r scale of the minnong511 page; the itwiki
   equation omits it. A is K x r, B is r x N, so the LoRA product is X A B.
@@ -46,6 +47,7 @@ Readings where the pages are silent (each pinned or flagged in the tests):
 from __future__ import annotations
 
 import math
+from fractions import Fraction
 
 import numpy as np
 from scipy.stats import norm
@@ -204,11 +206,54 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
 # Level 2: double quantization of the absmax constants (itwiki "QLoRA", DQ)
 # ---------------------------------------------------------------------------
 
+def f32_round(x: Fraction) -> np.float32:
+    """The fp32 value nearest to the non-negative rational x (IEEE round to nearest,
+    ties to even), for x below the largest finite fp32. Written from the definition:
+    find the binade [2^E, 2^(E+1)) holding x (E >= -126, since subnormals share the
+    spacing of the smallest normal binade), count x in units of that binade's spacing
+    2^(E-23), and round the count to an integer."""
+    x = Fraction(x)
+    if x < 0:
+        raise ValueError("f32_round takes non-negative values")
+    if x == 0:
+        return np.float32(0.0)
+    E = x.numerator.bit_length() - x.denominator.bit_length()
+    while Fraction(2) ** E > x:
+        E -= 1
+    while Fraction(2) ** (E + 1) <= x:
+        E += 1
+    E = max(E, -126)
+    ulp = Fraction(2) ** (E - 23)
+    units = x / ulp
+    n = units.numerator // units.denominator
+    rest = units - n
+    if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return np.float32(float(n * ulp))   # n <= 2^24: an fp32 value, converted exactly
+
+
+def exact_sum_f32(values: np.ndarray) -> Fraction:
+    """The exact sum of fp32 values >= 0, as a rational. Each value is sig * 2^(e - 150)
+    with sig its 24-bit significand and e its biased exponent (1 for subnormals); the
+    significands of each exponent are summed as integers (exactly), then combined."""
+    u = np.asarray(values, np.float32).ravel().view(np.uint32)
+    if np.any(u >> 31) or np.any(((u >> 23) & 0xFF) == 0xFF):
+        raise ValueError("exact_sum_f32 takes finite values >= 0")
+    e = (u >> 23) & 0xFF
+    sig = (u & 0x7FFFFF) | np.where(e > 0, 0x800000, 0).astype(np.uint32)
+    e = np.maximum(e, 1)
+    total = 0
+    for ev in np.unique(e[sig > 0]):
+        total += int(sig[e == ev].astype(np.int64).sum()) << int(ev)
+    return Fraction(total, 1 << 150)
+
+
 def constants_mean(absmax: np.ndarray) -> np.float32:
-    """One mean per tensor: the fp64 sum of all block constants over their count,
-    rounded once to fp32."""
-    a = np.asarray(absmax, np.float32).astype(np.float64)
-    return np.float32(np.sum(a) / a.size)
+    """One mean per tensor: the arithmetic mean of all block constants, taken exactly
+    (exact sum over their count) and rounded once to fp32. It does not depend on the
+    order of the constants, whatever their range."""
+    a = np.asarray(absmax, np.float32).ravel()
+    return f32_round(exact_sum_f32(a) / a.size)
 
 
 def double_quantize(absmax: np.ndarray, dq_block: int = DQ_BLOCK):

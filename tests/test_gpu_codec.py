@@ -51,6 +51,37 @@ def test_ragged_and_small_shapes(shape):
     compare_full(W, bf16=True)
 
 
+def test_mean_exact_for_wide_range_constants():
+    """Block absmax values from 2^-60 to 2^10 (fp32 input): the fp64 sum of such constants
+    is not exact and depends on its order, but the mean is defined as the exact
+    arithmetic mean rounded once to fp32, so the GPU must match the oracle bit for bit
+    (and the constants and codes with it). Also a tensor of 2^17 blocks with a few tiny
+    blocks among normal ones, and a subnormal block."""
+    rng = np.random.default_rng(33)
+    n_rows, k = 512, 1024                     # 8192 blocks
+    W = rng.normal(0, 1, (n_rows, k)).astype(np.float32)
+    scale = 2.0 ** rng.integers(-60, 11, n_rows * k // 64)
+    W = (W.reshape(-1, 64) * scale[:, None]).astype(np.float32).reshape(n_rows, k)
+    W[7, 64:128] = np.float32(2.0 ** -140)    # a block of subnormals
+    W[9, :64] = 0.0
+    q, ref = compare_full(W, bf16=False)
+    a64 = ref["absmax"].astype(np.float64)
+    assert len({float(np.cumsum(a64[rng.permutation(a64.size)])[-1]) for _ in range(6)}) > 1
+
+    g = np.random.default_rng(34)
+    W2 = g.normal(0, 0.02, (512, 16384)).astype(np.float32)
+    W2[::67, ::4096] *= np.float32(2.0 ** -40)
+    q2 = quantize_on_gpu(W2, bf16=False)
+    codes, absmax = O.quantize_blocks(W2[:8], O.nf4_levels())   # codes on sampled rows
+    full_absmax = np.max(np.abs(W2.reshape(-1, 64)), axis=1)
+    c2, c1, mean = O.double_quantize(full_absmax)
+    assert q2.mean.cpu().numpy().view(np.uint32)[0] == np.float32(mean).view(np.uint32)
+    assert np.array_equal(q2.c2.cpu().numpy(), c2)
+    assert np.array_equal(q2.c1.cpu().numpy().view(np.uint32), c1.view(np.uint32))
+    got_codes = q2.codes.cpu().numpy()[: 8 * 16384 // 2]
+    assert np.array_equal(got_codes, O.pack_nibbles(codes))
+
+
 def test_edge_values():
     rng = np.random.default_rng(21)
     W = rng.normal(0, 0.02, (40, 640)).astype(np.float32)

@@ -182,6 +182,54 @@ def test_dq_block_max_maps_to_unit_code_and_mean_is_global():
     assert np.max(np.abs(s - absmax)) < np.max(c1) / 8
 
 
+def test_f32_round_matches_correctly_rounded_conversion():
+    """Rational -> fp32 rounding against numpy's fp64 -> fp32 conversion (one correct
+    rounding from an exact fp64 value), over normals, subnormals and exact ties."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    d = np.concatenate([
+        rng.uniform(0, 1, 3000) * 2.0 ** rng.integers(-149, 120, 3000),
+        rng.uniform(0, 2.0 ** -126, 500),                       # subnormal range
+    ])
+    f = np.float32(rng.uniform(1, 2, 500)) * np.float32(2.0) ** rng.integers(-140, 100, 500)
+    ties = f.astype(np.float64) + np.spacing(f).astype(np.float64) / 2  # exact fp32 midpoints
+    for v in np.concatenate([d, ties, [0.0, 2.0 ** -149, 2.0 ** -150, 3 * 2.0 ** -151]]):
+        assert O.f32_round(Fraction(float(v))) == np.float32(v), v
+    # a value just above an fp32 midpoint whose fp64 rounding lands on the midpoint:
+    # two roundings go down (to even), one correct rounding goes up
+    m = np.float32(1.0)
+    x = Fraction(1) + Fraction(1, 2 ** 24) + Fraction(1, 2 ** 60)
+    assert np.float32(float(x)) == m
+    assert O.f32_round(x) == np.nextafter(m, np.float32(2))
+
+
+def test_exact_sum_and_mean_are_exact_and_order_free():
+    """The mean of the block constants is their exact arithmetic mean rounded once,
+    whatever their range: brute force with Fractions, and invariance under reordering
+    where an fp64 running sum is not."""
+    from fractions import Fraction
+    rng = np.random.default_rng(9)
+    a = (rng.uniform(1, 2, 4000) * 2.0 ** rng.integers(-60, 11, 4000)).astype(np.float32)
+    a[::97] = 0.0
+    a[5] = np.float32(2.0 ** -149)            # smallest subnormal
+    a[6] = np.float32(1.5 * 2.0 ** -130)      # subnormal
+    brute = sum((Fraction(float(v)) for v in a), Fraction(0))
+    assert O.exact_sum_f32(a) == brute
+    mean = O.constants_mean(a)
+    assert mean == O.f32_round(brute / a.size)
+    perm = rng.permutation(a.size)
+    assert O.constants_mean(a[perm]) == mean
+    # an fp64 running sum is order-dependent on these data; the exact mean is not
+    sums = {float(np.cumsum(a[rng.permutation(a.size)].astype(np.float64))[-1]) for _ in range(8)}
+    assert len(sums) > 1
+    # equal constants: the mean is the constant itself
+    assert O.constants_mean(np.full(1000, np.float32(0.0371))) == np.float32(0.0371)
+    # narrow-range data, where the fp64 sum is exact and its rounding cannot tie, give
+    # the same mean as the fp64 formula
+    b = rng.uniform(0.03, 0.09, 5000).astype(np.float32)
+    assert O.constants_mean(b) == np.float32(np.sum(b.astype(np.float64)) / b.size)
+
+
 def test_dq_codes_match_brute_force_over_t8():
     rng = np.random.default_rng(2)
     absmax = rng.uniform(0.02, 0.2, 600).astype(np.float32)

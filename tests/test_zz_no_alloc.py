@@ -50,12 +50,13 @@ def test_static_scratch_decode_matches_workspace_path(M, N, K, r):
 
 
 def test_static_scratch_with_fewer_k_splits():
-    """N = 16384 at M = 16: the planned K splits of fp32 partial sums do not all fit
-    the 4 MiB array, so the entry point uses fewer; results must not change."""
+    """M = 8 tokens on a 16384 x 16384 weight: the usual plan's fp32 partial sums (8 K
+    splits) do not fit the 4 MiB array, so the entry point plans with 7; the results
+    must not change."""
     need_gpu()
     g = torch.Generator(device="cuda")
     g.manual_seed(7)
-    M, N, K, r, scale = 16, 16384, 8192, 16, 2.0
+    M, N, K, r, scale = 8, 16384, 16384, 16, 2.0
     q = qlora.qlora_quantize_nf4_dq((torch.randn(N, K, generator=g, device="cuda") * 0.02)
                                     .to(torch.bfloat16))
     X = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
@@ -67,6 +68,7 @@ def test_static_scratch_with_fewer_k_splits():
         T = torch.full_like(T_ref, float("nan"))
         _static_fwd(X, q, A, B, r, scale, Y, T)
         torch.cuda.synchronize()
+        assert qlora.qlora_device_error() == 0
         assert_close(host(Y), host(Y_ref), bf16_out=True, what="Y")
         assert_close(host(T), host(T_ref), what="T")
 
@@ -87,3 +89,35 @@ def test_static_scratch_rejects_oversize_and_large_m():
     big = list(args)
     big[1] = 17
     assert L.qlora_linear_fwd_decode_static(*big) == 2           # QLORA_ERR_SHAPE
+
+
+def test_static_scratch_argument_errors_match_workspace_path():
+    """r, scale and alignment errors come back before anything is enqueued, with the
+    status qlora_linear_fwd gives for the same arguments."""
+    need_gpu()
+    M, N, K = 4, 256, 1024
+    q = qlora.NF4Weight.empty(N, K)
+    X = torch.zeros(M, K, dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros(K, 64, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(64, N, dtype=torch.bfloat16, device="cuda")
+    Y = torch.zeros(M * N + 8, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(qlora.qlora_linear_fwd_workspace_size(M, N, K, 16), dtype=torch.uint8,
+                     device="cuda")
+    L = qlora.lib()
+
+    def both(r, scale, y_ptr):
+        common = (ctypes.c_void_p(X.data_ptr()), M, q.c_struct(), ctypes.c_void_p(A.data_ptr()),
+                  ctypes.c_void_p(B.data_ptr()), r, ctypes.c_float(scale), ctypes.c_void_p(y_ptr),
+                  None)
+        st = L.qlora_linear_fwd_decode_static(*common, None)
+        ref = L.qlora_linear_fwd(*common, ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
+        return st, ref
+
+    y = Y.data_ptr()
+    for r, scale, y_ptr, want in [(4, 1.0, y, 1), (12, 1.0, y, 1), (16, float("nan"), y, 1),
+                                  (16, float("inf"), y, 1), (16, 1.0, y + 2, 3)]:
+        st, ref = both(r, scale, y_ptr)
+        assert st == ref == want, (r, scale, y_ptr - y, st, ref)
+    torch.cuda.synchronize()
+    assert qlora.qlora_device_error() == 0
+
