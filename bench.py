@@ -550,7 +550,8 @@ def stack_65b(device, warmup, steps, layers=80, M=8192, r=RANK_R, alpha=ALPHA):
     double-quantized constants resident at once (about 33 GB for 80 layers), LoRA r on each;
     one step is the forward and backward (dX, dA, dB) of every linear at M tokens. Inputs
     and upstream gradients are synthetic and shared by the layers (one buffer per shape);
-    every linear has its own weight, adapter and gradient buffers. Prints one JSON line."""
+    every linear has its own weight, adapter and gradient buffers. Returns the record (with
+    the clocks seen during its timed steps); frees its buffers."""
     from bit_nf4_quantized_unpack_b200 import inputs, qlora
     g = torch.Generator(device=device)
     g.manual_seed(4)
@@ -598,20 +599,28 @@ def stack_65b(device, warmup, steps, layers=80, M=8192, r=RANK_R, alpha=ALPHA):
     torch.cuda.synchronize()
     if qlora.qlora_device_error() != 0:
         raise RuntimeError("a kernel reported a timed-out wait")
+    clocks = ClockSampler(device)
+    clocks.start()
+    clocks.mark()
     launches0 = qlora.qlora_launch_count()
     ms = time_steps(step, steps, 1)
     launches = qlora.qlora_launch_count() - launches0
+    clk = clocks.stop()
     flops = layers * layer_flops(inputs.LLAMA65B_LINEARS, M, r)
-    print(json.dumps({"metric": "QLoRA 65B-shaped stack fwd+bwd TFLOP/s (M=8192)",
-                      "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
-                      "steps": steps, "warmup": warmup, "ms_per_step": ms,
-                      "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-                      "config": {"workload": f"{layers} layers x (q,k,v,o 8192x8192, gate/up "
-                                             f"8192->22016, down 22016->8192), NF4-DQ, LoRA "
-                                             f"r={r} alpha={alpha}; M={M} tokens",
-                                 "packed_weight_bytes": packed, "flops_per_step": flops,
-                                 "peak_mem_gb": torch.cuda.max_memory_allocated() / 1e9},
-                      "gpu_launches": launches}), flush=True)
+    rec = {"metric": "QLoRA 65B-shaped stack fwd+bwd TFLOP/s (M=8192)",
+           "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
+           "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"{layers} layers x (q,k,v,o 8192x8192, gate/up "
+                                  f"8192->22016, down 22016->8192), NF4-DQ, LoRA "
+                                  f"r={r} alpha={alpha}; M={M} tokens",
+                      "packed_weight_bytes": packed, "flops_per_step": flops,
+                      "peak_mem_gb": torch.cuda.max_memory_allocated() / 1e9,
+                      "l2": "inputs larger than L2 (33 GB of weights per step)"},
+           "gpu_launches": launches, "clocks": clk}
+    del lins, xs, dys, ys, dxs, wf, wb
+    torch.cuda.empty_cache()
+    return rec
 
 
 def profile_linear(device, scale, warmup, steps):
@@ -701,11 +710,18 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stack-65b", action="store_true",
+                    help="leave the 65B-shaped stack (1 warm-up + 2 steps) out of the default run")
     ap.add_argument("--decode-m", type=int, default=1,
                     help="tokens of the --profile-decode forward (1..16)")
+    ap.add_argument("--decode-n", type=int, default=8192,
+                    help="weight rows (out) of the --profile-decode forward")
+    ap.add_argument("--decode-k", type=int, default=28672,
+                    help="weight columns (in) of the --profile-decode forward")
     ap.add_argument("--profile-decode", action="store_true",
-                    help="only run the M=1 forward of an 8192x28672 weight --steps times "
-                         "(no graph): a small, self-contained case for profiler captures")
+                    help="only run the M-token forward of one n x k weight (8192x28672 unless "
+                         "--decode-n/-k say otherwise) --steps times (no graph): a small, "
+                         "self-contained case for profiler captures")
     ap.add_argument("--profile-dequant", action="store_true",
                     help="only run the double dequantization of a 4096x11008 weight (for ncu)")
     ap.add_argument("--profile-optimizer", action="store_true",
@@ -746,13 +762,14 @@ def main():
         profile_dequant(device, args.warmup, args.steps)
         return
     if args.stack_65b:
-        stack_65b(device, args.warmup, args.steps)
+        print(json.dumps(stack_65b(device, args.warmup, args.steps)), flush=True)
         return
     if args.profile_linear:
         profile_linear(device, scale, args.warmup, args.steps)
         return
     if args.profile_decode:
-        profile_decode(device, args.warmup, args.steps, M=args.decode_m)
+        profile_decode(device, args.warmup, args.steps, n=args.decode_n, k=args.decode_k,
+                       M=args.decode_m)
         return
     L = build_layer(device, seed=3 + 1000 * rank)
     flops = layer_flops(inputs.LLAMA7B_LINEARS, M_TOKENS, RANK_R)
@@ -793,13 +810,16 @@ def main():
     peaks, peaks_src = load_peaks()
     achieved = fused_flops / (fused_ms / 1e3) / 1e12
     # DRAM bytes per FLOP of the fused kernel from its ncu capture (gate linear, forward and
-    # dX; profiles/k_fused_nf4_gemm_gate_11008x4096_m4096.md), scaled to this step's
-    # average launch
+    # dX), scaled to this step's average launch
     traffic = FUSED_DRAM_BYTES_PER_FLOP * fused_flops / len(events)
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    # each launch is timed alone between its events, so the burst peak is the denominator;
+    # the sustained one is given beside it
+    peak = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", peak))
     roofline = {"bound": "tensor", "kernel": "k_fused_nf4_gemm (forward + dX)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{peaks_src} bf16_tflops_sustained",
+                "peak_source": f"{peaks_src} bf16_tflops (burst)",
+                "peak_sustained": sustained, "frac_of_sustained": achieved / sustained,
                 "fused_share_of_step": fused_ms / args.steps / ms, "traffic": traffic,
                 "traffic_unit": "bytes per launch (scaled from the ncu capture)"}
 
@@ -835,6 +855,10 @@ def main():
             if isinstance(v, dict):
                 v["frac_of_hbm"] = v["GBps"] / hbm
 
+    stack = None
+    if rank == 0 and world == 1 and not args.no_stack_65b:
+        stack = stack_65b(device, 1, 2)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, secs, desc = oracle_sample()
@@ -853,7 +877,8 @@ def main():
                            "l2": "inputs larger than L2 (weights + activations ~1.3 GB per step)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches,
-                "clocks": clk, "decode": decode, "codec": codec, "optimizer": optim}
+                "clocks": clk, "decode": decode, "codec": codec, "optimizer": optim,
+                "stack_65b": stack}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

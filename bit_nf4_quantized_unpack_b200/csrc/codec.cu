@@ -71,14 +71,91 @@ __device__ __forceinline__ float absmax3(float a, float b, float c) {
   return d;
 }
 
+// fl32(S / n) (round to nearest, ties to even) for S = sum_e bins[e] * 2^(e - 150), the
+// exact sum of the block constants, and n >= 1 of them (n < 2^32). One thread; exact
+// integer arithmetic on 32-bit digits `d` (14 of them, caller's scratch): the 256 bins
+// give A = S * 2^150 (< 2^311); the quotient q = floor(A * 2^64 / n) then holds S / n as
+// q * 2^-214 to at least 33 significant bits, and the bits of q below the kept 24 (or
+// below 2^-149 for a subnormal result) with the remainder decide the rounding.
+__device__ float exact_mean_f32(const unsigned long long* bins, int64_t n, uint32_t* d) {
+  constexpr int kD = 14;
+  for (int i = 0; i < kD; ++i) d[i] = 0u;
+  for (int e = 1; e < 256; ++e) {
+    const unsigned long long v = bins[e];
+    if (!v) continue;
+    // add v * 2^(e + 64): three digits from (e + 64) / 32 on, then the carry
+    const int w = (e + 64) >> 5, sh = (e + 64) & 31;
+    const uint64_t p0 = (v << sh) & 0xFFFFFFFFull;
+    const uint64_t p1 = (v >> (32 - sh)) & 0xFFFFFFFFull;
+    const uint64_t p2 = sh ? (v >> (64 - sh)) : 0ull;
+    uint64_t t = static_cast<uint64_t>(d[w]) + p0;
+    d[w] = static_cast<uint32_t>(t);
+    t = static_cast<uint64_t>(d[w + 1]) + p1 + (t >> 32);
+    d[w + 1] = static_cast<uint32_t>(t);
+    t = static_cast<uint64_t>(d[w + 2]) + p2 + (t >> 32);
+    d[w + 2] = static_cast<uint32_t>(t);
+    for (int k = w + 3; (t >> 32) && k < kD; ++k) {
+      t = static_cast<uint64_t>(d[k]) + (t >> 32);
+      d[k] = static_cast<uint32_t>(t);
+    }
+  }
+  const uint64_t nn = static_cast<uint64_t>(n);
+  uint64_t rem = 0;
+  for (int k = kD - 1; k >= 0; --k) {  // q = d / n, from the most significant digit
+    const uint64_t cur = (rem << 32) | d[k];
+    d[k] = static_cast<uint32_t>(cur / nn);
+    rem = cur % nn;
+  }
+  int top = -1;  // most significant set bit of q
+  for (int k = kD - 1; k >= 0 && top < 0; --k)
+    if (d[k]) top = 32 * k + 31 - __clz(d[k]);
+  if (top < 0) return 0.f;
+  auto nonzero_below = [&](int nbits) -> bool {  // any of q's bits 0 .. nbits - 1
+    for (int k = 0; 32 * k < nbits; ++k) {
+      const int nb = min(32, nbits - 32 * k);
+      if (d[k] & (nb == 32 ? 0xFFFFFFFFu : ((1u << nb) - 1u))) return true;
+    }
+    return false;
+  };
+  if (top < 65) {  // below 2^-149: 0, or the smallest subnormal when above half of it
+    const bool above_half = top == 64 && (rem != 0 || nonzero_below(64));
+    return above_half ? __uint_as_float(1u) : 0.f;
+  }
+  // the 64-bit window of q whose top bit is bit `top` (bits top - 63 .. top)
+  auto window = [&](int hi_bit) -> uint64_t {  // bits hi_bit - 63 .. hi_bit
+    const int lo = hi_bit - 63;
+    const int k = lo >> 5, sh = lo & 31;  // lo may be negative: those bits are zero
+    auto dig = [&](int i) -> uint64_t { return (i >= 0 && i < kD) ? d[i] : 0u; };
+    const uint64_t x = dig(k) | (dig(k + 1) << 32), y = dig(k + 2);
+    return sh ? ((x >> sh) | (y << (64 - sh))) : x;
+  };
+  // fp32 keeps bits [lsb, top]: 24 bits, or down to 2^-149 (bit 65 of q)
+  const int lsb = max(top - 23, 65);
+  const int nkeep = top - lsb + 1;  // 1 .. 24
+  const uint64_t win = window(top);
+  uint32_t sig = static_cast<uint32_t>(win >> (64 - nkeep));
+  const uint32_t guard = static_cast<uint32_t>(win >> (63 - nkeep)) & 1u;
+  // sticky: the bits below the guard (q bits 0 .. lsb - 2) and the remainder
+  const uint32_t sticky = (rem != 0 || nonzero_below(lsb - 1)) ? 1u : 0u;
+  if (guard && (sticky || (sig & 1u))) ++sig;
+  if (lsb == 65) return __uint_as_float(sig);  // subnormal (sig == 2^23: smallest normal)
+  int ebits = top - 214 + 127;                   // biased exponent of the binade
+  if (sig == 0x1000000u) {                       // rounding carried into the next binade
+    sig >>= 1;
+    ++ebits;
+  }
+  return __uint_as_float((static_cast<uint32_t>(ebits) << 23) | (sig & 0x7FFFFFu));
+}
+
 // Level 1: one 64-block per group of kQuantLanes = 4 lanes (16 elements per lane). Writes
 // the packed codes and the fp32 absmax of each block, and adds every absmax, exactly, into
 // 256 integer bins (one per fp32 exponent) for the mean: absmax = sig * 2^(e - 150) with
 // sig its 24-bit significand and e its biased exponent (1 for subnormals), and bin e sums
 // the sig of its exponent as a 64-bit integer (at most 2^31 blocks of 2^24 each). The CTA
 // sums into shared bins, then adds its nonzero bins into the global ones (zeroed before
-// the launch). Integer sums do not depend on their order, so the mean is the same for
-// any schedule and any range of constants.
+// the launch); the last CTA to finish forms the mean from them. Integer sums do not
+// depend on their order, so the mean is the same for any schedule and any range of
+// constants.
 //
 // x = fl32(w / absmax) is computed with Markstein's correction step (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000 processor", IBM J.
@@ -95,7 +172,8 @@ template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
     k_quantize_blocks(const T* __restrict__ W, int64_t nblocks,
                       const __grid_constant__ Nf4BucketTable tab, uint8_t* __restrict__ codes,
-                      float* __restrict__ absmax, unsigned long long* __restrict__ bins) {
+                      float* __restrict__ absmax, unsigned long long* __restrict__ bins,
+                      float* __restrict__ mean_out) {
   const int lane = threadIdx.x & 31;
   const int sub = lane & (kQuantLanes - 1);
   const unsigned gmask = ((1u << kQuantLanes) - 1u) << (lane & (32 - kQuantLanes));
@@ -176,89 +254,36 @@ __global__ void __launch_bounds__(kQuantThreads)
   __syncthreads();
   for (int i = threadIdx.x; i < 256; i += blockDim.x)
     if (sbins[i]) atomicAdd(bins + i, sbins[i]);
-}
-
-// fl32(S / n) (round to nearest, ties to even) for S = sum_e bins[e] * 2^(e - 150), the
-// exact sum of the block constants, and n >= 1 of them. One thread; exact integer
-// arithmetic: the 256 bins give a 320-bit integer A = S * 2^150, the quotient
-// q = floor(A * 2^64 / n) (448 bits, 32-bit digits, remainder kept) then holds S / n as
-// q * 2^-214 to at least 33 significant bits, and its bits below the kept 24 (or below
-// 2^-149 for a subnormal result) decide the rounding.
-__device__ float exact_mean_f32(const unsigned long long* bins, int64_t n) {
-  constexpr int kD = 14;  // 32-bit digits of A * 2^64 (A < 2^311)
-  uint32_t d[kD];
-#pragma unroll 1
-  for (int i = 0; i < kD; ++i) d[i] = 0u;
-#pragma unroll 1
-  for (int e = 1; e < 256; ++e) {
-    const unsigned long long v = bins[e];
-    if (!v) continue;
-    // add v * 2^(e + 64): digits from (e + 64) / 32 on, shifted by (e + 64) % 32
-    const int w = (e + 64) >> 5, sh = (e + 64) & 31;
-    uint64_t carry = 0;
-    const uint64_t parts[3] = {(v << sh) & 0xFFFFFFFFull, (v >> (32 - sh)) & 0xFFFFFFFFull,
-                               sh ? (v >> (64 - sh)) : 0ull};
-    for (int k = w; k < kD; ++k) {
-      const uint64_t add = (k - w < 3) ? parts[k - w] : 0ull;
-      if (add == 0 && carry == 0 && k - w >= 3) break;
-      const uint64_t t = static_cast<uint64_t>(d[k]) + add + carry;
-      d[k] = static_cast<uint32_t>(t);
-      carry = t >> 32;
-    }
-  }
-  // q = d / n, long division from the most significant digit (n < 2^32)
-  const uint64_t nn = static_cast<uint64_t>(n);
-  uint64_t rem = 0;
-  for (int k = kD - 1; k >= 0; --k) {
-    const uint64_t cur = (rem << 32) | d[k];
-    d[k] = static_cast<uint32_t>(cur / nn);
-    rem = cur % nn;
-  }
-  int top = -1;  // index of the most significant set bit of q
-  for (int k = kD - 1; k >= 0 && top < 0; --k)
-    if (d[k]) top = 32 * k + 31 - __clz(d[k]);
-  if (top < 0) return 0.f;
-  auto bit = [&](int p) -> uint32_t { return p < 0 ? 0u : (d[p >> 5] >> (p & 31)) & 1u; };
-  // value = q * 2^-214; its binade 2^(top - 214); fp32 keeps 24 bits, and nothing below
-  // 2^-149 (bit 65 of q)
-  const int lsb = max(top - 23, 65);
-  uint32_t sig = 0;
-  for (int p = top; p >= lsb; --p) sig = (sig << 1) | bit(p);
-  const uint32_t guard = bit(lsb - 1);
-  uint32_t sticky = rem != 0 ? 1u : 0u;
-  for (int p = lsb - 2; p >= 0 && !sticky; --p) sticky |= bit(p);
-  if (guard && (sticky || (sig & 1u))) ++sig;
-  if (lsb == 65) return __uint_as_float(sig);  // subnormal (sig == 2^23: smallest normal)
-  int ebits = top - 214 + 127;                   // biased exponent of the binade
-  if (sig == 0x1000000u) {                       // rounding carried into the next binade
-    sig >>= 1;
-    ++ebits;
-  }
-  return __uint_as_float((static_cast<uint32_t>(ebits) << 23) | (sig & 0x7FFFFFu));
-}
-
-// Level 2: the one mean of all block constants, then one warp per 256-block of constants,
-// 8 constants per lane. Launched as the programmatic dependent of level 1: every CTA forms
-// the mean itself from level 1's exponent bins (exact sum, one rounding to fp32), and
-// CTA 0 stores it.
-// The E4M3 code of each y = fl32(cc / c1) comes from t8_nearest_codes2.
-__global__ void __launch_bounds__(256)
-    k_double_quantize(const float* __restrict__ absmax, int64_t nblocks,
-                      const unsigned long long* __restrict__ bins, float* __restrict__ mean_out,
-                      const T8Thresholds th, uint8_t* __restrict__ c2, float* __restrict__ c1) {
-  __shared__ float sth[kT8Size - 1];
-  __shared__ unsigned long long sbins[256];
-  __shared__ float mean_s;
-  for (int i = threadIdx.x; i < kT8Size - 1; i += blockDim.x) sth[i] = th.t[i];
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // level 1's absmax and bins
+  // the last CTA to add its bins forms the mean (the bins and the counter were zeroed
+  // before the launch)
+  __threadfence();
+  __syncthreads();
+  __shared__ int last;
+  if (threadIdx.x == 0) last = atomicAdd(reinterpret_cast<unsigned int*>(bins + 256), 1u) ==
+                               gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
   for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = __ldcg(bins + i);
   __syncthreads();
   if (threadIdx.x == 0) {
-    mean_s = exact_mean_f32(sbins, nblocks);
-    if (blockIdx.x == 0) mean_out[0] = mean_s;
+    __shared__ uint32_t digits[14];
+    mean_out[0] = exact_mean_f32(sbins, nblocks, digits);
   }
+}
+
+// Level 2: one warp per 256-block of constants, 8 constants per lane, centred on the
+// mean that level 1 formed. Launched as the programmatic dependent of level 1.
+// The E4M3 code of each y = fl32(cc / c1) comes from t8_nearest_codes2.
+__global__ void __launch_bounds__(256)
+    k_double_quantize(const float* __restrict__ absmax, int64_t nblocks,
+                      const float* __restrict__ mean_in, const T8Thresholds th,
+                      uint8_t* __restrict__ c2, float* __restrict__ c1) {
+  __shared__ float sth[kT8Size - 1];
+  for (int i = threadIdx.x; i < kT8Size - 1; i += blockDim.x) sth[i] = th.t[i];
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // level 1's absmax and mean
   __syncthreads();
-  const float mean = mean_s;
+  const float mean = __ldcg(mean_in);
   const int lane = threadIdx.x & 31;
   const int64_t ndq = (nblocks + 255) / 256;
   for (int64_t b = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; b < ndq;
@@ -301,7 +326,7 @@ __global__ void __launch_bounds__(256)
               uint4* __restrict__ out) {
   __shared__ float lut[16];
   __shared__ float t8[256];  // T8 by E4M3 code
-  if (threadIdx.x < 16) lut[threadIdx.x] = code_level<CB>(threadIdx.x);
+  if (threadIdx.x < 16) lut[threadIdx.x] = code_level_rt<CB>(threadIdx.x);
   for (int e = threadIdx.x; e < 256; e += blockDim.x) t8[e] = t8_value(e);
   __syncthreads();
   const float mean = *mean_p;
@@ -362,7 +387,7 @@ cudaError_t quant_ctas(int64_t nblocks, int* ctas) {
 
 size_t quantize_workspace_bytes(int64_t n, int64_t k) {
   const int64_t nblocks = n * k / 64;
-  return align_up(static_cast<size_t>(nblocks) * 4, 256) + 256 * sizeof(unsigned long long);
+  return align_up(static_cast<size_t>(nblocks) * 4, 256) + 257 * sizeof(unsigned long long);
 }
 
 cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, int codebook,
@@ -375,15 +400,17 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   int ctas = 0;
   cudaError_t e = w_bf16 ? quant_ctas<uint16_t>(nblocks, &ctas) : quant_ctas<float>(nblocks, &ctas);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(bins, 0, 256 * sizeof(unsigned long long), st);
+  e = cudaMemsetAsync(bins, 0, 257 * sizeof(unsigned long long), st);  // bins and CTA count
   if (e != cudaSuccess) return e;
   note_launches(2);  // blocks, then the mean and double quantization
   if (w_bf16)
     k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, bins);
+        static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, bins,
+        mean);
   else
     k_quantize_blocks<float><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, bins);
+        static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, bins,
+        mean);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t ndq = (nblocks + 255) / 256;
@@ -400,8 +427,7 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k_double_quantize, static_cast<const float*>(absmax), nblocks,
-                            static_cast<const unsigned long long*>(bins), mean, t8_thresholds(), c2,
-                            c1);
+                            static_cast<const float*>(mean), t8_thresholds(), c2, c1);
 }
 
 cudaError_t launch_dequant(const qlora_nf4_weight& w, uint16_t* out, cudaStream_t st) {

@@ -46,9 +46,19 @@ constexpr int kUnitK = 256;  // K covered by one warp step (4 lanes x 64)
 // (lane (g, t) reads 16 bytes of block t of token g) then spreads over all eight 16-byte
 // bank groups.
 constexpr int kXBlkStride = 144;
-constexpr int kXStageMax = 48 * 1024;
+constexpr int kXStageMax = 80 * 1024;
 constexpr uint32_t kPairTabBytes = 65536;
-constexpr uint32_t kDecSmemMax = 2 * kPairTabBytes + kXStageMax + 1024;
+// A T share stages up to kTChunkRows rows of A at a time.
+constexpr int kTChunkRows = 64;
+__host__ __device__ constexpr int a_chunk_bytes(int r) { return kTChunkRows * r * 2; }
+// Dynamic shared memory: the 64 KB pair table at a 64 KB-aligned address (up to 64 KB of
+// alignment slack below it), the X stage, T8 (1 KB) and the A chunk; the last three are
+// placed in the slack when they fit there, else above the table.
+__host__ __device__ constexpr uint32_t dec_smem_bytes(int xs_bytes, int r) {
+  return 2 * kPairTabBytes + static_cast<uint32_t>(xs_bytes) + 1024u +
+         static_cast<uint32_t>(a_chunk_bytes(r));
+}
+constexpr uint32_t kDecSmemMax = dec_smem_bytes(kXStageMax, 64);
 
 struct DecodeArgs {
   const uint8_t* codes;
@@ -105,6 +115,17 @@ __device__ __forceinline__ void sts_b128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ uint2 lds_b64x2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
 }
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
@@ -391,7 +412,19 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   }
   const int64_t sstride = static_cast<int64_t>(a.row_groups) * M * kRowsPerWarp;
   const float* p0 = a.part + static_cast<int64_t>(rg) * M * kRowsPerWarp + lane;
-  for (int s = 0; s < a.splits; ++s) {
+  // four splits per step (all their loads in flight), added in a fixed order
+  int s = 0;
+  for (; s + 4 <= a.splits; s += 4) {
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+      if (m < M) {
+        const float* q = p0 + s * sstride + m * kRowsPerWarp;
+        const float v0 = __ldcg(q), v1 = __ldcg(q + sstride);
+        const float v2 = __ldcg(q + 2 * sstride), v3 = __ldcg(q + 3 * sstride);
+        y[m] += (v0 + v1) + (v2 + v3);
+      }
+  }
+  for (; s < a.splits; ++s) {
 #pragma unroll
     for (int m = 0; m < 16; ++m)
       if (m < M) y[m] += __ldcg(p0 + s * sstride + m * kRowsPerWarp);
@@ -418,61 +451,75 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
 
 // ---------------------------------------------------------------- T = X A
 // The CTA's share of T: rows [k0, k1) of A (inside its split, so X comes from the stage).
-// Lane (jq, tg): columns 4 jq .. 4 jq + 3 of A, tokens tg, tg + tgn, ... (at most 8).
+// Rows of A are staged kTChunkRows at a time with asynchronous 16-byte copies (one
+// latency round per chunk). Lane (jq, kq): columns 4 jq .. 4 jq + 3 of A, row octets kq,
+// kq + kqn, ... of the chunk, every token; the kqn lanes of a column group then add
+// their sums with shuffles and lane kq = 0 adds them into T.
 __device__ __forceinline__ void decode_t_share(const uint16_t* __restrict__ A, float* T,
                                                float* T_save, int* t_count, int shares, int r,
                                                int M, int xs_tok, int64_t kbeg, int64_t k0,
-                                               int64_t k1, int lane, uint32_t xs) {
-  int jqn = 2;  // lanes per token: a power of two with 4 jqn >= r
+                                               int64_t k1, int lane, uint32_t xs, uint32_t as) {
+  int jqn = 2;  // lanes per row: a power of two with 4 jqn >= r
   while (jqn * 4 < r) jqn <<= 1;
-  const int tgn = 32 / jqn;  // token groups (>= 2)
-  const int jq = lane & (jqn - 1), tg = lane / jqn;
+  const int kqn = 32 / jqn;  // lanes along the rows (>= 2)
+  const int jq = lane & (jqn - 1), kq = lane / jqn;
   const int j0 = jq * 4;
   const bool jlive = j0 < r;  // r is a multiple of 8, so j0 + 3 < r as well
-  float acc[8][4];
+  float acc[16][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int m = 0; m < 16; ++m)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
-  if (jlive) {
-    for (int64_t k = k0; k < k1; k += 8) {  // k0, k1 are multiples of 8
-      float av[8][4];
+    for (int c = 0; c < 4; ++c) acc[m][c] = 0.f;
+  for (int64_t kc = k0; kc < k1; kc += kTChunkRows) {  // k0, k1 are multiples of 8
+    const int rows = static_cast<int>(lmin(kTChunkRows, k1 - kc));
+    const int pieces = rows * r / 8;  // 16-byte pieces of the chunk
+    for (int i = lane; i < pieces; i += 32) cp_async16(as + 16 * i, A + kc * r + 8 * i);
+    cp_async_wait_all();
+    __syncwarp();
+    if (jlive) {
+      for (int o = kq; o < rows / 8; o += kqn) {
+        float av[8][4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(A + (k + e) * r + j0));
-        av[e][0] = bf16_to_f32(v.x & 0xFFFFu);
-        av[e][1] = bf16_to_f32(v.x >> 16);
-        av[e][2] = bf16_to_f32(v.y & 0xFFFFu);
-        av[e][3] = bf16_to_f32(v.y >> 16);
-      }
-      const int64_t kk = k - kbeg;
-      const uint32_t xo = static_cast<uint32_t>((kk >> 6) * kXBlkStride + (kk & 63) * 2);
+        for (int e = 0; e < 8; ++e) {
+          const uint2 v = lds_b64x2(as + static_cast<uint32_t>(((8 * o + e) * r + j0) * 2));
+          av[e][0] = bf16_to_f32(v.x & 0xFFFFu);
+          av[e][1] = bf16_to_f32(v.x >> 16);
+          av[e][2] = bf16_to_f32(v.y & 0xFFFFu);
+          av[e][3] = bf16_to_f32(v.y >> 16);
+        }
+        const int64_t kk = kc + 8 * o - kbeg;
+        const uint32_t xo = static_cast<uint32_t>((kk >> 6) * kXBlkStride + (kk & 63) * 2);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int m = tg + i * tgn;
-        if (m < M) {
-          const uint4 xv = lds_b128(xs + static_cast<uint32_t>(m * xs_tok) + xo);
-          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        for (int m = 0; m < 16; ++m) {
+          if (m < M) {
+            const uint4 xv = lds_b128(xs + static_cast<uint32_t>(m * xs_tok) + xo);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float x = bf16_to_f32((e & 1) ? (xw[e >> 1] >> 16) : (xw[e >> 1] & 0xFFFFu));
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t xw = (e >> 1) == 0 ? xv.x : (e >> 1) == 1 ? xv.y : (e >> 1) == 2 ? xv.z : xv.w;
+              const float x = bf16_to_f32((e & 1) ? (xw >> 16) : (xw & 0xFFFFu));
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[i][c] = fmaf(x, av[e][c], acc[i][c]);
+              for (int c = 0; c < 4; ++c) acc[m][c] = fmaf(x, av[e][c], acc[m][c]);
+            }
           }
         }
       }
     }
+    __syncwarp();  // the chunk is read before the next one overwrites it
   }
-  // T was zeroed by k_decode_prep
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (jlive && k0 < k1) {
+  for (int off = jqn; off < 32; off <<= 1)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int m = tg + i * tgn;
+    for (int m = 0; m < 16; ++m)
       if (m < M)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) atomicAdd(T + m * r + j0 + c, acc[i][c]);
-    }
+        for (int c = 0; c < 4; ++c) acc[m][c] += __shfl_xor_sync(0xFFFFFFFFu, acc[m][c], off);
+  // T was zeroed by k_decode_prep
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (jlive && kq == 0 && k0 < k1) {
+#pragma unroll
+    for (int m = 0; m < 16; ++m)
+      if (m < M)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) atomicAdd(T + m * r + j0 + c, acc[m][c]);
   }
   __threadfence();
   __syncwarp();
@@ -491,11 +538,21 @@ __global__ void __launch_bounds__(dec_threads(kTall), 1) k_decode_gemv(const Dec
   extern __shared__ __align__(16) uint8_t dsm[];
   const uint32_t sbase = smem_u32(dsm);
   const uint32_t tab = (sbase + kPairTabBytes - 1) & ~(kPairTabBytes - 1);
-  // the X stage and T8 go below the table when they fit there, else above it
-  const uint32_t need = static_cast<uint32_t>(a.xs_bytes) + 1024u;
-  const uint32_t xs_off = (tab - sbase >= need) ? 0u : (tab - sbase) + kPairTabBytes;
+  // the X stage, T8 and the A chunk go below the table while they fit there, else above
+  uint32_t lo_used = 0, hi_used = (tab - sbase) + kPairTabBytes;
+  auto place = [&](uint32_t bytes) {
+    if (lo_used + bytes <= tab - sbase) {
+      lo_used += bytes;
+      return lo_used - bytes;
+    }
+    hi_used += bytes;
+    return hi_used - bytes;
+  };
+  const uint32_t xs_off = place(static_cast<uint32_t>(a.xs_bytes));
+  const uint32_t t8_off = place(1024u);
+  const uint32_t as_off = place(static_cast<uint32_t>(a_chunk_bytes(a.r)));
   const uint32_t xs = sbase + xs_off;
-  float* t8 = reinterpret_cast<float*>(dsm + xs_off + a.xs_bytes);
+  float* t8 = reinterpret_cast<float*>(dsm + t8_off);
   uint8_t* tabp = dsm + (tab - sbase);
   const int split = blockIdx.x % a.splits, cidx = blockIdx.x / a.splits;
   const int u0 = split * a.units_per;
@@ -505,19 +562,42 @@ __global__ void __launch_bounds__(dec_threads(kTall), 1) k_decode_gemv(const Dec
   const int nblk = static_cast<int>((kend - kbeg) / 64);  // K is a multiple of 64
   const int M = static_cast<int>(a.M);
 
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
-  // 256 entries x 16 copies; thread i writes entry i / 16, copy i % 16
-  for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
-    const int e = i >> 4, cp = i & 15;
-    *reinterpret_cast<float2*>(tabp + e * 256 + CB * 128 + cp * 8) =
-        make_float2(code_level<CB>(e & 15), code_level<CB>(e >> 4));
+  // X columns [kbeg, kend) of every token, 16 bytes per thread and step: the loads of
+  // four steps are issued before their stores
+  {
+    const int n16 = M * nblk * 8;
+    for (int i0 = threadIdx.x; i0 < n16; i0 += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) {
+          const int m = i / (nblk * 8), rem = i - m * (nblk * 8);
+          v[u] = __ldg(reinterpret_cast<const uint4*>(a.X + m * a.K + kbeg + rem * 8));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n16) {
+          const int m = i / (nblk * 8), rem = i - m * (nblk * 8);
+          sts_b128(xs + static_cast<uint32_t>(m * a.xs_tok + (rem >> 3) * kXBlkStride +
+                                               (rem & 7) * 16),
+                   v[u]);
+        }
+      }
+    }
   }
-  // X columns [kbeg, kend) of every token, 16 bytes per thread and step
-  for (int i = threadIdx.x; i < M * nblk * 8; i += blockDim.x) {
-    const int m = i / (nblk * 8), rem = i - m * (nblk * 8);
-    const int b = rem >> 3, c = rem & 7;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.X + m * a.K + kbeg + b * 64 + c * 8));
-    sts_b128(xs + static_cast<uint32_t>(m * a.xs_tok + b * kXBlkStride + c * 16), v);
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
+  // 256 entries x 16 copies; thread i writes entry i / 16, copy i % 16 (its low level
+  // index (i / 16) % 16 is the same at every step)
+  {
+    const float lo = code_level_rt<CB>((threadIdx.x >> 4) & 15);
+    for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
+      const int e = i >> 4, cp = i & 15;
+      *reinterpret_cast<float2*>(tabp + e * 256 + CB * 128 + cp * 8) =
+          make_float2(lo, code_level_rt<CB>(e >> 4));
+    }
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -528,7 +608,7 @@ __global__ void __launch_bounds__(dec_threads(kTall), 1) k_decode_gemv(const Dec
     const int64_t k0 = lmin(kend, kbeg + cidx * share);
     const int64_t k1 = lmin(kend, k0 + share);
     decode_t_share(a.A, a.T, a.T_save, a.t_count, a.splits * a.cps, a.r, M, a.xs_tok, kbeg, k0,
-                   k1, lane, xs);
+                   k1, lane, xs, sbase + as_off);
     return;
   }
   const uint32_t lane_bits =
@@ -666,7 +746,7 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.splits * p.cps));
   cfg.blockDim = dim3(dec_threads(s.M > 8));
-  cfg.dynamicSmemBytes = 2 * kPairTabBytes + static_cast<uint32_t>(a.xs_bytes) + 1024;
+  cfg.dynamicSmemBytes = dec_smem_bytes(a.xs_bytes, s.r);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -29,6 +29,17 @@ __device__ __forceinline__ float code_level(int i) {
 }
 __device__ __forceinline__ float nf4_level(int i) { return code_level<0>(i); }
 
+// code_level for an index only known at run time, through selects over the constant
+// levels (an indexed local array would live in local memory).
+template <int CB>
+__device__ __forceinline__ float code_level_rt(int i) {
+  float v = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if (i == j) v = code_level<CB>(j);
+  return v;
+}
+
 // Value of an OCP FP8 E4M3 bit pattern (exact in fp32).
 __device__ __forceinline__ float e4m3_value(uint32_t b) {
   const uint32_t e = (b >> 3) & 15u, m = b & 7u;

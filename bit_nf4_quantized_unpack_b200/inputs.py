@@ -72,3 +72,16 @@ def linear_case(seed, M, N, K, r, alpha, w_fp32=False, outlier_frac=0.0):
     X = normal(rng, (M, K), 1.0, bf16=True)
     dY = normal(rng, (M, N), 1.0, bf16=True)
     return dict(W=W, A=A, B=B, X=X, dY=dY, r=r, alpha=float(alpha), scale=alpha / r)
+
+
+def decode_case(N, K, r=16, alpha=32.0, seed=2):
+    """The decode workload on one weight: W [N, K] ~N(0, 0.02) bf16, A, B ~N(0, 0.02),
+    X [16, K] ~N(0, 1) bf16, drawn in that order; a decode step of M <= 16 tokens takes
+    the first M rows of X."""
+    rng = np.random.default_rng(seed)
+    W = weight(rng, N, K, bf16=True)
+    A = normal(rng, (K, r), 0.02, bf16=True)
+    B = normal(rng, (r, N), 0.02, bf16=True)
+    X = normal(rng, (16, K), 1.0, bf16=True)
+    return dict(W=W, A=A, B=B, X=X, r=r, alpha=float(alpha), scale=alpha / r)
+

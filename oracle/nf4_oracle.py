@@ -168,12 +168,19 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
 # Level 1: blockwise absmax + NF4 codes (itwiki "QLoRA", NF4 section)
 # ---------------------------------------------------------------------------
 
+def block_absmax(w: np.ndarray, block: int = BLOCK) -> np.ndarray:
+    """Absolute maximum of each block of ``block`` consecutive weights (row-major
+    flattening), fp32 [n / block]."""
+    w = np.asarray(w, np.float32).reshape(-1, block)
+    return np.max(np.abs(w), axis=1).astype(np.float32)
+
+
 def quantize_blocks(w: np.ndarray, levels: np.ndarray, block: int = BLOCK):
     """Flatten row-major into blocks of ``block`` weights, divide each block by its
     absolute maximum (fp32, IEEE division) and take the nearest level.
     Returns (codes uint8 [n], absmax fp32 [n / block])."""
     w = np.asarray(w, np.float32).reshape(-1, block)
-    absmax = np.max(np.abs(w), axis=1)
+    absmax = block_absmax(w, block)
     x = np.zeros_like(w)
     live = absmax > 0
     x[live] = w[live] / absmax[live, None]           # fp32 / fp32, correctly rounded

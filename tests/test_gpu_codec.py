@@ -82,6 +82,17 @@ def test_mean_exact_for_wide_range_constants():
     assert np.array_equal(got_codes, O.pack_nibbles(codes))
 
 
+def test_mean_rounding_edges():
+    """Means at the bottom of the fp32 range, where the exact mean is rounded to a
+    subnormal, to the smallest subnormal or to zero: the GPU's division of the exact sum
+    must round as the oracle does."""
+    for tiny, zeros in [(2.0 ** -149, 1), (2.0 ** -149, 2), (3 * 2.0 ** -149, 3), (2.0 ** -149, 3),
+                        (3 * 2.0 ** -149, 5), (2.0 ** -126, 7), (1.5 * 2.0 ** -140, 63)]:
+        W = np.zeros((1 + zeros, 64), np.float32)
+        W[0, 17] = np.float32(tiny)
+        compare_full(W, bf16=False)
+
+
 def test_edge_values():
     rng = np.random.default_rng(21)
     W = rng.normal(0, 0.02, (40, 640)).astype(np.float32)

@@ -7,7 +7,8 @@ device array inside the library instead of a caller workspace. This test calls i
 through the C ABI twice in a row and compares each result with the workspace-based
 entry point, qlora_linear_fwd, within the parity tolerance of the other tests; the
 second call also shows that what the first call left in the shared array does not
-leak into the next result. The file is named to be collected last.
+leak into the next result. Each result is also compared with the oracle on sampled rows
+of the weight. The file is named to be collected last.
 """
 import ctypes
 
@@ -16,7 +17,9 @@ import pytest
 import torch
 
 from bit_nf4_quantized_unpack_b200 import inputs, qlora
-from tests.gpu_util import assert_close, host, need_gpu, to_dev_bf16
+from oracle import nf4_oracle as O
+from tests.gpu_util import (assert_close, assert_weight_matches_oracle, host, need_gpu,
+                            oracle_sampled_weight, to_dev_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -47,6 +50,18 @@ def test_static_scratch_decode_matches_workspace_path(M, N, K, r):
         assert qlora.qlora_device_error() == 0
         assert_close(host(Y), host(Y_ref), bf16_out=True, what=f"Y (call {call})")
         assert_close(host(T), host(T_ref), what=f"T (call {call})")
+        # and directly against the oracle, on sampled rows of W
+        rows = np.unique(np.random.default_rng(M).choice(N, min(N, 48), replace=False))
+        q_ref, codes_rows, codes_cols = oracle_sampled_weight(case["W"], rows, [0])
+        assert_weight_matches_oracle(q, q_ref, rows, [0], codes_rows, codes_cols)
+        Xh = host(X2).astype(np.float64)
+        A64, B64 = (np.asarray(case[k], np.float64) for k in ("A", "B"))
+        T64 = Xh @ A64
+        Wr = O.double_dequant_rows(q_ref, rows).astype(np.float64)
+        Y64 = Xh @ Wr.T + case["scale"] * (T64 @ B64[:, rows])
+        assert_close(host(Y)[:, rows], O.bf16_round(Y64.astype(np.float32)), bf16_out=True,
+                     what=f"Y against the oracle (call {call})")
+        assert_close(host(T), T64, what=f"T against the oracle (call {call})")
 
 
 def test_static_scratch_with_fewer_k_splits():
