@@ -71,71 +71,116 @@ __device__ __forceinline__ float absmax3(float a, float b, float c) {
   return d;
 }
 
+// fl32(S / n), rounded once to nearest (ties to even), for S >= 0 exact in fp64 and
+// 1 <= n < 2^53. q = fl64(S / n) is within half an fp64 ulp of S / n, so the correctly
+// rounded fp32 is fl32(q) or a neighbour: only where S / n lies on the other side of
+// (or on) an fp32 midpoint m around q can they differ, and the sign of m n - S, exact
+// from one fused multiply-add (m has at most 25 significant bits), tells which.
+__device__ float round_div_f32(double S, int64_t n) {
+  const double dn = static_cast<double>(n);
+  const double q = S / dn;
+  float f = __double2float_rn(q);
+  const float up = __uint_as_float(__float_as_uint(f) + 1u);
+  const double m_hi = 0.5 * (static_cast<double>(f) + static_cast<double>(up));
+  const double d_hi = fma(m_hi, dn, -S);  // < 0: S / n above the midpoint
+  if (d_hi < 0.0 || (d_hi == 0.0 && (__float_as_uint(f) & 1u))) return up;
+  if (f > 0.f) {
+    const float dnv = __uint_as_float(__float_as_uint(f) - 1u);
+    const double m_lo = 0.5 * (static_cast<double>(dnv) + static_cast<double>(f));
+    const double d_lo = fma(m_lo, dn, -S);  // > 0: S / n below the midpoint
+    if (d_lo > 0.0 || (d_lo == 0.0 && (__float_as_uint(f) & 1u))) return dnv;
+  }
+  return f;
+}
+
 // fl32(S / n) (round to nearest, ties to even) for S = sum_e bins[e] * 2^(e - 150), the
-// exact sum of the block constants, and n >= 1 of them (n < 2^32). One thread; exact
-// integer arithmetic on 32-bit digits `d` (14 of them, caller's scratch): the 256 bins
-// give A = S * 2^150 (< 2^311); the quotient q = floor(A * 2^64 / n) then holds S / n as
-// q * 2^-214 to at least 33 significant bits, and the bits of q below the kept 24 (or
-// below 2^-149 for a subnormal result) with the remainder decide the rounding.
-__device__ float exact_mean_f32(const unsigned long long* bins, int64_t n, uint32_t* d) {
+// exact sum of the block constants, and n >= 1 of them (n < 2^32). Exact integer
+// arithmetic on 32-bit digits: A = S * 2^150 (< 2^311) scaled by 2^64 fills 14 digits;
+// the quotient q = floor(A * 2^64 / n) then holds S / n as q * 2^-214 to at least 33
+// significant bits, and the bits of q below the kept 24 (or below 2^-149 for a
+// subnormal result) with the remainder decide the rounding.
+// The CTA's threads add the bins into per-digit 64-bit sums (`acc`, 16 entries, zeroed
+// by the caller; bin e adds to three digits, and no digit sum can reach 2^41), then
+// thread 0 propagates the carries and divides; returns the mean in thread 0.
+__device__ float exact_mean_f32(const unsigned long long* bins, int64_t n,
+                                unsigned long long* acc) {
   constexpr int kD = 14;
-  for (int i = 0; i < kD; ++i) d[i] = 0u;
-  for (int e = 1; e < 256; ++e) {
+  for (int e = 1 + threadIdx.x; e < 256; e += blockDim.x) {
     const unsigned long long v = bins[e];
     if (!v) continue;
-    // add v * 2^(e + 64): three digits from (e + 64) / 32 on, then the carry
-    const int w = (e + 64) >> 5, sh = (e + 64) & 31;
-    const uint64_t p0 = (v << sh) & 0xFFFFFFFFull;
-    const uint64_t p1 = (v >> (32 - sh)) & 0xFFFFFFFFull;
-    const uint64_t p2 = sh ? (v >> (64 - sh)) : 0ull;
-    uint64_t t = static_cast<uint64_t>(d[w]) + p0;
-    d[w] = static_cast<uint32_t>(t);
-    t = static_cast<uint64_t>(d[w + 1]) + p1 + (t >> 32);
-    d[w + 1] = static_cast<uint32_t>(t);
-    t = static_cast<uint64_t>(d[w + 2]) + p2 + (t >> 32);
-    d[w + 2] = static_cast<uint32_t>(t);
-    for (int k = w + 3; (t >> 32) && k < kD; ++k) {
-      t = static_cast<uint64_t>(d[k]) + (t >> 32);
-      d[k] = static_cast<uint32_t>(t);
-    }
+    const int w = (e + 64) >> 5, sh = (e + 64) & 31;  // v * 2^(e + 64)
+    atomicAdd(acc + w, (v << sh) & 0xFFFFFFFFull);
+    atomicAdd(acc + w + 1, (v >> (32 - sh)) & 0xFFFFFFFFull);
+    if (sh) atomicAdd(acc + w + 2, v >> (64 - sh));
   }
+  __syncthreads();
+  if (threadIdx.x != 0) return 0.f;
+  uint32_t d[kD];
+  unsigned long long carry = 0;
+#pragma unroll
+  for (int k = 0; k < kD; ++k) {
+    const unsigned long long t = acc[k] + carry;
+    d[k] = static_cast<uint32_t>(t);
+    carry = t >> 32;
+  }
+  // q = d / n from the most significant digit; each 64-by-32-bit step estimates the
+  // quotient digit in fp64 (within one of the truth, as cur < n * 2^32 < 2^64) and
+  // corrects it exactly
   const uint64_t nn = static_cast<uint64_t>(n);
+  const double rn = 1.0 / static_cast<double>(nn);
   uint64_t rem = 0;
-  for (int k = kD - 1; k >= 0; --k) {  // q = d / n, from the most significant digit
+#pragma unroll
+  for (int k = kD - 1; k >= 0; --k) {
     const uint64_t cur = (rem << 32) | d[k];
-    d[k] = static_cast<uint32_t>(cur / nn);
-    rem = cur % nn;
+    uint64_t q = static_cast<uint64_t>(static_cast<double>(cur) * rn);
+    if (q > 0xFFFFFFFFull) q = 0xFFFFFFFFull;
+    int64_t r = static_cast<int64_t>(cur - q * nn);
+    while (r < 0) {
+      --q;
+      r += static_cast<int64_t>(nn);
+    }
+    while (r >= static_cast<int64_t>(nn)) {
+      ++q;
+      r -= static_cast<int64_t>(nn);
+    }
+    d[k] = static_cast<uint32_t>(q);
+    rem = static_cast<uint64_t>(r);
   }
   int top = -1;  // most significant set bit of q
-  for (int k = kD - 1; k >= 0 && top < 0; --k)
-    if (d[k]) top = 32 * k + 31 - __clz(d[k]);
+#pragma unroll
+  for (int k = kD - 1; k >= 0; --k)
+    if (top < 0 && d[k]) top = 32 * k + 31 - __clz(d[k]);
   if (top < 0) return 0.f;
+  auto dig = [&](int i) -> uint64_t {
+    uint64_t v = 0;
+#pragma unroll
+    for (int k = 0; k < kD; ++k)
+      if (k == i) v = d[k];
+    return v;
+  };
   auto nonzero_below = [&](int nbits) -> bool {  // any of q's bits 0 .. nbits - 1
-    for (int k = 0; 32 * k < nbits; ++k) {
+    bool any = false;
+#pragma unroll
+    for (int k = 0; k < kD; ++k) {
       const int nb = min(32, nbits - 32 * k);
-      if (d[k] & (nb == 32 ? 0xFFFFFFFFu : ((1u << nb) - 1u))) return true;
+      if (nb > 0) any |= (d[k] & (nb >= 32 ? 0xFFFFFFFFu : ((1u << nb) - 1u))) != 0u;
     }
-    return false;
+    return any;
   };
   if (top < 65) {  // below 2^-149: 0, or the smallest subnormal when above half of it
     const bool above_half = top == 64 && (rem != 0 || nonzero_below(64));
     return above_half ? __uint_as_float(1u) : 0.f;
   }
   // the 64-bit window of q whose top bit is bit `top` (bits top - 63 .. top)
-  auto window = [&](int hi_bit) -> uint64_t {  // bits hi_bit - 63 .. hi_bit
-    const int lo = hi_bit - 63;
-    const int k = lo >> 5, sh = lo & 31;  // lo may be negative: those bits are zero
-    auto dig = [&](int i) -> uint64_t { return (i >= 0 && i < kD) ? d[i] : 0u; };
-    const uint64_t x = dig(k) | (dig(k + 1) << 32), y = dig(k + 2);
-    return sh ? ((x >> sh) | (y << (64 - sh))) : x;
-  };
+  const int lo = top - 63;
+  const int k0 = lo >> 5, sh = lo & 31;
+  const uint64_t x = dig(k0) | (dig(k0 + 1) << 32), y = dig(k0 + 2);
+  const uint64_t win = sh ? ((x >> sh) | (y << (64 - sh))) : x;
   // fp32 keeps bits [lsb, top]: 24 bits, or down to 2^-149 (bit 65 of q)
   const int lsb = max(top - 23, 65);
   const int nkeep = top - lsb + 1;  // 1 .. 24
-  const uint64_t win = window(top);
   uint32_t sig = static_cast<uint32_t>(win >> (64 - nkeep));
   const uint32_t guard = static_cast<uint32_t>(win >> (63 - nkeep)) & 1u;
-  // sticky: the bits below the guard (q bits 0 .. lsb - 2) and the remainder
   const uint32_t sticky = (rem != 0 || nonzero_below(lsb - 1)) ? 1u : 0u;
   if (guard && (sticky || (sig & 1u))) ++sig;
   if (lsb == 65) return __uint_as_float(sig);  // subnormal (sig == 2^23: smallest normal)
@@ -147,15 +192,22 @@ __device__ float exact_mean_f32(const unsigned long long* bins, int64_t n, uint3
   return __uint_as_float((static_cast<uint32_t>(ebits) << 23) | (sig & 0x7FFFFFu));
 }
 
+// Clears the accumulators of the mean (sum, exponent range, CTA counter) of level 1, its
+// programmatic dependent, which waits for this grid before it adds to them.
+__global__ void __launch_bounds__(32) k_quantize_prep(unsigned long long* acc) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (threadIdx.x < 4) acc[threadIdx.x] = 0ull;
+}
+
 // Level 1: one 64-block per group of kQuantLanes = 4 lanes (16 elements per lane). Writes
-// the packed codes and the fp32 absmax of each block, and adds every absmax, exactly, into
-// 256 integer bins (one per fp32 exponent) for the mean: absmax = sig * 2^(e - 150) with
-// sig its 24-bit significand and e its biased exponent (1 for subnormals), and bin e sums
-// the sig of its exponent as a 64-bit integer (at most 2^31 blocks of 2^24 each). The CTA
-// sums into shared bins, then adds its nonzero bins into the global ones (zeroed before
-// the launch); the last CTA to finish forms the mean from them. Integer sums do not
-// depend on their order, so the mean is the same for any schedule and any range of
-// constants.
+// the packed codes and the fp32 absmax of each block; the last CTA to finish forms the
+// mean of all absmax, exactly: the CTAs add their absmax in fp64 and keep the smallest and
+// largest exponent e (biased, 1 for subnormals) of the nonzero ones. Every absmax is then
+// a multiple of g = 2^(e_min - 150) below 2^(e_max - 126), so when e_max - e_min +
+// log2(n) <= 28 every partial sum is an integer multiple of g below 2^53 g: exact in
+// fp64, whatever the order. The last CTA then rounds S / n to fp32 exactly
+// (round_div_f32). Otherwise it re-reads all absmax and sums them as integers per
+// exponent (exact_mean_f32). The sums and the counter are cleared by k_quantize_prep.
 //
 // x = fl32(w / absmax) is computed with Markstein's correction step (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000 processor", IBM J.
@@ -172,24 +224,26 @@ template <typename T>
 __global__ void __launch_bounds__(kQuantThreads)
     k_quantize_blocks(const T* __restrict__ W, int64_t nblocks,
                       const __grid_constant__ Nf4BucketTable tab, uint8_t* __restrict__ codes,
-                      float* __restrict__ absmax, unsigned long long* __restrict__ bins,
+                      float* __restrict__ absmax, unsigned long long* __restrict__ acc_g,
                       float* __restrict__ mean_out) {
   const int lane = threadIdx.x & 31;
   const int sub = lane & (kQuantLanes - 1);
   const unsigned gmask = ((1u << kQuantLanes) - 1u) << (lane & (32 - kQuantLanes));
   const int64_t per_cta = kQuantThreads / kQuantLanes;
   __shared__ BucketSmem sb;
-  __shared__ unsigned long long sbins[256];
+  __shared__ unsigned long long sbins[256];  // the wide-range mean of the last CTA
   for (int i = threadIdx.x; i < kCodeBuckets; i += blockDim.x) {
     sb.thr[i] = tab.thr[i];
     sb.code[i] = tab.code[i];
   }
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
   __syncthreads();
   // the double quantization may be scheduled now; it waits for this grid's results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t stride = static_cast<int64_t>(gridDim.x) * per_cta;
   int64_t b = blockIdx.x * per_cta + threadIdx.x / kQuantLanes;
+  // this thread's part of the mean: fp64 sum and exponent range of its nonzero absmax
+  double sum_d = 0.0;
+  uint32_t e_lo = 255u, e_hi = 0u;
   // the next two blocks' elements are in flight while this one is coded
   Raw8<T> n0[kQuantChunks], n1[kQuantChunks];
 #pragma unroll
@@ -245,31 +299,74 @@ __global__ void __launch_bounds__(kQuantThreads)
       reinterpret_cast<uint2*>(codes + b * 32)[sub] = make_uint2(packed[0], packed[1 % kQuantChunks]);
     if (sub == 0) {
       absmax[b] = m;
-      const uint32_t u = __float_as_uint(m);  // m >= 0
-      const uint32_t e = u >> 23;
-      const uint32_t sig = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-      if (sig) atomicAdd(&sbins[e ? e : 1u], static_cast<unsigned long long>(sig));
+      const uint32_t e = __float_as_uint(m) >> 23;  // m >= 0
+      const uint32_t eb = e ? e : 1u;
+      sum_d += static_cast<double>(m);
+      e_lo = m > 0.f ? min(e_lo, eb) : e_lo;
+      e_hi = m > 0.f ? max(e_hi, eb) : e_hi;
     }
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    if (sbins[i]) atomicAdd(bins + i, sbins[i]);
-  // the last CTA to add its bins forms the mean (the bins and the counter were zeroed
-  // before the launch)
-  __threadfence();
+  // the CTA's sum and range, then into the global accumulators
+  __shared__ double red_d[kQuantThreads / 32];
+  __shared__ uint32_t red_lo[kQuantThreads / 32], red_hi[kQuantThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum_d += __shfl_xor_sync(0xFFFFFFFFu, sum_d, o);
+    e_lo = min(e_lo, __shfl_xor_sync(0xFFFFFFFFu, e_lo, o));
+    e_hi = max(e_hi, __shfl_xor_sync(0xFFFFFFFFu, e_hi, o));
+  }
+  if (lane == 0) {
+    red_d[threadIdx.x / 32] = sum_d;
+    red_lo[threadIdx.x / 32] = e_lo;
+    red_hi[threadIdx.x / 32] = e_hi;
+  }
   __syncthreads();
   __shared__ int last;
-  if (threadIdx.x == 0) last = atomicAdd(reinterpret_cast<unsigned int*>(bins + 256), 1u) ==
-                               gridDim.x - 1;
+  if (threadIdx.x == 0) {
+    double cs = 0.0;
+    uint32_t lo = 255u, hi = 0u;
+    for (int i = 0; i < kQuantThreads / 32; ++i) {
+      cs += red_d[i];
+      lo = min(lo, red_lo[i]);
+      hi = max(hi, red_hi[i]);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the accumulators are cleared
+    atomicAdd(reinterpret_cast<double*>(acc_g), cs);
+    atomicMax(reinterpret_cast<unsigned int*>(acc_g + 1), 255u - lo);  // cleared to 0
+    atomicMax(reinterpret_cast<unsigned int*>(acc_g + 2), hi);
+    __threadfence();
+    last = atomicAdd(reinterpret_cast<unsigned int*>(acc_g + 3), 1u) == gridDim.x - 1;
+  }
   __syncthreads();
   if (!last) return;
   __threadfence();
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = __ldcg(bins + i);
-  __syncthreads();
+  __shared__ int wide;
+  __shared__ double total;
   if (threadIdx.x == 0) {
-    __shared__ uint32_t digits[14];
-    mean_out[0] = exact_mean_f32(sbins, nblocks, digits);
+    total = __ldcg(reinterpret_cast<const double*>(acc_g));
+    const int lo = 255 - static_cast<int>(__ldcg(reinterpret_cast<const unsigned int*>(acc_g + 1)));
+    const int hi = static_cast<int>(__ldcg(reinterpret_cast<const unsigned int*>(acc_g + 2)));
+    int lg = 0;  // ceil(log2 n)
+    while ((int64_t{1} << lg) < nblocks) ++lg;
+    wide = total > 0.0 && hi - lo + lg > 28;
+    if (!wide) mean_out[0] = total > 0.0 ? round_div_f32(total, nblocks) : 0.f;
   }
+  __syncthreads();
+  if (!wide) return;
+  // wide range: exact integer sums per exponent over all constants
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
+  __syncthreads();
+  for (int64_t j = threadIdx.x; j < nblocks; j += blockDim.x) {
+    const uint32_t u = __float_as_uint(__ldcg(absmax + j));
+    const uint32_t e = u >> 23;
+    const uint32_t sig = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+    if (sig) atomicAdd(&sbins[e ? e : 1u], static_cast<unsigned long long>(sig));
+  }
+  __shared__ unsigned long long digit_sums[16];
+  if (threadIdx.x < 16) digit_sums[threadIdx.x] = 0ull;
+  __syncthreads();
+  const float mean = exact_mean_f32(sbins, nblocks, digit_sums);
+  if (threadIdx.x == 0) mean_out[0] = mean;
 }
 
 // Level 2: one warp per 256-block of constants, 8 constants per lane, centred on the
@@ -387,7 +484,7 @@ cudaError_t quant_ctas(int64_t nblocks, int* ctas) {
 
 size_t quantize_workspace_bytes(int64_t n, int64_t k) {
   const int64_t nblocks = n * k / 64;
-  return align_up(static_cast<size_t>(nblocks) * 4, 256) + 257 * sizeof(unsigned long long);
+  return align_up(static_cast<size_t>(nblocks) * 4, 256) + 4 * sizeof(unsigned long long);
 }
 
 cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, int codebook,
@@ -400,19 +497,29 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   int ctas = 0;
   cudaError_t e = w_bf16 ? quant_ctas<uint16_t>(nblocks, &ctas) : quant_ctas<float>(nblocks, &ctas);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(bins, 0, 257 * sizeof(unsigned long long), st);  // bins and CTA count
-  if (e != cudaSuccess) return e;
-  note_launches(2);  // blocks, then the mean and double quantization
-  if (w_bf16)
-    k_quantize_blocks<uint16_t><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const uint16_t*>(W), nblocks, code_buckets(codebook), codes, absmax, bins,
-        mean);
-  else
-    k_quantize_blocks<float><<<ctas, kQuantThreads, 0, st>>>(
-        static_cast<const float*>(W), nblocks, code_buckets(codebook), codes, absmax, bins,
-        mean);
+  note_launches(3);  // clearing, blocks, then the double quantization
+  k_quantize_prep<<<1, 32, 0, st>>>(bins);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  {
+    cudaLaunchConfig_t c1cfg = {};
+    c1cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+    c1cfg.blockDim = dim3(kQuantThreads);
+    c1cfg.stream = st;
+    cudaLaunchAttribute a1[1];
+    a1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a1[0].val.programmaticStreamSerializationAllowed = 1;
+    c1cfg.attrs = a1;
+    c1cfg.numAttrs = 1;
+    const Nf4BucketTable& tab = code_buckets(codebook);
+    e = w_bf16 ? cudaLaunchKernelEx(&c1cfg, k_quantize_blocks<uint16_t>,
+                                    static_cast<const uint16_t*>(W), nblocks, tab, codes, absmax,
+                                    bins, mean)
+               : cudaLaunchKernelEx(&c1cfg, k_quantize_blocks<float>,
+                                    static_cast<const float*>(W), nblocks, tab, codes, absmax,
+                                    bins, mean);
+    if (e != cudaSuccess) return e;
+  }
   const int64_t ndq = (nblocks + 255) / 256;
   int64_t g = (ndq + 7) / 8;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;

@@ -234,18 +234,6 @@ __device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases<kG
     }
 }
 
-// 64 bf16 of one token's row of the X stage (block `blk` of the split), as 32 pairs.
-__device__ __forceinline__ void lds_x64(uint32_t addr, uint32_t (&x)[32]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint4 v = lds_b128(addr + 16 * i);
-    x[4 * i] = v.x;
-    x[4 * i + 1] = v.y;
-    x[4 * i + 2] = v.z;
-    x[4 * i + 3] = v.w;
-  }
-}
-
 // One unit: bit (2 q + h) of kPermMask selects the permute table for the row block of
 // rows (q, h); the others go through the pair table. xs0 / xs1: this lane's tokens' rows
 // of the X stage.
@@ -258,9 +246,6 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
   const int blk = (u - u0) * (kUnitK / 64) + t;  // block of the split
   const bool kv = blk < nblk;                    // false past the end of K
   const uint32_t xoff = static_cast<uint32_t>(min(blk, nblk - 1) * kXBlkStride);
-  uint32_t xa[32], xb[32];
-  lds_x64(xs0 + xoff, xa);
-  if (kTall) lds_x64(xs1 + xoff, xb);
 #pragma unroll
   for (int q = 0; q < kGroups; ++q) {
     Nf4Lut lut[2];
@@ -276,6 +261,9 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
     }
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
+      // this word's 8 columns of X for the lane's token(s), just before their MMAs
+      const uint4 xa = lds_b128(xs0 + xoff + 16 * w);
+      const uint4 xb = kTall ? lds_b128(xs1 + xoff + 16 * w) : xa;
       uint32_t o0[4], o1[4];
       const uint32_t w0 = w < 4 ? (&c.q[q][0][0].x)[w] : (&c.q[q][0][1].x)[w - 4];
       const uint32_t w1 = w < 4 ? (&c.q[q][1][0].x)[w] : (&c.q[q][1][1].x)[w - 4];
@@ -287,13 +275,11 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
         lut_decode8(w1, lut[1], o1);
       else
         pair_decode8(w1, lane_bits, s2[1], o1);
-      mma_bf16_16816(acc[q][0], o0[0], o1[0], o0[1], o1[1], xa[4 * w], xa[4 * w + 1]);
-      mma_bf16_16816(acc[q][0], o0[2], o1[2], o0[3], o1[3], xa[4 * w + 2], xa[4 * w + 3]);
+      mma_bf16_16816(acc[q][0], o0[0], o1[0], o0[1], o1[1], xa.x, xa.y);
+      mma_bf16_16816(acc[q][0], o0[2], o1[2], o0[3], o1[3], xa.z, xa.w);
       if (kTall) {
-        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[0], o1[0], o0[1], o1[1], xb[4 * w],
-                       xb[4 * w + 1]);
-        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[2], o1[2], o0[3], o1[3], xb[4 * w + 2],
-                       xb[4 * w + 3]);
+        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
+        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
       }
     }
   }
