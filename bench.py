@@ -253,21 +253,54 @@ def layer_step(L, scale, world, events=None, pool=None):
             qlora.qlora_profile_events(events[-1][0], events[-1][1])
         qlora.qlora_linear_fwd(xs[INPUT_OF[lin["name"]]], lin["q"], lin["A"], lin["B"], scale,
                                Y=lin["Y"], T=lin["T"], workspace=L["ws_f"])
-    for lin in reversed(L["layer"]):
+    slices = linear_grad_slices(L["grads"], L["layer"]) if world > 1 else None
+    pending = []
+    for idx in reversed(range(len(L["layer"]))):
+        lin = L["layer"][idx]
         if events is not None:
             events.append((*pool.pop(), "dgrad", lin))
             qlora.qlora_profile_events(events[-1][0], events[-1][1])
         qlora.qlora_linear_bwd(lin["dY"], xs[INPUT_OF[lin["name"]]], lin["T"], lin["q"], lin["A"],
                                lin["B"], scale, dX=lin["dX"], dA=lin["dA"], dB=lin["dB"],
                                workspace=L["ws_b"])
+        # this linear's dA and dB are final: sum them over the ranks while the next
+        # linear's backward runs
+        pending.append(allreduce_linear_grads_async(slices[idx] if slices else None, world))
     if events is not None:
         qlora.qlora_profile_events(None, None)
-    allreduce_lora_grads(L["grads"], world)
+    wait_all(pending)
+
+
+def linear_grad_slices(grads, layer, r=RANK_R):
+    """Each linear's [dA | dB] slice of the flat gradient buffer (dA then dB, linear after
+    linear)."""
+    out, off = [], 0
+    for lin in layer:
+        n = lin["k"] * r + r * lin["n"]
+        out.append(grads[off:off + n])
+        off += n
+    return out
+
+
+def allreduce_linear_grads_async(grad, world):
+    """The data-parallel exchange of one linear: its LoRA gradients summed over the ranks
+    by an all-reduce issued as soon as its backward is enqueued (the collective runs on its
+    own stream after that work). Returns the pending work, or None on one rank."""
+    if world > 1:
+        return torch.distributed.all_reduce(grad, async_op=True)
+    return None
+
+
+def wait_all(pending):
+    """The current stream waits for every pending collective of the step."""
+    for w in pending:
+        if w is not None:
+            w.wait()
 
 
 def allreduce_lora_grads(grads, world):
-    """Data-parallel exchange of one step: the LoRA gradients of all linears live in one
-    flat fp32 buffer, summed over the ranks with a single all-reduce."""
+    """The whole step's LoRA gradients (one flat fp32 buffer) summed over the ranks in one
+    blocking all-reduce."""
     if world > 1:
         torch.distributed.all_reduce(grads)
 

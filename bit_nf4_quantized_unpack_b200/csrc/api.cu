@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" entry points: host-side validation (nothing is launched
 // when an argument is rejected), dispatch to the kernels, and host utilities.
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -332,6 +333,120 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   q = check_device();
   if (q != QLORA_OK) return q;
   return gemm_backward(dY, X, T_saved, w, A, B, s, dX, dA, dB, workspace, st);
+}
+
+// ---- column (N) sharding of W
+
+qlora_status qlora_shard_rows(int64_t n_out, int64_t k_in, int32_t world, int32_t rank,
+                              int64_t* row0, int64_t* rows) {
+  if (!row0 || !rows || world < 1 || rank < 0 || rank >= world) return QLORA_ERR_INVALID_ARG;
+  if (n_out < 1 || k_in < 64 || k_in % 64 != 0 || n_out % 8 != 0) return QLORA_ERR_SHAPE;
+  // a cut at row n keeps the shard's 256-constant blocks of c1 whole and its c1 16-byte
+  // aligned when n * k_in is a multiple of 4 * 256 * 64 = 65536; rows come in multiples of 8
+  int64_t g = k_in, h = 65536;
+  while (h) {
+    const int64_t t = g % h;
+    g = h;
+    h = t;
+  }
+  // g divides 65536, so the rows per cut are a power of two; at least 8
+  const int64_t unit = std::max<int64_t>(65536 / g, 8);
+  const int64_t units = n_out / unit;
+  if (units < world) {
+    set_last_error("qlora_shard_rows: fewer whole cut units than shards");
+    return QLORA_ERR_SHAPE;
+  }
+  const int64_t u0 = units * rank / world, u1 = units * (rank + 1) / world;
+  *row0 = u0 * unit;
+  *rows = (rank == world - 1) ? n_out - *row0 : (u1 - u0) * unit;
+  return QLORA_OK;
+}
+
+qlora_status qlora_shard_weight(qlora_nf4_weight w, int64_t row0, int64_t rows,
+                                qlora_nf4_weight* out) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  qlora_status q = check_weight(w);
+  if (q != QLORA_OK) return q;
+  if (row0 < 0 || rows < 8 || rows % 8 != 0 || row0 + rows > w.n_out) return QLORA_ERR_SHAPE;
+  if ((row0 * w.k_in) % 65536 != 0) {
+    set_last_error("qlora_shard_weight: row0 * k_in must be a multiple of 65536");
+    return QLORA_ERR_SHAPE;
+  }
+  *out = w;
+  out->codes = w.codes + row0 * (w.k_in / 2);
+  out->c2 = w.c2 + row0 * (w.k_in / 64);
+  out->c1 = w.c1 + row0 * w.k_in / 16384;
+  out->n_out = rows;
+  return QLORA_OK;
+}
+
+size_t qlora_linear_bwd_shard_g_workspace_size(int64_t M, int64_t n_shard, int r) {
+  if (M < 0 || n_shard < 8 || r < 8 || r > 64) return 0;
+  return gemm_shard_g_workspace(LinearShape{M, n_shard, 64, r, 1.f});
+}
+
+qlora_status qlora_linear_bwd_shard_g(const uint16_t* dY, int64_t M, int64_t n_shard,
+                                      const uint16_t* B, int r, float* G_part, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (M < 0 || M > (int64_t{1} << 31) || n_shard < 8 || n_shard % 8 != 0) return QLORA_ERR_SHAPE;
+  if (r < 8 || r > 64 || r % 8 != 0) return QLORA_ERR_INVALID_ARG;
+  if (!G_part) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(G_part)) return QLORA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M == 0) return QLORA_OK;
+  if (!dY || !B) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(B)) return QLORA_ERR_ALIGN;
+  const LinearShape s{M, n_shard, 64, r, 1.f};
+  if (!workspace || workspace_bytes < gemm_shard_g_workspace(s)) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+  qlora_status q = check_device();
+  if (q != QLORA_OK) return q;
+  return gemm_shard_g(dY, B, s, G_part, workspace, st);
+}
+
+size_t qlora_linear_bwd_shard_workspace_size(int64_t M, int64_t n_shard, int64_t k_in, int r) {
+  if (M < 0 || n_shard < 1 || k_in < 64 || r < 8 || r > 64) return 0;
+  return gemm_shard_bwd_workspace(LinearShape{M, n_shard, k_in, r, 1.f});
+}
+
+qlora_status qlora_linear_bwd_shard(const uint16_t* dY, const uint16_t* X, const float* T_saved,
+                                    const float* G, int64_t M, qlora_nf4_weight w,
+                                    const uint16_t* A, const uint16_t* B, int r, float scale,
+                                    int32_t lora_in_dx, float* dX_part, float* dA, float* dB,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  qlora_status q = check_linear(M, w, r, scale);
+  if (q != QLORA_OK) return q;
+  if (!dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dA) || !aligned16(dB)) return QLORA_ERR_ALIGN;
+  const LinearShape s{M, w.n_out, w.k_in, r, scale};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M == 0) {  // empty batch: zero gradients, nothing to add to dX
+    q = check_device();
+    if (q != QLORA_OK) return q;
+    cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(w.k_in) * r * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(w.n_out) * r * 4, st);
+    return cuda_status(e);
+  }
+  if (!dY || !X || !G || !A || !B) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(G) || !aligned16(A) || !aligned16(B) ||
+      (dX_part && !aligned16(dX_part)) || (T_saved && !aligned16(T_saved)))
+    return QLORA_ERR_ALIGN;
+  if (!workspace || workspace_bytes < gemm_shard_bwd_workspace(s)) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QLORA_ERR_ALIGN;
+  q = check_device();
+  if (q != QLORA_OK) return q;
+  return gemm_shard_bwd(dY, X, T_saved, G, w, A, B, s, lora_in_dx != 0, dX_part, dA, dB,
+                        workspace, st);
+}
+
+qlora_status qlora_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, void* stream) {
+  if (n < 0 || n % 4 != 0) return QLORA_ERR_SHAPE;
+  if (n == 0) return QLORA_OK;
+  if (!src || !dst) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return QLORA_ERR_ALIGN;
+  qlora_status q = check_device();
+  if (q != QLORA_OK) return q;
+  return cuda_status(launch_to_bf16(src, dst, n, static_cast<cudaStream_t>(stream)));
 }
 
 qlora_status qlora_selftest_wait_timeout(void* stream) {

@@ -92,6 +92,7 @@ struct FusedArgs {
   int row_tiles;      // tiles along the D rows (weight side)
   int num_tiles;      // row_tiles x token tiles
   uint16_t* out;      // [M, out_ld] bf16
+  bool out_f32;       // write fp32 [M, out_ld] through tm_out instead (dgrad partial sums)
   int64_t out_ld;     // N (forward) or K (dgrad)
   int64_t out_rows;   // valid D rows: N (forward) or K (dgrad)
   int codebook;       // 4-bit codebook of the codes (0 NF4, 1 uniform)
@@ -466,6 +467,38 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         // one's TMEM load, before its conversion and store
         const int64_t left = (args.M - m0 - h * kHalfCols + 31) / 32;
         const int nchunks = left < kHalfCols / 32 ? static_cast<int>(left) : kHalfCols / 32;
+        if (args.out_f32) {
+          // fp32 output: one 32 x 32 chunk fills the warp's whole 4 KB stage, as
+          // stage[token][row] (a 32-lane store per token is one 128-byte row), then one
+          // unswizzled TMA tile store; the stage is reused once that store has read it
+#pragma unroll 1
+          for (int c = 0; c < nchunks; ++c) {
+            const int64_t mb = m0 + h * kHalfCols + c * 32;
+            const uint32_t stage_s = smem_u32(stage2);
+            if (chunks >= 1 && lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+            ++chunks;
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, v);  // row quarter * 32 + lane, 32 tokens
+            tmem_ld_wait();
+            if (c == nchunks - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[h]);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              asm volatile("st.shared.b32 [%0], %1;" ::"r"(stage_s + j * 128 + lane * 4), "r"(v[j])
+                           : "memory");
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && obase < args.out_rows) {
+              tma_store_2d(&tm_out, stage2, static_cast<int>(obase), static_cast<int>(mb));
+              bulk_commit_group();
+            }
+          }
+          continue;
+        }
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
           const int64_t mb = m0 + h * kHalfCols + c * 32;
@@ -854,6 +887,39 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// G and T of a column-sharded backward (plain fp32 [M, r]; G summed over the shards) as
+// the bf16 operand pairs of the fused dX kernel and the grouped dA/dB GEMM: scale G as
+// hi | lo ([M, 128]), G as hi | lo and T as hi | lo (the arithmetic of k_finalize_rank).
+__global__ void k_rank_from_plain(const float* __restrict__ G, const float* __restrict__ T,
+                                  int64_t M, int r, float scale, uint16_t* __restrict__ gs,
+                                  uint16_t* __restrict__ ghl, uint16_t* __restrict__ thl) {
+  griddep_wait_and_release();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= M * 64) return;
+  const int64_t m = i >> 6;
+  const int j = static_cast<int>(i & 63);
+  const float g = j < r ? G[m * r + j] : 0.f;
+  const float t = j < r ? T[m * r + j] : 0.f;
+  auto hilo = [&](uint16_t* out, float v) {
+    const uint16_t hi = bf16_bits_rn(v);
+    out[m * 128 + j] = hi;
+    out[m * 128 + 64 + j] = bf16_bits_rn(v - __uint_as_float(static_cast<uint32_t>(hi) << 16));
+  };
+  hilo(gs, g * scale);
+  hilo(ghl, g);
+  hilo(thl, t);
+}
+
+// dst[i] = bf16_rn(src[i]), four per thread (n % 4 == 0, 16-byte aligned).
+__global__ void k_to_bf16(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t n4) {
+  griddep_wait_and_release();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = make_uint2(pack_bf16x2_rn(v.x, v.y), pack_bf16x2_rn(v.z, v.w));
+  }
+}
+
 // Stacked rows of a grouped launch: the first problem padded to whole tiles, then the second.
 inline int64_t stacked_rows(int64_t rows0, int64_t rows1) { return align_up(rows0, 128) + rows1; }
 
@@ -1036,6 +1102,7 @@ qlora_status gemm_forward(const uint16_t* X, const qlora_nf4_weight& w, const ui
   a.M = s.M;
   a.ext_mmas = (s.r + 15) / 16;
   a.out = Y;
+  a.out_f32 = false;
   a.out_ld = s.N;
   a.out_rows = s.N;
   a.err = device_error_word();
@@ -1113,6 +1180,7 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
     a.M = s.M;
     a.ext_mmas = (s.r + 15) / 16;
     a.out = dX;
+    a.out_f32 = false;
     a.out_ld = s.K;
     a.out_rows = s.K;
     a.err = device_error_word();
@@ -1133,6 +1201,111 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
   }
   QL_TRY(e);
   return QLORA_OK;
+}
+
+// ---- column (N) sharding of W: the backward of one shard
+size_t gemm_shard_g_workspace(const LinearShape& s) {
+  return align_up(partial_floats(s.M, s.N, 64) * sizeof(float), 256) + 256;
+}
+
+qlora_status gemm_shard_g(const uint16_t* dY, const uint16_t* B, const LinearShape& s,
+                          float* G_part, void* ws, cudaStream_t st) {
+  float* part = static_cast<float*>(ws);
+  CUtensorMap ta, tb;
+  QL_MAP(&ta, kBF16, dY, s.N, s.M, s.N * 2, 64, 128, kSW128);  // dY K-major (over n)
+  QL_MAP(&tb, kBF16, B, s.N, s.r, s.N * 2, 64, 64, kSW128);    // B [r, N] K-major
+  int splits = 0;
+  QL_TRY((run_lora_gemm<false, false, 64>(ta, tb, s.M, s.N, part, st, &splits)));
+  QL_TRY(launch_pdl(k_finalize_rank, dim3(blocks_for(s.M * 64, 256)), dim3(256), 0, st, part,
+                    splits, plan_split(s.M, s.N).rows_pad, s.M, s.r, s.scale, G_part, nullptr,
+                    nullptr, nullptr, nullptr));
+  return QLORA_OK;
+}
+
+size_t gemm_shard_bwd_workspace(const LinearShape& s) {
+  float *p, *t;
+  uint16_t *g, *gh, *th;
+  return bwd_layout(s, nullptr, &p, &g, &gh, &th, &t);
+}
+
+qlora_status gemm_shard_bwd(const uint16_t* dY, const uint16_t* X, const float* T_saved,
+                            const float* G, const qlora_nf4_weight& w, const uint16_t* A,
+                            const uint16_t* B, const LinearShape& s, bool lora_in_dx,
+                            float* dX_part, float* dA, float* dB, void* ws, cudaStream_t st) {
+  float *part, *tbuf;
+  uint16_t *gs, *ghl, *thl;
+  bwd_layout(s, ws, &part, &gs, &ghl, &thl, &tbuf);
+  const float* t = T_saved;
+  if (!t) {
+    qlora_status q = lora_down_T(X, A, s, part, tbuf, nullptr, st);
+    if (q != QLORA_OK) return q;
+    t = tbuf;
+  }
+  QL_TRY(launch_pdl(k_rank_from_plain, dim3(blocks_for(s.M * 64, 256)), dim3(256), 0, st, G, t,
+                    s.M, s.r, s.scale, gs, ghl, thl));
+  CUtensorMap xa, xw, xx, xo, ga, gb, ga1, gb1;
+  if (dX_part) {
+    QL_MAP(&xa, kBF16, dY, s.N, s.M, s.N * 2, 64, 256, kSW128);
+    QL_MAP(&xw, kBF16, A, s.r, s.K, s.r * 2, 64, 128, kSW128);   // A [K, r] K-major
+    QL_MAP(&xx, kBF16, gs, 128, s.M, 256, 64, 256, kSW128);      // scale G, bf16 hi | lo
+    // fp32 dX partial sums [M, K]: 32 x 32 boxes, no swizzle
+    QL_MAP(&xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dX_part, s.K, s.M, s.K * 4, 32, 32,
+           CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  QL_MAP(&ga, kBF16, X, s.K, s.M, s.K * 2, 64, 64, kSW128);
+  QL_MAP(&gb, kBF16, ghl, 128, s.M, 256, 64, 64, kSW128);
+  QL_MAP(&ga1, kBF16, dY, s.N, s.M, s.N * 2, 64, 64, kSW128);
+  QL_MAP(&gb1, kBF16, thl, 128, s.M, 256, 64, 64, kSW128);
+  SideStream* side = nullptr;
+  if (dX_part) QL_TRY(side_stream(st, &side));
+  cudaStream_t gst = st;
+  if (side) {
+    QL_TRY(cudaEventRecord(side->fork, st));
+    QL_TRY(cudaStreamWaitEvent(side->st, side->fork, 0));
+    gst = side->st;
+  }
+  cudaError_t e = cudaSuccess;
+  if (dX_part) {
+    FusedArgs a;
+    a.codebook = w.codebook;
+    a.codes = w.codes;
+    a.c2 = w.c2;
+    a.c1 = w.c1;
+    a.mean = w.mean;
+    a.N = s.N;
+    a.K = s.K;
+    a.M = s.M;
+    a.ext_mmas = lora_in_dx ? (s.r + 15) / 16 : 0;
+    a.out = nullptr;
+    a.out_f32 = true;
+    a.out_ld = s.K;
+    a.out_rows = s.K;
+    a.err = device_error_word();
+    e = run_fused<Mode::kDgrad>(xa, xw, xx, xo, a, st);
+  }
+  int splits = 0;
+  if (e == cudaSuccess)
+    e = run_lora_gemm<true, true, 128>(ga, gb, s.K, s.M, part, gst, &splits, &ga1, &gb1, s.N);
+  if (e == cudaSuccess) {
+    const int64_t stacked = stacked_rows(s.K, s.N);
+    e = launch_pdl(k_finalize_grad, dim3(blocks_for(stacked, kGradRows)), dim3(256), 0, gst,
+                   part, splits, plan_split(stacked, s.M).rows_pad,
+                   static_cast<int64_t>(align_up(s.K, 128)), s.K, dA, s.N, dB, s.r, s.scale);
+  }
+  if (side) {
+    cudaError_t ej = cudaEventRecord(side->join, side->st);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, side->join, 0);
+    if (e == cudaSuccess) e = ej;
+  }
+  QL_TRY(e);
+  return QLORA_OK;
+}
+
+cudaError_t launch_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t st) {
+  const int64_t n4 = n / 4;
+  const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, static_cast<int64_t>(num_sms()) * 8);
+  return launch_pdl(k_to_bf16, dim3(static_cast<unsigned>(std::max<int64_t>(blocks, 1))), dim3(256),
+                    0, st, reinterpret_cast<const float4*>(src), reinterpret_cast<uint2*>(dst), n4);
 }
 
 }  // namespace qlora

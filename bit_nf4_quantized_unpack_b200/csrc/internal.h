@@ -75,6 +75,20 @@ qlora_status gemm_backward(const uint16_t* dY, const uint16_t* X, const float* T
                            const LinearShape& s, uint16_t* dX, float* dA, float* dB, void* ws,
                            cudaStream_t st);
 
+// Column (N) sharding of W (gemm.cu): the backward of one shard, whose weight is rows
+// [row0, row0 + N) of W. gemm_shard_g: G_part = dY B^T (fp32, unscaled); once G is summed
+// over the shards, gemm_shard_bwd: dX_part = dY W_hat (+ scale G A^T when lora_in_dx) in
+// fp32, dA = scale X^T G, dB = scale T^T dY. launch_to_bf16 rounds a summed dX.
+size_t gemm_shard_g_workspace(const LinearShape& s);
+qlora_status gemm_shard_g(const uint16_t* dY, const uint16_t* B, const LinearShape& s,
+                          float* G_part, void* ws, cudaStream_t st);
+size_t gemm_shard_bwd_workspace(const LinearShape& s);
+qlora_status gemm_shard_bwd(const uint16_t* dY, const uint16_t* X, const float* T_saved,
+                            const float* G, const qlora_nf4_weight& w, const uint16_t* A,
+                            const uint16_t* B, const LinearShape& s, bool lora_in_dx,
+                            float* dX_part, float* dA, float* dB, void* ws, cudaStream_t st);
+cudaError_t launch_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t st);
+
 // ---- launchers (decode.cu) ------------------------------------------------------
 constexpr int64_t kDecodeMaxM = 16;
 // Workspace of the decode kernels, or 0 when they cannot run the shape (the fused GEMM

@@ -71,6 +71,15 @@ _SIGNATURES = {
     "qlora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
     "qlora_linear_bwd": (_i32, [_vp, _vp, _vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32, _vp, _vp,
                                 _vp, _vp, _sz, _vp]),
+    "qlora_shard_rows": (_i32, [_i64, _i64, _i32, _i32, ctypes.POINTER(ctypes.c_int64),
+                                ctypes.POINTER(ctypes.c_int64)]),
+    "qlora_shard_weight": (_i32, [CNF4Weight, _i64, _i64, ctypes.c_void_p]),
+    "qlora_linear_bwd_shard_g_workspace_size": (_sz, [_i64, _i64, _i32]),
+    "qlora_linear_bwd_shard_g": (_i32, [_vp, _i64, _i64, _vp, _i32, _vp, _vp, _sz, _vp]),
+    "qlora_linear_bwd_shard_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
+    "qlora_linear_bwd_shard": (_i32, [_vp, _vp, _vp, _vp, _i64, CNF4Weight, _vp, _vp, _i32, _f32,
+                                      _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_f32_to_bf16": (_i32, [_vp, _vp, _i64, _vp]),
     "qlora_selftest_wait_timeout": (_i32, [_vp]),
     "qlora_adamw_state_bytes": (_sz, [_i64, _i32]),
     "qlora_adamw_step": (_i32, [_vp, _vp, _vp, _i64, _i32, _vp, _sz, CAdamwHparams, _vp]),
@@ -288,6 +297,70 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None, 
                                   _ptr(ws), ws.numel(), _stream()),
            "qlora_linear_bwd")
     return (dX if need_dX else None), dA, dB
+
+
+def qlora_shard_rows(n_out: int, k_in: int, world: int, rank: int):
+    """(row0, rows) of shard `rank` of `world` for a column (N) split of an n_out x k_in
+    weight: near-equal parts cut only where row * k_in % 65536 == 0."""
+    r0, rows = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(lib().qlora_shard_rows(n_out, k_in, world, rank, ctypes.byref(r0), ctypes.byref(rows)),
+           "qlora_shard_rows")
+    return int(r0.value), int(rows.value)
+
+
+def qlora_shard_weight(w: NF4Weight, row0: int, rows: int) -> NF4Weight:
+    """Rows [row0, row0 + rows) of w as a weight of its own: views of w's buffers (no copy),
+    checked by the library (cuts where row0 * k_in % 65536 == 0)."""
+    out = CNF4Weight()
+    _check(lib().qlora_shard_weight(w.c_struct(), row0, rows, ctypes.byref(out)), "qlora_shard_weight")
+    k = w.k_in
+    view = NF4Weight(w.codes[row0 * k // 2:(row0 + rows) * k // 2],
+                     w.c2[row0 * k // 64:(row0 + rows) * k // 64],
+                     w.c1[row0 * k // 16384:-(-(row0 + rows) * k // 16384)],
+                     w.mean, rows, k, w.codebook)
+    assert view.codes.data_ptr() == out.codes and view.c1.data_ptr() == out.c1
+    return view
+
+
+def qlora_linear_bwd_shard_g(dY: torch.Tensor, B: torch.Tensor, G_part: torch.Tensor | None = None):
+    """G_part [M, r] fp32 = dY B^T for one shard's dY [M, n_shard] and B [r, n_shard]."""
+    M, n = dY.shape
+    r = B.shape[0]
+    G_part = G_part if G_part is not None else torch.empty(M, r, dtype=torch.float32, device=dY.device)
+    need = int(lib().qlora_linear_bwd_shard_g_workspace_size(M, n, r))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dY.device)
+    _check(lib().qlora_linear_bwd_shard_g(_ptr(_as_bits(dY)), M, n, _ptr(_as_bits(B)), r, _ptr(G_part),
+                                          _ptr(ws), ws.numel(), _stream()), "qlora_linear_bwd_shard_g")
+    return G_part
+
+
+def qlora_linear_bwd_shard(dY: torch.Tensor, X: torch.Tensor, T: torch.Tensor | None,
+                           G: torch.Tensor, w: NF4Weight, A: torch.Tensor, B: torch.Tensor,
+                           scale: float, lora_in_dx: bool, need_dX: bool = True):
+    """One shard's (dX_part fp32 [M, K] or None, dA [K, r], dB [r, n_shard]) given G summed
+    over the shards; dX_part carries scale G A^T only when lora_in_dx."""
+    M = X.shape[0]
+    r = A.shape[1]
+    dev = X.device
+    dXp = torch.empty(M, w.k_in, dtype=torch.float32, device=dev) if need_dX else None
+    dA = torch.empty(w.k_in, r, dtype=torch.float32, device=dev)
+    dB = torch.empty(r, w.n_out, dtype=torch.float32, device=dev)
+    need = int(lib().qlora_linear_bwd_shard_workspace_size(M, w.n_out, w.k_in, r))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().qlora_linear_bwd_shard(_ptr(_as_bits(dY)), _ptr(_as_bits(X)), _ptr(T), _ptr(G), M,
+                                        w.c_struct(), _ptr(_as_bits(A)), _ptr(_as_bits(B)), r,
+                                        float(scale), int(bool(lora_in_dx)), _ptr(dXp), _ptr(dA),
+                                        _ptr(dB), _ptr(ws), ws.numel(), _stream()),
+           "qlora_linear_bwd_shard")
+    return dXp, dA, dB
+
+
+def qlora_f32_to_bf16(src: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16_rn of an fp32 tensor (numel % 4 == 0)."""
+    out = out if out is not None else torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    _check(lib().qlora_f32_to_bf16(_ptr(src), _ptr(_as_bits(out)), src.numel(), _stream()),
+           "qlora_f32_to_bf16")
+    return out
 
 
 def qlora_profile_events(before=None, after=None):

@@ -311,6 +311,81 @@ qlora_status qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, const float
                               size_t workspace_bytes, void *stream);
 
 /*
+ * Column (N) sharding of W across GPUs. The layer's backward (itwiki "QLoRA", section
+ * "계산 방식": dX flows to the previous layer, gradients only for A and B) splits along
+ * the output features: a shard holds rows [row0, row0 + n_shard) of the quantized W and
+ * the matching columns of B, dY and Y, while X, A and T are whole on every shard. Then
+ *   Y_shard = X W_hat_shard^T + scale T B_shard        (qlora_linear_fwd on the shard)
+ *   G       = sum over shards of dY_shard B_shard^T     (a cross-shard sum)
+ *   dX      = bf16(sum over shards of dY_shard W_hat_shard + scale G A^T)
+ *   dA      = scale X^T G,   dB_shard = scale T^T dY_shard.
+ * One step of a sharded backward: qlora_linear_bwd_shard_g on every shard, a sum of the
+ * G_part over the shards (the caller's collective, e.g. an NCCL all-reduce), then
+ * qlora_linear_bwd_shard on every shard with exactly one shard adding the LoRA term
+ * (lora_in_dx = 1), a sum of the dX_part, and qlora_f32_to_bf16 of that sum.
+ *
+ * qlora_shard_rows: rows [*row0, *row0 + *rows) of an n_out x k_in weight for shard `rank`
+ * of `world`: near-equal parts cut only where row * k_in is a multiple of 65536, so that
+ * each shard's 256-constant blocks of c1 are whole (the one mean stays the tensor's) and
+ * its c1 stays 16-byte aligned; the last shard takes the remainder. Host only.
+ * Errors: QLORA_ERR_INVALID_ARG for NULL outputs or rank outside [0, world);
+ * QLORA_ERR_SHAPE when there are fewer whole cuts than shards (or n_out % 8 != 0).
+ */
+qlora_status qlora_shard_rows(int64_t n_out, int64_t k_in, int32_t world, int32_t rank,
+                              int64_t *row0, int64_t *rows);
+
+/*
+ * qlora_shard_weight: *out = the view of rows [row0, row0 + rows) of w as a weight of its
+ * own (pointers into w's buffers; nothing is copied or allocated; w keeps ownership).
+ * Errors: those of the weight checks; QLORA_ERR_SHAPE unless row0 * k_in % 65536 == 0,
+ * rows % 8 == 0 and the rows lie inside w. Host only.
+ */
+qlora_status qlora_shard_weight(qlora_nf4_weight w, int64_t row0, int64_t rows,
+                                qlora_nf4_weight *out);
+
+/* Device bytes of workspace qlora_linear_bwd_shard_g needs. */
+size_t qlora_linear_bwd_shard_g_workspace_size(int64_t M, int64_t n_shard, int r);
+
+/*
+ * qlora_linear_bwd_shard_g: G_part [M, r] fp32 (device, overwritten) = dY B^T for one
+ * shard's dY [M, n_shard] and B [r, n_shard] (bf16 device), unscaled.
+ * Errors: QLORA_ERR_SHAPE unless n_shard >= 8, n_shard % 8 == 0, 0 <= M <= 2^31;
+ * QLORA_ERR_INVALID_ARG for r outside {8, ..., 64} or NULL pointers; QLORA_ERR_ALIGN,
+ * QLORA_ERR_WORKSPACE as elsewhere. M == 0 enqueues nothing.
+ */
+qlora_status qlora_linear_bwd_shard_g(const uint16_t *dY, int64_t M, int64_t n_shard,
+                                      const uint16_t *B, int r, float *G_part, void *workspace,
+                                      size_t workspace_bytes, void *stream);
+
+/* Device bytes of workspace qlora_linear_bwd_shard needs. */
+size_t qlora_linear_bwd_shard_workspace_size(int64_t M, int64_t n_shard, int64_t k_in, int r);
+
+/*
+ * qlora_linear_bwd_shard: the rest of one shard's backward, given G [M, r] fp32 (device)
+ * summed over all shards.
+ *   dX_part [M, K] fp32 device (overwritten), or NULL to skip:
+ *           dY W_hat_shard, plus scale G A^T when lora_in_dx != 0 (set it on one shard);
+ *           computed on the tensor cores like qlora_linear_bwd's dX, but left in fp32
+ *           for the cross-shard sum
+ *   dA [K, r] fp32 (overwritten) = scale X^T G (the same on every shard)
+ *   dB [r, n_shard] fp32 (overwritten) = scale T^T dY_shard
+ * w is the shard's weight (qlora_shard_weight); dY [M, n_shard], X [M, K], A [K, r],
+ * B [r, n_shard] bf16; T_saved [M, r] fp32 or NULL (recomputed from X and A).
+ * Errors: as qlora_linear_bwd. M == 0 writes zeros to dA and dB.
+ */
+qlora_status qlora_linear_bwd_shard(const uint16_t *dY, const uint16_t *X, const float *T_saved,
+                                    const float *G, int64_t M, qlora_nf4_weight w,
+                                    const uint16_t *A, const uint16_t *B, int r, float scale,
+                                    int32_t lora_in_dx, float *dX_part, float *dA, float *dB,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * qlora_f32_to_bf16: dst[i] = bf16_rn(src[i]) for i < n (device, n % 4 == 0, 16-byte
+ * aligned), e.g. dX from the sum of the shards' dX_part.
+ */
+qlora_status qlora_f32_to_bf16(const float *src, uint16_t *dst, int64_t n, void *stream);
+
+/*
  * qlora_selftest_wait_timeout: a test hook for the failure path that every kernel's
  * bounded waits share (not part of the method). Enqueues on `stream` one small kernel
  * whose only wait, on an mbarrier that nothing arrives at, runs out after the library's

@@ -1,5 +1,6 @@
 """The multi-GPU host logic of bench.py, run as two gloo ranks on the CPU: the
-data-parallel all-reduce of the flat LoRA-gradient buffer and the max-over-ranks
+data-parallel all-reduce of the LoRA gradients (the flat buffer at once, and linear by
+linear with asynchronous all-reduces in the backward's order) and the max-over-ranks
 timing reduction. (Only one GPU is available to this test suite; the NCCL path runs
 the same calls.)"""
 import os
@@ -29,7 +30,23 @@ def _worker(rank, world, port, out):
         gathered = [torch.zeros(1000) for _ in range(world)]
         dist.all_gather(gathered, local)
         ms = bench.max_over_ranks(1.5 + rank, world, "cpu")
-        out.put((rank, torch.allclose(grads, sum(gathered), atol=1e-5), ms))
+        ok = torch.allclose(grads, sum(gathered), atol=1e-5)
+        # per linear: the [dA | dB] slices of a 7-linear layout, summed one by one in the
+        # backward's order (last linear first) by asynchronous all-reduces
+        layer = [dict(k=k, n=n) for k, n in ((64, 32), (64, 32), (64, 32), (64, 64), (64, 96),
+                                              (64, 96), (96, 64))]
+        numel = sum(l["k"] * 4 + 4 * l["n"] for l in layer)
+        flat = torch.randn(numel, generator=g)
+        ref = [torch.zeros(numel) for _ in range(world)]
+        dist.all_gather(ref, flat.clone())
+        slices = bench.linear_grad_slices(flat, layer, r=4)
+        assert sum(sl.numel() for sl in slices) == numel
+        assert slices[0].data_ptr() == flat.data_ptr()
+        pending = [bench.allreduce_linear_grads_async(slices[i], world)
+                   for i in reversed(range(len(layer)))]
+        bench.wait_all(pending)
+        ok = ok and torch.allclose(flat, sum(ref), atol=1e-5)
+        out.put((rank, ok, ms))
     finally:
         dist.destroy_process_group()
 
