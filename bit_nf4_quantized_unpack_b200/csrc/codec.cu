@@ -47,21 +47,42 @@ struct Raw8<uint16_t> {  // bf16
 
 // NF4 code of x in [-1, 1] from the bucket table in shared memory, given
 // bk = fl32(16 x + 16 + 1.5 * 2^23): that number lies in [2^23, 2^24), where the ulp is 1,
-// so its low mantissa bits hold the bucket round-half-even(16 x + 16). The table is two
-// arrays of 4-byte words (fp32 thresholds, codes) at a fixed distance, so that one address
-// serves both loads; 33 words occupy 32 banks, so the lanes of a warp rarely conflict.
-// The unsigned clamp keeps any bit pattern (a NaN from a non-finite input) inside the table.
+// so its low mantissa bits hold the bucket round-half-even(16 x + 16) (0..32). The table
+// is two arrays of 64 4-byte words (negated fp32 thresholds, codes) at a fixed distance,
+// so that one address serves both loads, indexed by the low six bits of bk: any bit
+// pattern (a NaN from a non-finite input) stays inside it. Entries 33-63 are -inf
+// (no threshold) and code 0.
+constexpr int kBucketSlots = 64;
 struct BucketSmem {
-  float thr[kCodeBuckets];
-  uint32_t code[kCodeBuckets];
+  float nthr[kBucketSlots];  // -threshold
+  uint32_t code[kBucketSlots];
 };
 constexpr float kBucketBias = 16.0f + 12582912.0f;  // S + 1.5 * 2^23
-__device__ __forceinline__ uint32_t bucket_code(float x, float bk, const BucketSmem& sb) {
-  const uint32_t idx = min(__float_as_uint(bk), 0x4B400000u + (kCodeBuckets - 1)) - 0x4B400000u;
-  return sb.code[idx] + (x >= sb.thr[idx] ? 1u : 0u);
+__device__ __forceinline__ uint32_t bucket_index(float bk) {
+  return __float_as_uint(bk) & (kBucketSlots - 1);
 }
 __device__ __forceinline__ uint32_t bucket_code(float x, const BucketSmem& sb) {
-  return bucket_code(x, __fmaf_rn(x, static_cast<float>(kBucketScale), kBucketBias), sb);
+  const uint32_t idx = bucket_index(__fmaf_rn(x, static_cast<float>(kBucketScale), kBucketBias));
+  return sb.code[idx] + (-x <= sb.nthr[idx] ? 1u : 0u);
+}
+
+// Eight codes packed as one 32-bit word (element 2j in the low nibble of byte j, 2j+1 in
+// the high one) from the bucket codes cw[i] (0..15, low byte) and d[i] = fl32(x_i -
+// thr_i): x >= thr exactly when d is not negative (the sign of a rounded difference is
+// that of the exact one, and x == thr gives +0; no threshold is zero), and then the code
+// is one above the bucket's (at most 14 where the bucket holds a threshold, so the
+// nibble does not carry). The sign bytes come from prmt's sign-replicating selectors
+// (0xFF where d < 0).
+__device__ __forceinline__ uint32_t pack_codes8(const uint32_t (&cw)[8], const float (&d)[8]) {
+  const uint32_t ce = prmt(prmt(cw[0], cw[2], 0x0040u), prmt(cw[4], cw[6], 0x0040u), 0x5410u);
+  const uint32_t co = prmt(prmt(cw[1], cw[3], 0x0040u), prmt(cw[5], cw[7], 0x0040u), 0x5410u);
+  uint32_t di[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) di[i] = __float_as_uint(d[i]);
+  const uint32_t se = prmt(prmt(di[0], di[2], 0x00FBu), prmt(di[4], di[6], 0x00FBu), 0x5410u);
+  const uint32_t so = prmt(prmt(di[1], di[3], 0x00FBu), prmt(di[5], di[7], 0x00FBu), 0x5410u);
+  const uint32_t neg = (se & 0x0F0F0F0Fu) | (so & 0xF0F0F0F0u);  // 0xF where x < thr
+  return ce + (co << 4) + (0x11111111u & ~neg);
 }
 
 // max(|a|, |b|, |c|) in one three-input max (sm_100).
@@ -232,9 +253,9 @@ __global__ void __launch_bounds__(kQuantThreads)
   const int64_t per_cta = kQuantThreads / kQuantLanes;
   __shared__ BucketSmem sb;
   __shared__ unsigned long long sbins[256];  // the wide-range mean of the last CTA
-  for (int i = threadIdx.x; i < kCodeBuckets; i += blockDim.x) {
-    sb.thr[i] = tab.thr[i];
-    sb.code[i] = tab.code[i];
+  for (int i = threadIdx.x; i < kBucketSlots; i += blockDim.x) {
+    sb.nthr[i] = i < kCodeBuckets ? -tab.thr[i] : __int_as_float(0xFF800000);
+    sb.code[i] = i < kCodeBuckets ? tab.code[i] : 0u;
   }
   __syncthreads();
   // the double quantization may be scheduled now; it waits for this grid's results
@@ -275,17 +296,25 @@ __global__ void __launch_bounds__(kQuantThreads)
       const uint64_t kscale = f2_pack(kBucketScale, kBucketScale);
       const uint64_t kbias = f2_pack(kBucketBias, kBucketBias);
 #pragma unroll
-      for (int i = 0; i < kQuantPer / 2; ++i) {
-        const uint64_t w = f2_pack(v[2 * i], v[2 * i + 1]);
-        const uint64_t q = f2_mul(w, rr);
-        const uint64_t e = f2_fma(q, nm, w);  // w - q m, exact
-        const uint64_t x = f2_fma(e, rr, q);  // fl32(w / m)
-        const uint64_t bk = f2_fma(x, kscale, kbias);
-        float x0, x1, b0, b1;
-        f2_unpack(x, x0, x1);
-        f2_unpack(bk, b0, b1);
-        packed[i / 4] |= bucket_code(x0, b0, sb) << (8 * (i % 4));
-        packed[i / 4] |= bucket_code(x1, b1, sb) << (8 * (i % 4) + 4);
+      for (int h = 0; h < kQuantChunks; ++h) {
+        uint32_t cw[8];
+        float d[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint64_t w = f2_pack(v[8 * h + 2 * i], v[8 * h + 2 * i + 1]);
+          const uint64_t q = f2_mul(w, rr);
+          const uint64_t e = f2_fma(q, nm, w);  // w - q m, exact
+          const uint64_t x = f2_fma(e, rr, q);  // fl32(w / m)
+          const uint64_t bk = f2_fma(x, kscale, kbias);
+          float b0, b1;
+          f2_unpack(bk, b0, b1);
+          const uint32_t i0 = bucket_index(b0), i1 = bucket_index(b1);
+          cw[2 * i] = sb.code[i0];
+          cw[2 * i + 1] = sb.code[i1];
+          const uint64_t df = f2_add(x, f2_pack(sb.nthr[i0], sb.nthr[i1]));  // fl32(x - thr)
+          f2_unpack(df, d[2 * i], d[2 * i + 1]);
+        }
+        packed[h] = pack_codes8(cw, d);
       }
     } else {  // absmax zero or below 2^-64: plain IEEE division (x = 0 for a zero block)
 #pragma unroll

@@ -11,8 +11,7 @@
 //   (split c % splits) and the row groups c / splits, + cps, ... of it. It stages the
 //   split's columns of X in shared memory once (padded so that the MMA operand loads are
 //   conflict-free), then
-//   * its weight warps each take one group of 16 (M <= 8) or 32 weight rows over the
-//     split: lanes stream 32 bytes of packed codes per row with 128-bit loads (the next
+//   * its weight warps each take one group of 16 weight rows over the split: lanes stream 32 bytes of packed codes per row with 128-bit loads (the next
 //     256-wide unit while the current one is expanded), double-dequantize them straight
 //     into the A fragments of mma.m16n8k16 (X is the B operand; the dequantized weight
 //     never leaves registers) and store the split's partial sums; the last warp of a row
@@ -32,13 +31,13 @@
 namespace qlora {
 namespace {
 
-// Weight rows per warp: one 16-row MMA group for M <= 8, two for M > 8 (the X fragments
-// of 16 tokens are then shared by twice the rows).
-__host__ __device__ constexpr int rows_per_warp(bool tall) { return tall ? 32 : 16; }
-// One CTA per SM: 16 warps at <= 128 registers (M <= 8) or 8 at <= 255 (M > 8); the last
-// warp of a CTA computes its share of T, the others take weight rows.
-__host__ __device__ constexpr int dec_threads(bool tall) { return tall ? 256 : 512; }
-__host__ __device__ constexpr int weight_warps(bool tall) { return dec_threads(tall) / 32 - 1; }
+// Weight rows per warp task: one 16-row MMA group (for M > 8 the warp issues a second MMA
+// per step for tokens 8..15 with the same A fragments).
+constexpr int kRowsPerWarp = 16;
+// One CTA per SM: 16 warps at <= 128 registers; the last warp of a CTA computes its share
+// of T, the others take weight rows.
+constexpr int kDecThreads = 512;
+constexpr int kWeightWarps = kDecThreads / 32 - 1;
 constexpr int kUnitK = 256;  // K covered by one warp step (4 lanes x 64)
 
 // X stage: each 64-column block of a token's row takes 128 bytes at a 144-byte stride,
@@ -72,11 +71,11 @@ struct DecodeArgs {
   int r;
   float scale;
   int splits, units_per, nunits;  // K is cut into `splits` ranges of `units_per` 256-units
-  int row_groups;                 // groups of rows_per_warp(M > 8) rows of W
+  int row_groups;                 // groups of kRowsPerWarp rows of W
   int cps;                        // CTAs per split (grid = splits x cps)
   int xs_tok;                     // bytes between token rows of the X stage
   int xs_bytes;                   // bytes of the X stage (M x xs_tok)
-  float* part;      // [splits][row_groups][M][rows per warp] partial sums of X W_hat^T
+  float* part;      // [splits][row_groups][M][kRowsPerWarp] partial sums of X W_hat^T
   float* T;         // [M][r] T = X A (zeroed by k_decode_prep)
   float* T_save;    // optional copy of T for the backward pass
   int* counters;    // [row_groups] warps of the group that have stored their partials
@@ -188,21 +187,19 @@ __device__ __forceinline__ void pair_decode8(uint32_t w, uint32_t lane_bits, uin
 
 // Packed codes and block constants of one unit for this lane (rows beyond N are clamped
 // and K beyond the matrix is clamped; their scale is forced to zero later).
-template <int kGroups>
 struct UnitCodes {
-  uint4 q[kGroups][2][2];
-  uint32_t e2[kGroups][2];
-  float e1[kGroups][2];
+  uint4 q[2][2];  // [row g / g + 8][first / second 16 bytes]
+  uint32_t e2[2];
+  float e1[2];
 };
 
 // This lane's weight rows (clamped to the last row; their scale is forced to zero later)
 // as one base and 32-bit offsets from it, computed once per task.
-template <int kGroups>
 struct RowBases {
-  const uint8_t* code;           // codes of the first row
-  int64_t blk;                   // index of the first row's first 64-block
-  int coff[kGroups][2];          // code byte offset of each row from `code`
-  int boff[kGroups][2];          // block offset of each row from `blk`
+  const uint8_t* code;  // codes of row g
+  int64_t blk;          // index of row g's first 64-block
+  int coff;             // code byte offset of row g + 8 from `code`
+  int boff;             // block offset of row g + 8 from `blk`
 };
 
 // Streamed 16-byte load of packed codes that also asks L2 to fetch the whole 256-byte
@@ -215,82 +212,56 @@ __device__ __forceinline__ uint4 ldg_codes(const void* p) {
   return v;
 }
 
-template <int kGroups>
-__device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases<kGroups>& rb, int u,
-                                          int t, int bpr, UnitCodes<kGroups>& c) {
+__device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases& rb, int u, int t,
+                                          int bpr, UnitCodes& c) {
   const int kbi = min(u * (kUnitK / 64) + t, bpr - 1);  // 64-block of this lane (clamped)
   const uint8_t* base = rb.code + kbi * 32;
   const int64_t jb = rb.blk + kbi;
 #pragma unroll
-  for (int q = 0; q < kGroups; ++q)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint8_t* p = base + rb.coff[q][h];
-      c.q[q][h][0] = ldg_codes(p);
-      c.q[q][h][1] = ldg_codes(p + 16);
-      const int64_t j = jb + rb.boff[q][h];
-      c.e2[q][h] = __ldg(a.c2 + j);
-      c.e1[q][h] = __ldg(a.c1 + (j >> 8));
-    }
-}
-
-// One unit: bit (2 q + h) of kPermMask selects the permute table for the row block of
-// rows (q, h); the others go through the pair table. xs0 / xs1: this lane's tokens' rows
-// of the X stage.
-template <bool kTall, int CB, uint32_t kPermMask, int kGroups = kTall ? 2 : 1>
-__device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int u0,
-                                             int nblk, int g, int t, const UnitCodes<kGroups>& c,
-                                             const float* t8, float mean, uint32_t lane_bits,
-                                             uint32_t xs0, uint32_t xs1,
-                                             float (&acc)[kGroups][kTall ? 2 : 1][4]) {
-  const int blk = (u - u0) * (kUnitK / 64) + t;  // block of the split
-  const bool kv = blk < nblk;                    // false past the end of K
-  const uint32_t xoff = static_cast<uint32_t>(min(blk, nblk - 1) * kXBlkStride);
-#pragma unroll
-  for (int q = 0; q < kGroups; ++q) {
-    Nf4Lut lut[2];
-    uint64_t s2[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const bool live = kv && (rbase + q * 16 + g + 8 * h) < a.N;
-      const float s = live ? block_scale_tab(t8, c.e2[q][h], c.e1[q][h], mean) : 0.f;
-      if ((kPermMask >> (2 * q + h)) & 1u)
-        build_lut<CB>(s, lut[h]);
-      else
-        s2[h] = f2_pack(s, s);
-    }
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      // this word's 8 columns of X for the lane's token(s), just before their MMAs
-      const uint4 xa = lds_b128(xs0 + xoff + 16 * w);
-      const uint4 xb = kTall ? lds_b128(xs1 + xoff + 16 * w) : xa;
-      uint32_t o0[4], o1[4];
-      const uint32_t w0 = w < 4 ? (&c.q[q][0][0].x)[w] : (&c.q[q][0][1].x)[w - 4];
-      const uint32_t w1 = w < 4 ? (&c.q[q][1][0].x)[w] : (&c.q[q][1][1].x)[w - 4];
-      if ((kPermMask >> (2 * q)) & 1u)
-        lut_decode8(w0, lut[0], o0);
-      else
-        pair_decode8(w0, lane_bits, s2[0], o0);
-      if ((kPermMask >> (2 * q + 1)) & 1u)
-        lut_decode8(w1, lut[1], o1);
-      else
-        pair_decode8(w1, lane_bits, s2[1], o1);
-      mma_bf16_16816(acc[q][0], o0[0], o1[0], o0[1], o1[1], xa.x, xa.y);
-      mma_bf16_16816(acc[q][0], o0[2], o1[2], o0[3], o1[3], xa.z, xa.w);
-      if (kTall) {
-        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
-        mma_bf16_16816(acc[q][kTall ? 1 : 0], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
-      }
-    }
+  for (int h = 0; h < 2; ++h) {
+    const uint8_t* p = base + (h ? rb.coff : 0);
+    c.q[h][0] = ldg_codes(p);
+    c.q[h][1] = ldg_codes(p + 16);
+    const int64_t j = jb + (h ? rb.boff : 0);
+    c.e2[h] = __ldg(a.c2 + j);
+    c.e1[h] = __ldg(a.c1 + (j >> 8));
   }
 }
 
-// Which row blocks of a pair of units take the permute table: M <= 8, row g + 8 of every
-// unit (one half); M > 8, row g + 8 of the first 16-row group in even units and of the
-// second in odd ones (one quarter).
-template <bool kTall> struct PermMasks;
-template <> struct PermMasks<false> { static constexpr uint32_t even = 2u, odd = 2u; };
-template <> struct PermMasks<true> { static constexpr uint32_t even = 2u, odd = 8u; };
+// One unit: the codes of row g go through the pair table, those of row g + 8 through the
+// permute table (half the weights each). xs0 / xs1: this lane's tokens' rows of the X
+// stage (tokens g and, for M > 8, g + 8).
+template <bool kTall, int CB>
+__device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int u0,
+                                             int nblk, int g, int t, const UnitCodes& c,
+                                             const float* t8, float mean, uint32_t lane_bits,
+                                             uint32_t xs0, uint32_t xs1,
+                                             float (&acc)[kTall ? 2 : 1][4]) {
+  const int blk = (u - u0) * (kUnitK / 64) + t;  // block of the split
+  const bool kv = blk < nblk;                    // false past the end of K
+  const uint32_t xoff = static_cast<uint32_t>(min(blk, nblk - 1) * kXBlkStride);
+  const bool live0 = kv && (rbase + g) < a.N, live1 = kv && (rbase + g + 8) < a.N;
+  const float s0 = live0 ? block_scale_tab(t8, c.e2[0], c.e1[0], mean) : 0.f;
+  const float s1 = live1 ? block_scale_tab(t8, c.e2[1], c.e1[1], mean) : 0.f;
+  const uint64_t s2 = f2_pack(s0, s0);
+  Nf4Lut lut;
+  build_lut<CB>(s1, lut);
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    // this word's 8 columns of X for the lane's token(s), just before their MMAs
+    const uint4 xa = lds_b128(xs0 + xoff + 16 * w);
+    uint32_t o0[4], o1[4];
+    pair_decode8(w < 4 ? (&c.q[0][0].x)[w] : (&c.q[0][1].x)[w - 4], lane_bits, s2, o0);
+    lut_decode8(w < 4 ? (&c.q[1][0].x)[w] : (&c.q[1][1].x)[w - 4], lut, o1);
+    mma_bf16_16816(acc[0], o0[0], o1[0], o0[1], o1[1], xa.x, xa.y);
+    mma_bf16_16816(acc[0], o0[2], o1[2], o0[3], o1[3], xa.z, xa.w);
+    if (kTall) {
+      const uint4 xb = lds_b128(xs1 + xoff + 16 * w);
+      mma_bf16_16816(acc[kTall ? 1 : 0], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
+      mma_bf16_16816(acc[kTall ? 1 : 0], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
+    }
+  }
+}
 
 // Bounded wait of a finisher for every T share of the call (lane 0 spins; false on
 // timeout, after recording it).
@@ -317,8 +288,6 @@ template <bool kTall, int CB>
 __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, int split,
                                                    int nblk, int lane, const float* t8,
                                                    uint32_t lane_bits, uint32_t xs) {
-  constexpr int kGroups = kTall ? 2 : 1;
-  constexpr int kRowsPerWarp = rows_per_warp(kTall);
   const int g = lane >> 2, t = lane & 3;
   const int u0 = split * a.units_per;
   const int u1 = min(a.nunits, u0 + a.units_per);
@@ -327,38 +296,31 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   const uint32_t xs0 = xs + static_cast<uint32_t>(min(g, static_cast<int>(a.M) - 1) * a.xs_tok);
   const uint32_t xs1 =
       xs + static_cast<uint32_t>(min(g + 8, static_cast<int>(a.M) - 1) * a.xs_tok);
-  float acc[kGroups][kTall ? 2 : 1][4];
+  float acc[kTall ? 2 : 1][4];
 #pragma unroll
-  for (int q = 0; q < kGroups; ++q)
+  for (int h = 0; h < (kTall ? 2 : 1); ++h)
 #pragma unroll
-    for (int h = 0; h < (kTall ? 2 : 1); ++h)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[q][h][i] = 0.f;
+    for (int i = 0; i < 4; ++i) acc[h][i] = 0.f;
 
   const int bpr = static_cast<int>(a.K / 64);
-  RowBases<kGroups> rb;
+  RowBases rb;
   const int64_t row_g = lmin(rbase + g, a.N - 1);
   rb.code = a.codes + row_g * (a.K / 2);
   rb.blk = row_g * bpr;
-#pragma unroll
-  for (int q = 0; q < kGroups; ++q)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int dr = static_cast<int>(lmin(rbase + q * 16 + g + 8 * h, a.N - 1) - row_g);
-      rb.coff[q][h] = dr * static_cast<int>(a.K / 2);
-      rb.boff[q][h] = dr * bpr;
-    }
+  const int dr = static_cast<int>(lmin(rbase + g + 8, a.N - 1) - row_g);
+  rb.coff = dr * static_cast<int>(a.K / 2);
+  rb.boff = dr * bpr;
   // two code buffers: the loads of unit u + 1 are in flight while unit u is expanded
-  UnitCodes<kGroups> cb0, cb1;
+  UnitCodes cb0, cb1;
   if (u0 < u1) load_unit(a, rb, u0, t, bpr, cb0);
   for (int u = u0; u < u1; u += 2) {
     if (u + 1 < u1) load_unit(a, rb, u + 1, t, bpr, cb1);
-    compute_unit<kTall, CB, PermMasks<kTall>::even>(a, rbase, u, u0, nblk, g, t, cb0, t8, mean,
-                                                     lane_bits, xs0, xs1, acc);
+    compute_unit<kTall, CB>(a, rbase, u, u0, nblk, g, t, cb0, t8, mean, lane_bits, xs0, xs1,
+                            acc);
     if (u + 1 < u1) {
       if (u + 2 < u1) load_unit(a, rb, u + 2, t, bpr, cb0);
-      compute_unit<kTall, CB, PermMasks<kTall>::odd>(a, rbase, u + 1, u0, nblk, g, t, cb1, t8,
-                                                      mean, lane_bits, xs0, xs1, acc);
+      compute_unit<kTall, CB>(a, rbase, u + 1, u0, nblk, g, t, cb1, t8, mean, lane_bits, xs0,
+                              xs1, acc);
     }
   }
 
@@ -367,15 +329,13 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   const int64_t M = a.M;
   float* pp = a.part + (static_cast<int64_t>(split) * a.row_groups + rg) * M * kRowsPerWarp;
 #pragma unroll
-  for (int q = 0; q < kGroups; ++q)
+  for (int hm = 0; hm < (kTall ? 2 : 1); ++hm)
 #pragma unroll
-    for (int hm = 0; hm < (kTall ? 2 : 1); ++hm)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int rl = q * 16 + g + 8 * (i >> 1);
-        const int m = 8 * hm + 2 * t + (i & 1);
-        if (m < M) pp[m * kRowsPerWarp + rl] = acc[q][hm][i];
-      }
+    for (int i = 0; i < 4; ++i) {
+      const int rl = g + 8 * (i >> 1);
+      const int m = 8 * hm + 2 * t + (i & 1);
+      if (m < M) pp[m * kRowsPerWarp + rl] = acc[hm][i];
+    }
 
   // the counters come zeroed from k_decode_prep
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -520,7 +480,7 @@ __device__ __forceinline__ void decode_t_share(const uint16_t* __restrict__ A, f
 
 // ---------------------------------------------------------------- the main kernel
 template <bool kTall, int CB>  // kTall: M > 8 (tokens 8..15 in the upper fragment rows); CB: codebook
-__global__ void __launch_bounds__(dec_threads(kTall), 1) k_decode_gemv(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, 1) k_decode_gemv(const DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t dsm[];
   const uint32_t sbase = smem_u32(dsm);
   const uint32_t tab = (sbase + kPairTabBytes - 1) & ~(kPairTabBytes - 1);
@@ -587,7 +547,7 @@ __global__ void __launch_bounds__(dec_threads(kTall), 1) k_decode_gemv(const Dec
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kW = weight_warps(kTall);
+  constexpr int kW = kWeightWarps;
   if (warp == kW) {
     // this CTA's share of the split's rows of A
     const int64_t share = ((kend - kbeg + a.cps - 1) / a.cps + 7) / 8 * 8;
@@ -614,8 +574,7 @@ int x_stage_tok(int units_per) {
 }
 
 size_t part_bytes(const DecodePlan& p, const LinearShape& s) {
-  return align_up(static_cast<size_t>(p.splits) * p.row_groups * s.M * rows_per_warp(s.M > 8) * 4,
-                  256);
+  return align_up(static_cast<size_t>(p.splits) * p.row_groups * s.M * kRowsPerWarp * 4, 256);
 }
 size_t t_bytes(const LinearShape& s) { return align_up(static_cast<size_t>(s.M) * s.r * 4, 256); }
 size_t counter_bytes(const DecodePlan& p) {
@@ -636,10 +595,8 @@ size_t decode_scratch_bytes(const DecodePlan& p, const LinearShape& s) {
 DecodePlan plan_decode(const LinearShape& s, size_t max_scratch = ~size_t{0}) {
   DecodePlan p;
   p.nunits = static_cast<int>((s.K + kUnitK - 1) / kUnitK);
-  const bool tall = s.M > 8;
-  const int rows = rows_per_warp(tall);
-  p.row_groups = static_cast<int>((s.N + rows - 1) / rows);
-  const int64_t W = weight_warps(tall);
+  p.row_groups = static_cast<int>((s.N + kRowsPerWarp - 1) / kRowsPerWarp);
+  const int64_t W = kWeightWarps;
   const int64_t sms = num_sms();
   const int64_t max_splits =
       std::max<int64_t>(1, std::min<int64_t>(p.nunits, s.K / (16 * std::max<int64_t>(1, s.M))));
@@ -731,7 +688,7 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   if (e != cudaSuccess) return cuda_status(e);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.splits * p.cps));
-  cfg.blockDim = dim3(dec_threads(s.M > 8));
+  cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = dec_smem_bytes(a.xs_bytes, s.r);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

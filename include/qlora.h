@@ -266,13 +266,13 @@ qlora_status qlora_linear_fwd(const uint16_t *X, int64_t M, qlora_nf4_weight w,
  *   Scratch: a fixed 4 MiB array in device memory inside this library, which every
  *   GPU that loads the library holds until the process exits. A call splits K into
  *   s ranges and needs
- *       align256(s * ceil(N / R) * R * M * 4) + align256(M * r * 4)
- *       + align256(4 * ceil(N / R) + 4)  bytes,   R = 16 rows (M <= 8) or 32 (M > 8),
+ *       align256(s * ceil(N / 16) * 16 * M * 4) + align256(M * r * 4)
+ *       + align256(4 * ceil(N / 16) + 4)  bytes
  *   for fp32 partial sums, T and the arrival counters. It takes the number of splits
  *   its planner prefers when that fits, else the best that fits. The fewest splits it can
- *   run is ceil(ceil(K / 256) / u) with u = 85, 42, 28, 21, 17, 14, 12, 10, 9, 8, 7, 7,
- *   6, 5, 5, 5 for M = 1 .. 16 (a split's columns of X are staged in 48 KB of shared
- *   memory); when even that does not fit the array, the call is rejected with
+ *   run is ceil(ceil(K / 256) / u) with u = 142, 71, 47, 35, 28, 23, 20, 17, 15, 14, 12,
+ *   11, 10, 10, 9, 8 for M = 1 .. 16 (a split's columns of X are staged in at most 80 KB
+ *   of shared memory); when even that does not fit the array, the call is rejected with
  *   QLORA_ERR_WORKSPACE (qlora_last_error() gives the shape), and M > 16 with
  *   QLORA_ERR_SHAPE. Argument errors are checked as in qlora_linear_fwd and give its
  *   status codes.

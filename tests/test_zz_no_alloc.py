@@ -65,13 +65,13 @@ def test_static_scratch_decode_matches_workspace_path(M, N, K, r):
 
 
 def test_static_scratch_with_fewer_k_splits():
-    """M = 8 tokens on a 16384 x 16384 weight: the usual plan's fp32 partial sums (8 K
-    splits) do not fit the 4 MiB array, so the entry point plans with 7; the results
-    must not change."""
+    """M = 16 tokens on an 8192 x 11008 weight: the usual plan's fp32 partial sums (8 K
+    splits, 4.2 MB) do not fit the 4 MiB array, so the entry point plans with 7; the
+    results must not change."""
     need_gpu()
     g = torch.Generator(device="cuda")
     g.manual_seed(7)
-    M, N, K, r, scale = 8, 16384, 16384, 16, 2.0
+    M, N, K, r, scale = 16, 8192, 11008, 16, 2.0
     q = qlora.qlora_quantize_nf4_dq((torch.randn(N, K, generator=g, device="cuda") * 0.02)
                                     .to(torch.bfloat16))
     X = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
