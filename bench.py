@@ -720,6 +720,24 @@ def profile_dequant(device, warmup, steps, n=4096, k=11008):
     torch.cuda.synchronize()
 
 
+def profile_quant(device, warmup, steps):
+    """The quantization (NF4 codes and double-quantized constants, bf16 in) of the three
+    Llama-7B weight shapes, --steps passes after --warmup, for ncu captures."""
+    from bit_nf4_quantized_unpack_b200 import qlora
+    g = torch.Generator(device=device)
+    g.manual_seed(9)
+    Ws, Qs, wss = [], [], []
+    for n, k in [(4096, 4096), (4096, 11008), (11008, 4096)]:
+        Ws.append((torch.randn(n, k, generator=g, device=device) * 0.02).to(torch.bfloat16))
+        Qs.append(qlora.NF4Weight.empty(n, k, device))
+        wss.append(torch.empty(qlora.qlora_quantize_workspace_size(n, k), dtype=torch.uint8,
+                               device=device))
+    for _ in range(warmup + steps):
+        for W, q, ws in zip(Ws, Qs, wss):
+            qlora.qlora_quantize_nf4_dq(W, out=q, workspace=ws)
+    torch.cuda.synchronize()
+
+
 def profile_optimizer(device, warmup, steps, n=40_000_000, state_bits=8):
     """The paged AdamW step (8-bit states by default) on n LoRA-sized fp32 parameters, for
     ncu captures (0.72 GB moved per 8-bit step, beyond L2)."""
@@ -757,6 +775,9 @@ def main():
                          "self-contained case for profiler captures")
     ap.add_argument("--profile-dequant", action="store_true",
                     help="only run the double dequantization of a 4096x11008 weight (for ncu)")
+    ap.add_argument("--profile-quant", action="store_true",
+                    help="only run the quantization of the three Llama-7B weight shapes "
+                         "--steps times (for ncu)")
     ap.add_argument("--profile-optimizer", action="store_true",
                     help="only run the 8-bit AdamW step on 40M parameters (for ncu)")
     ap.add_argument("--profile-merge", action="store_true",
@@ -787,6 +808,9 @@ def main():
     scale = ALPHA / RANK_R
     if args.profile_merge:
         profile_merge(device, args.warmup, args.steps)
+        return
+    if args.profile_quant:
+        profile_quant(device, args.warmup, args.steps)
         return
     if args.profile_optimizer:
         profile_optimizer(device, args.warmup, args.steps)

@@ -49,7 +49,10 @@ constexpr int kXStageMax = 80 * 1024;
 constexpr uint32_t kPairTabBytes = 65536;
 // A T share stages up to kTChunkRows rows of A at a time.
 constexpr int kTChunkRows = 64;
+constexpr int kPrefetchRank = 16;  // ranks of B a finisher fetches before it knows it is one
 __host__ __device__ constexpr int a_chunk_bytes(int r) { return kTChunkRows * r * 2; }
+// the finishers stage T (M x r fp32) in the same area
+static_assert(4 * kDecodeMaxM <= 2 * kTChunkRows, "T fits the A-chunk area");
 // Dynamic shared memory: the 64 KB pair table at a 64 KB-aligned address (up to 64 KB of
 // alignment slack below it), the X stage, T8 (1 KB) and the A chunk; the last three are
 // placed in the slack when they fit there, else above the table.
@@ -125,6 +128,16 @@ __device__ __forceinline__ uint2 lds_b64x2(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
+}
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
@@ -287,7 +300,8 @@ __device__ __forceinline__ bool wait_t_complete(const DecodeArgs& a, int lane) {
 template <bool kTall, int CB>
 __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, int split,
                                                    int nblk, int lane, const float* t8,
-                                                   uint32_t lane_bits, uint32_t xs) {
+                                                   uint32_t lane_bits, uint32_t xs,
+                                                   uint32_t ts) {
   const int g = lane >> 2, t = lane & 3;
   const int u0 = split * a.units_per;
   const int u1 = min(a.nunits, u0 + a.units_per);
@@ -337,62 +351,96 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
       if (m < M) pp[m * kRowsPerWarp + rl] = acc[hm][i];
     }
 
-  // the counters come zeroed from k_decode_prep
+  // The finisher's operands that are ready now: B[j][row] for the first kPrefetchRank j of
+  // this lane's row (lane (rl, half) = (lane % 16, lane / 16)), as bf16 pairs; in flight
+  // while the arrival is counted.
+  const int rl = lane & 15, half = lane >> 4;
+  const int64_t row = rbase + rl;
+  const int64_t rowc = lmin(row, a.N - 1);
+  const int r = a.r;
+  uint32_t bq[kPrefetchRank / 2];
+#pragma unroll
+  for (int i = 0; i < kPrefetchRank / 2; ++i)
+    if (2 * i < r)
+      bq[i] = static_cast<uint32_t>(__ldg(a.B + (2 * i) * a.N + rowc)) |
+              (static_cast<uint32_t>(__ldg(a.B + (2 * i + 1) * a.N + rowc)) << 16);
+
+  // Arrival: the warp's partial sums are ordered before the count (release), and the
+  // last warp of the row group sees every other warp's (acquire). The counters come
+  // zeroed from k_decode_prep.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __threadfence();
   __syncwarp();
   int last = 0;
-  if (lane == 0) last = atomicAdd(a.counters + rg, 1) == a.splits - 1;
+  if (lane == 0) last = atom_add_acq_rel_gpu(a.counters + rg, 1) == a.splits - 1;
   last = __shfl_sync(0xFFFFFFFFu, last, 0);
   if (!last) return;
-  __threadfence();  // the other warps' partial sums are visible from here on
   if (!wait_t_complete(a, lane)) return;
+  __syncwarp();
 
-  const int64_t row = rbase + lane;
-  if (lane >= kRowsPerWarp || row >= a.N) return;
-  float y[16], lora[16];
+  // T (complete now) into the CTA's A-chunk area of shared memory, by asynchronous copies
+  // in flight with the partial-sum loads below. This CTA's T warp has stopped using the
+  // area (it counted its share in after its last chunk), and every finisher of the CTA
+  // writes the same values there.
+  const int mr = static_cast<int>(M) * r;  // a multiple of 8
+  for (int e = 4 * lane; e < mr; e += 128) cp_async16(ts + 4 * e, a.T + e);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+
+  // the splits' partial sums of tokens m = half, half + 2, ..., added four splits at a
+  // time in a fixed order
+  float y[8];
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    y[m] = 0.f;
-    lora[m] = 0.f;
-  }
+  for (int i = 0; i < 8; ++i) y[i] = 0.f;
   const int64_t sstride = static_cast<int64_t>(a.row_groups) * M * kRowsPerWarp;
-  const float* p0 = a.part + static_cast<int64_t>(rg) * M * kRowsPerWarp + lane;
-  // four splits per step (all their loads in flight), added in a fixed order
+  const float* p0 = a.part + static_cast<int64_t>(rg) * M * kRowsPerWarp + rl;
   int s = 0;
   for (; s + 4 <= a.splits; s += 4) {
 #pragma unroll
-    for (int m = 0; m < 16; ++m)
+    for (int i = 0; i < 8; ++i) {
+      const int m = 2 * i + half;
       if (m < M) {
         const float* q = p0 + s * sstride + m * kRowsPerWarp;
         const float v0 = __ldcg(q), v1 = __ldcg(q + sstride);
         const float v2 = __ldcg(q + 2 * sstride), v3 = __ldcg(q + 3 * sstride);
-        y[m] += (v0 + v1) + (v2 + v3);
+        y[i] += (v0 + v1) + (v2 + v3);
       }
+    }
   }
   for (; s < a.splits; ++s) {
 #pragma unroll
-    for (int m = 0; m < 16; ++m)
-      if (m < M) y[m] += __ldcg(p0 + s * sstride + m * kRowsPerWarp);
+    for (int i = 0; i < 8; ++i) {
+      const int m = 2 * i + half;
+      if (m < M) y[i] += __ldcg(p0 + s * sstride + m * kRowsPerWarp);
+    }
   }
-  const int r = a.r;
-  for (int j = 0; j < r; j += 4) {
-    float bv[4];
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();
+
+  if (row >= a.N) return;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) bv[i] = bf16_to_f32(__ldg(a.B + (j + i) * a.N + row));
+  for (int i = 0; i < 8; ++i) {
+    const int m = 2 * i + half;
+    if (m < M) {
+      float lora = 0.f;
 #pragma unroll
-    for (int m = 0; m < 16; ++m)
-      if (m < M) {
-        const float4 tv = __ldcg(reinterpret_cast<const float4*>(a.T + m * r + j));
-        lora[m] = fmaf(tv.x, bv[0], lora[m]);
-        lora[m] = fmaf(tv.y, bv[1], lora[m]);
-        lora[m] = fmaf(tv.z, bv[2], lora[m]);
-        lora[m] = fmaf(tv.w, bv[3], lora[m]);
+      for (int j4 = 0; j4 < kPrefetchRank / 4; ++j4)
+        if (4 * j4 < r) {
+          const uint4 tv = lds_b128(ts + static_cast<uint32_t>((m * r + 4 * j4) * 4));
+          const uint32_t b01 = bq[2 * j4], b23 = bq[2 * j4 + 1];
+          lora = fmaf(__uint_as_float(tv.x), bf16_to_f32(b01 & 0xFFFFu), lora);
+          lora = fmaf(__uint_as_float(tv.y), bf16_to_f32(b01 >> 16), lora);
+          lora = fmaf(__uint_as_float(tv.z), bf16_to_f32(b23 & 0xFFFFu), lora);
+          lora = fmaf(__uint_as_float(tv.w), bf16_to_f32(b23 >> 16), lora);
+        }
+      for (int j = kPrefetchRank; j < r; j += 4) {  // ranks above kPrefetchRank
+        const uint4 tv = lds_b128(ts + static_cast<uint32_t>((m * r + j) * 4));
+        lora = fmaf(__uint_as_float(tv.x), bf16_to_f32(__ldg(a.B + j * a.N + rowc)), lora);
+        lora = fmaf(__uint_as_float(tv.y), bf16_to_f32(__ldg(a.B + (j + 1) * a.N + rowc)), lora);
+        lora = fmaf(__uint_as_float(tv.z), bf16_to_f32(__ldg(a.B + (j + 2) * a.N + rowc)), lora);
+        lora = fmaf(__uint_as_float(tv.w), bf16_to_f32(__ldg(a.B + (j + 3) * a.N + rowc)), lora);
       }
+      a.Y[m * a.N + row] = bf16_bits_rn(y[i] + a.scale * lora);
+    }
   }
-#pragma unroll
-  for (int m = 0; m < 16; ++m)
-    if (m < M) a.Y[m * a.N + row] = bf16_bits_rn(y[m] + a.scale * lora[m]);
 }
 
 // ---------------------------------------------------------------- T = X A
@@ -458,22 +506,22 @@ __device__ __forceinline__ void decode_t_share(const uint16_t* __restrict__ A, f
       if (m < M)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[m][c] += __shfl_xor_sync(0xFFFFFFFFu, acc[m][c], off);
-  // T was zeroed by k_decode_prep
+  // T was zeroed by k_decode_prep; one 4-wide reduction per token and column quad (all
+  // CTAs add into the same M x r floats, so fewer, wider operations queue less at L2)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (jlive && kq == 0 && k0 < k1) {
 #pragma unroll
     for (int m = 0; m < 16; ++m)
-      if (m < M)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) atomicAdd(T + m * r + j0 + c, acc[m][c]);
+      if (m < M) red_add_v4(T + m * r + j0, acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
   }
-  __threadfence();
+  // the share is counted after its additions (release); the last share's warp sees all
+  // of T (acquire) and copies it out
   __syncwarp();
   int last = 0;
-  if (lane == 0) last = atomicAdd(t_count, 1) == shares - 1;
+  if (lane == 0) last = atom_add_acq_rel_gpu(t_count, 1) == shares - 1;
   last = __shfl_sync(0xFFFFFFFFu, last, 0);
   if (last && T_save) {
-    __threadfence();
+    __syncwarp();
     for (int e = lane; e < M * r; e += 32) T_save[e] = __ldcg(T + e);
   }
 }
@@ -560,7 +608,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode_gemv(const DecodeArgs
   const uint32_t lane_bits =
       static_cast<uint32_t>((lane & 15) * 8 + CB * 128) | (tab & 0x00FF0000u);
   for (int rg = cidx + a.cps * warp; rg < a.row_groups; rg += a.cps * kW)
-    decode_weight_task<kTall, CB>(a, rg, split, nblk, lane, t8, lane_bits, xs);
+    decode_weight_task<kTall, CB>(a, rg, split, nblk, lane, t8, lane_bits, xs, sbase + as_off);
 }
 
 // ---------------------------------------------------------------- host side

@@ -185,8 +185,9 @@ size_t qlora_quantize_workspace_size(int64_t n_out, int64_t k_in);
  * Errors: QLORA_ERR_SHAPE unless n_out >= 1, k_in >= 64, k_in % 64 == 0 and
  *         n_out * k_in <= 2^37 (at most 2^31 blocks);
  *         QLORA_ERR_INVALID_ARG for a NULL pointer or unknown dtype.
- * The workspace also holds the 256 integer sums of the mean; the call clears them
- * with cudaMemsetAsync on `stream` before the kernels run.
+ * The workspace also holds, after the absmax array, the accumulators of the mean (an
+ * fp64 sum, the exponent range and a CTA count: four 64-bit words); the call clears
+ * them with a small kernel on `stream` before the level-1 kernel adds to them.
  * Inputs must be finite.
  */
 qlora_status qlora_quantize_nf4_dq(const void *W, qlora_dtype w_dtype, int64_t n_out,

@@ -176,7 +176,8 @@ def test_graph_replay_matches_eager():
 def test_launch_count_per_call():
     """The library counts its own kernels: 3 per GEMM-path forward (T, its finalize, the
     fused GEMM), 5 per backward with T saved (G, its finalize, the fused dX GEMM, the
-    grouped dA/dB GEMM and its finalize), 2 per decode-path forward."""
+    grouped dA/dB GEMM and its finalize), 2 per decode-path forward, 3 per quantization
+    (clearing its accumulators, level 1, the double quantization)."""
     case = inputs.linear_case(51, 300, 256, 512, 16, alpha=32)
     q = qlora.qlora_quantize_nf4_dq(to_dev_bf16(case["W"]))
     Xd, Ad, Bd, dYd = (to_dev_bf16(case[k]) for k in ("X", "A", "B", "dY"))
@@ -187,5 +188,7 @@ def test_launch_count_per_call():
     n2 = qlora.qlora_launch_count()
     qlora.qlora_linear_fwd(Xd[:4].contiguous(), q, Ad, Bd, case["scale"])
     n3 = qlora.qlora_launch_count()
+    qlora.qlora_quantize_nf4_dq(to_dev_bf16(case["W"]))
+    n4 = qlora.qlora_launch_count()
     torch.cuda.synchronize()
-    assert (n1 - n0, n2 - n1, n3 - n2) == (3, 5, 2)
+    assert (n1 - n0, n2 - n1, n3 - n2, n4 - n3) == (3, 5, 2, 3)
