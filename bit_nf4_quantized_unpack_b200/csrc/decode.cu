@@ -5,8 +5,10 @@
 //                                           alpha/r from page "quantization", minnong511)
 //
 // Two launches per call:
-// k_decode_prep: zeroes T and the arrival counters of the call (one small CTA; it lets the
-//   main kernel launch at once).
+// k_decode_prep: zeroes T and the arrival counters of the call. It is a programmatic
+//   dependent of whatever ran before on the stream (it launches while that kernel drains
+//   and waits for it to complete before it writes), and it lets the main kernel launch at
+//   once.
 // k_decode_gemv (its programmatic dependent): one CTA per SM. CTA c owns one K split
 //   (split c % splits) and the row groups c / splits, + cps, ... of it. It stages the
 //   split's columns of X in shared memory once (padded so that the MMA operand loads are
@@ -148,9 +150,11 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 // ---------------------------------------------------------------- call set-up
 __global__ void __launch_bounds__(256) k_decode_prep(float* T, int mr, int* counters, int nc,
                                                      int* t_count) {
-  // the main kernel may launch now; it waits for this grid before it touches T or the
-  // counters
+  // the main kernel may launch now (it waits for this grid before it reads its inputs);
+  // this grid waits for the kernel before it (which may still read T or the counters of
+  // the previous call) before it writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int stride = gridDim.x * blockDim.x;
   const int i0 = blockIdx.x * blockDim.x + threadIdx.x;
   for (int i = i0; i < mr; i += stride) T[i] = 0.f;
@@ -368,7 +372,6 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   // Arrival: the warp's partial sums are ordered before the count (release), and the
   // last warp of the row group sees every other warp's (acquire). The counters come
   // zeroed from k_decode_prep.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncwarp();
   int last = 0;
   if (lane == 0) last = atom_add_acq_rel_gpu(a.counters + rg, 1) == a.splits - 1;
@@ -508,7 +511,6 @@ __device__ __forceinline__ void decode_t_share(const uint16_t* __restrict__ A, f
         for (int c = 0; c < 4; ++c) acc[m][c] += __shfl_xor_sync(0xFFFFFFFFu, acc[m][c], off);
   // T was zeroed by k_decode_prep; one 4-wide reduction per token and column quad (all
   // CTAs add into the same M x r floats, so fewer, wider operations queue less at L2)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (jlive && kq == 0 && k0 < k1) {
 #pragma unroll
     for (int m = 0; m < 16; ++m)
@@ -556,6 +558,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode_gemv(const DecodeArgs
   const int nblk = static_cast<int>((kend - kbeg) / 64);  // K is a multiple of 64
   const int M = static_cast<int>(a.M);
 
+  // the next kernel on the stream may launch now (a programmatic dependent waits for this
+  // grid to complete before it reads what it writes)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the constant tables: T8 and the pair table, 256 entries x 16 copies; thread i writes
+  // entry i / 16, copy i % 16 (its low level index (i / 16) % 16 is the same at every step)
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
+  {
+    const float lo = code_level_rt<CB>((threadIdx.x >> 4) & 15);
+    for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
+      const int e = i >> 4, cp = i & 15;
+      *reinterpret_cast<float2*>(tabp + e * 256 + CB * 128 + cp * 8) =
+          make_float2(lo, code_level_rt<CB>(e >> 4));
+    }
+  }
+  // k_decode_prep, and so every kernel before it on the stream, is complete from here on:
+  // X, A and the cleared T and counters are ready
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // X columns [kbeg, kend) of every token, 16 bytes per thread and step: the loads of
   // four steps are issued before their stores
   {
@@ -580,17 +599,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode_gemv(const DecodeArgs
                    v[u]);
         }
       }
-    }
-  }
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) t8[i] = t8_value(i);
-  // 256 entries x 16 copies; thread i writes entry i / 16, copy i % 16 (its low level
-  // index (i / 16) % 16 is the same at every step)
-  {
-    const float lo = code_level_rt<CB>((threadIdx.x >> 4) & 15);
-    for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x) {
-      const int e = i >> 4, cp = i & 15;
-      *reinterpret_cast<float2*>(tabp + e * 256 + CB * 128 + cp * 8) =
-          make_float2(lo, code_level_rt<CB>(e >> 4));
     }
   }
   __syncthreads();
@@ -731,8 +739,19 @@ qlora_status launch_decode(const uint16_t* X, const qlora_nf4_weight& w, const u
   note_launches(2);  // the set-up kernel and the main kernel
   const int mr = static_cast<int>(s.M) * s.r;
   const int prep_ctas = std::max(1, std::min(num_sms(), (p.row_groups + 2047) / 2048));
-  k_decode_prep<<<prep_ctas, 256, 0, st>>>(a.T, mr, a.counters, p.row_groups, a.t_count);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  {
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(static_cast<unsigned>(prep_ctas));
+    pc.blockDim = dim3(256);
+    pc.stream = st;
+    cudaLaunchAttribute pa[1];
+    pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pa[0].val.programmaticStreamSerializationAllowed = 1;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&pc, k_decode_prep, a.T, mr, a.counters, p.row_groups, a.t_count);
+  }
   if (e != cudaSuccess) return cuda_status(e);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.splits * p.cps));
