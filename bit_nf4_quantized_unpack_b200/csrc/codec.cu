@@ -214,9 +214,12 @@ __device__ float exact_mean_f32(const unsigned long long* bins, int64_t n,
 }
 
 // Clears the accumulators of the mean (sum, exponent range, CTA counter) of level 1, its
-// programmatic dependent, which waits for this grid before it adds to them.
+// programmatic dependent, which waits for this grid before it reads its inputs. It is
+// itself a programmatic dependent of the kernel before it on the stream and waits for it
+// to complete before it writes.
 __global__ void __launch_bounds__(32) k_quantize_prep(unsigned long long* acc) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (threadIdx.x < 4) acc[threadIdx.x] = 0ull;
 }
 
@@ -260,6 +263,9 @@ __global__ void __launch_bounds__(kQuantThreads)
   __syncthreads();
   // the double quantization may be scheduled now; it waits for this grid's results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // k_quantize_prep, and every kernel before it on the stream, is complete from here on:
+  // W is ready, the accumulators are cleared, and no earlier call still reads the absmax
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t stride = static_cast<int64_t>(gridDim.x) * per_cta;
   int64_t b = blockIdx.x * per_cta + threadIdx.x / kQuantLanes;
   // this thread's part of the mean: fp64 sum and exponent range of its nonzero absmax
@@ -359,7 +365,6 @@ __global__ void __launch_bounds__(kQuantThreads)
       lo = min(lo, red_lo[i]);
       hi = max(hi, red_hi[i]);
     }
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // the accumulators are cleared
     atomicAdd(reinterpret_cast<double*>(acc_g), cs);
     atomicMax(reinterpret_cast<unsigned int*>(acc_g + 1), 255u - lo);  // cleared to 0
     atomicMax(reinterpret_cast<unsigned int*>(acc_g + 2), hi);
@@ -527,9 +532,19 @@ cudaError_t launch_quantize(const void* W, bool w_bf16, int64_t n, int64_t k, in
   cudaError_t e = w_bf16 ? quant_ctas<uint16_t>(nblocks, &ctas) : quant_ctas<float>(nblocks, &ctas);
   if (e != cudaSuccess) return e;
   note_launches(3);  // clearing, blocks, then the double quantization
-  k_quantize_prep<<<1, 32, 0, st>>>(bins);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  {
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(1);
+    pc.blockDim = dim3(32);
+    pc.stream = st;
+    cudaLaunchAttribute pa[1];
+    pa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pa[0].val.programmaticStreamSerializationAllowed = 1;
+    pc.attrs = pa;
+    pc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&pc, k_quantize_prep, bins);
+    if (e != cudaSuccess) return e;
+  }
   {
     cudaLaunchConfig_t c1cfg = {};
     c1cfg.gridDim = dim3(static_cast<unsigned>(ctas));
