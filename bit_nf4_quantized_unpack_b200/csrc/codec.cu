@@ -429,13 +429,22 @@ __global__ void __launch_bounds__(256)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    // y = fl32(cc / c1): Markstein's correction step on one correctly rounded reciprocal
+    // (as in level 1; exact for c1 >= 2^-64 wherever |y| > 2^-36, and every |y| below
+    // that has the zero entry's code either way), plain IEEE division for smaller c1
+    const bool fast = m >= 0x1p-64f;
+    const float rc = fast ? __frcp_rn(m) : 0.f;
+    auto quot = [&](float c) {
+      if (fast) {
+        const float q = __fmul_rn(c, rc);
+        return __fmaf_rn(__fmaf_rn(-q, m, c), rc, q);
+      }
+      return m > 0.f ? __fdiv_rn(c, m) : 0.f;
+    };
     uint32_t out[2] = {0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      const float y0 = (m > 0.f) ? __fdiv_rn(cc[i], m) : 0.f;
-      const float y1 = (m > 0.f) ? __fdiv_rn(cc[i + 1], m) : 0.f;
-      out[i / 4] |= t8_nearest_codes2(y0, y1, sth) << (8 * (i % 4));
-    }
+    for (int i = 0; i < 8; i += 2)
+      out[i / 4] |= t8_nearest_codes2(quot(cc[i]), quot(cc[i + 1]), sth) << (8 * (i % 4));
     if (j0 + 8 <= nblocks) {
       reinterpret_cast<uint2*>(c2 + j0)[0] = make_uint2(out[0], out[1]);
     } else {
