@@ -246,9 +246,9 @@ __device__ __forceinline__ void load_unit(const DecodeArgs& a, const RowBases& r
 }
 
 // One unit: the codes of row g go through the pair table, those of row g + 8 through the
-// permute table (half the weights each). xs0 / xs1: this lane's tokens' rows of the X
-// stage (tokens g and, for M > 8, g + 8).
-template <bool kTall, int CB>
+// permute table, or through the pair table as well when kAllPair. xs0 / xs1: this lane's
+// tokens' rows of the X stage (tokens g and, for M > 8, g + 8).
+template <bool kTall, int CB, bool kAllPair>
 __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase, int u, int u0,
                                              int nblk, int g, int t, const UnitCodes& c,
                                              const float* t8, float mean, uint32_t lane_bits,
@@ -261,15 +261,19 @@ __device__ __forceinline__ void compute_unit(const DecodeArgs& a, int64_t rbase,
   const float s0 = live0 ? block_scale_tab(t8, c.e2[0], c.e1[0], mean) : 0.f;
   const float s1 = live1 ? block_scale_tab(t8, c.e2[1], c.e1[1], mean) : 0.f;
   const uint64_t s2 = f2_pack(s0, s0);
+  const uint64_t s2b = f2_pack(s1, s1);
   Nf4Lut lut;
-  build_lut<CB>(s1, lut);
+  if (!kAllPair) build_lut<CB>(s1, lut);
 #pragma unroll
   for (int w = 0; w < 8; ++w) {
     // this word's 8 columns of X for the lane's token(s), just before their MMAs
     const uint4 xa = lds_b128(xs0 + xoff + 16 * w);
     uint32_t o0[4], o1[4];
     pair_decode8(w < 4 ? (&c.q[0][0].x)[w] : (&c.q[0][1].x)[w - 4], lane_bits, s2, o0);
-    lut_decode8(w < 4 ? (&c.q[1][0].x)[w] : (&c.q[1][1].x)[w - 4], lut, o1);
+    if (kAllPair)
+      pair_decode8(w < 4 ? (&c.q[1][0].x)[w] : (&c.q[1][1].x)[w - 4], lane_bits, s2b, o1);
+    else
+      lut_decode8(w < 4 ? (&c.q[1][0].x)[w] : (&c.q[1][1].x)[w - 4], lut, o1);
     mma_bf16_16816(acc[0], o0[0], o1[0], o0[1], o1[1], xa.x, xa.y);
     mma_bf16_16816(acc[0], o0[2], o1[2], o0[3], o1[3], xa.z, xa.w);
     if (kTall) {
@@ -328,17 +332,20 @@ __device__ __forceinline__ void decode_weight_task(const DecodeArgs& a, int rg, 
   const int dr = static_cast<int>(lmin(rbase + g + 8, a.N - 1) - row_g);
   rb.coff = dr * static_cast<int>(a.K / 2);
   rb.boff = dr * bpr;
-  // two code buffers: the loads of unit u + 1 are in flight while unit u is expanded
+  // two code buffers: the loads of unit u + 1 are in flight while unit u is expanded.
+  // Which table each row takes: M <= 8, row g + 8 of odd units through the pair table too
+  // (three quarters pair table); M > 8, half and half (its second X fragment loads take
+  // shared-memory bandwidth of their own).
   UnitCodes cb0, cb1;
   if (u0 < u1) load_unit(a, rb, u0, t, bpr, cb0);
   for (int u = u0; u < u1; u += 2) {
     if (u + 1 < u1) load_unit(a, rb, u + 1, t, bpr, cb1);
-    compute_unit<kTall, CB>(a, rbase, u, u0, nblk, g, t, cb0, t8, mean, lane_bits, xs0, xs1,
-                            acc);
+    compute_unit<kTall, CB, false>(a, rbase, u, u0, nblk, g, t, cb0, t8, mean, lane_bits, xs0,
+                                   xs1, acc);
     if (u + 1 < u1) {
       if (u + 2 < u1) load_unit(a, rb, u + 2, t, bpr, cb0);
-      compute_unit<kTall, CB>(a, rbase, u + 1, u0, nblk, g, t, cb1, t8, mean, lane_bits, xs0,
-                              xs1, acc);
+      compute_unit<kTall, CB, !kTall>(a, rbase, u + 1, u0, nblk, g, t, cb1, t8, mean, lane_bits,
+                                      xs0, xs1, acc);
     }
   }
 
