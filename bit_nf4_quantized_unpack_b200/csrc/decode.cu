@@ -649,7 +649,7 @@ size_t decode_scratch_bytes(const DecodePlan& p, const LinearShape& s) {
 
 // K splits and CTAs per split. CTA c takes split c % splits and row groups c / splits,
 // + cps, ...; each of its weight warps one row group at a time over the whole split. The
-// choice minimises the units of the busiest warp (each task charged two extra units for
+// choice minimises the units of the busiest warp (each task charged one extra unit for
 // its pipeline fill and its partial-sum store, and a CTA with fewer than three quarters
 // of its weight warps busy charged for the bandwidth it leaves unused), subject to the X
 // stage fitting its shared-memory budget, at most K / (16 M) splits (the partial sums,
@@ -681,7 +681,7 @@ DecodePlan plan_decode(const LinearShape& s, size_t max_scratch = ~size_t{0}) {
     const int64_t tasks = (per_cta + W - 1) / W;
     const int64_t busy = std::min<int64_t>(per_cta, W);
     const double want = 0.75 * static_cast<double>(W);
-    const double cost = static_cast<double>(tasks * (up + 2)) *
+    const double cost = static_cast<double>(tasks * (up + 1)) *
                         (static_cast<double>(busy) < want ? want / static_cast<double>(busy) : 1.0);
     if (best_cost < 0.0 || cost < best_cost) {
       best_cost = cost;
