@@ -58,6 +58,22 @@ def test_decode_path_small_m(M):
     run_case(inputs.linear_case(200 + M, M, 256, 2048, 16, alpha=32))
 
 
+@pytest.mark.parametrize("M,N,K,r", [
+    (2, 136, 576, 8),      # last 16-row group half full; K ends 64 columns into a 256-wide unit
+    (3, 1024, 2048, 64),
+    (7, 264, 1280, 16),
+    (8, 512, 4096, 16),    # the largest M of the one-MMA-per-step kernel
+    (9, 136, 576, 8),      # the smallest M of the two-MMA kernel, ragged as above
+    (12, 1024, 3072, 32),
+    (15, 256, 2048, 64),
+    (16, 48000, 256, 16),  # one K split: 21 row groups per CTA, so some warps take two
+])
+def test_decode_path_shapes(M, N, K, r):
+    """The decode kernels at token counts between the bench's, with ragged row groups and
+    units, every rank class, and warps that take more than one row group."""
+    run_case(inputs.linear_case(300 + M, M, N, K, r, alpha=2 * r))
+
+
 def test_zero_weight_isolates_lora_term():
     case = inputs.linear_case(7, 300, 256, 512, 16, alpha=32)
     case["W"] = np.zeros_like(case["W"])
