@@ -240,7 +240,9 @@ __global__ void __launch_bounds__(32) k_quantize_prep(unsigned long long* acc) {
 // once in the packed f32x2 form. For m >= 2^-64, 1/m is finite and the
 // residual stays exact for every |x| above 2^-36, far below the smallest threshold
 // magnitude (0.04); blocks with a smaller absmax take plain IEEE division.
-// The code of x comes from the 33-bucket table (two shared-memory loads and one compare).
+// The code of x comes from the bucket table: two shared-memory loads per weight, the
+// threshold test as the sign of one f32x2 difference per two weights, and the byte
+// permutes of pack_codes8 per eight.
 constexpr int kQuantLanes = 4;
 constexpr int kQuantPer = 64 / kQuantLanes;  // elements per lane
 constexpr int kQuantChunks = kQuantPer / 8;  // 8-element loads (and 32-bit code words) per lane

@@ -9,18 +9,20 @@
 //   dependent of whatever ran before on the stream (it launches while that kernel drains
 //   and waits for it to complete before it writes), and it lets the main kernel launch at
 //   once.
-// k_decode_gemv (its programmatic dependent): one CTA per SM. CTA c owns one K split
-//   (split c % splits) and the row groups c / splits, + cps, ... of it. It stages the
-//   split's columns of X in shared memory once (padded so that the MMA operand loads are
-//   conflict-free), then
-//   * its weight warps each take one group of 16 weight rows over the split: lanes stream 32 bytes of packed codes per row with 128-bit loads (the next
-//     256-wide unit while the current one is expanded), double-dequantize them straight
-//     into the A fragments of mma.m16n8k16 (X is the B operand; the dequantized weight
-//     never leaves registers) and store the split's partial sums; the last warp of a row
-//     group to finish adds the splits up, adds scale * T B and writes bf16 Y;
+// k_decode_gemv (its programmatic dependent): one CTA of 16 warps per SM. CTA c owns one
+//   K split (split c % splits) and the row groups c / splits, + cps, ... of it. It builds
+//   its constant tables, waits for k_decode_prep, stages the split's columns of X in
+//   shared memory once (padded so that the MMA operand loads are conflict-free), then
+//   * its 15 weight warps each take one group of 16 weight rows over the split: lanes
+//     stream 32 bytes of packed codes per row with 128-bit loads (the next 256-wide unit
+//     while the current one is expanded), double-dequantize them straight into the A
+//     fragments of mma.m16n8k16 (X is the B operand; the dequantized weight never leaves
+//     registers) and store the split's partial sums; the last warp of a row group to
+//     arrive adds the splits up in a fixed order, adds scale * T B and writes bf16 Y;
 //   * its last warp computes T = X A over its share of the split's rows from the staged X
-//     and adds it into T with fp32 atomics (so T's summation order varies from run to
-//     run, within fp32 rounding); the finishers wait, bounded, until every share is in.
+//     and adds it into T with fp32 reductions (so T's summation order varies from run to
+//     run, within fp32 rounding; Y's does not); the finishers wait, bounded, until every
+//     share is in.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(256) k_decode_prep(float* T, int mr, int* coun
 //
 // Two ways to expand a 64-block of codes, both giving bf16_rn(fl32(L[code] * s)) bit for
 // bit; a warp uses both so that neither the integer ALU nor the shared-memory pipe
-// alone bounds it:
+// alone bounds it (three quarters pair table for M <= 8, half for M > 8):
 //  * the pair table: every byte of codes (two weights) is the index of a shared-memory
 //    entry holding the two fp32 levels; one packed fp32 multiply by s and one bf16x2
 //    conversion give the operand pair. Per byte: one byte permute to form the address,
