@@ -273,21 +273,19 @@ __global__ void __launch_bounds__(kQuantThreads)
   // this thread's part of the mean: fp64 sum and exponent range of its nonzero absmax
   double sum_d = 0.0;
   uint32_t e_lo = 255u, e_hi = 0u;
-  // the next two blocks' elements are in flight while this one is coded
-  Raw8<T> n0[kQuantChunks], n1[kQuantChunks];
+  // the next block's elements are in flight while this one is coded (one buffer: a second
+  // one, rotated by register copies, measured slower)
+  Raw8<T> n0[kQuantChunks];
 #pragma unroll
-  for (int h = 0; h < kQuantChunks; ++h) {
+  for (int h = 0; h < kQuantChunks; ++h)
     if (b < nblocks) n0[h].load(W + b * 64 + sub * kQuantPer + h * 8);
-    if (b + stride < nblocks) n1[h].load(W + (b + stride) * 64 + sub * kQuantPer + h * 8);
-  }
   for (; b < nblocks; b += stride) {
     float v[kQuantPer];
 #pragma unroll
     for (int h = 0; h < kQuantChunks; ++h) n0[h].values(*reinterpret_cast<float(*)[8]>(v + 8 * h));
 #pragma unroll
     for (int h = 0; h < kQuantChunks; ++h) {
-      n0[h] = n1[h];
-      if (b + 2 * stride < nblocks) n1[h].load(W + (b + 2 * stride) * 64 + sub * kQuantPer + h * 8);
+      if (b + stride < nblocks) n0[h].load(W + (b + stride) * 64 + sub * kQuantPer + h * 8);
     }
     float m = fmaxf(fabsf(v[kQuantPer - 2]), fabsf(v[kQuantPer - 1]));
 #pragma unroll
