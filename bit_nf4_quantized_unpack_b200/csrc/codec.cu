@@ -421,10 +421,19 @@ __global__ void __launch_bounds__(256)
        b += static_cast<int64_t>(gridDim.x) * blockDim.x / 32) {
     const int64_t j0 = b * 256 + lane * 8;
     float cc[8];
+    if (j0 + 8 <= nblocks) {  // two 16-byte loads (the absmax array is 256-byte aligned)
+      const float4 a0 = reinterpret_cast<const float4*>(absmax + j0)[0];
+      const float4 a1 = reinterpret_cast<const float4*>(absmax + j0)[1];
+      cc[0] = a0.x; cc[1] = a0.y; cc[2] = a0.z; cc[3] = a0.w;
+      cc[4] = a1.x; cc[5] = a1.y; cc[6] = a1.z; cc[7] = a1.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cc[i] = (j0 + i < nblocks) ? absmax[j0 + i] : mean;
+    }
     float m = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      cc[i] = (j0 + i < nblocks) ? __fsub_rn(absmax[j0 + i], mean) : 0.f;
+      cc[i] = __fsub_rn(cc[i], mean);  // 0 past the end
       m = fmaxf(m, fabsf(cc[i]));
     }
 #pragma unroll
