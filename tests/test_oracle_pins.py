@@ -414,3 +414,35 @@ def test_uniform_codebook_through_the_double_quantized_path():
     assert codes.min() == 0 and codes.max() == 15    # every block's max maps to +-1
     rows = np.array([0, 31, 63])
     np.testing.assert_array_equal(O.double_dequant_rows(q, rows), O.double_dequant(q)[rows])
+
+
+def test_block_absmax_brute_force():
+    """Block absmax against a plain loop over each 64-block (row-major flattening)."""
+    rng = np.random.default_rng(31)
+    w = (rng.standard_normal((6, 192)) * 0.02).astype(np.float32)
+    w[2, 70] = -0.9                      # a negative extreme sets its block's absmax
+    got = O.block_absmax(w)
+    flat = w.ravel()
+    want = [max(abs(float(v)) for v in flat[i:i + 64]) for i in range(0, flat.size, 64)]
+    assert got.dtype == np.float32 and np.array_equal(got, np.float32(want))
+    assert got[(2 * 192 + 70) // 64] == np.float32(0.9)
+
+
+def test_sampled_weight_helper_matches_full_quantization():
+    """The full-size GPU tests build their reference weight with oracle_sampled_weight
+    (every constant, codes on sampled rows and 64-column blocks only). On a small weight
+    it must give the full quantization's constants and codes there."""
+    from tests.gpu_util import oracle_sampled_weight
+    rng = np.random.default_rng(37)
+    N, K = 40, 512
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    rows, blocks = np.array([0, 7, 39]), np.array([0, 3, 7])
+    q_ref, codes_rows, codes_cols = oracle_sampled_weight(W, rows, blocks)
+    full = O.quantize_nf4_dq(W)
+    assert np.array_equal(q_ref["c2"], full["c2"]) and np.array_equal(q_ref["c1"], full["c1"])
+    assert q_ref["mean"] == full["mean"]
+    codes = full["codes"].reshape(N, K // 2)
+    assert np.array_equal(codes_rows, codes[rows])
+    assert np.array_equal(codes_cols, np.concatenate([codes[:, 32 * b:32 * (b + 1)] for b in blocks], 1))
+    # and the reference weight's rows equal the full double dequantization there
+    assert np.array_equal(O.double_dequant_rows(q_ref, rows), O.double_dequant(full)[rows])
